@@ -1,0 +1,422 @@
+#!/usr/bin/env python3
+"""Benchmark of the CKDA forward on B200.
+
+One step = one ckda_chunk_fwd over the 1.3B-model-shaped layer workload
+(B=8, T=4096, H=16, d_k=d_v=128, bf16 q/k/v, fp32 alpha/beta/state, S0 = 0, output
+o and S_T), inputs resident in HBM. Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank processes its own full
+layer batch (the path shards over independent (batch, head) sequences with no
+exchange), timing is the max over ranks and `value` counts all ranks' tokens.
+`--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CKDA fwd tokens/s at H=16,d=128,T=4096; % of tensor-core/HBM roofline"
+WORKLOAD = dict(B=8, T=4096, H=16, dk=128, dv=128)
+BYTES_PER_TOKEN_HEAD = 2 * 128 * 2 + 128 * 2 + 128 * 4 + 4 + 128 * 4   # q,k,v bf16; alpha, beta, o fp32
+FLOPS_PER_TOKEN_HEAD = 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128         # minimal count, chunk 64
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extras", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    """Hash of the sources of the chunk kernel; the committed DRAM-traffic figure is
+    only reported while it matches."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "delta_rule_attention_ckda_b200", "csrc")
+    for rel in ["ckda_api.cu", "kernels/common.cuh", "kernels/chunk_tc.cuh", "kernels/tc_primitives.cuh",
+                "kernels/recurrent.cuh", "kernels/decode.cuh"]:
+        p = os.path.join(csrc, rel)
+        if os.path.exists(p):
+            with open(p, "rb") as f:
+                h.update(rel.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel_key):
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d.get(kernel_key)
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            return float(ent["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import torch
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(device_index)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.gpu], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(inp, n_seq, threads=None):
+    """Run the fp64 oracle on the first n_seq (b, h) sequences of the workload."""
+    import oracle
+    B, T, H, dk, dv = inp.shape
+    pairs = [(i // H, i % H) for i in range(n_seq)]
+    q = torch_stack(inp.q, pairs)
+    k = torch_stack(inp.k, pairs)
+    v = torch_stack(inp.v, pairs)
+    a = torch_stack(inp.alpha, pairs)
+    import torch
+    b = torch.stack([inp.beta[bb, :, h] for bb, h in pairs])[:, :, None]
+    if threads:
+        oracle.set_threads(threads)
+    t0 = time.perf_counter()
+    oracle.oracle_fwd(q, k, v, a, b, None)
+    return time.perf_counter() - t0
+
+
+def torch_stack(x, pairs):
+    import torch
+    return torch.stack([x[b, :, h] for b, h in pairs])[:, :, None]
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(inp, target_s=12.0):
+    import oracle
+    oracle.build()
+    cores = cpu_cores()
+    oracle.set_threads(cores)
+    B, T, H, dk, dv = inp.shape
+    t1 = oracle_sample(inp, min(cores, B * H))       # calibration: one sequence per core
+    per_round = max(t1, 1e-3)
+    rounds = max(1, min(int(target_s / per_round), (B * H) // min(cores, B * H)))
+    n_seq = min(B * H, rounds * min(cores, B * H))
+    dt = oracle_sample(inp, n_seq)
+    tokens = n_seq * T / H            # token-heads / H = tokens with all heads
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_seq} of {B * H} (batch, head) sequences x T={T} of the layer workload, "
+                      f"fp64 sequential loop, OpenMP over sequences, {dt:.2f} s wall",
+            "seconds": dt}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def reference_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from ckda_inputs import make_workload
+    import oracle
+    oracle.build()
+    inp = make_workload("layer")
+    B, T, H, dk, dv = inp.shape
+    cores = cpu_cores()
+    oracle.set_threads(cores)
+    n_seq = min(B * H, cores)
+    for _ in range(args.warmup):
+        oracle_sample(inp, n_seq)
+    times = [oracle_sample(inp, n_seq) for _ in range(args.steps)]
+    tot = sum(times)
+    tokens = n_seq * T / H * args.steps
+    value = tokens / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "layer B=8 T=4096 H=16 dk=dv=128", **WORKLOAD,
+                       "sample_per_step": f"{n_seq} (batch, head) sequences x T={T}"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {n_seq} of {B * H} sequences x T={T}, fp64 oracle"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_launches(fn, steps, stream):
+    import torch
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        fn()
+    ev1.record(stream)
+    ev1.synchronize()
+    return ev0.elapsed_time(ev1) / 1e3
+
+
+def ours_arm(args):
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    import delta_rule_attention_ckda_b200 as ck
+    from ckda_inputs import make_workload
+    ck.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    inp = make_workload("layer")
+    B, T, H, dk, dv = inp.shape
+    q, k, v, a, b = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
+    o = torch.empty(B, T, H, dv, device=dev)
+    ST = torch.empty(B, H, dk, dv, device=dev)
+    wsb = ck.workspace_bytes(B, T, H, dk, dv)
+    ws = torch.empty(max(wsb, 16), device=dev, dtype=torch.uint8)
+    path = "chunk_tc" if ck.chunk_path(B, T, H, dk, dv) == ck.PATH_CHUNK_TC else "recurrent"
+
+    def step():
+        ck.chunk_fwd(q, k, v, a, b, None, o=o, S_T=ST, workspace=ws if wsb else None)
+
+    for _ in range(args.warmup):
+        step()
+    assert ck.get_device_error() == 0
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    sampler.start()
+    time.sleep(0.15)
+    barrier(world)
+    secs = time_launches(step, args.steps, stream)
+    barrier(world)
+    clocks = sampler.stop()
+    if ck.get_device_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+    secs = max_over_ranks(secs, world)
+    tokens = B * T * world * args.steps
+    value = tokens / secs
+    per_launch = secs / args.steps
+    alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD + B * H * dk * dv * 4
+    hbm, src = peaks()
+    achieved = alg_bytes / per_launch / 1e9
+    kernel_key = f"chunk_fwd_{path}_layer"
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": committed_traffic(kernel_key),
+            "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6.65 TB/s",
+            "kernel": kernel_key, "alg_bytes_per_launch": alg_bytes,
+            "tflops_minimal": B * T * H * FLOPS_PER_TOKEN_HEAD / per_launch / 1e12}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_launch,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "layer B=8 T=4096 H=16 dk=dv=128 chunk=64", **WORKLOAD,
+                       "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
+                       "path": path, "l2": "inputs larger than L2 (~950 MB per step vs 126 MB), no flush",
+                       "state": "S0 = 0 (not read), S_T written"},
+            "roofline": roof, "gpu_launches": args.steps, "clocks": clocks}
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_measure(ck, inp, dev, stream, world, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    if not args.no_extras:
+        line["decode"] = decode_measure(ck, dev, stream, world)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_measure(ck, inp, dev, stream, world, args):
+    """Same metric through the public Python API with pinned host buffers; every step
+    copies its inputs host->device and reads o and S_T back."""
+    import torch
+    B, T, H, dk, dv = inp.shape
+    hq, hk, hv, ha, hb = (x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
+    ho = torch.empty(B, T, H, dv, pin_memory=True)
+    hS = torch.empty(B, H, dk, dv, pin_memory=True)
+    dq, dk_, dv_, da, db = (torch.empty_like(x, device=dev) for x in (hq, hk, hv, ha, hb))
+
+    def step():
+        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (da, ha), (db, hb)):
+            d.copy_(h, non_blocking=True)
+        o, S = ck.chunk_fwd(dq, dk_, dv_, da, db, None)
+        ho.copy_(o, non_blocking=True)
+        hS.copy_(S, non_blocking=True)
+
+    step()
+    n = max(3, min(args.steps, 5))
+    barrier(world)
+    secs = time_launches(step, n, stream)
+    secs = max_over_ranks(secs, world)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, hb))
+    d2h = ho.numel() * 4 + hS.numel() * 4
+    return {"value": B * T * world * n / secs, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n}
+
+
+def decode_measure(ck, dev, stream, world):
+    """The decode workload: 256 sequences x 16 heads, d = 128, fp32 state updated in
+    place, 1024 calls (call t reads input set t % 64)."""
+    import torch
+    from ckda_inputs import DECODE, make_decode_pool
+    pool = make_decode_pool()
+    P, N, H, D = DECODE["pool"], DECODE["N"], DECODE["H"], DECODE["dk"]
+    dq, dk_, dv_, da, db = (x.to(dev) for x in (pool.q, pool.k, pool.v, pool.alpha, pool.beta))
+    S = pool.S0.to(dev)
+    o = torch.empty(N, H, D, device=dev)
+    calls = DECODE["steps"]
+    for t in range(8):
+        ck.decode_step(dq[t % P], dk_[t % P], dv_[t % P], da[t % P], db[t % P], S, o=o)
+    barrier(world)
+    it = iter(range(calls))
+
+    def one():
+        t = next(it)
+        ck.decode_step(dq[t % P], dk_[t % P], dv_[t % P], da[t % P], db[t % P], S, o=o)
+
+    secs = time_launches(one, calls, stream)
+    assert ck.get_device_error() == 0
+    secs = max_over_ranks(secs, world)
+    per = secs / calls
+    bytes_call = N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4)
+    hbm, src = peaks()
+    gbs = bytes_call / per / 1e9
+    return {"workload": "decode N=256 H=16 d=128 fp32 state, 1024 calls", "us_per_call": per * 1e6,
+            "tokens_per_s": N * world / per, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+                                                         "unit": "GB/s", "frac": gbs / hbm,
+                                                         "alg_bytes_per_launch": bytes_call,
+                                                         "kernel": "decode128"},
+            "gpu_launches": calls}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return ours_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,178 @@
+"""ctypes binding of libckda.so (argument marshalling only; every step runs in CUDA).
+
+The functions here take torch CUDA tensors, check dtype/shape/contiguity on the host,
+and pass raw device pointers plus the current CUDA stream to the C ABI declared in
+include/ckda.h. There is no fallback: if the library is missing or the tensors are
+not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libckda.so")
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported request", 3: "pointer not 16-byte aligned",
+          4: "CUDA error", 5: "device wait timed out", 6: "workspace missing or too small"}
+F32, BF16 = 0, 1
+PATH_RECURRENT, PATH_CHUNK_TC = 0, 1
+
+
+class CkdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, 'unknown')} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libckda.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libckda.so not found at {path}; run delta_rule_attention_ckda_b200/build.py")
+    lib = ctypes.CDLL(path)
+    vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ckda_abi_version.restype = i
+    lib.ckda_status_string.argtypes = [i]
+    lib.ckda_status_string.restype = ctypes.c_char_p
+    lib.ckda_chunk_fwd_workspace_bytes.argtypes = [i] * 6
+    lib.ckda_chunk_fwd_workspace_bytes.restype = sz
+    lib.ckda_chunk_fwd_path.argtypes = [i] * 6
+    lib.ckda_chunk_fwd_path.restype = i
+    lib.ckda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 6 + [vp, sz, vp]
+    lib.ckda_chunk_fwd.restype = i
+    lib.ckda_recurrent_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 6 + [vp]
+    lib.ckda_recurrent_fwd.restype = i
+    lib.ckda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 5 + [vp]
+    lib.ckda_decode_step.restype = i
+    lib.ckda_get_device_error.argtypes = [vp]
+    lib.ckda_get_device_error.restype = i
+    _lib = lib
+    return lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _raise(status: int, where: str):
+    if status != 0:
+        raise CkdaError(status, where)
+
+
+def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    return int(load().ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
+
+
+def chunk_path(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    return int(load().ckda_chunk_fwd_path(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
+
+
+def _fwd_common(q, k, v, alpha, beta, S0, o, S_T):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _check(q, "q", (B, T, H, dk))
+    _check(k, "k", (B, T, H, dk), dt)
+    _check(v, "v", (B, T, H, dv), dt)
+    _check(alpha, "alpha", (B, T, H, dk), torch.float32)
+    _check(beta, "beta", (B, T, H), torch.float32)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    if o is None:
+        o = torch.empty(B, T, H, dv, device=q.device, dtype=torch.float32)
+    _check(o, "o", (B, T, H, dv), torch.float32)
+    if S_T is not None:
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32)
+    return B, T, H, dk, dv, _dt(q), o
+
+
+def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
+              workspace=None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """ckda_chunk_fwd. Returns (o, S_T). Allocates o / S_T / workspace with torch when
+    not given (the library itself never allocates)."""
+    B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
+    if S_T is None and want_state:
+        S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
+    lib = load()
+    need = int(lib.ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt))
+    if need and workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ckda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o),
+                            _ptr(S_T), B, T, H, dk, dv, dt, _ptr(workspace), wbytes, _stream(stream))
+    _raise(st, "ckda_chunk_fwd")
+    return o, S_T
+
+
+def recurrent_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """ckda_recurrent_fwd (fp32 SIMT token-by-token kernel). Returns (o, S_T)."""
+    B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
+    if S_T is None and want_state:
+        S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
+    st = load().ckda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                   _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _stream(stream))
+    _raise(st, "ckda_recurrent_fwd")
+    return o, S_T
+
+
+def decode_step(q, k, v, alpha, beta, S, *, o=None, stream=None) -> torch.Tensor:
+    """ckda_decode_step: updates S [N,H,dk,dv] in place, returns o [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _check(q, "q", (N, H, dk))
+    _check(k, "k", (N, H, dk), dt)
+    _check(v, "v", (N, H, dv), dt)
+    _check(alpha, "alpha", (N, H, dk), torch.float32)
+    _check(beta, "beta", (N, H), torch.float32)
+    _check(S, "S", (N, H, dk, dv), torch.float32)
+    if o is None:
+        o = torch.empty(N, H, dv, device=q.device, dtype=torch.float32)
+    _check(o, "o", (N, H, dv), torch.float32)
+    st = load().ckda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                                 _ptr(o), N, H, dk, dv, _dt(q), _stream(stream))
+    _raise(st, "ckda_decode_step")
+    return o
+
+
+def get_device_error(stream=None) -> int:
+    """ckda_get_device_error: synchronises the stream; returns the status code."""
+    return int(load().ckda_get_device_error(_stream(stream)))

@@ -1,0 +1,182 @@
+// Host side of the CKDA C ABI (see include/ckda.h): argument validation, path
+// selection and kernel launches. Nothing here allocates device memory.
+#include "ckda.h"
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "kernels/common.cuh"
+#include "kernels/recurrent.cuh"
+#include "kernels/decode.cuh"
+#include "kernels/chunk_tc.cuh"
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool dims_ok(int dk, int dv) {
+    return dk >= 1 && dk <= CKDA_MAX_D && dv >= 1 && dv <= CKDA_MAX_D;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+ckda_status_t launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+// T = 0: S_T <- S0 (or zero).
+ckda_status_t copy_state(const float* S0, float* S_T, size_t n, cudaStream_t st) {
+    if (S_T == nullptr || S_T == S0) return CKDA_OK;
+    cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, n * sizeof(float), cudaMemcpyDeviceToDevice, st)
+                       : cudaMemsetAsync(S_T, 0, n * sizeof(float), st);
+    return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+template <typename TIn>
+ckda_status_t launch_recurrent(const TIn* q, const TIn* k, const TIn* v, const float* alpha,
+                               const float* beta, const float* S0, float* o, float* S_T,
+                               int B, int T, int H, int dk, int dv, cudaStream_t st) {
+    const int cols = dv <= 32 ? 32 : (dv <= 64 ? 64 : 128);
+    // Few sequences: split the columns over more CTAs (one warp each).
+    const long long seqs = (long long)B * H;
+    const int cols_per_cta = (seqs * ((dv + cols - 1) / cols) < 148) ? 32 : cols;
+    dim3 grid((unsigned)seqs, (unsigned)((dv + cols_per_cta - 1) / cols_per_cta));
+    dim3 block((unsigned)cols_per_cta);
+#define CKDA_LAUNCH_REC(DKT)                                                                  \
+    ckda::recurrent_fwd_kernel<DKT, TIn><<<grid, block, 0, st>>>(q, k, v, alpha, beta, S0, o, \
+                                                                  S_T, T, H, dk, dv, cols_per_cta)
+    if (dk <= 16) CKDA_LAUNCH_REC(16);
+    else if (dk <= 32) CKDA_LAUNCH_REC(32);
+    else if (dk <= 64) CKDA_LAUNCH_REC(64);
+    else CKDA_LAUNCH_REC(128);
+#undef CKDA_LAUNCH_REC
+    return launch_status();
+}
+
+ckda_status_t check_fwd_args(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, const float* o,
+                             const float* S_T, int B, int T, int H, int dk, int dv,
+                             ckda_dtype_t dt) {
+    if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
+    if (dt != CKDA_F32 && dt != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
+    const bool any_tokens = (long long)B * T * H > 0;
+    if (any_tokens && (!q || !k || !v || !alpha || !beta || !o)) return CKDA_ERR_INVALID_ARG;
+    const void* ptrs[8] = {q, k, v, alpha, beta, S0, o, S_T};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return CKDA_ERR_MISALIGNED;
+    return CKDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ckda_abi_version(void) { return CKDA_ABI_VERSION; }
+
+const char* ckda_status_string(ckda_status_t s) {
+    switch (s) {
+        case CKDA_OK: return "ok";
+        case CKDA_ERR_INVALID_ARG: return "invalid argument";
+        case CKDA_ERR_UNSUPPORTED: return "unsupported request";
+        case CKDA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case CKDA_ERR_CUDA: return "CUDA error";
+        case CKDA_ERR_TIMEOUT: return "device wait timed out";
+        case CKDA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+ckda_path_t ckda_chunk_fwd_path(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {
+    (void)B; (void)T; (void)H;
+    return ckda::chunk_tc_supported(dk, dv, dt) ? CKDA_PATH_CHUNK_TC : CKDA_PATH_RECURRENT;
+}
+
+size_t ckda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {
+    if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return 0;
+    if (ckda_chunk_fwd_path(B, T, H, dk, dv, dt) != CKDA_PATH_CHUNK_TC) return 0;
+    return ckda::chunk_tc_workspace_bytes(B, T, H, dk, dv);
+}
+
+ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, const float* S0,
+                                 float* o, float* S_T, int B, int T, int H, int dk, int dv,
+                                 ckda_dtype_t dt, void* stream) {
+    ckda_status_t s = check_fwd_args(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt);
+    if (s != CKDA_OK) return s;
+    cudaStream_t st = as_stream(stream);
+    if ((long long)B * H == 0) return CKDA_OK;
+    if (T == 0) return copy_state(S0, S_T, (size_t)B * H * dk * dv, st);
+    if (dt == CKDA_BF16)
+        return launch_recurrent(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                static_cast<const __nv_bfloat16*>(v), alpha, beta, S0, o, S_T, B, T, H,
+                                dk, dv, st);
+    return launch_recurrent(static_cast<const float*>(q), static_cast<const float*>(k),
+                            static_cast<const float*>(v), alpha, beta, S0, o, S_T, B, T, H, dk, dv, st);
+}
+
+ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, float* o, float* S_T, int B,
+                             int T, int H, int dk, int dv, ckda_dtype_t dt, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    ckda_status_t s = check_fwd_args(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt);
+    if (s != CKDA_OK) return s;
+    const size_t need = ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return CKDA_ERR_MISALIGNED;
+    cudaStream_t st = as_stream(stream);
+    if ((long long)B * H == 0) return CKDA_OK;
+    if (T == 0) return copy_state(S0, S_T, (size_t)B * H * dk * dv, st);
+    if (ckda_chunk_fwd_path(B, T, H, dk, dv, dt) == CKDA_PATH_CHUNK_TC) {
+        cudaError_t e = ckda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
+                                              static_cast<const __nv_bfloat16*>(k),
+                                              static_cast<const __nv_bfloat16*>(v), alpha, beta,
+                                              S0, o, S_T, B, T, H, dk, dv, workspace, st);
+        return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+    }
+    return ckda_recurrent_fwd(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt, stream);
+}
+
+ckda_status_t ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                               const float* beta, float* S, float* o, int N, int H, int dk,
+                               int dv, ckda_dtype_t dt, void* stream) {
+    if (N < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
+    if (dt != CKDA_F32 && dt != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
+    const long long seqs = (long long)N * H;
+    if (seqs == 0) return CKDA_OK;
+    if (seqs > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !S || !o) return CKDA_ERR_INVALID_ARG;
+    const void* ptrs[7] = {q, k, v, alpha, beta, S, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return CKDA_ERR_MISALIGNED;
+    cudaStream_t st = as_stream(stream);
+    if (dk == 128 && dv == 128) {
+        if (dt == CKDA_BF16)
+            ckda::decode128_kernel<__nv_bfloat16><<<(unsigned)seqs, 256, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                static_cast<const __nv_bfloat16*>(v), alpha, beta, S, o);
+        else
+            ckda::decode128_kernel<float><<<(unsigned)seqs, 256, 0, st>>>(
+                static_cast<const float*>(q), static_cast<const float*>(k),
+                static_cast<const float*>(v), alpha, beta, S, o);
+        return launch_status();
+    }
+    // Other sizes: a decode step is the recurrent forward with T = 1, S in place.
+    return ckda_recurrent_fwd(q, k, v, alpha, beta, S, o, S, N, 1, H, dk, dv, dt, stream);
+}
+
+ckda_status_t ckda_get_device_error(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CKDA_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, ckda::g_error_word, sizeof(word)) != cudaSuccess)
+        return CKDA_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(ckda::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+        return CKDA_ERR_CUDA;
+    if (word & ckda::kErrTimeout) return CKDA_ERR_TIMEOUT;
+    return CKDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// Token-by-token CKDA forward on CUDA cores, fp32 (any d_k, d_v <= 128).
+//
+// Recurrence (blog post "One update, one quarter-turn", section "The mirror"):
+//   S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T,  o_t = S_t^T q_t,
+// evaluated in delta form: S <- Diag(a)S; u = b (v - S^T k); S <- S + k u^T; o = S^T q.
+//
+// The columns of S evolve independently (every operation above acts on S from the
+// left or adds k u^T column by column), so each thread owns one state column
+// S[:, j] in registers and needs no reduction across threads: y_j = S[:,j].k and
+// o_j = S[:,j].q are thread-local dot products. A CTA of up to 128 threads covers up
+// to 128 columns of one (b, h) and stages TB tokens of k, q, alpha in shared memory
+// (broadcast reads). Rows beyond d_k are padded with k = q = alpha = 0, which keeps
+// them exactly zero.
+#pragma once
+#include "common.cuh"
+
+namespace ckda {
+
+template <int DK, typename TIn>
+__global__ void __launch_bounds__(128)
+recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                     const TIn* __restrict__ v, const float* __restrict__ alpha,
+                     const float* __restrict__ beta, const float* S0,
+                     float* __restrict__ o, float* ST,
+                     int T, int H, int dk, int dv, int cols_per_cta) {
+    constexpr int TB = 16;                       // tokens staged per batch
+    __shared__ float sk[TB][DK], sq[TB][DK], sa[TB][DK];
+    __shared__ float sv[TB][128];
+    __shared__ float sb[TB];
+
+    const int bh = blockIdx.x;
+    const int b = bh / H, h = bh % H;
+    const int j = blockIdx.y * cols_per_cta + threadIdx.x;
+    const bool active = (threadIdx.x < cols_per_cta) && (j < dv);
+    const size_t state_base = (size_t)bh * dk * dv;
+
+    float s[DK];
+#pragma unroll
+    for (int i = 0; i < DK; ++i)
+        s[i] = (active && S0 != nullptr && i < dk) ? S0[state_base + (size_t)i * dv + j] : 0.f;
+
+    for (int t0 = 0; t0 < T; t0 += TB) {
+        const int nt = min(TB, T - t0);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < nt * DK; idx += blockDim.x) {
+            const int tt = idx / DK, i = idx % DK;
+            const size_t tok = ((size_t)b * T + t0 + tt) * H + h;
+            const bool in = i < dk;
+            sk[tt][i] = in ? ld_in(k + tok * dk + i) : 0.f;
+            sq[tt][i] = in ? ld_in(q + tok * dk + i) : 0.f;
+            sa[tt][i] = in ? __ldg(alpha + tok * dk + i) : 0.f;
+        }
+        if (threadIdx.x < nt) sb[threadIdx.x] = __ldg(beta + ((size_t)b * T + t0 + threadIdx.x) * H + h);
+        for (int tt = 0; tt < nt; ++tt) {
+            const size_t tok = ((size_t)b * T + t0 + tt) * H + h;
+            sv[tt][threadIdx.x] = active ? ld_in(v + tok * dv + j) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int tt = 0; tt < nt; ++tt) {
+            float y = 0.f;
+#pragma unroll
+            for (int i = 0; i < DK; ++i) {
+                s[i] *= sa[tt][i];
+                y = fmaf(s[i], sk[tt][i], y);
+            }
+            const float u = sb[tt] * (sv[tt][threadIdx.x] - y);
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < DK; ++i) {
+                s[i] = fmaf(sk[tt][i], u, s[i]);
+                acc = fmaf(s[i], sq[tt][i], acc);
+            }
+            if (active) o[(((size_t)b * T + t0 + tt) * H + h) * dv + j] = acc;
+        }
+    }
+    if (active && ST != nullptr) {
+#pragma unroll
+        for (int i = 0; i < DK; ++i)
+            if (i < dk) ST[state_base + (size_t)i * dv + j] = s[i];
+    }
+}
+
+}  // namespace ckda

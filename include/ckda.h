@@ -1,0 +1,156 @@
+/*
+ * ckda.h - C ABI of the CKDA (Complex Kimi Delta Attention) forward library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (Complex KDA: Understanding and Enhancing the Expressivity of Kimi
+ * Delta Attention, as summarised by the blog post "One update, one quarter-turn",
+ * section "The mirror", and by the ai.info summary, "What This Paper Is About"):
+ * for every (batch b, head h) a d_k x d_v state S evolves token by token as
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t                   (read after the update, no 1/sqrt(d) scale)
+ *
+ * with a signed per-channel gate alpha_t in [-1,1]^{d_k}, a step beta_t in [0,2]
+ * and a unit key ||k_t|| = 1 (ai.info summary, "Key Contributions", Theorem 1).
+ * Those ranges are preconditions on device data and are NOT checked; values outside
+ * them (beta > 2, |alpha| > 1) are computed as given.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All pointers are DEVICE pointers owned by the caller. The library allocates no
+ *   device memory and keeps no per-call state; the only global state is one device
+ *   error word per GPU (see ckda_get_device_error) and cached kernel attributes.
+ * - Layout is contiguous row-major, head-interleaved:
+ *       q, k, alpha : [B, T, H, d_k]     v, o : [B, T, H, d_v]     beta : [B, T, H]
+ *       S0, S_T, S  : [B, H, d_k, d_v]   (d_v fastest)
+ *   q, k, v have the dtype named by `dt`; alpha, beta, states and o are fp32.
+ * - Every base pointer must be 16-byte aligned (CKDA_ERR_MISALIGNED otherwise).
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   Calls are asynchronous on that stream and never synchronise the host, except
+ *   ckda_get_device_error.
+ * - Argument errors return before anything is launched. A failed launch returns
+ *   CKDA_ERR_CUDA. Device-side failures (a bounded wait that ran out) are recorded
+ *   in the device error word and reported by ckda_get_device_error.
+ * - 1 <= d_k, d_v <= 128. T >= 0 (T = 0 writes S_T = S0 and no o).
+ *
+ * This header needs no CUDA or torch header.
+ */
+#ifndef CKDA_H_
+#define CKDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CKDA_API __attribute__((visibility("default")))
+#else
+#define CKDA_API
+#endif
+
+#define CKDA_MAX_D 128
+#define CKDA_ABI_VERSION 1
+
+typedef enum {
+    CKDA_OK = 0,
+    CKDA_ERR_INVALID_ARG = 1,   /* null required pointer, bad size, bad dtype        */
+    CKDA_ERR_UNSUPPORTED = 2,   /* valid request the library cannot serve            */
+    CKDA_ERR_MISALIGNED = 3,    /* a base pointer is not 16-byte aligned             */
+    CKDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed              */
+    CKDA_ERR_TIMEOUT = 5,       /* a device-side bounded wait ran out                */
+    CKDA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required        */
+} ckda_status_t;
+
+typedef enum {
+    CKDA_F32 = 0,               /* q, k, v are float32                               */
+    CKDA_BF16 = 1               /* q, k, v are bfloat16                              */
+} ckda_dtype_t;
+
+/* Which kernel family ckda_chunk_fwd selects for a problem. */
+typedef enum {
+    CKDA_PATH_RECURRENT = 0,    /* fp32 SIMT token-by-token kernel (any d <= 128)    */
+    CKDA_PATH_CHUNK_TC = 1      /* chunked WY/UT kernel on tcgen05 tensor cores      */
+} ckda_path_t;
+
+/* Version of this ABI (CKDA_ABI_VERSION). */
+CKDA_API int ckda_abi_version(void);
+
+/* Human-readable name of a status code; never NULL, static storage. */
+CKDA_API const char* ckda_status_string(ckda_status_t status);
+
+/*
+ * Bytes of device workspace ckda_chunk_fwd needs for this problem (may be 0).
+ * Invalid sizes return 0; ckda_chunk_fwd then rejects them.
+ */
+CKDA_API size_t ckda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
+
+/* The path ckda_chunk_fwd takes for these sizes (for tests and reporting). */
+CKDA_API ckda_path_t ckda_chunk_fwd_path(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
+
+/*
+ * Chunked forward (prefill / training forward without gradients).
+ * Evaluates the recurrence above for all T tokens of every (b, h) and writes every
+ * o_t and, if S_T != NULL, the final state. The tensor-core path splits the sequence
+ * into chunks of 64 tokens and evaluates each chunk in the WY/UT form (the
+ * "Chunk-WY" kernels named on the thelatestinai card) with the signed gate carried
+ * as sign parity plus log-magnitude (ai.info summary, "Methodology": sign separated
+ * from the log-space gate magnitude); other shapes take the recurrent path. Both
+ * compute the same map; results agree with the sequential fp64 definition within
+ * rounding.
+ *   q, k     [B,T,H,dk] dt        v      [B,T,H,dv] dt
+ *   alpha    [B,T,H,dk] fp32      beta   [B,T,H]    fp32
+ *   S0       [B,H,dk,dv] fp32 or NULL (zero initial state)
+ *   o        [B,T,H,dv] fp32 out
+ *   S_T      [B,H,dk,dv] fp32 out or NULL; may equal S0 (in-place update)
+ *   workspace: device buffer of at least ckda_chunk_fwd_workspace_bytes(...) bytes,
+ *              owned by the caller (NULL allowed when that size is 0).
+ * o must not overlap any input. Returns CKDA_OK or an error status (nothing launched
+ * on argument errors).
+ */
+CKDA_API ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v,
+                             const float* alpha, const float* beta, const float* S0,
+                             float* o, float* S_T,
+                             int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Token-by-token forward on CUDA cores in fp32 (the recurrent path of
+ * ckda_chunk_fwd, callable directly). Same arguments and semantics as
+ * ckda_chunk_fwd, no workspace. Each thread keeps one state column resident in
+ * registers; the state is read once and written once.
+ */
+CKDA_API ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, const float* S0,
+                                 float* o, float* S_T,
+                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                 void* stream);
+
+/*
+ * One recurrent decode step for N independent sequences (blog post "One update,
+ * one quarter-turn", section "The whiteboard": each token erases a little and writes
+ * a little into a fixed-size state). Updates S in place and writes o:
+ *     S <- (I - beta k k^T) Diag(alpha) S + beta k v^T,   o = S^T q   (new S)
+ *   q, k   [N,H,dk] dt      v [N,H,dv] dt      alpha [N,H,dk] fp32   beta [N,H] fp32
+ *   S      [N,H,dk,dv] fp32, read and written exactly once per element
+ *   o      [N,H,dv] fp32 out (must not overlap S)
+ */
+CKDA_API ckda_status_t ckda_decode_step(const void* q, const void* k, const void* v,
+                               const float* alpha, const float* beta,
+                               float* S, float* o,
+                               int N, int H, int dk, int dv, ckda_dtype_t dt, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this GPU's device error word.
+ * Returns CKDA_OK, CKDA_ERR_TIMEOUT (a bounded device wait ran out; the kernel
+ * returned early and its outputs are invalid) or CKDA_ERR_CUDA (a sticky CUDA error;
+ * the context is unusable).
+ */
+CKDA_API ckda_status_t ckda_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CKDA_H_ */

@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol include/ckda.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ckda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from delta_rule_attention_ckda_b200 import build
+    build.build()
+    import delta_rule_attention_ckda_b200 as ck
+    return ck.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"CKDA_API\s+[\w\s\*]+?\b(ckda_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ["ckda_chunk_fwd", "ckda_decode_step", "ckda_chunk_fwd_workspace_bytes",
+                 "ckda_status_string", "ckda_get_device_error", "ckda_recurrent_fwd"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_exports_match_nm(lib):
+    import subprocess
+    import delta_rule_attention_ckda_b200 as ck
+    out = subprocess.run(["nm", "-D", "--defined-only", ck.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ckda_\w+)", out))
+    assert set(declared_symbols()) <= exported
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.ckda_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.ckda_status_string(99) == b"unknown status"
+    assert lib.ckda_abi_version() == 1
+
+
+NULL = None
+
+
+def call_fwd(lib, fn, q=NULL, k=NULL, v=NULL, a=NULL, b=NULL, S0=NULL, o=NULL, ST=NULL,
+             B=1, T=4, H=1, dk=16, dv=16, dt=1):
+    args = [ctypes.c_void_p(x) if x is not None else None for x in (q, k, v, a, b, S0, o, ST)]
+    if fn == "ckda_chunk_fwd":
+        return lib.ckda_chunk_fwd(*args, B, T, H, dk, dv, dt, None, 0, None)
+    return lib.ckda_recurrent_fwd(*args, B, T, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("fn", ["ckda_chunk_fwd", "ckda_recurrent_fwd"])
+def test_rejects_bad_sizes_before_launch(lib, fn):
+    # none of these reaches a launch, so the fake pointers are never dereferenced
+    p = 0x10000
+    assert call_fwd(lib, fn, p, p, p, p, p, None, p, None, dk=0) == 1
+    assert call_fwd(lib, fn, p, p, p, p, p, None, p, None, dv=129) == 1
+    assert call_fwd(lib, fn, p, p, p, p, p, None, p, None, B=-1) == 1
+    assert call_fwd(lib, fn, p, p, p, p, p, None, p, None, T=-5) == 1
+    assert call_fwd(lib, fn, p, p, p, p, p, None, p, None, dt=7) == 1
+
+
+@pytest.mark.parametrize("fn", ["ckda_chunk_fwd", "ckda_recurrent_fwd"])
+def test_rejects_null_and_misaligned(lib, fn):
+    p = 0x10000
+    assert call_fwd(lib, fn, None, p, p, p, p, None, p, None) == 1       # q missing
+    assert call_fwd(lib, fn, p, p, p, p, p, None, None, None) == 1       # o missing
+    assert call_fwd(lib, fn, p + 4, p, p, p, p, None, p, None) == 3      # q misaligned
+    assert call_fwd(lib, fn, p, p, p, p, p, p + 8, p, None) == 3         # S0 misaligned
+    assert call_fwd(lib, fn, p, p, p, p, p, None, p, p + 2) == 3         # S_T misaligned
+
+
+def test_decode_rejects(lib):
+    p = ctypes.c_void_p(0x10000)
+    bad = ctypes.c_void_p(0x10004)
+    assert lib.ckda_decode_step(p, p, p, p, p, p, p, 4, 2, 0, 16, 1, None) == 1
+    assert lib.ckda_decode_step(p, p, p, p, p, p, p, 4, 2, 16, 200, 1, None) == 1
+    assert lib.ckda_decode_step(p, p, p, p, p, None, p, 4, 2, 16, 16, 1, None) == 1
+    assert lib.ckda_decode_step(p, p, p, p, p, bad, p, 4, 2, 16, 16, 1, None) == 3
+    assert lib.ckda_decode_step(p, p, p, p, p, p, p, 4, 2, 16, 16, 3, None) == 1
+
+
+def test_empty_problems_launch_nothing(lib):
+    # B*H == 0 returns OK without touching CUDA
+    assert call_fwd(lib, "ckda_chunk_fwd", None, None, None, None, None, None, None, None,
+                    B=0) == 0
+    assert lib.ckda_decode_step(None, None, None, None, None, None, None, 0, 4, 16, 16, 1,
+                                None) == 0
+
+
+def test_workspace_query_and_path(lib):
+    assert lib.ckda_chunk_fwd_workspace_bytes(1, 10, 1, 0, 16, 1) == 0
+    for dt in (0, 1):
+        assert lib.ckda_chunk_fwd_path(2, 100, 4, 16, 16, dt) in (0, 1)
+    # fp32 inputs always take the recurrent path (the tensor-core path is bf16-only)
+    assert lib.ckda_chunk_fwd_path(8, 4096, 16, 128, 128, 0) == 0
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    import delta_rule_attention_ckda_b200 as ck
+    x = torch.zeros(1, 4, 1, 16)
+    with pytest.raises(ValueError):
+        ck.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
