@@ -10,6 +10,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libckda.so")
+SELFTEST_LIB = os.path.join(PKG, "libckda_selftest.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
@@ -17,8 +18,7 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std
          "-Xptxas", "-warn-spills"]
 
 
-def sources():
-    return [os.path.join(CSRC, "ckda_api.cu")]
+TARGETS = {LIB: "ckda_api.cu", SELFTEST_LIB: "selftest.cu"}
 
 
 def _newest_input():
@@ -28,16 +28,22 @@ def _newest_input():
     return max(os.path.getmtime(f) for f in files)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def _build_one(lib: str, src: str, force: bool, verbose: bool, extra) -> None:
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= _newest_input():
+        return
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           *sources(), "-o", tmp, "-lcuda"]
+           os.path.join(CSRC, src), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Build libckda.so and the test-only libckda_selftest.so; returns libckda.so's path."""
+    for lib, src in TARGETS.items():
+        _build_one(lib, src, force, verbose, extra)
     return LIB
 
 
