@@ -1,23 +1,675 @@
-// Chunked WY/UT CKDA forward on tcgen05 tensor cores (sm_100a).
+// Chunked WY/UT CKDA forward on tcgen05 tensor cores (sm_100a), d_k = d_v = 128.
+//
+// Recurrence (blog post "One update, one quarter-turn", section "The mirror"):
+//   S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T,   o_t = S_t^T q_t.
+//
+// Chunk form (C = 64 tokens, S0 = state entering the chunk, r, s positions in it):
+//   Gamma_r = prod_{j<=r} a_j, carried as a sign parity and a log2-magnitude sum,
+//             because a signed gate has no logarithm (ai.info summary, "Methodology":
+//             sign separated from the log-space gate magnitude);
+//   A_rs    = b_r k_r^T Diag(Gamma_r/Gamma_s) k_s   (s < r),
+//   P_rs    =     q_r^T Diag(Gamma_r/Gamma_s) k_s   (s <= r),
+//   T       = (I + A)^{-1} Diag(b)                   (UT transform, forward solve),
+//   U~ = T V,  W = T (Gamma (.) K),  U = U~ - W S0,
+//   O  = (Gamma (.) Q) S0 + P U,
+//   S_C = Diag(Gamma_C) S0 + ((Gamma_C/Gamma) (.) K)^T U.
+// In exact arithmetic this equals the token loop; the WY/UT evaluation is the
+// "Chunk-WY" scheme the thelatestinai card names, derived here for the signed gate.
+//
+// B200 mapping. One CTA (256 threads) owns one (batch, head) and walks its chunks in
+// order. Everything is computed transposed, so the 128 feature rows sit on the 128
+// TMEM lanes: the fp32 state lives in TMEM as S^T for the whole sequence and never
+// round-trips HBM. Every product runs on tcgen05 with bf16 operands; operands that
+// are not raw bf16 inputs are split x = hi + lo (two bf16) and each product is the
+// three passes hi*hi + hi*lo + lo*hi (about 16 significant bits), which the fp32-state
+// tolerance needs. Raw V stays exact in one bf16 operand. Inputs arrive by TMA (no
+// multicast) with 128-byte swizzle; tokens past the end read as zero and get gate 1.
+//
+// Pairwise gate ratios use one reference (token 31 of the chunk): left factors
+// 2^{L_r - L_ref}, right factors 2^{L_ref - L_s}. When a chunk's gates decay so fast
+// that those factors would leave the safe exponent range, that chunk computes A and P
+// pair by pair on CUDA cores instead (exact, slow, rare).
 #pragma once
 #include "common.cuh"
+#include "tc_primitives.cuh"
+#include "tc_host.cuh"
 
 namespace ckda {
 
-inline bool chunk_tc_supported(int dk, int dv, int dt) {
-    (void)dk; (void)dv; (void)dt;
-    return false;
+namespace ctc {
+
+constexpr int C = 64;        // chunk length
+constexpr int D = 128;       // d_k = d_v
+constexpr int NT = 256;      // threads per CTA
+
+// log2-domain limits of the single-reference factorisation
+constexpr float kLgFloor = -100.f;    // floor of log2|a| per token (a = 0 allowed)
+constexpr float kRefRange = 96.f;     // |L_r - L_ref| bound for the fast path
+constexpr float kChunkRange = 124.f;  // -L_C bound for the fast path
+
+// shared-memory map (bytes from a 1024-aligned base)
+constexpr uint32_t SM_K = 0;            // k tile: 2 TMA boxes [64 tok][64 ch] bf16
+constexpr uint32_t SM_Q = 16384;        // q tile
+constexpr uint32_t SM_V = 32768;        // v tile (MN-major A operand of V^T T^T)
+constexpr uint32_t SM_AL = 49152;       // alpha tile: 4 boxes [64 tok][32 ch] fp32
+constexpr uint32_t SM_AMAT = 49152;     //   reused: A (fp32 64x64, column-swizzled)
+constexpr uint32_t SM_T = 65536;        //   reused: [T_hi ; T_lo] K-major [128 n][64 s]
+constexpr uint32_t SM_XHI = 81920;      // X = [k e1 ; q e1] MN-major, 2 blocks [128 c][64 r]
+constexpr uint32_t SM_XLO = 114688;
+constexpr uint32_t SM_YHI = 147456;     // Y = k e2, MN-major [128 c][64 s]
+constexpr uint32_t SM_YLO = 163840;
+constexpr uint32_t SM_C1HI = 81920;     //   reused after the A/P MMA: [W^T | Q~^T] MN-major
+constexpr uint32_t SM_C1LO = 114688;
+constexpr uint32_t SM_KPHI = 147456;    //   reused: K' = (Gamma_C/Gamma) k, K-major [128 c][64 s]
+constexpr uint32_t SM_KPLO = 163840;
+constexpr uint32_t SM_PHI = 180224;     // P K-major [64 r][64 s]
+constexpr uint32_t SM_PLO = 188416;
+constexpr uint32_t SM_XINV = 196608;    // (I + A)^{-1}, fp32 [64][65]
+constexpr uint32_t SM_YTMP = SM_XINV + 64 * 65 * 4;   // 3 x 16 x 16 fp32
+constexpr uint32_t SM_SMALL = SM_YTMP + 3 * 256 * 4;
+constexpr uint32_t SM_BYTES = SM_SMALL + 4096;
+constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;       // + alignment slack
+
+// slow-path scratch (only when the fast path is refused): L and sign per (r, c)
+constexpr uint32_t SM_SLOW_L = SM_XHI;                 // fp32 [64][128]
+constexpr uint32_t SM_SLOW_S = SM_XLO;                 // fp32 [64][128] (+1 / -1)
+
+// TMEM column map (512 columns allocated)
+constexpr uint32_t TM_S = 0;          // S^T fp32 accumulator [d_v lanes][d_k cols]
+constexpr uint32_t TM_D1 = 128;       // [A ; P] 128 x 64
+constexpr uint32_t TM_DR = 128;       // S0^T [W^T | Q~^T] 128 x 128 (cols 192.. become O)
+constexpr uint32_t TM_O = 192;
+constexpr uint32_t TM_KTHI = 192;     // (Gamma k)^T hi, packed bf16, A operand
+constexpr uint32_t TM_KTLO = 224;
+constexpr uint32_t TM_DU = 256;       // V^T [T_hi^T | T_lo^T]
+constexpr uint32_t TM_DW = 384;       // (Gamma k)^T [T_hi^T | T_lo^T] + lo part
+constexpr uint32_t TM_SAHI = 384;     // S0^T hi / lo packed bf16 (A operand of C1)
+constexpr uint32_t TM_SALO = 448;
+constexpr uint32_t TM_UAHI = 384;     // U^T hi / lo packed bf16 (A operand of C2)
+constexpr uint32_t TM_UALO = 416;
+
+constexpr uint32_t kTmaBytes = 10 * 8192;    // 6 bf16 boxes + 4 fp32 boxes
+
+// Byte address (from tile base) of the 16-byte chunk `ch` (0..7) of row `row` in a
+// tile of 128-byte rows with 128-byte swizzle.
+__device__ __forceinline__ uint32_t chunk_off(int row, int ch) {
+    return (uint32_t)row * 128u + ((uint32_t)(ch ^ (row & 7)) << 4);
 }
+
+__device__ __forceinline__ float ld_bf16_tile(const uint8_t* tile, int r, int c) {
+    // TMA box layout: boxes of 64 channels, [64 tokens][128 B]
+    const uint32_t off = (uint32_t)(c >> 6) * 8192u + tc::swz128((uint32_t)r * 128u + (uint32_t)(c & 63) * 2u);
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
+}
+
+__device__ __forceinline__ float ld_alpha_tile(const uint8_t* tile, int r, int c) {
+    const uint32_t off = (uint32_t)(c >> 5) * 8192u + tc::swz128((uint32_t)r * 128u + (uint32_t)(c & 31) * 4u);
+    return *reinterpret_cast<const float*>(tile + off);
+}
+
+// Split 32 fp32 values into hi/lo bf16 and store them as four 16-byte chunks
+// (chunks 4h .. 4h+3) of row `row` in two swizzled tiles.
+__device__ __forceinline__ void store_split_row32(uint8_t* hi_tile, uint8_t* lo_tile, int row, int h,
+                                                  const float (&x)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t ph[4], pl[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __nv_bfloat16 h0, l0, h1, l1;
+            tc::split_bf16(x[8 * q + 2 * e], h0, l0);
+            tc::split_bf16(x[8 * q + 2 * e + 1], h1, l1);
+            ph[e] = tc::pack_bf16(h0, h1);
+            pl[e] = tc::pack_bf16(l0, l1);
+        }
+        const uint32_t off = chunk_off(row, 4 * h + q);
+        *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    }
+}
+
+// Split 8 fp32 values into hi/lo bf16 and store them as 16-byte chunk `ch` of row `row`.
+__device__ __forceinline__ void store_split8(uint8_t* hi_tile, uint8_t* lo_tile, int row, int ch,
+                                             const float (&x)[8]) {
+    uint32_t ph[4], pl[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        __nv_bfloat16 h0, l0, h1, l1;
+        tc::split_bf16(x[2 * e], h0, l0);
+        tc::split_bf16(x[2 * e + 1], h1, l1);
+        ph[e] = tc::pack_bf16(h0, h1);
+        pl[e] = tc::pack_bf16(l0, l1);
+    }
+    const uint32_t off = chunk_off(row, ch);
+    *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+    *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+}
+
+// Split 32 fp32 values (consecutive K positions) into packed bf16 pairs for a TMEM A operand.
+__device__ __forceinline__ void split_pack32(const float (&x)[32], uint32_t (&hi)[16], uint32_t (&lo)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        __nv_bfloat16 h0, l0, h1, l1;
+        tc::split_bf16(x[2 * e], h0, l0);
+        tc::split_bf16(x[2 * e + 1], h1, l1);
+        hi[e] = tc::pack_bf16(h0, h1);
+        lo[e] = tc::pack_bf16(l0, l1);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&r)[N]) {
+    tc::tmem_ld32<N>(taddr, r);
+}
+
+__device__ __forceinline__ void tmem_st_f32x32(uint32_t taddr, const float (&x)[32]) {
+    uint32_t a[16], b[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        a[e] = __float_as_uint(x[e]);
+        b[e] = __float_as_uint(x[16 + e]);
+    }
+    tc::tmem_st32<16>(taddr, a);
+    tc::tmem_st32<16>(taddr + 16, b);
+}
+
+// Every thread waits on the barrier; returns true if any thread of the CTA timed out.
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
+    const bool ok = tc::mbar_wait(bar, parity);
+    return __syncthreads_or(!ok) != 0;
+}
+
+__device__ __forceinline__ void sync_for_mma() {
+    // make generic-proxy shared-memory writes and tcgen05.st visible to the MMA issuer
+    tc::tmem_st_wait();
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+}
+
+}  // namespace ctc
+
+// ------------------------------------------------------------------------------ kernel
+
+__global__ void __launch_bounds__(ctc::NT, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
+                const float* __restrict__ beta, const float* S0, float* __restrict__ o, float* ST,
+                int T, int H) {
+    using namespace ctc;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar_tma, bar_mma;
+    __shared__ uint32_t tmem_base_s;
+
+    float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
+    float* sh_gC = sh_beta + 64;                                         // [128] Gamma_C
+    float* sh_Lx = sh_gC + 128;                                          // [128]
+    float* sh_LC = sh_Lx + 128;                                          // [128]
+    uint32_t* sh_px = reinterpret_cast<uint32_t*>(sh_LC + 128);          // [128]
+    uint32_t* sh_pC = sh_px + 128;                                       // [128]
+    float* amat = reinterpret_cast<float*>(sm + SM_AMAT);
+    float* xinv = reinterpret_cast<float*>(sm + SM_XINV);
+    float* ytmp = reinterpret_cast<float*>(sm + SM_YTMP);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, hh = warp >> 2;
+    const int m = quarter * 32 + lane;            // TMEM lane = channel / feature / row
+    const int bh = blockIdx.x;
+    const int b = bh / H, h = bh % H;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+
+    if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
+    if (tid == 0) {
+        tc::mbar_init(&bar_tma, 1);
+        tc::mbar_init(&bar_mma, 1);
+        tc::fence_mbar_init();
+        tc::prefetch_tensormap(&map_k);
+        tc::prefetch_tensormap(&map_q);
+        tc::prefetch_tensormap(&map_v);
+        tc::prefetch_tensormap(&map_a);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = tmem_base_s;
+    const uint32_t tl = tm + lane_base;           // this warp's lane quarter
+
+    auto issue_loads = [&](int t0) {
+        tc::mbar_arrive_expect_tx(&bar_tma, kTmaBytes);
+        for (int i = 0; i < 2; ++i) {
+            tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma, 64 * i, h, t0, b);
+            tc::tma_load_4d(sm + SM_Q + i * 8192, &map_q, &bar_tma, 64 * i, h, t0, b);
+            tc::tma_load_4d(sm + SM_V + i * 8192, &map_v, &bar_tma, 64 * i, h, t0, b);
+        }
+        for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma, 32 * i, h, t0, b);
+    };
+    if (tid == 0) issue_loads(0);
+
+    // initial state -> S^T accumulator (lane d_v, columns d_k)
+    {
+        const size_t sb = (size_t)bh * D * D;
+        for (int cb = 0; cb < 2; ++cb) {
+            float x[32];
+            const int c0 = 64 * hh + 32 * cb;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = S0 ? S0[sb + (size_t)(c0 + i) * D + m] : 0.f;
+            tmem_st_f32x32(tl + TM_S + c0, x);
+        }
+        tc::tmem_st_wait();
+    }
+
+    const uint32_t sbase = tc::smem_u32(sm);
+    uint32_t mma_phase = 0;
+    bool failed = false;
+    const int nchunks = (T + C - 1) / C;
+
+    for (int ck = 0; ck < nchunks && !failed; ++ck) {
+        const int t0 = ck * C;
+        const int nvalid = min(C, T - t0);
+        if (tid < C) sh_beta[tid] = (tid < nvalid) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
+        if (wait_all(&bar_tma, ck & 1)) { failed = true; break; }
+
+        // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
+        float g[32], kp[32];      // Gamma_r and Gamma_C / Gamma_r, signed
+        uint32_t par = 0;
+        float Lref, LC;
+        uint32_t pref, pC;
+        {
+            float run = 0.f;
+            uint32_t p = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int r = 32 * hh + i;
+                const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
+                run += fmaxf(log2f(fabsf(a)), kLgFloor);
+                p ^= (a < 0.f) ? 1u : 0u;
+                g[i] = run;                       // local cumulative log2 magnitude
+                par |= p << i;
+            }
+            if (hh == 0) { sh_Lx[m] = run; sh_px[m] = p; }
+            __syncthreads();
+            int bad = 0;
+            if (hh == 1) {
+                Lref = sh_Lx[m];
+                pref = sh_px[m];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) g[i] += Lref;
+                if (pref) par = ~par;
+                LC = g[31];
+                pC = par >> 31;
+                sh_LC[m] = LC;
+                sh_pC[m] = pC;
+                bad = (-Lref > kRefRange) || (Lref - LC > kRefRange) || (-LC > kChunkRange);
+            }
+            const bool slow = __syncthreads_or(bad) != 0;
+            if (hh == 0) {
+                Lref = g[31];
+                pref = par >> 31;
+                LC = sh_LC[m];
+                pC = sh_pC[m];
+                const float gC = exp2f(LC);
+                sh_gC[m] = pC ? -gC : gC;
+            }
+            // g <- Gamma_r, kp <- Gamma_C / Gamma_r (signed)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t pr = (par >> i) & 1u;
+                const float Lr = g[i];
+                if (slow) {
+                    reinterpret_cast<float*>(sm + SM_SLOW_L)[(32 * hh + i) * D + m] = Lr;
+                    reinterpret_cast<float*>(sm + SM_SLOW_S)[(32 * hh + i) * D + m] = pr ? -1.f : 1.f;
+                }
+                const float gr = exp2f(Lr);
+                const float kr = exp2f(LC - Lr);
+                g[i] = pr ? -gr : gr;
+                kp[i] = (pr ^ pC) ? -kr : kr;
+            }
+
+            // X = [k e1 ; q e1], Y = k e2 with e1 = Gamma_r / Gamma_ref, e2 = Gamma_ref / Gamma_r
+            const float inv_gref = (pref ? -1.f : 1.f) * exp2f(-Lref);
+            const float kref_ratio = ((pref ^ pC) ? -1.f : 1.f) * exp2f(Lref - LC);
+            if (!slow) {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float xk[8], xq[8], yk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 8 * q8 + e, r = 32 * hh + i;
+                        const float kv = ld_bf16_tile(sm + SM_K, r, m);
+                        const float qv = ld_bf16_tile(sm + SM_Q, r, m);
+                        const float e1 = g[i] * inv_gref;
+                        const float e2 = kp[i] * kref_ratio;
+                        xk[e] = kv * e1;
+                        xq[e] = qv * e1;
+                        yk[e] = kv * e2;
+                    }
+                    store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xk);
+                    store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xq);
+                    store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
+                }
+            }
+            // (Gamma k)^T into TMEM as the A operand of W^T = K~^T T^T
+            {
+                float kt[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) kt[i] = ld_bf16_tile(sm + SM_K, 32 * hh + i, m) * g[i];
+                uint32_t hi[16], lo[16];
+                split_pack32(kt, hi, lo);
+                tc::tmem_st32<16>(tl + TM_KTHI + 16 * hh, hi);
+                tc::tmem_st32<16>(tl + TM_KTLO + 16 * hh, lo);
+            }
+            sync_for_mma();
+
+            // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact slow path
+            if (!slow) {
+                if (tid == 0) {
+                    const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
+                    const uint32_t xa[3] = {sbase + SM_XHI, sbase + SM_XHI, sbase + SM_XLO};
+                    const uint32_t yb[3] = {sbase + SM_YHI, sbase + SM_YLO, sbase + SM_YHI};
+                    for (int ps = 0; ps < 3; ++ps)
+                        for (int ks = 0; ks < 8; ++ks)
+                            tc::mma_ss(tm + TM_D1, tc::sdesc(xa[ps] + ks * 2048, 16384, 1024),
+                                       tc::sdesc(yb[ps] + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
+                    tc::mma_commit(&bar_mma);
+                }
+                if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
+                mma_phase ^= 1u;
+                tc::tc_fence_after();
+                // ---------------- P3: A (fp32 for the solve) and P (hi/lo) out of TMEM
+                float d1[32];
+                tmem_ld<32>(tl + TM_D1 + 32 * hh, d1);
+                tc::tmem_ld_wait();
+                if (m < C) {
+                    const int r = m;
+                    const float br = sh_beta[r];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int s = 32 * hh + i;
+                        amat[r * 64 + (s ^ (r & 31))] = (s < r) ? br * d1[i] : 0.f;
+                    }
+                } else {
+                    const int r = m - C;
+                    float pv[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) pv[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
+                    store_split_row32(sm + SM_PHI, sm + SM_PLO, r, hh, pv);
+                }
+            } else {
+                // exact pairwise evaluation: 64 x 64 pairs, 128 channels each
+                const float* Ls = reinterpret_cast<const float*>(sm + SM_SLOW_L);
+                const float* Ss = reinterpret_cast<const float*>(sm + SM_SLOW_S);
+                __syncthreads();
+                for (int e = tid; e < C * C; e += NT) {
+                    const int r = e >> 6, s = e & 63;
+                    float accA = 0.f, accP = 0.f;
+                    if (s <= r) {
+                        for (int c = 0; c < D; ++c) {
+                            const float w = Ss[r * D + c] * Ss[s * D + c] * exp2f(Ls[r * D + c] - Ls[s * D + c]);
+                            const float ks = ld_bf16_tile(sm + SM_K, s, c) * w;
+                            accA = fmaf(ld_bf16_tile(sm + SM_K, r, c), ks, accA);
+                            accP = fmaf(ld_bf16_tile(sm + SM_Q, r, c), ks, accP);
+                        }
+                    }
+                    amat[r * 64 + (s ^ (r & 31))] = (s < r) ? sh_beta[r] * accA : 0.f;
+                    // P row r, column s: written as hi/lo pairs one element at a time
+                    __nv_bfloat16 ph, pl;
+                    tc::split_bf16(accP, ph, pl);
+                    const uint32_t off = chunk_off(r, s >> 3) + (uint32_t)(s & 7) * 2u;
+                    *reinterpret_cast<__nv_bfloat16*>(sm + SM_PHI + off) = ph;
+                    *reinterpret_cast<__nv_bfloat16*>(sm + SM_PLO + off) = pl;
+                }
+            }
+            // phase 2 of the gate: Q~^T (block 1 of the C1 operand) and K' (reusing X/Y space)
+            __syncthreads();     // slow-path scratch (X/Y region) fully consumed
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                float xq[8], xk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * q8 + e, r = 32 * hh + i;
+                    xq[e] = ld_bf16_tile(sm + SM_Q, r, m) * g[i];
+                    xk[e] = ld_bf16_tile(sm + SM_K, r, m) * kp[i];
+                }
+                store_split8(sm + SM_C1HI + 16384, sm + SM_C1LO + 16384, m, 4 * hh + q8, xq);
+                store_split8(sm + SM_KPHI, sm + SM_KPLO, m, 4 * hh + q8, xk);
+            }
+        }
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();
+        __syncthreads();
+
+        // ---------------- P4: T = (I + A)^{-1} Diag(beta), blocked 16 x 16
+        if (tid < 64) {
+            const int I = tid >> 4, j = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * I + rr;
+                float acc = (rr == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int ss = 0; ss < rr; ++ss) {
+                    const int s = 16 * I + ss;
+                    acc -= amat[r * 64 + (s ^ (r & 31))] * x[ss];
+                }
+                x[rr] = (rr < j) ? 0.f : acc;
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) xinv[(16 * I + rr) * 65 + 16 * I + j] = x[rr];
+        }
+        __syncthreads();
+        for (int I = 1; I < 4; ++I) {
+            for (int e = tid; e < I * 256; e += NT) {
+                const int J = e >> 8, rr = (e >> 4) & 15, jj = e & 15;
+                const int r = 16 * I + rr;
+                float acc = 0.f;
+                for (int K = J; K < I; ++K)
+#pragma unroll
+                    for (int mm = 0; mm < 16; ++mm) {
+                        const int s = 16 * K + mm;
+                        acc = fmaf(amat[r * 64 + (s ^ (r & 31))], xinv[s * 65 + 16 * J + jj], acc);
+                    }
+                ytmp[e] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < I * 256; e += NT) {
+                const int J = e >> 8, rr = (e >> 4) & 15, jj = e & 15;
+                float acc = 0.f;
+                for (int mm = 0; mm <= rr; ++mm)
+                    acc = fmaf(xinv[(16 * I + rr) * 65 + 16 * I + mm], ytmp[J * 256 + mm * 16 + jj], acc);
+                xinv[(16 * I + rr) * 65 + 16 * J + jj] = -acc;
+            }
+            __syncthreads();
+        }
+        {
+            // T = X Diag(beta): thread -> row r = tid / 4, columns 16 (tid % 4) .. +15
+            const int r = tid >> 2, q4 = tid & 3;
+            uint32_t ph[8], pl[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int s0 = 16 * q4 + 2 * e;
+                const float v0 = (s0 <= r) ? xinv[r * 65 + s0] * sh_beta[s0] : 0.f;
+                const float v1 = (s0 + 1 <= r) ? xinv[r * 65 + s0 + 1] * sh_beta[s0 + 1] : 0.f;
+                __nv_bfloat16 h0, l0, h1, l1;
+                tc::split_bf16(v0, h0, l0);
+                tc::split_bf16(v1, h1, l1);
+                ph[e] = tc::pack_bf16(h0, h1);
+                pl[e] = tc::pack_bf16(l0, l1);
+            }
+            uint8_t* tt = sm + SM_T;
+            *reinterpret_cast<uint4*>(tt + chunk_off(r, 2 * q4)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+            *reinterpret_cast<uint4*>(tt + chunk_off(r, 2 * q4 + 1)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
+            *reinterpret_cast<uint4*>(tt + chunk_off(64 + r, 2 * q4)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+            *reinterpret_cast<uint4*>(tt + chunk_off(64 + r, 2 * q4 + 1)) = make_uint4(pl[4], pl[5], pl[6], pl[7]);
+        }
+        sync_for_mma();
+
+        // ---------------- P5: U~^T = V^T [T_hi^T | T_lo^T],  W^T = K~^T [..] + K~lo^T T_hi^T
+        if (tid == 0) {
+            const uint32_t iu = tc::idesc_bf16(128, 128, 1, 0);
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_ss(tm + TM_DU, tc::sdesc(sbase + SM_V + ks * 2048, 8192, 1024),
+                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iu, ks != 0);
+            const uint32_t iw = tc::idesc_bf16(128, 128, 0, 0);
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_ts(tm + TM_DW, tm + TM_KTHI + ks * 8, tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw,
+                           ks != 0);
+            const uint32_t iw2 = tc::idesc_bf16(128, 64, 0, 0);
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_ts(tm + TM_DW, tm + TM_KTLO + ks * 8, tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw2, 1);
+            tc::mma_commit(&bar_mma);
+        }
+        if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
+        mma_phase ^= 1u;
+        tc::tc_fence_after();
+        // inputs of this chunk are consumed: prefetch the next chunk
+        if (tid == 0 && ck + 1 < nchunks) issue_loads(t0 + C);
+
+        // ---------------- P6: W^T -> C1 operand block 0; S0^T -> TMEM A operand; S *= Gamma_C
+        {
+            float w0[32], w1[32];
+            tmem_ld<32>(tl + TM_DW + 32 * hh, w0);
+            tmem_ld<32>(tl + TM_DW + 64 + 32 * hh, w1);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w0[i] += w1[i];
+            store_split_row32(sm + SM_C1HI, sm + SM_C1LO, m, hh, w0);
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+            const int c0 = 64 * hh + 32 * cb;
+            float s[32];
+            tmem_ld<32>(tl + TM_S + c0, s);
+            tc::tmem_ld_wait();
+            uint32_t hi[16], lo[16];
+            split_pack32(s, hi, lo);
+            tc::tmem_st32<16>(tl + TM_SAHI + c0 / 2, hi);
+            tc::tmem_st32<16>(tl + TM_SALO + c0 / 2, lo);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[i] *= sh_gC[c0 + i];
+            tmem_st_f32x32(tl + TM_S + c0, s);
+        }
+        sync_for_mma();
+
+        // ---------------- P7: D_R = S0^T [W^T | Q~^T]  (3 passes)
+        if (tid == 0) {
+            const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
+            const uint32_t aa[3] = {tm + TM_SAHI, tm + TM_SAHI, tm + TM_SALO};
+            const uint32_t bb[3] = {sbase + SM_C1HI, sbase + SM_C1LO, sbase + SM_C1HI};
+            for (int ps = 0; ps < 3; ++ps)
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_ts(tm + TM_DR, aa[ps] + ks * 8, tc::sdesc(bb[ps] + ks * 2048, 16384, 1024), idesc,
+                               (ps | ks) != 0);
+            tc::mma_commit(&bar_mma);
+        }
+        if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
+        mma_phase ^= 1u;
+        tc::tc_fence_after();
+
+        // ---------------- P8: U^T = U~^T - (S0^T W^T) -> TMEM A operand
+        {
+            float ua[32], ub[32], ws[32];
+            tmem_ld<32>(tl + TM_DU + 32 * hh, ua);
+            tmem_ld<32>(tl + TM_DU + 64 + 32 * hh, ub);
+            tmem_ld<32>(tl + TM_DR + 32 * hh, ws);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ua[i] = (ua[i] + ub[i]) - ws[i];
+            uint32_t hi[16], lo[16];
+            split_pack32(ua, hi, lo);
+            tc::tmem_st32<16>(tl + TM_UAHI + 16 * hh, hi);
+            tc::tmem_st32<16>(tl + TM_UALO + 16 * hh, lo);
+        }
+        sync_for_mma();
+
+        // ---------------- P9: O^T += U^T P^T ;  S^T += U^T K'  (3 passes each)
+        if (tid == 0) {
+            const uint32_t io = tc::idesc_bf16(128, 64, 0, 0);
+            const uint32_t is = tc::idesc_bf16(128, 128, 0, 0);
+            const uint32_t aa[3] = {tm + TM_UAHI, tm + TM_UAHI, tm + TM_UALO};
+            const uint32_t pb[3] = {sbase + SM_PHI, sbase + SM_PLO, sbase + SM_PHI};
+            const uint32_t kb[3] = {sbase + SM_KPHI, sbase + SM_KPLO, sbase + SM_KPHI};
+            for (int ps = 0; ps < 3; ++ps)
+                for (int ks = 0; ks < 4; ++ks) {
+                    tc::mma_ts(tm + TM_O, aa[ps] + ks * 8, tc::sdesc(pb[ps] + ks * 32, 16, 1024), io, 1);
+                    tc::mma_ts(tm + TM_S, aa[ps] + ks * 8, tc::sdesc(kb[ps] + ks * 32, 16, 1024), is, 1);
+                }
+            tc::mma_commit(&bar_mma);
+        }
+        if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
+        mma_phase ^= 1u;
+        tc::tc_fence_after();
+
+        // ---------------- P10: o rows of this chunk
+        {
+            float ov[32];
+            tmem_ld<32>(tl + TM_O + 32 * hh, ov);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int r = 32 * hh + i;
+                if (r < nvalid) o[(((size_t)b * T + t0 + r) * H + h) * D + m] = ov[i];
+            }
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+    }
+
+    // final state
+    if (!failed && ST != nullptr) {
+        const size_t sb = (size_t)bh * D * D;
+        for (int cb = 0; cb < 2; ++cb) {
+            const int c0 = 64 * hh + 32 * cb;
+            float x[32];
+            tmem_ld<32>(tl + TM_S + c0, x);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ST[sb + (size_t)(c0 + i) * D + m] = x[i];
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tm, 512);
+        tc::tmem_relinquish();
+    }
+}
+
+// ------------------------------------------------------------------------------ host
+
+inline bool chunk_tc_supported(int dk, int dv, int dt) { return dt == 1 && dk == 128 && dv == 128; }
 
 inline size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv) {
     (void)B; (void)T; (void)H; (void)dk; (void)dv;
     return 0;
 }
 
-inline cudaError_t launch_chunk_tc(const __nv_bfloat16*, const __nv_bfloat16*, const __nv_bfloat16*,
-                                   const float*, const float*, const float*, float*, float*,
-                                   int, int, int, int, int, void*, cudaStream_t) {
-    return cudaErrorNotSupported;
+inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                   const float* alpha, const float* beta, const float* S0, float* o, float* ST,
+                                   int B, int T, int H, int dk, int dv, void* workspace, cudaStream_t st) {
+    (void)workspace;
+    if (dk != 128 || dv != 128) return cudaErrorNotSupported;
+    CUtensorMap mk, mq, mv, ma;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!tc::make_map_bthd(&mk, k, bf, 2, B, T, H, dk, 64, 64) || !tc::make_map_bthd(&mq, q, bf, 2, B, T, H, dk, 64, 64) ||
+        !tc::make_map_bthd(&mv, v, bf, 2, B, T, H, dv, 64, 64) ||
+        !tc::make_map_bthd(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dk, 32, 64))
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)ctc::SMEM_ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    chunk_tc_kernel<<<(unsigned)(B * H), ctc::NT, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, beta, S0, o, ST, T, H);
+    return cudaGetLastError();
 }
 
 }  // namespace ckda

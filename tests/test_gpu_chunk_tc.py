@@ -1,0 +1,105 @@
+"""Parity of the tensor-core chunk path (bf16 q/k/v, d_k = d_v = 128) against the
+fp64 oracle, at the workloads' full sizes (sampled sequences) and on edge cases.
+Tolerance: max-abs error <= 3e-3 * RMS(oracle) for o and for the final state."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ckda_inputs import make_inputs, make_workload
+from parity_util import TAU_BF16, check, gather_pairs, oracle_on_pairs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ck():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from delta_rule_attention_ckda_b200 import build
+    build.build()
+    import delta_rule_attention_ckda_b200 as m
+    m.load()
+    return m
+
+
+def run_chunk(ck, inp, S0=True):
+    q, k, v, a, b, s0 = to_dev(inp)
+    o, ST = ck.chunk_fwd(q, k, v, a, b, s0 if S0 else None)
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    return o, ST
+
+
+def test_tc_path_is_selected(ck):
+    assert ck.chunk_path(8, 4096, 16, 128, 128, torch.bfloat16) == ck.PATH_CHUNK_TC
+    assert ck.chunk_path(8, 4096, 16, 128, 128, torch.float32) == ck.PATH_RECURRENT
+
+
+@pytest.mark.parametrize("T", [1, 2, 31, 32, 33, 63, 64, 65, 127, 128, 129, 300])
+def test_lengths_and_ragged_tails(ck, T):
+    inp = make_inputs(2, T, 2, 128, 128, torch.bfloat16, seed=T, gate="tanh15", s0_std=0.05)
+    o, ST = run_chunk(ck, inp)
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check(f"T={T}/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check(f"T={T}/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
+@pytest.mark.parametrize("gate", ["tanh0", "tanh15", "signmag"])
+def test_gate_distributions(ck, gate):
+    inp = make_inputs(2, 700, 3, 128, 128, torch.bfloat16, seed=77, gate=gate, s0_std=0.1)
+    o, ST = run_chunk(ck, inp)
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check(f"{gate}/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check(f"{gate}/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
+def test_extreme_decay_takes_exact_path(ck):
+    """Gates near zero in some chunks push the log-magnitude range past the single-
+    reference limits; those chunks are evaluated pair by pair and must stay exact."""
+    inp = make_inputs(1, 256, 2, 128, 128, torch.bfloat16, seed=5, gate="tanh15", s0_std=0.3)
+    inp.alpha[0, 70:75, :, :40] = 1e-20         # chunk 1: L drops by ~330 in log2
+    inp.alpha[0, 130, 0, :] = 0.0               # chunk 2: exact zeros (floored)
+    inp.alpha[0, 131, 0, :] = -1e-35
+    inp.alpha[0, 200:230, 1, 5:9] = -0.02       # chunk 3: long fast decay, signed
+    o, ST = run_chunk(ck, inp)
+    assert torch.isfinite(o).all() and torch.isfinite(ST).all()
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check("extreme/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check("extreme/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
+def test_small_workload_shape_padded(ck):
+    """bf16, many heads, short sequences: exercises many CTAs with one chunk each."""
+    inp = make_inputs(4, 40, 37, 128, 128, torch.bfloat16, seed=8, gate="tanh15", s0_std=0.05)
+    o, ST = run_chunk(ck, inp)
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check("many-heads/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check("many-heads/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
+def test_layer_workload_full_size(ck):
+    """B=8, T=4096, H=16, d=128, S0 = 0 (the bench's launch), checked on sampled
+    (batch, head) sequences against the oracle."""
+    inp = make_workload("layer")
+    o, ST = run_chunk(ck, inp, S0=False)
+    pairs = [(0, 0), (3, 7), (7, 15), (5, 2)]
+    o_ref, S_ref = oracle_on_pairs(inp, pairs)
+    got_o, got_S = gather_pairs(o, ST, pairs)
+    check("layer/o", got_o, o_ref, TAU_BF16)
+    check("layer/S", got_S, S_ref, TAU_BF16)
+
+
+def test_long_workload_full_size(ck):
+    """B=1, T=65536, H=16, d=128 with a random initial state: error must not grow
+    over 1024 chunks of state propagation. Two sampled heads against the oracle."""
+    inp = make_workload("long")
+    o, ST = run_chunk(ck, inp)
+    pairs = [(0, 3), (0, 12)]
+    o_ref, S_ref = oracle_on_pairs(inp, pairs)
+    got_o, got_S = gather_pairs(o, ST, pairs)
+    check("long/o", got_o, o_ref, TAU_BF16)
+    check("long/S", got_S, S_ref, TAU_BF16)
+    # late tokens are as accurate as early ones (no drift over 1024 chunks)
+    for sl in (slice(0, 4096), slice(61440, 65536)):
+        check(f"long/o[{sl.start}:]", got_o[:, sl], o_ref[:, sl], TAU_BF16)
