@@ -16,19 +16,32 @@
 // In exact arithmetic this equals the token loop; the WY/UT evaluation is the
 // "Chunk-WY" scheme the thelatestinai card names, derived here for the signed gate.
 //
+// Gate factoring. With a reference token ref (31) per chunk and per channel,
+//   e1_r = Gamma_r / Gamma_ref,  e2_s = Gamma_ref / Gamma_s,
+//   g_ref = Gamma_ref,  kappa = Gamma_C / Gamma_ref,
+// every gate product above splits into per-token factors and per-channel constants:
+//   Gamma_r/Gamma_s = e1_r e2_s,  Gamma_r = e1_r g_ref,  Gamma_C/Gamma_s = e2_s kappa,
+//   Gamma_C = g_ref kappa.
+// So one pair of token tiles X = [k e1 ; q e1] and Y = k e2 serves every product:
+//   [A ; P] from X Y^T;  W / g_ref from (k e1) T^T;  O from S0 Diag(g_ref) and q e1;
+//   the state update from S0 Diag(g_ref) + U^T (k e2), which is S_C Diag(1/kappa).
+// The TMEM accumulator therefore holds S Diag(1/kappa_prev); each chunk rescales it
+// by kappa_prev * g_ref (a per-column factor, folded into the pass that copies the
+// state into the MMA operand), and the final write multiplies by the last kappa.
+//
 // B200 mapping. One CTA (256 threads) owns one (batch, head) and walks its chunks in
-// order. Everything is computed transposed, so the 128 feature rows sit on the 128
-// TMEM lanes: the fp32 state lives in TMEM as S^T for the whole sequence and never
+// order. Everything is computed transposed so the 128 feature rows sit on the 128
+// TMEM lanes: the fp32 state lives in TMEM for the whole sequence and never
 // round-trips HBM. Every product runs on tcgen05 with bf16 operands; operands that
 // are not raw bf16 inputs are split x = hi + lo (two bf16) and each product is the
 // three passes hi*hi + hi*lo + lo*hi (about 16 significant bits), which the fp32-state
-// tolerance needs. Raw V stays exact in one bf16 operand. Inputs arrive by TMA (no
+// tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by TMA (no
 // multicast) with 128-byte swizzle; tokens past the end read as zero and get gate 1.
 //
-// Pairwise gate ratios use one reference (token 31 of the chunk): left factors
-// 2^{L_r - L_ref}, right factors 2^{L_ref - L_s}. When a chunk's gates decay so fast
-// that those factors would leave the safe exponent range, that chunk computes A and P
-// pair by pair on CUDA cores instead (exact, slow, rare).
+// Exponent safety. e1 and e2 stay inside [2^-96, 2^96] unless a chunk's gates decay
+// very fast; such a chunk computes A and P pair by pair on CUDA cores (exact), uses
+// the unfactored tiles (k Gamma, q Gamma, k Gamma_C/Gamma) with g_ref = kappa = 1,
+// and applies Gamma_C to the state directly.
 #pragma once
 #include "common.cuh"
 #include "tc_primitives.cuh"
@@ -52,40 +65,30 @@ constexpr uint32_t SM_K = 0;            // k tile: 2 TMA boxes [64 tok][64 ch] b
 constexpr uint32_t SM_Q = 16384;        // q tile
 constexpr uint32_t SM_V = 32768;        // v tile (MN-major A operand of V^T T^T)
 constexpr uint32_t SM_AL = 49152;       // alpha tile: 4 boxes [64 tok][32 ch] fp32
-constexpr uint32_t SM_AMAT = 49152;     //   reused: A (fp32 64x64, column-swizzled)
-constexpr uint32_t SM_T = 65536;        //   reused: [T_hi ; T_lo] K-major [128 n][64 s]
-constexpr uint32_t SM_XHI = 81920;      // X = [k e1 ; q e1] MN-major, 2 blocks [128 c][64 r]
-constexpr uint32_t SM_XLO = 114688;
-constexpr uint32_t SM_YHI = 147456;     // Y = k e2, MN-major [128 c][64 s]
+constexpr uint32_t SM_AX = 0;           //   after the gate: A, then (I + A)^{-1}, fp32 [64][64]
+constexpr uint32_t SM_T = 16384;        //   after the gate: [T_hi ; T_lo] K-major [128 n][64 s]
+constexpr uint32_t SM_SLOWL = 49152;    //   slow path only: L fp32 [64][128]
+constexpr uint32_t SM_XHI = 81920;      // X hi: block 0 = k e1 (later W^T), block 1 = q e1, [128 c][64 r]
+constexpr uint32_t SM_XLO = 114688;     // X lo
+constexpr uint32_t SM_YHI = 147456;     // Y = k e2, [128 c][64 s] (MN-major for A/P, K-major for S)
 constexpr uint32_t SM_YLO = 163840;
-constexpr uint32_t SM_C1HI = 81920;     //   reused after the A/P MMA: [W^T | Q~^T] MN-major
-constexpr uint32_t SM_C1LO = 114688;
-constexpr uint32_t SM_KPHI = 147456;    //   reused: K' = (Gamma_C/Gamma) k, K-major [128 c][64 s]
-constexpr uint32_t SM_KPLO = 163840;
 constexpr uint32_t SM_PHI = 180224;     // P K-major [64 r][64 s]
 constexpr uint32_t SM_PLO = 188416;
-constexpr uint32_t SM_XINV = 196608;    // (I + A)^{-1}, fp32 [64][65]
-constexpr uint32_t SM_YTMP = SM_XINV + 64 * 65 * 4;   // 3 x 16 x 16 fp32
-constexpr uint32_t SM_SMALL = SM_YTMP + 3 * 256 * 4;
-constexpr uint32_t SM_BYTES = SM_SMALL + 4096;
+constexpr uint32_t SM_RT = 196608;      // solve temporary, fp32 [16][48]
+constexpr uint32_t SM_SMALL = SM_RT + 16 * 48 * 4;
+constexpr uint32_t SM_BYTES = SM_SMALL + 8192;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;       // + alignment slack
 
-// slow-path scratch (only when the fast path is refused): L and sign per (r, c)
-constexpr uint32_t SM_SLOW_L = SM_XHI;                 // fp32 [64][128]
-constexpr uint32_t SM_SLOW_S = SM_XLO;                 // fp32 [64][128] (+1 / -1)
-
 // TMEM column map (512 columns allocated)
-constexpr uint32_t TM_S = 0;          // S^T fp32 accumulator [d_v lanes][d_k cols]
+constexpr uint32_t TM_S = 0;          // state accumulator S^T Diag(1/kappa) [d_v lanes][d_k cols]
 constexpr uint32_t TM_D1 = 128;       // [A ; P] 128 x 64
-constexpr uint32_t TM_DR = 128;       // S0^T [W^T | Q~^T] 128 x 128 (cols 192.. become O)
-constexpr uint32_t TM_O = 192;
-constexpr uint32_t TM_KTHI = 192;     // (Gamma k)^T hi, packed bf16, A operand
-constexpr uint32_t TM_KTLO = 224;
+constexpr uint32_t TM_DR = 128;       // (S0 Diag g)^T [W^T/g | (q e1)^T] 128 x 128
+constexpr uint32_t TM_O = 192;        //   its second half accumulates O^T
 constexpr uint32_t TM_DU = 256;       // V^T [T_hi^T | T_lo^T]
-constexpr uint32_t TM_DW = 384;       // (Gamma k)^T [T_hi^T | T_lo^T] + lo part
-constexpr uint32_t TM_SAHI = 384;     // S0^T hi / lo packed bf16 (A operand of C1)
+constexpr uint32_t TM_DW = 384;       // (k e1)^T [T_hi^T | T_lo^T] + lo part
+constexpr uint32_t TM_SAHI = 384;     // (S0 Diag g)^T hi / lo, packed bf16 (A operand)
 constexpr uint32_t TM_SALO = 448;
-constexpr uint32_t TM_UAHI = 384;     // U^T hi / lo packed bf16 (A operand of C2)
+constexpr uint32_t TM_UAHI = 384;     // U^T hi / lo, packed bf16 (A operand)
 constexpr uint32_t TM_UALO = 416;
 
 constexpr uint32_t kTmaBytes = 10 * 8192;    // 6 bf16 boxes + 4 fp32 boxes
@@ -96,70 +99,41 @@ __device__ __forceinline__ uint32_t chunk_off(int row, int ch) {
     return (uint32_t)row * 128u + ((uint32_t)(ch ^ (row & 7)) << 4);
 }
 
+// Element (r, c) of a bf16 TMA tile made of 64-channel boxes [64 tokens][128 B].
 __device__ __forceinline__ float ld_bf16_tile(const uint8_t* tile, int r, int c) {
-    // TMA box layout: boxes of 64 channels, [64 tokens][128 B]
     const uint32_t off = (uint32_t)(c >> 6) * 8192u + tc::swz128((uint32_t)r * 128u + (uint32_t)(c & 63) * 2u);
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
 }
 
+// Element (r, c) of the fp32 alpha tile made of 32-channel boxes [64 tokens][128 B].
 __device__ __forceinline__ float ld_alpha_tile(const uint8_t* tile, int r, int c) {
     const uint32_t off = (uint32_t)(c >> 5) * 8192u + tc::swz128((uint32_t)r * 128u + (uint32_t)(c & 31) * 4u);
     return *reinterpret_cast<const float*>(tile + off);
 }
 
-// Split 32 fp32 values into hi/lo bf16 and store them as four 16-byte chunks
-// (chunks 4h .. 4h+3) of row `row` in two swizzled tiles.
-__device__ __forceinline__ void store_split_row32(uint8_t* hi_tile, uint8_t* lo_tile, int row, int h,
-                                                  const float (&x)[32]) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t ph[4], pl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            __nv_bfloat16 h0, l0, h1, l1;
-            tc::split_bf16(x[8 * q + 2 * e], h0, l0);
-            tc::split_bf16(x[8 * q + 2 * e + 1], h1, l1);
-            ph[e] = tc::pack_bf16(h0, h1);
-            pl[e] = tc::pack_bf16(l0, l1);
-        }
-        const uint32_t off = chunk_off(row, 4 * h + q);
-        *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-        *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-    }
+// (a, b) -> packed bf16 hi pair and packed bf16 lo pair, a + b exact to ~16 bits each.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Split 8 fp32 values into hi/lo bf16 and store them as 16-byte chunk `ch` of row `row`.
-__device__ __forceinline__ void store_split8(uint8_t* hi_tile, uint8_t* lo_tile, int row, int ch,
-                                             const float (&x)[8]) {
+// Split 8 fp32 values and store them as 16-byte chunk `ch` of row `row` (hi and lo tiles).
+__device__ __forceinline__ void store_split8(uint8_t* hi_tile, uint8_t* lo_tile, int row, int ch, const float* x) {
     uint32_t ph[4], pl[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        tc::split_bf16(x[2 * e], h0, l0);
-        tc::split_bf16(x[2 * e + 1], h1, l1);
-        ph[e] = tc::pack_bf16(h0, h1);
-        pl[e] = tc::pack_bf16(l0, l1);
-    }
+    for (int e = 0; e < 4; ++e) split2(x[2 * e], x[2 * e + 1], ph[e], pl[e]);
     const uint32_t off = chunk_off(row, ch);
     *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
     *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
 }
 
-// Split 32 fp32 values (consecutive K positions) into packed bf16 pairs for a TMEM A operand.
+// Split 32 fp32 values (consecutive K positions) into packed bf16 pairs (TMEM A operand).
 __device__ __forceinline__ void split_pack32(const float (&x)[32], uint32_t (&hi)[16], uint32_t (&lo)[16]) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        __nv_bfloat16 h0, l0, h1, l1;
-        tc::split_bf16(x[2 * e], h0, l0);
-        tc::split_bf16(x[2 * e + 1], h1, l1);
-        hi[e] = tc::pack_bf16(h0, h1);
-        lo[e] = tc::pack_bf16(l0, l1);
-    }
-}
-
-template <int N>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&r)[N]) {
-    tc::tmem_ld32<N>(taddr, r);
+    for (int e = 0; e < 16; ++e) split2(x[2 * e], x[2 * e + 1], hi[e], lo[e]);
 }
 
 __device__ __forceinline__ void tmem_st_f32x32(uint32_t taddr, const float (&x)[32]) {
@@ -179,14 +153,17 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
     return __syncthreads_or(!ok) != 0;
 }
 
+// Make generic-proxy shared-memory writes and tcgen05.st visible to the MMA issuer.
 __device__ __forceinline__ void sync_for_mma() {
-    // make generic-proxy shared-memory writes and tcgen05.st visible to the MMA issuer
     tc::tmem_st_wait();
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
 }
+
+// fp32 [64][64] matrix with XOR-swizzled columns (conflict-free row and column access)
+__device__ __forceinline__ int ax_idx(int r, int s) { return r * 64 + (s ^ (r & 31)); }
 
 }  // namespace ctc
 
@@ -204,14 +181,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     __shared__ uint32_t tmem_base_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
-    float* sh_gC = sh_beta + 64;                                         // [128] Gamma_C
-    float* sh_Lx = sh_gC + 128;                                          // [128]
-    float* sh_LC = sh_Lx + 128;                                          // [128]
-    uint32_t* sh_px = reinterpret_cast<uint32_t*>(sh_LC + 128);          // [128]
+    float* sh_fa = sh_beta + 64;            // [128] factor for the state operand copy
+    float* sh_fs = sh_fa + 128;             // [128] factor for the state accumulator
+    float* sh_kref = sh_fs + 128;           // [128] kappa of the last chunk
+    float* sh_Lx = sh_kref + 128;           // [128] exchange: L at token 31
+    float* sh_LC = sh_Lx + 128;             // [128] exchange: L at token 63
+    uint32_t* sh_px = reinterpret_cast<uint32_t*>(sh_LC + 128);        // [128]
     uint32_t* sh_pC = sh_px + 128;                                       // [128]
-    float* amat = reinterpret_cast<float*>(sm + SM_AMAT);
-    float* xinv = reinterpret_cast<float*>(sm + SM_XINV);
-    float* ytmp = reinterpret_cast<float*>(sm + SM_YTMP);
+    uint32_t* sh_sign = sh_pC + 128;        // [64][4] slow path: sign bits per (token, channel)
+    float* ax = reinterpret_cast<float*>(sm + SM_AX);
+    float* rt = reinterpret_cast<float*>(sm + SM_RT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, hh = warp >> 2;
@@ -230,6 +209,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::prefetch_tensormap(&map_v);
         tc::prefetch_tensormap(&map_a);
     }
+    if (tid < D) sh_kref[tid] = 1.f;
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -246,8 +226,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma, 32 * i, h, t0, b);
     };
     if (tid == 0) issue_loads(0);
+    auto load_beta = [&](int t0) -> float {
+        return (tid < C && t0 + tid < T) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
+    };
+    float beta_next = load_beta(0);
 
-    // initial state -> S^T accumulator (lane d_v, columns d_k)
+    // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
     {
         const size_t sb = (size_t)bh * D * D;
         for (int cb = 0; cb < 2; ++cb) {
@@ -268,244 +252,242 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     for (int ck = 0; ck < nchunks && !failed; ++ck) {
         const int t0 = ck * C;
         const int nvalid = min(C, T - t0);
-        if (tid < C) sh_beta[tid] = (tid < nvalid) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
+        if (tid < C) sh_beta[tid] = beta_next;
         if (wait_all(&bar_tma, ck & 1)) { failed = true; break; }
 
         // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
-        float g[32], kp[32];      // Gamma_r and Gamma_C / Gamma_r, signed
-        uint32_t par = 0;
-        float Lref, LC;
-        uint32_t pref, pC;
+        bool slow;
         {
+            float L[32];
+            uint32_t par = 0;
             float run = 0.f;
             uint32_t p = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int r = 32 * hh + i;
                 const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
-                run += fmaxf(log2f(fabsf(a)), kLgFloor);
+                run += fmaxf(__log2f(fabsf(a)), kLgFloor);
                 p ^= (a < 0.f) ? 1u : 0u;
-                g[i] = run;                       // local cumulative log2 magnitude
+                L[i] = run;
                 par |= p << i;
             }
             if (hh == 0) { sh_Lx[m] = run; sh_px[m] = p; }
             __syncthreads();
+            float Lref, LC;
+            uint32_t pref, pC;
             int bad = 0;
             if (hh == 1) {
                 Lref = sh_Lx[m];
                 pref = sh_px[m];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) g[i] += Lref;
+                for (int i = 0; i < 32; ++i) L[i] += Lref;
                 if (pref) par = ~par;
-                LC = g[31];
+                LC = L[31];
                 pC = par >> 31;
                 sh_LC[m] = LC;
                 sh_pC[m] = pC;
                 bad = (-Lref > kRefRange) || (Lref - LC > kRefRange) || (-LC > kChunkRange);
             }
-            const bool slow = __syncthreads_or(bad) != 0;
+            slow = __syncthreads_or(bad) != 0;
             if (hh == 0) {
-                Lref = g[31];
+                Lref = L[31];
                 pref = par >> 31;
                 LC = sh_LC[m];
                 pC = sh_pC[m];
-                const float gC = exp2f(LC);
-                sh_gC[m] = pC ? -gC : gC;
-            }
-            // g <- Gamma_r, kp <- Gamma_C / Gamma_r (signed)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const uint32_t pr = (par >> i) & 1u;
-                const float Lr = g[i];
-                if (slow) {
-                    reinterpret_cast<float*>(sm + SM_SLOW_L)[(32 * hh + i) * D + m] = Lr;
-                    reinterpret_cast<float*>(sm + SM_SLOW_S)[(32 * hh + i) * D + m] = pr ? -1.f : 1.f;
-                }
-                const float gr = exp2f(Lr);
-                const float kr = exp2f(LC - Lr);
-                g[i] = pr ? -gr : gr;
-                kp[i] = (pr ^ pC) ? -kr : kr;
-            }
-
-            // X = [k e1 ; q e1], Y = k e2 with e1 = Gamma_r / Gamma_ref, e2 = Gamma_ref / Gamma_r
-            const float inv_gref = (pref ? -1.f : 1.f) * exp2f(-Lref);
-            const float kref_ratio = ((pref ^ pC) ? -1.f : 1.f) * exp2f(Lref - LC);
-            if (!slow) {
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float xk[8], xq[8], yk[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = 8 * q8 + e, r = 32 * hh + i;
-                        const float kv = ld_bf16_tile(sm + SM_K, r, m);
-                        const float qv = ld_bf16_tile(sm + SM_Q, r, m);
-                        const float e1 = g[i] * inv_gref;
-                        const float e2 = kp[i] * kref_ratio;
-                        xk[e] = kv * e1;
-                        xq[e] = qv * e1;
-                        yk[e] = kv * e2;
-                    }
-                    store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xk);
-                    store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xq);
-                    store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
-                }
-            }
-            // (Gamma k)^T into TMEM as the A operand of W^T = K~^T T^T
-            {
-                float kt[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) kt[i] = ld_bf16_tile(sm + SM_K, 32 * hh + i, m) * g[i];
-                uint32_t hi[16], lo[16];
-                split_pack32(kt, hi, lo);
-                tc::tmem_st32<16>(tl + TM_KTHI + 16 * hh, hi);
-                tc::tmem_st32<16>(tl + TM_KTLO + 16 * hh, lo);
-            }
-            sync_for_mma();
-
-            // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact slow path
-            if (!slow) {
-                if (tid == 0) {
-                    const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
-                    const uint32_t xa[3] = {sbase + SM_XHI, sbase + SM_XHI, sbase + SM_XLO};
-                    const uint32_t yb[3] = {sbase + SM_YHI, sbase + SM_YLO, sbase + SM_YHI};
-                    for (int ps = 0; ps < 3; ++ps)
-                        for (int ks = 0; ks < 8; ++ks)
-                            tc::mma_ss(tm + TM_D1, tc::sdesc(xa[ps] + ks * 2048, 16384, 1024),
-                                       tc::sdesc(yb[ps] + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
-                    tc::mma_commit(&bar_mma);
-                }
-                if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
-                mma_phase ^= 1u;
-                tc::tc_fence_after();
-                // ---------------- P3: A (fp32 for the solve) and P (hi/lo) out of TMEM
-                float d1[32];
-                tmem_ld<32>(tl + TM_D1 + 32 * hh, d1);
-                tc::tmem_ld_wait();
-                if (m < C) {
-                    const int r = m;
-                    const float br = sh_beta[r];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int s = 32 * hh + i;
-                        amat[r * 64 + (s ^ (r & 31))] = (s < r) ? br * d1[i] : 0.f;
-                    }
+                const float kprev = sh_kref[m];
+                const float gC = (pC ? -1.f : 1.f) * exp2f(LC);
+                if (!slow) {
+                    const float gref = (pref ? -1.f : 1.f) * exp2f(Lref);
+                    const float kappa = ((pref ^ pC) ? -1.f : 1.f) * exp2f(LC - Lref);
+                    sh_fa[m] = kprev * gref;
+                    sh_fs[m] = kprev * gref;
+                    sh_kref[m] = kappa;
                 } else {
-                    const int r = m - C;
-                    float pv[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) pv[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
-                    store_split_row32(sm + SM_PHI, sm + SM_PLO, r, hh, pv);
-                }
-            } else {
-                // exact pairwise evaluation: 64 x 64 pairs, 128 channels each
-                const float* Ls = reinterpret_cast<const float*>(sm + SM_SLOW_L);
-                const float* Ss = reinterpret_cast<const float*>(sm + SM_SLOW_S);
-                __syncthreads();
-                for (int e = tid; e < C * C; e += NT) {
-                    const int r = e >> 6, s = e & 63;
-                    float accA = 0.f, accP = 0.f;
-                    if (s <= r) {
-                        for (int c = 0; c < D; ++c) {
-                            const float w = Ss[r * D + c] * Ss[s * D + c] * exp2f(Ls[r * D + c] - Ls[s * D + c]);
-                            const float ks = ld_bf16_tile(sm + SM_K, s, c) * w;
-                            accA = fmaf(ld_bf16_tile(sm + SM_K, r, c), ks, accA);
-                            accP = fmaf(ld_bf16_tile(sm + SM_Q, r, c), ks, accP);
-                        }
-                    }
-                    amat[r * 64 + (s ^ (r & 31))] = (s < r) ? sh_beta[r] * accA : 0.f;
-                    // P row r, column s: written as hi/lo pairs one element at a time
-                    __nv_bfloat16 ph, pl;
-                    tc::split_bf16(accP, ph, pl);
-                    const uint32_t off = chunk_off(r, s >> 3) + (uint32_t)(s & 7) * 2u;
-                    *reinterpret_cast<__nv_bfloat16*>(sm + SM_PHI + off) = ph;
-                    *reinterpret_cast<__nv_bfloat16*>(sm + SM_PLO + off) = pl;
+                    sh_fa[m] = kprev;
+                    sh_fs[m] = kprev * gC;
+                    sh_kref[m] = 1.f;
                 }
             }
-            // phase 2 of the gate: Q~^T (block 1 of the C1 operand) and K' (reusing X/Y space)
-            __syncthreads();     // slow-path scratch (X/Y region) fully consumed
+            // per-token factors: fast path e1 = Gamma_r/Gamma_ref, e2 = Gamma_ref/Gamma_r;
+            // slow path e1 = Gamma_r, e2 = Gamma_C/Gamma_r
+            const float lo1 = slow ? 0.f : Lref;
+            const float lo2 = slow ? LC : Lref;
+            const uint32_t ps1 = slow ? 0u : pref;
+            const uint32_t ps2 = slow ? pC : pref;
+            if (slow) {
+                float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i];
+            }
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
-                float xq[8], xk[8];
+                float xk[8], xq[8], yk[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int i = 8 * q8 + e, r = 32 * hh + i;
-                    xq[e] = ld_bf16_tile(sm + SM_Q, r, m) * g[i];
-                    xk[e] = ld_bf16_tile(sm + SM_K, r, m) * kp[i];
+                    const uint32_t pr = (par >> i) & 1u;
+                    const float e1 = ((pr ^ ps1) ? -1.f : 1.f) * exp2f(L[i] - lo1);
+                    const float e2 = ((pr ^ ps2) ? -1.f : 1.f) * exp2f(lo2 - L[i]);
+                    const float kv = ld_bf16_tile(sm + SM_K, r, m);
+                    const float qv = ld_bf16_tile(sm + SM_Q, r, m);
+                    xk[e] = kv * e1;
+                    xq[e] = qv * e1;
+                    yk[e] = kv * e2;
                 }
-                store_split8(sm + SM_C1HI + 16384, sm + SM_C1LO + 16384, m, 4 * hh + q8, xq);
-                store_split8(sm + SM_KPHI, sm + SM_KPLO, m, 4 * hh + q8, xk);
+                store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xk);
+                store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xq);
+                store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
+            }
+            if (slow) {
+                // sign bits of Gamma per (token, channel): word [r][m/32], bit m%32
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const unsigned bits = __ballot_sync(0xffffffffu, (par >> i) & 1u);
+                    if (lane == 0) sh_sign[(32 * hh + i) * 4 + quarter] = bits;
+                }
+            }
+        }
+        sync_for_mma();
+
+        // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact pairwise path
+        if (!slow) {
+            if (tid == 0) {
+                const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
+                const uint32_t xa[3] = {sbase + SM_XHI, sbase + SM_XHI, sbase + SM_XLO};
+                const uint32_t yb[3] = {sbase + SM_YHI, sbase + SM_YLO, sbase + SM_YHI};
+                for (int ps = 0; ps < 3; ++ps)
+                    for (int ks = 0; ks < 8; ++ks)
+                        tc::mma_ss(tm + TM_D1, tc::sdesc(xa[ps] + ks * 2048, 16384, 1024),
+                                   tc::sdesc(yb[ps] + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
+                tc::mma_commit(&bar_mma);
+            }
+            if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
+            mma_phase ^= 1u;
+            tc::tc_fence_after();
+            // ---------------- P3: A (fp32, into the k-tile space) and P (hi/lo) out of TMEM
+            float d1[32];
+            tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
+            tc::tmem_ld_wait();
+            if (m < C) {
+                const int r = m;
+                const float br = sh_beta[r];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int s = 32 * hh + i;
+                    ax[ax_idx(r, s)] = (s < r) ? br * d1[i] : 0.f;
+                }
+            } else {
+                const int r = m - C;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) d1[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_PHI, sm + SM_PLO, r, 4 * hh + q8, d1 + 8 * q8);
+            }
+        } else {
+            // exact pairwise evaluation: 64 x 64 pairs, 128 channels each
+            const float* Ls = reinterpret_cast<const float*>(sm + SM_SLOWL);
+            float va[16], vp[16];
+#pragma unroll 1
+            for (int j = 0; j < 16; ++j) {
+                const int e = tid + NT * j, r = e >> 6, s = e & 63;
+                float accA = 0.f, accP = 0.f;
+                if (s <= r) {
+                    for (int c = 0; c < D; ++c) {
+                        const uint32_t sg = ((sh_sign[r * 4 + (c >> 5)] ^ sh_sign[s * 4 + (c >> 5)]) >> (c & 31)) & 1u;
+                        const float w = (sg ? -1.f : 1.f) * exp2f(Ls[r * D + c] - Ls[s * D + c]);
+                        const float ksw = ld_bf16_tile(sm + SM_K, s, c) * w;
+                        accA = fmaf(ld_bf16_tile(sm + SM_K, r, c), ksw, accA);
+                        accP = fmaf(ld_bf16_tile(sm + SM_Q, r, c), ksw, accP);
+                    }
+                }
+                va[j] = (s < r) ? sh_beta[r] * accA : 0.f;
+                vp[j] = accP;
+            }
+            __syncthreads();      // k, q tiles fully read before A overwrites them
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int e = tid + NT * j, r = e >> 6, s = e & 63;
+                ax[ax_idx(r, s)] = va[j];
+                uint32_t hpair, lpair;
+                split2(vp[j], 0.f, hpair, lpair);
+                const uint32_t off = chunk_off(r, s >> 3) + (uint32_t)(s & 7) * 2u;
+                *reinterpret_cast<uint16_t*>(sm + SM_PHI + off) = (uint16_t)(hpair & 0xffffu);
+                *reinterpret_cast<uint16_t*>(sm + SM_PLO + off) = (uint16_t)(lpair & 0xffffu);
             }
         }
         tc::tmem_ld_wait();
         tc::tc_fence_before();
         __syncthreads();
 
-        // ---------------- P4: T = (I + A)^{-1} Diag(beta), blocked 16 x 16
-        if (tid < 64) {
-            const int I = tid >> 4, j = tid & 15;
+        // ---------------- P4: T = (I + A)^{-1} Diag(beta), blocked 16 x 16, in place
+        // diagonal blocks: warp I inverts block I, lane j < 16 solves column j
+        if (warp < 4 && lane < 16) {
+            const int I = warp, j = lane;
             float x[16];
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * I + rr;
-                float acc = (rr == j) ? 1.f : 0.f;
+                float acc0 = (rr == j) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-                for (int ss = 0; ss < rr; ++ss) {
-                    const int s = 16 * I + ss;
-                    acc -= amat[r * 64 + (s ^ (r & 31))] * x[ss];
+                for (int ss = 0; ss < rr; ss += 2) {
+                    acc0 -= ax[ax_idx(r, 16 * I + ss)] * x[ss];
+                    if (ss + 1 < rr) acc1 -= ax[ax_idx(r, 16 * I + ss + 1)] * x[ss + 1];
                 }
-                x[rr] = (rr < j) ? 0.f : acc;
+                x[rr] = (rr < j) ? 0.f : acc0 + acc1;
             }
+            __syncwarp(0x0000ffffu);
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) xinv[(16 * I + rr) * 65 + 16 * I + j] = x[rr];
+            for (int rr = 0; rr < 16; ++rr) ax[ax_idx(16 * I + rr, 16 * I + j)] = x[rr];
         }
         __syncthreads();
-        for (int I = 1; I < 4; ++I) {
-            for (int e = tid; e < I * 256; e += NT) {
-                const int J = e >> 8, rr = (e >> 4) & 15, jj = e & 15;
+        // block rows I = 1..3: R = -A_{I,<I} X_{<I}, then X_{I,<I} = X_II R.
+        // Thread (rr = tid / 16, cc = tid % 16) owns columns cc + 16 J of row 16 I + rr.
+        {
+            const int rr = tid >> 4, cc = tid & 15;
+#pragma unroll
+            for (int I = 1; I < 4; ++I) {
                 const int r = 16 * I + rr;
-                float acc = 0.f;
-                for (int K = J; K < I; ++K)
+                float acc[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+                for (int K = 0; K < I; ++K) {
 #pragma unroll
                     for (int mm = 0; mm < 16; ++mm) {
-                        const int s = 16 * K + mm;
-                        acc = fmaf(amat[r * 64 + (s ^ (r & 31))], xinv[s * 65 + 16 * J + jj], acc);
+                        const int kk = 16 * K + mm;
+                        const float a = ax[ax_idx(r, kk)];
+#pragma unroll
+                        for (int J = 0; J <= K; ++J) acc[J] = fmaf(a, ax[ax_idx(kk, 16 * J + cc)], acc[J]);
                     }
-                ytmp[e] = acc;
+                }
+#pragma unroll
+                for (int J = 0; J < I; ++J) rt[rr * 48 + 16 * J + cc] = -acc[J];
+                __syncthreads();
+                float xo[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+                for (int mm = 0; mm < 16; ++mm) {
+                    const float xd = ax[ax_idx(r, 16 * I + mm)];       // X_II (zero above the diagonal)
+#pragma unroll
+                    for (int J = 0; J < I; ++J) xo[J] = fmaf(xd, rt[mm * 48 + 16 * J + cc], xo[J]);
+                }
+#pragma unroll
+                for (int J = 0; J < I; ++J) ax[ax_idx(r, 16 * J + cc)] = xo[J];
+                __syncthreads();
             }
-            __syncthreads();
-            for (int e = tid; e < I * 256; e += NT) {
-                const int J = e >> 8, rr = (e >> 4) & 15, jj = e & 15;
-                float acc = 0.f;
-                for (int mm = 0; mm <= rr; ++mm)
-                    acc = fmaf(xinv[(16 * I + rr) * 65 + 16 * I + mm], ytmp[J * 256 + mm * 16 + jj], acc);
-                xinv[(16 * I + rr) * 65 + 16 * J + jj] = -acc;
-            }
-            __syncthreads();
         }
         {
             // T = X Diag(beta): thread -> row r = tid / 4, columns 16 (tid % 4) .. +15
             const int r = tid >> 2, q4 = tid & 3;
-            uint32_t ph[8], pl[8];
+            float v[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int s0 = 16 * q4 + 2 * e;
-                const float v0 = (s0 <= r) ? xinv[r * 65 + s0] * sh_beta[s0] : 0.f;
-                const float v1 = (s0 + 1 <= r) ? xinv[r * 65 + s0 + 1] * sh_beta[s0 + 1] : 0.f;
-                __nv_bfloat16 h0, l0, h1, l1;
-                tc::split_bf16(v0, h0, l0);
-                tc::split_bf16(v1, h1, l1);
-                ph[e] = tc::pack_bf16(h0, h1);
-                pl[e] = tc::pack_bf16(l0, l1);
+            for (int e = 0; e < 16; ++e) {
+                const int s = 16 * q4 + e;
+                v[e] = (s <= r) ? ax[ax_idx(r, s)] * sh_beta[s] : 0.f;
             }
-            uint8_t* tt = sm + SM_T;
-            *reinterpret_cast<uint4*>(tt + chunk_off(r, 2 * q4)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-            *reinterpret_cast<uint4*>(tt + chunk_off(r, 2 * q4 + 1)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
-            *reinterpret_cast<uint4*>(tt + chunk_off(64 + r, 2 * q4)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-            *reinterpret_cast<uint4*>(tt + chunk_off(64 + r, 2 * q4 + 1)) = make_uint4(pl[4], pl[5], pl[6], pl[7]);
+            store_split8(sm + SM_T, sm + SM_T + 8192, r, 2 * q4, v);
+            store_split8(sm + SM_T, sm + SM_T + 8192, r, 2 * q4 + 1, v + 8);
         }
         sync_for_mma();
 
-        // ---------------- P5: U~^T = V^T [T_hi^T | T_lo^T],  W^T = K~^T [..] + K~lo^T T_hi^T
+        // ---------------- P5: U~^T = V^T [T_hi^T | T_lo^T],  W^T/g = (k e1)^T [..] + lo part
         if (tid == 0) {
             const uint32_t iu = tc::idesc_bf16(128, 128, 1, 0);
             for (int ks = 0; ks < 4; ++ks)
@@ -513,28 +495,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                            tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iu, ks != 0);
             const uint32_t iw = tc::idesc_bf16(128, 128, 0, 0);
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ts(tm + TM_DW, tm + TM_KTHI + ks * 8, tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw,
-                           ks != 0);
+                tc::mma_ss(tm + TM_DW, tc::sdesc(sbase + SM_XHI + ks * 32, 16, 1024),
+                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw, ks != 0);
             const uint32_t iw2 = tc::idesc_bf16(128, 64, 0, 0);
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ts(tm + TM_DW, tm + TM_KTLO + ks * 8, tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw2, 1);
+                tc::mma_ss(tm + TM_DW, tc::sdesc(sbase + SM_XLO + ks * 32, 16, 1024),
+                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw2, 1);
             tc::mma_commit(&bar_mma);
         }
         if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
         mma_phase ^= 1u;
         tc::tc_fence_after();
-        // inputs of this chunk are consumed: prefetch the next chunk
+        // this chunk's k, q, v, alpha and the solve scratch are consumed: prefetch the next chunk
         if (tid == 0 && ck + 1 < nchunks) issue_loads(t0 + C);
+        if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
 
-        // ---------------- P6: W^T -> C1 operand block 0; S0^T -> TMEM A operand; S *= Gamma_C
+        // ---------------- P6: W^T/g -> X block 0; state operand copy and rescale
         {
             float w0[32], w1[32];
-            tmem_ld<32>(tl + TM_DW + 32 * hh, w0);
-            tmem_ld<32>(tl + TM_DW + 64 + 32 * hh, w1);
+            tc::tmem_ld32<32>(tl + TM_DW + 32 * hh, w0);
+            tc::tmem_ld32<32>(tl + TM_DW + 64 + 32 * hh, w1);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) w0[i] += w1[i];
-            store_split_row32(sm + SM_C1HI, sm + SM_C1LO, m, hh, w0);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, w0 + 8 * q8);
         }
         tc::tc_fence_before();
         __syncthreads();
@@ -542,24 +527,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
         for (int cb = 0; cb < 2; ++cb) {
             const int c0 = 64 * hh + 32 * cb;
-            float s[32];
-            tmem_ld<32>(tl + TM_S + c0, s);
+            float s[32], z[32];
+            tc::tmem_ld32<32>(tl + TM_S + c0, s);
             tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) z[i] = s[i] * sh_fa[c0 + i];
             uint32_t hi[16], lo[16];
-            split_pack32(s, hi, lo);
+            split_pack32(z, hi, lo);
             tc::tmem_st32<16>(tl + TM_SAHI + c0 / 2, hi);
             tc::tmem_st32<16>(tl + TM_SALO + c0 / 2, lo);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s[i] *= sh_gC[c0 + i];
+            for (int i = 0; i < 32; ++i) s[i] *= sh_fs[c0 + i];
             tmem_st_f32x32(tl + TM_S + c0, s);
         }
         sync_for_mma();
 
-        // ---------------- P7: D_R = S0^T [W^T | Q~^T]  (3 passes)
+        // ---------------- P7: D_R = (S0 Diag g)^T [W^T/g | (q e1)^T]  (3 passes)
         if (tid == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
             const uint32_t aa[3] = {tm + TM_SAHI, tm + TM_SAHI, tm + TM_SALO};
-            const uint32_t bb[3] = {sbase + SM_C1HI, sbase + SM_C1LO, sbase + SM_C1HI};
+            const uint32_t bb[3] = {sbase + SM_XHI, sbase + SM_XLO, sbase + SM_XHI};
             for (int ps = 0; ps < 3; ++ps)
                 for (int ks = 0; ks < 8; ++ks)
                     tc::mma_ts(tm + TM_DR, aa[ps] + ks * 8, tc::sdesc(bb[ps] + ks * 2048, 16384, 1024), idesc,
@@ -573,9 +560,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // ---------------- P8: U^T = U~^T - (S0^T W^T) -> TMEM A operand
         {
             float ua[32], ub[32], ws[32];
-            tmem_ld<32>(tl + TM_DU + 32 * hh, ua);
-            tmem_ld<32>(tl + TM_DU + 64 + 32 * hh, ub);
-            tmem_ld<32>(tl + TM_DR + 32 * hh, ws);
+            tc::tmem_ld32<32>(tl + TM_DU + 32 * hh, ua);
+            tc::tmem_ld32<32>(tl + TM_DU + 64 + 32 * hh, ub);
+            tc::tmem_ld32<32>(tl + TM_DR + 32 * hh, ws);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) ua[i] = (ua[i] + ub[i]) - ws[i];
@@ -586,13 +573,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
         sync_for_mma();
 
-        // ---------------- P9: O^T += U^T P^T ;  S^T += U^T K'  (3 passes each)
+        // ---------------- P9: O^T += U^T P^T ;  acc += U^T (k e2)  (3 passes each)
         if (tid == 0) {
             const uint32_t io = tc::idesc_bf16(128, 64, 0, 0);
             const uint32_t is = tc::idesc_bf16(128, 128, 0, 0);
             const uint32_t aa[3] = {tm + TM_UAHI, tm + TM_UAHI, tm + TM_UALO};
             const uint32_t pb[3] = {sbase + SM_PHI, sbase + SM_PLO, sbase + SM_PHI};
-            const uint32_t kb[3] = {sbase + SM_KPHI, sbase + SM_KPLO, sbase + SM_KPHI};
+            const uint32_t kb[3] = {sbase + SM_YHI, sbase + SM_YLO, sbase + SM_YHI};
             for (int ps = 0; ps < 3; ++ps)
                 for (int ks = 0; ks < 4; ++ks) {
                     tc::mma_ts(tm + TM_O, aa[ps] + ks * 8, tc::sdesc(pb[ps] + ks * 32, 16, 1024), io, 1);
@@ -607,7 +594,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // ---------------- P10: o rows of this chunk
         {
             float ov[32];
-            tmem_ld<32>(tl + TM_O + 32 * hh, ov);
+            tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -620,16 +607,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::tc_fence_after();
     }
 
-    // final state
+    // final state: S = acc Diag(kappa_last)
     if (!failed && ST != nullptr) {
         const size_t sb = (size_t)bh * D * D;
         for (int cb = 0; cb < 2; ++cb) {
             const int c0 = 64 * hh + 32 * cb;
             float x[32];
-            tmem_ld<32>(tl + TM_S + c0, x);
+            tc::tmem_ld32<32>(tl + TM_S + c0, x);
             tc::tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ST[sb + (size_t)(c0 + i) * D + m] = x[i];
+            for (int i = 0; i < 32; ++i) ST[sb + (size_t)(c0 + i) * D + m] = x[i] * sh_kref[c0 + i];
         }
     }
     tc::tc_fence_before();
