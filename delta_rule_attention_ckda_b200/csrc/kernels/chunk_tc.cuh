@@ -72,6 +72,7 @@ constexpr uint32_t SM_XHI = 81920;      // X hi: block 0 = k e1 (later W^T), blo
 constexpr uint32_t SM_XLO = 114688;     // X lo
 constexpr uint32_t SM_YHI = 147456;     // Y = k e2, [128 c][64 s] (MN-major for A/P, K-major for S)
 constexpr uint32_t SM_YLO = 163840;
+constexpr uint32_t SM_OT = 81920;       //   after C1: o tile fp32 [64 tok][128], TMA-stored
 constexpr uint32_t SM_PHI = 180224;     // P K-major [64 r][64 s]
 constexpr uint32_t SM_PLO = 188416;
 constexpr uint32_t SM_RT = 196608;      // solve temporary, fp32 [16][48]
@@ -172,8 +173,8 @@ __device__ __forceinline__ int ax_idx(int r, int s) { return r * 64 + (s ^ (r & 
 __global__ void __launch_bounds__(ctc::NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
-                const float* __restrict__ beta, const float* S0, float* __restrict__ o, float* ST,
-                int T, int H) {
+                const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta, const float* S0,
+                float* ST, int T, int H) {
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -208,6 +209,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::prefetch_tensormap(&map_q);
         tc::prefetch_tensormap(&map_v);
         tc::prefetch_tensormap(&map_a);
+        tc::prefetch_tensormap(&map_o);
     }
     if (tid < D) sh_kref[tid] = 1.f;
     tc::tc_fence_before();
@@ -253,6 +255,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         const int t0 = ck * C;
         const int nvalid = min(C, T - t0);
         if (tid < C) sh_beta[tid] = beta_next;
+        if (tid == 0) tc::bulk_wait_read0();     // the previous o tile has left the X region
         if (wait_all(&bar_tma, ck & 1)) { failed = true; break; }
 
         // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
@@ -591,21 +594,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         mma_phase ^= 1u;
         tc::tc_fence_after();
 
-        // ---------------- P10: o rows of this chunk
+        // ---------------- P10: o rows of this chunk -> shared tile [64 tok][128] -> TMA store
         {
             float ov[32];
             tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
             tc::tmem_ld_wait();
+            float* ot = reinterpret_cast<float*>(sm + SM_OT);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = 32 * hh + i;
-                if (r < nvalid) o[(((size_t)b * T + t0 + r) * H + h) * D + m] = ov[i];
-            }
+            for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
         }
+        tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncthreads();
         tc::tc_fence_after();
+        if (tid == 0) {
+            tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0, b);   // rows past T are skipped
+            tc::bulk_commit();
+        }
     }
+    if (tid == 0) tc::bulk_wait0();
 
     // final state: S = acc Diag(kappa_last)
     if (!failed && ST != nullptr) {
@@ -642,11 +649,13 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
                                    int B, int T, int H, int dk, int dv, void* workspace, cudaStream_t st) {
     (void)workspace;
     if (dk != 128 || dv != 128) return cudaErrorNotSupported;
-    CUtensorMap mk, mq, mv, ma;
+    CUtensorMap mk, mq, mv, ma, mo;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!tc::make_map_bthd(&mk, k, bf, 2, B, T, H, dk, 64, 64) || !tc::make_map_bthd(&mq, q, bf, 2, B, T, H, dk, 64, 64) ||
         !tc::make_map_bthd(&mv, v, bf, 2, B, T, H, dv, 64, 64) ||
-        !tc::make_map_bthd(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dk, 32, 64))
+        !tc::make_map_bthd(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dk, 32, 64) ||
+        !tc::make_map_bthd(&mo, o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dv, 128, 64,
+                           CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
@@ -655,7 +664,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    chunk_tc_kernel<<<(unsigned)(B * H), ctc::NT, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, beta, S0, o, ST, T, H);
+    chunk_tc_kernel<<<(unsigned)(B * H), ctc::NT, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H);
     return cudaGetLastError();
 }
 
