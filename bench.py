@@ -43,6 +43,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-extras", action="store_true")
+    p.add_argument("--batch", type=int, default=WORKLOAD["B"],
+                   help="batch size of the layer workload (smaller values for profiling captures)")
+    p.add_argument("--only", default="all", choices=["all", "chunk", "decode"],
+                   help="run only one of the two kernels (profiling captures)")
     return p.parse_args()
 
 
@@ -285,7 +289,12 @@ def ours_arm(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
 
-    inp = make_workload("layer")
+    if args.only == "decode":
+        line = {"decode": decode_measure(ck, dev, stream, world)}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+    inp = make_workload("layer", B=args.batch)
     B, T, H, dk, dv = inp.shape
     q, k, v, a, b = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
     o = torch.empty(B, T, H, dv, device=dev)
@@ -328,7 +337,7 @@ def ours_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_launch,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "layer B=8 T=4096 H=16 dk=dv=128 chunk=64", **WORKLOAD,
+            "config": {"workload": f"layer B={B} T={T} H={H} dk=dv={dk} chunk=64", **WORKLOAD, "B": B,
                        "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
                        "path": path, "l2": "inputs larger than L2 (~950 MB per step vs 126 MB), no flush",
                        "state": "S0 = 0 (not read), S_T written"},
@@ -338,7 +347,7 @@ def ours_arm(args):
         line["e2e"] = e2e_measure(ck, inp, dev, stream, world, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp)
-    if not args.no_extras:
+    if not args.no_extras and args.only == "all":
         line["decode"] = decode_measure(ck, dev, stream, world)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -407,7 +416,7 @@ def decode_measure(ck, dev, stream, world):
             "tokens_per_s": N * world / per, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
                                                          "unit": "GB/s", "frac": gbs / hbm,
                                                          "alg_bytes_per_launch": bytes_call,
-                                                         "kernel": "decode128"},
+                                                         "kernel": "decode128", "traffic": committed_traffic("decode128")},
             "gpu_launches": calls}
 
 
