@@ -72,7 +72,7 @@ constexpr uint32_t SM_XHI = 81920;      // X hi: block 0 = k e1 (later W^T), blo
 constexpr uint32_t SM_XLO = 114688;     // X lo
 constexpr uint32_t SM_YHI = 147456;     // Y = k e2, [128 c][64 s] (MN-major for A/P, K-major for S)
 constexpr uint32_t SM_YLO = 163840;
-constexpr uint32_t SM_OT = 81920;       //   after C1: o tile fp32 [64 tok][128], TMA-stored
+constexpr uint32_t SM_OT = 49152;       //   after the gate: o tile fp32 [64 tok][128], TMA-stored
 constexpr uint32_t SM_PHI = 180224;     // P K-major [64 r][64 s]
 constexpr uint32_t SM_PLO = 188416;
 constexpr uint32_t SM_RT = 196608;      // solve temporary, fp32 [16][48]
@@ -82,15 +82,15 @@ constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;       // + alignment slack
 
 // TMEM column map (512 columns allocated)
 constexpr uint32_t TM_S = 0;          // state accumulator S^T Diag(1/kappa) [d_v lanes][d_k cols]
-constexpr uint32_t TM_D1 = 128;       // [A ; P] 128 x 64
-constexpr uint32_t TM_DR = 128;       // (S0 Diag g)^T [W^T/g | (q e1)^T] 128 x 128
-constexpr uint32_t TM_O = 192;        //   its second half accumulates O^T
+constexpr uint32_t TM_SAHI = 128;     // (S0 Diag g)^T hi / lo, packed bf16 (A operand of C1)
+constexpr uint32_t TM_SALO = 192;
+constexpr uint32_t TM_UAHI = 128;     // U^T hi / lo, packed bf16 (A operand of the O / S MMAs)
+constexpr uint32_t TM_UALO = 160;
 constexpr uint32_t TM_DU = 256;       // V^T [T_hi^T | T_lo^T]
+constexpr uint32_t TM_D1 = 384;       // [A ; P] 128 x 64
 constexpr uint32_t TM_DW = 384;       // (k e1)^T [T_hi^T | T_lo^T] + lo part
-constexpr uint32_t TM_SAHI = 384;     // (S0 Diag g)^T hi / lo, packed bf16 (A operand)
-constexpr uint32_t TM_SALO = 448;
-constexpr uint32_t TM_UAHI = 384;     // U^T hi / lo, packed bf16 (A operand)
-constexpr uint32_t TM_UALO = 416;
+constexpr uint32_t TM_DR = 384;       // (S0 Diag g)^T [W^T/g | (q e1)^T] 128 x 128
+constexpr uint32_t TM_O = 448;        //   its second half accumulates O^T (read in the next chunk)
 
 constexpr uint32_t kTmaBytes = 10 * 8192;    // 6 bf16 boxes + 4 fp32 boxes
 
@@ -170,6 +170,12 @@ __device__ __forceinline__ int ax_idx(int r, int s) { return r * 64 + (s ^ (r & 
 
 // ------------------------------------------------------------------------------ kernel
 
+// Per-chunk schedule (one CTA per (batch, head), 8 warps). Each tcgen05 group commits to
+// its own mbarrier, so work that does not depend on an MMA runs while it executes:
+//   gate cumulation of chunk c          ||  O / state MMAs of chunk c-1
+//   o store of chunk c-1, state copy     ||  [A ; P] MMA of chunk c
+//   W^T epilogue                         ||  U~ MMA
+// and the next chunk's inputs are fetched by TMA once the U~ MMA has consumed V and T.
 __global__ void __launch_bounds__(ctc::NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
@@ -178,7 +184,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tma, bar_mma;
+    __shared__ uint64_t bar_tma, bar_ap, bar_w, bar_u, bar_c1, bar_c2;
     __shared__ uint32_t tmem_base_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
@@ -203,7 +209,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
     if (tid == 0) {
         tc::mbar_init(&bar_tma, 1);
-        tc::mbar_init(&bar_mma, 1);
+        tc::mbar_init(&bar_ap, 1);
+        tc::mbar_init(&bar_w, 1);
+        tc::mbar_init(&bar_u, 1);
+        tc::mbar_init(&bar_c1, 1);
+        tc::mbar_init(&bar_c2, 1);
         tc::fence_mbar_init();
         tc::prefetch_tensormap(&map_k);
         tc::prefetch_tensormap(&map_q);
@@ -233,6 +243,55 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     };
     float beta_next = load_beta(0);
 
+    // o rows of a finished chunk: TMEM -> shared tile [64 tok][128] fp32 in the alpha space.
+    // The TMA store itself is issued by thread 0 after the next CTA barrier.
+    auto stage_o = [&]() {
+        float ov[32];
+        tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
+        tc::tmem_ld_wait();
+        float* ot = reinterpret_cast<float*>(sm + SM_OT);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
+        tc::fence_proxy_async_smem();
+    };
+    // state copy into the C1 operand (scaled by fa) and rescale of the accumulator (by fs)
+    auto state_copy = [&](bool slow_chunk) {
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+            const int c0 = 64 * hh + 32 * cb;
+            float sv[32], z[32];
+            tc::tmem_ld32<32>(tl + TM_S + c0, sv);
+            tc::tmem_ld_wait();
+            const float4* fa4 = reinterpret_cast<const float4*>(sh_fa + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 f = fa4[i];
+                z[4 * i] = sv[4 * i] * f.x;
+                z[4 * i + 1] = sv[4 * i + 1] * f.y;
+                z[4 * i + 2] = sv[4 * i + 2] * f.z;
+                z[4 * i + 3] = sv[4 * i + 3] * f.w;
+            }
+            uint32_t hi[16], lo[16];
+            split_pack32(z, hi, lo);
+            tc::tmem_st32<16>(tl + TM_SAHI + c0 / 2, hi);
+            tc::tmem_st32<16>(tl + TM_SALO + c0 / 2, lo);
+            if (!slow_chunk) {
+                tmem_st_f32x32(tl + TM_S + c0, z);        // fast path: fs == fa
+            } else {
+                const float4* fs4 = reinterpret_cast<const float4*>(sh_fs + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 f = fs4[i];
+                    sv[4 * i] *= f.x;
+                    sv[4 * i + 1] *= f.y;
+                    sv[4 * i + 2] *= f.z;
+                    sv[4 * i + 3] *= f.w;
+                }
+                tmem_st_f32x32(tl + TM_S + c0, sv);
+            }
+        }
+    };
+
     // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
     {
         const size_t sb = (size_t)bh * D * D;
@@ -247,7 +306,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     }
 
     const uint32_t sbase = tc::smem_u32(sm);
-    uint32_t mma_phase = 0;
+    uint32_t ph_ap = 0, ph_w = 0, ph_u = 0, ph_c1 = 0, ph_c2 = 0;
     bool failed = false;
     const int nchunks = (T + C - 1) / C;
 
@@ -255,7 +314,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         const int t0 = ck * C;
         const int nvalid = min(C, T - t0);
         if (tid < C) sh_beta[tid] = beta_next;
-        if (tid == 0) tc::bulk_wait_read0();     // the previous o tile has left the X region
         if (wait_all(&bar_tma, ck & 1)) { failed = true; break; }
 
         // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
@@ -269,7 +327,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             for (int i = 0; i < 32; ++i) {
                 const int r = 32 * hh + i;
                 const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
-                run += fmaxf(__log2f(fabsf(a)), kLgFloor);
+                run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
                 p ^= (a < 0.f) ? 1u : 0u;
                 L[i] = run;
                 par |= p << i;
@@ -322,6 +380,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i];
             }
+            // the previous chunk's O / S MMAs read Y and P: wait for them before overwriting
+            if (ck > 0) {
+                if (wait_all(&bar_c2, ph_c2)) { failed = true; break; }
+                ph_c2 ^= 1u;
+                tc::tc_fence_after();
+            }
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
                 float xk[8], xq[8], yk[8];
@@ -329,8 +393,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 for (int e = 0; e < 8; ++e) {
                     const int i = 8 * q8 + e, r = 32 * hh + i;
                     const uint32_t pr = (par >> i) & 1u;
-                    const float e1 = ((pr ^ ps1) ? -1.f : 1.f) * exp2f(L[i] - lo1);
-                    const float e2 = ((pr ^ ps2) ? -1.f : 1.f) * exp2f(lo2 - L[i]);
+                    const float e1 = ((pr ^ ps1) ? -1.f : 1.f) * tc::ex2_approx(L[i] - lo1);
+                    const float e2 = ((pr ^ ps2) ? -1.f : 1.f) * tc::ex2_approx(lo2 - L[i]);
                     const float kv = ld_bf16_tile(sm + SM_K, r, m);
                     const float qv = ld_bf16_tile(sm + SM_Q, r, m);
                     xk[e] = kv * e1;
@@ -356,17 +420,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         if (!slow) {
             if (tid == 0) {
                 const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
-                const uint32_t xa[3] = {sbase + SM_XHI, sbase + SM_XHI, sbase + SM_XLO};
-                const uint32_t yb[3] = {sbase + SM_YHI, sbase + SM_YLO, sbase + SM_YHI};
-                for (int ps = 0; ps < 3; ++ps)
+#pragma unroll
+                for (int ps = 0; ps < 3; ++ps) {
+                    const uint32_t xa = sbase + (ps == 2 ? SM_XLO : SM_XHI);
+                    const uint32_t yb = sbase + (ps == 1 ? SM_YLO : SM_YHI);
+#pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        tc::mma_ss(tm + TM_D1, tc::sdesc(xa[ps] + ks * 2048, 16384, 1024),
-                                   tc::sdesc(yb[ps] + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
-                tc::mma_commit(&bar_mma);
+                        tc::mma_ss(tm + TM_D1, tc::sdesc(xa + ks * 2048, 16384, 1024),
+                                   tc::sdesc(yb + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
+                }
+                tc::mma_commit(&bar_ap);
             }
-            if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
-            mma_phase ^= 1u;
+            // while the MMA runs: the previous chunk's o tile and this chunk's state copy
+            if (ck > 0) stage_o();
+            state_copy(slow);
+            if (wait_all(&bar_ap, ph_ap)) { failed = true; break; }
+            ph_ap ^= 1u;
             tc::tc_fence_after();
+            if (tid == 0 && ck > 0) {
+                tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
+                tc::bulk_commit();
+            }
             // ---------------- P3: A (fp32, into the k-tile space) and P (hi/lo) out of TMEM
             float d1[32];
             tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
@@ -417,6 +491,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 *reinterpret_cast<uint16_t*>(sm + SM_PHI + off) = (uint16_t)(hpair & 0xffffu);
                 *reinterpret_cast<uint16_t*>(sm + SM_PLO + off) = (uint16_t)(lpair & 0xffffu);
             }
+            if (ck > 0) stage_o();
+            state_copy(slow);
+            __syncthreads();
+            if (tid == 0 && ck > 0) {
+                tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);
+                tc::bulk_commit();
+            }
         }
         tc::tmem_ld_wait();
         tc::tc_fence_before();
@@ -430,13 +511,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * I + rr;
-                float acc0 = (rr == j) ? 1.f : 0.f, acc1 = 0.f;
+                float acc[4] = {(rr == j) ? 1.f : 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int ss = 0; ss < rr; ss += 2) {
-                    acc0 -= ax[ax_idx(r, 16 * I + ss)] * x[ss];
-                    if (ss + 1 < rr) acc1 -= ax[ax_idx(r, 16 * I + ss + 1)] * x[ss + 1];
-                }
-                x[rr] = (rr < j) ? 0.f : acc0 + acc1;
+                for (int ss = 0; ss < rr; ++ss) acc[ss & 3] -= ax[ax_idx(r, 16 * I + ss)] * x[ss];
+                x[rr] = (rr < j) ? 0.f : (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
             __syncwarp(0x0000ffffu);
 #pragma unroll
@@ -444,76 +522,92 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
         __syncthreads();
         // block rows I = 1..3: R = -A_{I,<I} X_{<I}, then X_{I,<I} = X_II R.
-        // Thread (rr = tid / 16, cc = tid % 16) owns columns cc + 16 J of row 16 I + rr.
-        {
-            const int rr = tid >> 4, cc = tid & 15;
+        // Thread task = (row rr, column group g of 4); entries above the block diagonal are
+        // zero, so every task runs the same k range. Groups of 4 columns stay inside one
+        // 16-byte word of the column-swizzled layout (element j of logical group g of row k
+        // is at group g ^ ((k & 31) >> 2), position j ^ (k & 3)).
 #pragma unroll
-            for (int I = 1; I < 4; ++I) {
-                const int r = 16 * I + rr;
-                float acc[3] = {0.f, 0.f, 0.f};
+        for (int I = 1; I < 4; ++I) {
+            const int ng = 4 * I;
+            const bool act = tid < 16 * ng;
+            const int rr = tid / ng, g = tid % ng;
+            const int r = 16 * I + (act ? rr : 0);
+            if (act) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int K = 0; K < I; ++K) {
+                for (int k = 0; k < 16 * I; ++k) {
+                    const float a = ax[ax_idx(r, k)];
+                    const float4 xv = *reinterpret_cast<const float4*>(ax + k * 64 + 4 * (g ^ ((k & 31) >> 2)));
+                    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                    for (int mm = 0; mm < 16; ++mm) {
-                        const int kk = 16 * K + mm;
-                        const float a = ax[ax_idx(r, kk)];
-#pragma unroll
-                        for (int J = 0; J <= K; ++J) acc[J] = fmaf(a, ax[ax_idx(kk, 16 * J + cc)], acc[J]);
-                    }
+                    for (int jj = 0; jj < 4; ++jj) acc[jj] = fmaf(a, xs[jj ^ (k & 3)], acc[jj]);
                 }
-#pragma unroll
-                for (int J = 0; J < I; ++J) rt[rr * 48 + 16 * J + cc] = -acc[J];
-                __syncthreads();
-                float xo[3] = {0.f, 0.f, 0.f};
+                *reinterpret_cast<float4*>(rt + rr * 48 + 4 * g) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+            }
+            __syncthreads();
+            if (act) {
+                float xo[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int mm = 0; mm < 16; ++mm) {
                     const float xd = ax[ax_idx(r, 16 * I + mm)];       // X_II (zero above the diagonal)
-#pragma unroll
-                    for (int J = 0; J < I; ++J) xo[J] = fmaf(xd, rt[mm * 48 + 16 * J + cc], xo[J]);
+                    const float4 rv = *reinterpret_cast<const float4*>(rt + mm * 48 + 4 * g);
+                    xo[0] = fmaf(xd, rv.x, xo[0]);
+                    xo[1] = fmaf(xd, rv.y, xo[1]);
+                    xo[2] = fmaf(xd, rv.z, xo[2]);
+                    xo[3] = fmaf(xd, rv.w, xo[3]);
                 }
-#pragma unroll
-                for (int J = 0; J < I; ++J) ax[ax_idx(r, 16 * J + cc)] = xo[J];
-                __syncthreads();
+                // physical position p of logical element j is j ^ (r & 3)
+                float o0 = xo[0], o1 = xo[1], o2 = xo[2], o3 = xo[3];
+                if (r & 1) { float t = o0; o0 = o1; o1 = t; t = o2; o2 = o3; o3 = t; }
+                if (r & 2) { float t = o0; o0 = o2; o2 = t; t = o1; o1 = o3; o3 = t; }
+                *reinterpret_cast<float4*>(ax + r * 64 + 4 * (g ^ ((r & 31) >> 2))) = make_float4(o0, o1, o2, o3);
             }
+            __syncthreads();
         }
         {
             // T = X Diag(beta): thread -> row r = tid / 4, columns 16 (tid % 4) .. +15
             const int r = tid >> 2, q4 = tid & 3;
-            float v[16];
+            float v[16], bb[16];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 b4 = reinterpret_cast<const float4*>(sh_beta + 16 * q4)[e];
+                bb[4 * e] = b4.x; bb[4 * e + 1] = b4.y; bb[4 * e + 2] = b4.z; bb[4 * e + 3] = b4.w;
+            }
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int s = 16 * q4 + e;
-                v[e] = (s <= r) ? ax[ax_idx(r, s)] * sh_beta[s] : 0.f;
+                v[e] = (s <= r) ? ax[ax_idx(r, s)] * bb[e] : 0.f;
             }
             store_split8(sm + SM_T, sm + SM_T + 8192, r, 2 * q4, v);
             store_split8(sm + SM_T, sm + SM_T + 8192, r, 2 * q4 + 1, v + 8);
         }
         sync_for_mma();
 
-        // ---------------- P5: U~^T = V^T [T_hi^T | T_lo^T],  W^T/g = (k e1)^T [..] + lo part
+        // ---------------- P5: W^T/g = (k e1)^T [T_hi^T | T_lo^T] + lo part;  U~^T = V^T [..]
         if (tid == 0) {
-            const uint32_t iu = tc::idesc_bf16(128, 128, 1, 0);
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(tm + TM_DU, tc::sdesc(sbase + SM_V + ks * 2048, 8192, 1024),
-                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iu, ks != 0);
             const uint32_t iw = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 tc::mma_ss(tm + TM_DW, tc::sdesc(sbase + SM_XHI + ks * 32, 16, 1024),
                            tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw, ks != 0);
             const uint32_t iw2 = tc::idesc_bf16(128, 64, 0, 0);
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 tc::mma_ss(tm + TM_DW, tc::sdesc(sbase + SM_XLO + ks * 32, 16, 1024),
                            tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw2, 1);
-            tc::mma_commit(&bar_mma);
+            tc::mma_commit(&bar_w);
+            const uint32_t iu = tc::idesc_bf16(128, 128, 1, 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_ss(tm + TM_DU, tc::sdesc(sbase + SM_V + ks * 2048, 8192, 1024),
+                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iu, ks != 0);
+            tc::mma_commit(&bar_u);
         }
-        if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
-        mma_phase ^= 1u;
+        if (wait_all(&bar_w, ph_w)) { failed = true; break; }
+        ph_w ^= 1u;
         tc::tc_fence_after();
-        // this chunk's k, q, v, alpha and the solve scratch are consumed: prefetch the next chunk
-        if (tid == 0 && ck + 1 < nchunks) issue_loads(t0 + C);
-        if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
 
-        // ---------------- P6: W^T/g -> X block 0; state operand copy and rescale
+        // ---------------- P6: W^T/g -> X block 0, while the U~ MMA runs
         {
             float w0[32], w1[32];
             tc::tmem_ld32<32>(tl + TM_DW + 32 * hh, w0);
@@ -524,40 +618,33 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, w0 + 8 * q8);
         }
-        tc::tc_fence_before();
-        __syncthreads();
+        if (wait_all(&bar_u, ph_u)) { failed = true; break; }
+        ph_u ^= 1u;
         tc::tc_fence_after();
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-            const int c0 = 64 * hh + 32 * cb;
-            float s[32], z[32];
-            tc::tmem_ld32<32>(tl + TM_S + c0, s);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = s[i] * sh_fa[c0 + i];
-            uint32_t hi[16], lo[16];
-            split_pack32(z, hi, lo);
-            tc::tmem_st32<16>(tl + TM_SAHI + c0 / 2, hi);
-            tc::tmem_st32<16>(tl + TM_SALO + c0 / 2, lo);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[i] *= sh_fs[c0 + i];
-            tmem_st_f32x32(tl + TM_S + c0, s);
+        // this chunk's k, q, v, alpha and the solve scratch are consumed: prefetch the next chunk
+        if (tid == 0 && ck + 1 < nchunks) {
+            tc::bulk_wait_read0();               // the o tile in the alpha space has been read
+            issue_loads(t0 + C);
         }
+        if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
         sync_for_mma();
 
         // ---------------- P7: D_R = (S0 Diag g)^T [W^T/g | (q e1)^T]  (3 passes)
         if (tid == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
-            const uint32_t aa[3] = {tm + TM_SAHI, tm + TM_SAHI, tm + TM_SALO};
-            const uint32_t bb[3] = {sbase + SM_XHI, sbase + SM_XLO, sbase + SM_XHI};
-            for (int ps = 0; ps < 3; ++ps)
+#pragma unroll
+            for (int ps = 0; ps < 3; ++ps) {
+                const uint32_t aa = tm + (ps == 2 ? TM_SALO : TM_SAHI);
+                const uint32_t bb = sbase + (ps == 1 ? SM_XLO : SM_XHI);
+#pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_ts(tm + TM_DR, aa[ps] + ks * 8, tc::sdesc(bb[ps] + ks * 2048, 16384, 1024), idesc,
+                    tc::mma_ts(tm + TM_DR, aa + ks * 8, tc::sdesc(bb + ks * 2048, 16384, 1024), idesc,
                                (ps | ks) != 0);
-            tc::mma_commit(&bar_mma);
+            }
+            tc::mma_commit(&bar_c1);
         }
-        if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
-        mma_phase ^= 1u;
+        if (wait_all(&bar_c1, ph_c1)) { failed = true; break; }
+        ph_c1 ^= 1u;
         tc::tc_fence_after();
 
         // ---------------- P8: U^T = U~^T - (S0^T W^T) -> TMEM A operand
@@ -576,40 +663,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
         sync_for_mma();
 
-        // ---------------- P9: O^T += U^T P^T ;  acc += U^T (k e2)  (3 passes each)
+        // ---------------- P9: O^T += U^T P^T ;  acc += U^T (k e2)  (3 passes each, waited in the next chunk)
         if (tid == 0) {
             const uint32_t io = tc::idesc_bf16(128, 64, 0, 0);
             const uint32_t is = tc::idesc_bf16(128, 128, 0, 0);
-            const uint32_t aa[3] = {tm + TM_UAHI, tm + TM_UAHI, tm + TM_UALO};
-            const uint32_t pb[3] = {sbase + SM_PHI, sbase + SM_PLO, sbase + SM_PHI};
-            const uint32_t kb[3] = {sbase + SM_YHI, sbase + SM_YLO, sbase + SM_YHI};
-            for (int ps = 0; ps < 3; ++ps)
-                for (int ks = 0; ks < 4; ++ks) {
-                    tc::mma_ts(tm + TM_O, aa[ps] + ks * 8, tc::sdesc(pb[ps] + ks * 32, 16, 1024), io, 1);
-                    tc::mma_ts(tm + TM_S, aa[ps] + ks * 8, tc::sdesc(kb[ps] + ks * 32, 16, 1024), is, 1);
-                }
-            tc::mma_commit(&bar_mma);
-        }
-        if (wait_all(&bar_mma, mma_phase)) { failed = true; break; }
-        mma_phase ^= 1u;
-        tc::tc_fence_after();
-
-        // ---------------- P10: o rows of this chunk -> shared tile [64 tok][128] -> TMA store
-        {
-            float ov[32];
-            tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
-            tc::tmem_ld_wait();
-            float* ot = reinterpret_cast<float*>(sm + SM_OT);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
+            for (int ps = 0; ps < 3; ++ps) {
+                const uint32_t aa = tm + (ps == 2 ? TM_UALO : TM_UAHI);
+                const uint32_t pb = sbase + (ps == 1 ? SM_PLO : SM_PHI);
+                const uint32_t kb = sbase + (ps == 1 ? SM_YLO : SM_YHI);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    tc::mma_ts(tm + TM_O, aa + ks * 8, tc::sdesc(pb + ks * 32, 16, 1024), io, 1);
+                    tc::mma_ts(tm + TM_S, aa + ks * 8, tc::sdesc(kb + ks * 32, 16, 1024), is, 1);
+                }
+            }
+            tc::mma_commit(&bar_c2);
         }
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        tc::tc_fence_after();
-        if (tid == 0) {
-            tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0, b);   // rows past T are skipped
-            tc::bulk_commit();
+    }
+
+    // last chunk: its O / state MMAs, then its o tile
+    if (!failed && nchunks > 0) {
+        if (wait_all(&bar_c2, ph_c2)) {
+            failed = true;
+        } else {
+            tc::tc_fence_after();
+            if (tid == 0) tc::bulk_wait_read0();
+            __syncthreads();
+            stage_o();
+            __syncthreads();
+            if (tid == 0) {
+                tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, (nchunks - 1) * C, b);
+                tc::bulk_commit();
+            }
         }
     }
     if (tid == 0) tc::bulk_wait0();

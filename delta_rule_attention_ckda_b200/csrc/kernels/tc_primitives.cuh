@@ -243,6 +243,21 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// ---------------------------------------------------------------- SFU approximations
+// The hardware base-2 exponential and logarithm (PTX ex2.approx / lg2.approx, flush to
+// zero): about 2 ulp relative error, enough for gate factors that are then split into
+// 16-bit bf16 pairs. Results below the fp32 normal range flush to zero.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------- bf16 helpers
 
 // x = hi + lo with hi = bf16(x), lo = bf16(x - hi): a 16-bit-significand pair.
