@@ -16,18 +16,20 @@
 // In exact arithmetic this equals the token loop; the WY/UT evaluation is the
 // "Chunk-WY" scheme the thelatestinai card names, derived here for the signed gate.
 //
-// Gate factoring. With a reference token ref (31) per chunk and per channel,
-//   e1_r = Gamma_r / Gamma_ref,  e2_s = Gamma_ref / Gamma_s,
-//   g_ref = Gamma_ref,  kappa = Gamma_C / Gamma_ref,
+// Gate factoring. With a per-channel reference level R = L_C / 2 (the middle of the
+// chunk's log2-magnitude range; the signs stay with the tokens),
+//   e1_r = sgn_r 2^{L_r - R},  e2_s = sgn_s 2^{R - L_s},  g_ref = 2^R,  kappa = sgn_C 2^{L_C - R},
 // every gate product above splits into per-token factors and per-channel constants:
 //   Gamma_r/Gamma_s = e1_r e2_s,  Gamma_r = e1_r g_ref,  Gamma_C/Gamma_s = e2_s kappa,
-//   Gamma_C = g_ref kappa.
+//   Gamma_C = g_ref kappa,
+// and every factor lies in [2^{L_C/2}, 2^{-L_C/2}].
 // So one pair of token tiles X = [k e1 ; q e1] and Y = k e2 serves every product:
 //   [A ; P] from X Y^T;  W / g_ref from (k e1) T^T;  O from S0 Diag(g_ref) and q e1;
 //   the state update from S0 Diag(g_ref) + U^T (k e2), which is S_C Diag(1/kappa).
 // The TMEM accumulator therefore holds S Diag(1/kappa_prev); each chunk rescales it
 // by kappa_prev * g_ref (a per-column factor, folded into the pass that copies the
 // state into the MMA operand), and the final write multiplies by the last kappa.
+// Entries above the diagonal of X Y^T may overflow; they are never read.
 //
 // B200 mapping. One CTA (256 threads) owns one (batch, head) and walks its chunks in
 // order. Everything is computed transposed so the 128 feature rows sit on the 128
@@ -38,8 +40,9 @@
 // tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by TMA (no
 // multicast) with 128-byte swizzle; tokens past the end read as zero and get gate 1.
 //
-// Exponent safety. e1 and e2 stay inside [2^-96, 2^96] unless a chunk's gates decay
-// very fast; such a chunk computes A and P pair by pair on CUDA cores (exact), uses
+// Exponent safety. e1 and e2 stay inside [2^-96, 2^96] unless a chunk's gates decay by
+// more than 2^-192 in some channel; such a chunk computes A and P pair by pair on CUDA
+// cores (exact), uses
 // the unfactored tiles (k Gamma, q Gamma, k Gamma_C/Gamma) with g_ref = kappa = 1,
 // and applies Gamma_C to the state directly.
 #pragma once
@@ -57,8 +60,7 @@ constexpr int NT = 256;      // threads per CTA
 
 // log2-domain limits of the single-reference factorisation
 constexpr float kLgFloor = -100.f;    // floor of log2|a| per token (a = 0 allowed)
-constexpr float kRefRange = 96.f;     // |L_r - L_ref| bound for the fast path
-constexpr float kChunkRange = 124.f;  // -L_C bound for the fast path
+constexpr float kChunkRange = 192.f;  // -L_C bound for the fast path (factors within 2^{+-96})
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t SM_K = 0;            // k tile: 2 TMA boxes [64 tok][64 ch] bf16
@@ -188,14 +190,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     __shared__ uint32_t tmem_base_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
-    float* sh_fa = sh_beta + 64;            // [128] factor for the state operand copy
-    float* sh_fs = sh_fa + 128;             // [128] factor for the state accumulator
+    float* sh_fa = sh_beta + 64;            // [128] g_ref (operand copy = S g_ref)
+    float* sh_fs = sh_fa + 128;             // [128] g_ref, or Gamma_C on the exact path (accumulator)
     float* sh_kref = sh_fs + 128;           // [128] kappa of the last chunk
     float* sh_Lx = sh_kref + 128;           // [128] exchange: L at token 31
     float* sh_LC = sh_Lx + 128;             // [128] exchange: L at token 63
     uint32_t* sh_px = reinterpret_cast<uint32_t*>(sh_LC + 128);        // [128]
     uint32_t* sh_pC = sh_px + 128;                                       // [128]
     uint32_t* sh_sign = sh_pC + 128;        // [64][4] slow path: sign bits per (token, channel)
+    float* sh_kp = reinterpret_cast<float*>(sh_sign + 256);             // [128] kappa of the previous chunk
     float* ax = reinterpret_cast<float*>(sm + SM_AX);
     float* rt = reinterpret_cast<float*>(sm + SM_RT);
 
@@ -254,7 +257,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
         tc::fence_proxy_async_smem();
     };
-    // state copy into the C1 operand (scaled by fa) and rescale of the accumulator (by fs)
+    // state copy into the C1 operand and rescale of the accumulator. The accumulator holds
+    // S Diag(1/kappa_prev): first S = acc kappa_prev, then the operand S g_ref and the new
+    // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
+    // for fast-decaying channels although each factor and each result is in range.
     auto state_copy = [&](bool slow_chunk) {
 #pragma unroll
         for (int cb = 0; cb < 2; ++cb) {
@@ -262,10 +268,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             float sv[32], z[32];
             tc::tmem_ld32<32>(tl + TM_S + c0, sv);
             tc::tmem_ld_wait();
+            const float4* kp4 = reinterpret_cast<const float4*>(sh_kp + c0);
             const float4* fa4 = reinterpret_cast<const float4*>(sh_fa + c0);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
+                const float4 kk = kp4[i];
                 const float4 f = fa4[i];
+                sv[4 * i] *= kk.x;
+                sv[4 * i + 1] *= kk.y;
+                sv[4 * i + 2] *= kk.z;
+                sv[4 * i + 3] *= kk.w;
                 z[4 * i] = sv[4 * i] * f.x;
                 z[4 * i + 1] = sv[4 * i + 1] * f.y;
                 z[4 * i + 2] = sv[4 * i + 2] * f.z;
@@ -347,7 +359,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 pC = par >> 31;
                 sh_LC[m] = LC;
                 sh_pC[m] = pC;
-                bad = (-Lref > kRefRange) || (Lref - LC > kRefRange) || (-LC > kChunkRange);
+                bad = (-LC > kChunkRange);
             }
             slow = __syncthreads_or(bad) != 0;
             if (hh == 0) {
@@ -355,26 +367,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 pref = par >> 31;
                 LC = sh_LC[m];
                 pC = sh_pC[m];
-                const float kprev = sh_kref[m];
+                sh_kp[m] = sh_kref[m];
                 const float gC = (pC ? -1.f : 1.f) * exp2f(LC);
                 if (!slow) {
-                    const float gref = (pref ? -1.f : 1.f) * exp2f(Lref);
-                    const float kappa = ((pref ^ pC) ? -1.f : 1.f) * exp2f(LC - Lref);
-                    sh_fa[m] = kprev * gref;
-                    sh_fs[m] = kprev * gref;
+                    const float gref = exp2f(0.5f * LC);
+                    const float kappa = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
+                    sh_fa[m] = gref;
+                    sh_fs[m] = gref;
                     sh_kref[m] = kappa;
                 } else {
-                    sh_fa[m] = kprev;
-                    sh_fs[m] = kprev * gC;
+                    sh_fa[m] = 1.f;
+                    sh_fs[m] = gC;
                     sh_kref[m] = 1.f;
                 }
             }
             // per-token factors: fast path e1 = Gamma_r/Gamma_ref, e2 = Gamma_ref/Gamma_r;
             // slow path e1 = Gamma_r, e2 = Gamma_C/Gamma_r
-            const float lo1 = slow ? 0.f : Lref;
-            const float lo2 = slow ? LC : Lref;
-            const uint32_t ps1 = slow ? 0u : pref;
-            const uint32_t ps2 = slow ? pC : pref;
+            const float Rm = 0.5f * LC;                 // reference: middle of the chunk's log range
+            const float lo1 = slow ? 0.f : Rm;
+            const float lo2 = slow ? LC : Rm;
+            const uint32_t ps1 = 0u;
+            const uint32_t ps2 = slow ? pC : 0u;
             if (slow) {
                 float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
 #pragma unroll
@@ -461,35 +474,43 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_PHI, sm + SM_PLO, r, 4 * hh + q8, d1 + 8 * q8);
             }
         } else {
-            // exact pairwise evaluation: 64 x 64 pairs, 128 channels each
+            // exact pairwise evaluation: thread (row r, columns s = sq + 4 j), 128 channels each;
+            // row data is loaded once per channel and reused for the 16 columns
             const float* Ls = reinterpret_cast<const float*>(sm + SM_SLOWL);
+            const int r = tid >> 2, sq = tid & 3;
             float va[16], vp[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) va[j] = vp[j] = 0.f;
 #pragma unroll 1
-            for (int j = 0; j < 16; ++j) {
-                const int e = tid + NT * j, r = e >> 6, s = e & 63;
-                float accA = 0.f, accP = 0.f;
-                if (s <= r) {
-                    for (int c = 0; c < D; ++c) {
-                        const uint32_t sg = ((sh_sign[r * 4 + (c >> 5)] ^ sh_sign[s * 4 + (c >> 5)]) >> (c & 31)) & 1u;
-                        const float w = (sg ? -1.f : 1.f) * exp2f(Ls[r * D + c] - Ls[s * D + c]);
-                        const float ksw = ld_bf16_tile(sm + SM_K, s, c) * w;
-                        accA = fmaf(ld_bf16_tile(sm + SM_K, r, c), ksw, accA);
-                        accP = fmaf(ld_bf16_tile(sm + SM_Q, r, c), ksw, accP);
+            for (int c = 0; c < D; ++c) {
+                const float Lr = Ls[r * D + c];
+                const uint32_t sr = (sh_sign[r * 4 + (c >> 5)] >> (c & 31)) & 1u;
+                const float kr = ld_bf16_tile(sm + SM_K, r, c), qr = ld_bf16_tile(sm + SM_Q, r, c);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int sc = sq + 4 * j;
+                    if (sc <= r) {
+                        const uint32_t ss = (sh_sign[sc * 4 + (c >> 5)] >> (c & 31)) & 1u;
+                        const float w = ((sr ^ ss) ? -1.f : 1.f) * tc::ex2_approx(Lr - Ls[sc * D + c]);
+                        const float ksw = ld_bf16_tile(sm + SM_K, sc, c) * w;
+                        va[j] = fmaf(kr, ksw, va[j]);
+                        vp[j] = fmaf(qr, ksw, vp[j]);
                     }
                 }
-                va[j] = (s < r) ? sh_beta[r] * accA : 0.f;
-                vp[j] = accP;
             }
             __syncthreads();      // k, q tiles fully read before A overwrites them
+            {
+                const float br = sh_beta[r];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int e = tid + NT * j, r = e >> 6, s = e & 63;
-                ax[ax_idx(r, s)] = va[j];
-                uint32_t hpair, lpair;
-                split2(vp[j], 0.f, hpair, lpair);
-                const uint32_t off = chunk_off(r, s >> 3) + (uint32_t)(s & 7) * 2u;
-                *reinterpret_cast<uint16_t*>(sm + SM_PHI + off) = (uint16_t)(hpair & 0xffffu);
-                *reinterpret_cast<uint16_t*>(sm + SM_PLO + off) = (uint16_t)(lpair & 0xffffu);
+                for (int j = 0; j < 16; ++j) {
+                    const int sc = sq + 4 * j;
+                    ax[ax_idx(r, sc)] = (sc < r) ? br * va[j] : 0.f;
+                    uint32_t hpair, lpair;
+                    split2((sc <= r) ? vp[j] : 0.f, 0.f, hpair, lpair);
+                    const uint32_t offp = chunk_off(r, sc >> 3) + (uint32_t)(sc & 7) * 2u;
+                    *reinterpret_cast<uint16_t*>(sm + SM_PHI + offp) = (uint16_t)(hpair & 0xffffu);
+                    *reinterpret_cast<uint16_t*>(sm + SM_PLO + offp) = (uint16_t)(lpair & 0xffffu);
+                }
             }
             if (ck > 0) stage_o();
             state_copy(slow);

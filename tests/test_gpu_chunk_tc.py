@@ -69,6 +69,23 @@ def test_extreme_decay_takes_exact_path(ck):
     check("extreme/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
 
 
+@pytest.mark.parametrize("mag", [0.5, 0.2, 0.15, 0.1])
+def test_fast_decaying_channels(ck, mag):
+    """Channels whose gates shrink the state by up to 2^-210 per chunk: 0.5, 0.2 and 0.15
+    stay on the factored path (log2 range within the reference bounds), 0.1 does not.
+    Signs alternate, so the factored signs are exercised as well."""
+    inp = make_inputs(2, 320, 2, 128, 128, torch.bfloat16, seed=int(mag * 100), gate="tanh15",
+                      s0_std=0.2)
+    sgn = torch.where(torch.arange(320) % 3 == 0, -1.0, 1.0)[None, :, None, None]
+    inp.alpha[:, :, :, 96:] = mag * sgn
+    inp.alpha[1, 64:128, 0, :16] = mag
+    o, ST = run_chunk(ck, inp)
+    assert torch.isfinite(o).all() and torch.isfinite(ST).all()
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check(f"decay{mag}/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check(f"decay{mag}/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
 def test_small_workload_shape_padded(ck):
     """bf16, many heads, short sequences: exercises many CTAs with one chunk each."""
     inp = make_inputs(4, 40, 37, 128, 128, torch.bfloat16, seed=8, gate="tanh15", s0_std=0.05)
