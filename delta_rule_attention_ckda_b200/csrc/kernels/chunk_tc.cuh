@@ -64,23 +64,26 @@ constexpr float kChunkRange = 192.f;  // -L_C bound for the fast path (factors w
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t SM_K = 0;            // k tile: 2 TMA boxes [64 tok][64 ch] bf16
+constexpr uint32_t SM_AT = 0;           //   after the gate: A column-major, at[s][r] = A_rs, fp32 [64][64]
 constexpr uint32_t SM_Q = 16384;        // q tile
+constexpr uint32_t SM_T = 16384;        //   after the gate: [T_hi ; T_lo] K-major [128 n][64 s]
 constexpr uint32_t SM_V = 32768;        // v tile (MN-major A operand of V^T T^T)
 constexpr uint32_t SM_AL = 49152;       // alpha tile: 4 boxes [64 tok][32 ch] fp32
-constexpr uint32_t SM_AX = 0;           //   after the gate: A, then (I + A)^{-1}, fp32 [64][64]
-constexpr uint32_t SM_T = 16384;        //   after the gate: [T_hi ; T_lo] K-major [128 n][64 s]
 constexpr uint32_t SM_SLOWL = 49152;    //   slow path only: L fp32 [64][128]
+constexpr uint32_t SM_OT = 49152;       //   after the gate: o tile fp32 [64 tok][128], TMA-stored
 constexpr uint32_t SM_XHI = 81920;      // X hi: block 0 = k e1 (later W^T), block 1 = q e1, [128 c][64 r]
 constexpr uint32_t SM_XLO = 114688;     // X lo
 constexpr uint32_t SM_YHI = 147456;     // Y = k e2, [128 c][64 s] (MN-major for A/P, K-major for S)
 constexpr uint32_t SM_YLO = 163840;
-constexpr uint32_t SM_OT = 49152;       //   after the gate: o tile fp32 [64 tok][128], TMA-stored
 constexpr uint32_t SM_PHI = 180224;     // P K-major [64 r][64 s]
 constexpr uint32_t SM_PLO = 188416;
-constexpr uint32_t SM_RT = 196608;      // solve temporary, fp32 [16][48]
-constexpr uint32_t SM_SMALL = SM_RT + 16 * 48 * 4;
+constexpr uint32_t SM_XS = 196608;      // (I + A)^{-1}, fp32 row-major [64][XS_LD]; blocks above the
+constexpr int XS_LD = 68;               //   16 x 16 block diagonal stay zero for the whole kernel
+constexpr uint32_t SM_RS = SM_XS + 64 * XS_LD * 4;   // solve temporaries, fp32 [32][36]
+constexpr uint32_t SM_SMALL = SM_RS + 32 * 36 * 4;
 constexpr uint32_t SM_BYTES = SM_SMALL + 8192;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;       // + alignment slack
+static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
 
 // TMEM column map (512 columns allocated)
 constexpr uint32_t TM_S = 0;          // state accumulator S^T Diag(1/kappa) [d_v lanes][d_k cols]
@@ -165,9 +168,6 @@ __device__ __forceinline__ void sync_for_mma() {
     tc::tc_fence_after();
 }
 
-// fp32 [64][64] matrix with XOR-swizzled columns (conflict-free row and column access)
-__device__ __forceinline__ int ax_idx(int r, int s) { return r * 64 + (s ^ (r & 31)); }
-
 }  // namespace ctc
 
 // ------------------------------------------------------------------------------ kernel
@@ -199,8 +199,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     uint32_t* sh_pC = sh_px + 128;                                       // [128]
     uint32_t* sh_sign = sh_pC + 128;        // [64][4] slow path: sign bits per (token, channel)
     float* sh_kp = reinterpret_cast<float*>(sh_sign + 256);             // [128] kappa of the previous chunk
-    float* ax = reinterpret_cast<float*>(sm + SM_AX);
-    float* rt = reinterpret_cast<float*>(sm + SM_RT);
+    float* at = reinterpret_cast<float*>(sm + SM_AT);
+    float* xs = reinterpret_cast<float*>(sm + SM_XS);
+    float* rs = reinterpret_cast<float*>(sm + SM_RS);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, hh = warp >> 2;
@@ -225,6 +226,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::prefetch_tensormap(&map_o);
     }
     if (tid < D) sh_kref[tid] = 1.f;
+    // blocks of (I + A)^{-1} above the 16 x 16 block diagonal: zero once, never written again
+    for (int e = tid; e < 384; e += NT) {
+        int r, g;
+        if (e < 192) { r = e / 12; g = 4 + e % 12; }
+        else if (e < 320) { r = 16 + (e - 192) / 8; g = 8 + (e - 192) % 8; }
+        else { r = 32 + (e - 320) / 4; g = 12 + (e - 320) % 4; }
+        *reinterpret_cast<float4*>(xs + r * XS_LD + 4 * g) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -454,7 +463,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
                 tc::bulk_commit();
             }
-            // ---------------- P3: A (fp32, into the k-tile space) and P (hi/lo) out of TMEM
+            // ---------------- P3: A (fp32, column-major) and P (hi/lo) out of TMEM
             float d1[32];
             tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
             tc::tmem_ld_wait();
@@ -464,7 +473,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int s = 32 * hh + i;
-                    ax[ax_idx(r, s)] = (s < r) ? br * d1[i] : 0.f;
+                    at[s * 64 + r] = (s < r) ? br * d1[i] : 0.f;
                 }
             } else {
                 const int r = m - C;
@@ -504,7 +513,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int sc = sq + 4 * j;
-                    ax[ax_idx(r, sc)] = (sc < r) ? br * va[j] : 0.f;
+                    at[sc * 64 + r] = (sc < r) ? br * va[j] : 0.f;
                     uint32_t hpair, lpair;
                     split2((sc <= r) ? vp[j] : 0.f, 0.f, hpair, lpair);
                     const uint32_t offp = chunk_off(r, sc >> 3) + (uint32_t)(sc & 7) * 2u;
@@ -524,83 +533,110 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::tc_fence_before();
         __syncthreads();
 
-        // ---------------- P4: T = (I + A)^{-1} Diag(beta), blocked 16 x 16, in place
-        // diagonal blocks: warp I inverts block I, lane j < 16 solves column j
+        // ---------------- P4: T = (I + A)^{-1} Diag(beta): 16 x 16 diagonal blocks, then two
+        // doubling levels. With L = I + A split into 2 x 2 blocks, L^{-1} has the lower-left
+        // block -X_22 A_21 X_11 (X_ii the inverses of the diagonal blocks).
         if (warp < 4 && lane < 16) {
+            // diagonal block I, column j: right-looking forward substitution; column ss of
+            // A_II is contiguous in the column-major A, so each step is 4 broadcast loads
             const int I = warp, j = lane;
-            float x[16];
+            const float* acol = at + (16 * I) * 64 + 16 * I;
+            float acc[16];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * I + rr;
-                float acc[4] = {(rr == j) ? 1.f : 0.f, 0.f, 0.f, 0.f};
+            for (int rr = 0; rr < 16; ++rr) acc[rr] = (rr == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int ss = 0; ss < rr; ++ss) acc[ss & 3] -= ax[ax_idx(r, 16 * I + ss)] * x[ss];
-                x[rr] = (rr < j) ? 0.f : (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            for (int ss = 0; ss < 15; ++ss) {
+                const float xv = acc[ss];             // final value of x_ss (0 above the diagonal)
+                float a[16];
+#pragma unroll
+                for (int g = (ss + 1) >> 2; g < 4; ++g) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(acol + ss * 64 + 4 * g);
+                    a[4 * g] = t4.x; a[4 * g + 1] = t4.y; a[4 * g + 2] = t4.z; a[4 * g + 3] = t4.w;
+                }
+#pragma unroll
+                for (int rr = ss + 1; rr < 16; ++rr) acc[rr] = fmaf(-a[rr], xv, acc[rr]);
             }
-            __syncwarp(0x0000ffffu);
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) ax[ax_idx(16 * I + rr, 16 * I + j)] = x[rr];
+            for (int rr = 0; rr < 16; ++rr) xs[(16 * I + rr) * XS_LD + 16 * I + j] = acc[rr];
         }
         __syncthreads();
-        // block rows I = 1..3: R = -A_{I,<I} X_{<I}, then X_{I,<I} = X_II R.
-        // Thread task = (row rr, column group g of 4); entries above the block diagonal are
-        // zero, so every task runs the same k range. Groups of 4 columns stay inside one
-        // 16-byte word of the column-swizzled layout (element j of logical group g of row k
-        // is at group g ^ ((k & 31) >> 2), position j ^ (k & 3)).
-#pragma unroll
-        for (int I = 1; I < 4; ++I) {
-            const int ng = 4 * I;
-            const bool act = tid < 16 * ng;
-            const int rr = tid / ng, g = tid % ng;
-            const int r = 16 * I + (act ? rr : 0);
-            if (act) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int k = 0; k < 16 * I; ++k) {
-                    const float a = ax[ax_idx(r, k)];
-                    const float4 xv = *reinterpret_cast<const float4*>(ax + k * 64 + 4 * (g ^ ((k & 31) >> 2)));
-                    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) acc[jj] = fmaf(a, xs[jj ^ (k & 3)], acc[jj]);
-                }
-                *reinterpret_cast<float4*>(rt + rr * 48 + 4 * g) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-            }
-            __syncthreads();
-            if (act) {
-                float xo[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int mm = 0; mm < 16; ++mm) {
-                    const float xd = ax[ax_idx(r, 16 * I + mm)];       // X_II (zero above the diagonal)
-                    const float4 rv = *reinterpret_cast<const float4*>(rt + mm * 48 + 4 * g);
-                    xo[0] = fmaf(xd, rv.x, xo[0]);
-                    xo[1] = fmaf(xd, rv.y, xo[1]);
-                    xo[2] = fmaf(xd, rv.z, xo[2]);
-                    xo[3] = fmaf(xd, rv.w, xo[3]);
-                }
-                // physical position p of logical element j is j ^ (r & 3)
-                float o0 = xo[0], o1 = xo[1], o2 = xo[2], o3 = xo[3];
-                if (r & 1) { float t = o0; o0 = o1; o1 = t; t = o2; o2 = o3; o3 = t; }
-                if (r & 2) { float t = o0; o0 = o2; o2 = t; t = o1; o1 = o3; o3 = t; }
-                *reinterpret_cast<float4*>(ax + r * 64 + 4 * (g ^ ((r & 31) >> 2))) = make_float4(o0, o1, o2, o3);
-            }
-            __syncthreads();
-        }
+        // level 1 (blocks of 16 -> 32), pairs (0,1) and (2,3): R = A_10 X_00, X_10 = -X_11 R.
+        // Thread: pair pb, row r, columns 2 c2, 2 c2 + 1.
         {
-            // T = X Diag(beta): thread -> row r = tid / 4, columns 16 (tid % 4) .. +15
-            const int r = tid >> 2, q4 = tid & 3;
-            float v[16], bb[16];
+            const int pb = tid >> 7, r = (tid >> 3) & 15, c2 = tid & 7, o = 32 * pb;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 b4 = reinterpret_cast<const float4*>(sh_beta + 16 * q4)[e];
-                bb[4 * e] = b4.x; bb[4 * e + 1] = b4.y; bb[4 * e + 2] = b4.z; bb[4 * e + 3] = b4.w;
+            for (int k = 0; k < 16; ++k) {
+                const float a = at[(o + k) * 64 + o + 16 + r];
+                const float2 xv = *reinterpret_cast<const float2*>(xs + (o + k) * XS_LD + o + 2 * c2);
+                acc.x = fmaf(a, xv.x, acc.x);
+                acc.y = fmaf(a, xv.y, acc.y);
             }
+            *reinterpret_cast<float2*>(rs + pb * 320 + r * 20 + 2 * c2) = acc;
+            __syncthreads();
+            float2 xo = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int s = 16 * q4 + e;
-                v[e] = (s <= r) ? ax[ax_idx(r, s)] * bb[e] : 0.f;
+            for (int mm = 0; mm < 16; ++mm) {
+                const float xd = xs[(o + 16 + r) * XS_LD + o + 16 + mm];   // X_11, zero above the diagonal
+                const float2 rv = *reinterpret_cast<const float2*>(rs + pb * 320 + mm * 20 + 2 * c2);
+                xo.x = fmaf(xd, rv.x, xo.x);
+                xo.y = fmaf(xd, rv.y, xo.y);
             }
-            store_split8(sm + SM_T, sm + SM_T + 8192, r, 2 * q4, v);
-            store_split8(sm + SM_T, sm + SM_T + 8192, r, 2 * q4 + 1, v + 8);
+            *reinterpret_cast<float2*>(xs + (o + 16 + r) * XS_LD + o + 2 * c2) = make_float2(-xo.x, -xo.y);
+        }
+        __syncthreads();
+        // level 2 (32 -> 64): R = A[32:64, 0:32] X[0:32, 0:32], X[32:64, 0:32] = -X[32:64, 32:64] R.
+        // T = X Diag(beta) is split into the MMA operand as soon as a block of X is final.
+        {
+            // R: warp -> columns 4 w .. 4 w + 3, lane -> row; X[k][c] = 0 for k < c
+            const int cg = warp, r = lane;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int k = 4 * cg; k < 32; ++k) {
+                const float a = at[k * 64 + 32 + r];
+                const float4 xv = *reinterpret_cast<const float4*>(xs + k * XS_LD + 4 * cg);
+                acc.x = fmaf(a, xv.x, acc.x);
+                acc.y = fmaf(a, xv.y, acc.y);
+                acc.z = fmaf(a, xv.z, acc.z);
+                acc.w = fmaf(a, xv.w, acc.w);
+            }
+            *reinterpret_cast<float4*>(rs + r * 36 + 4 * cg) = acc;
+            // final blocks of T: rows 0..31 x columns 0..31 and rows 32..63 x columns 32..63
+            // (16-byte chunk ch of row tr), and the zero block rows 0..31 x columns 32..63
+            {
+                const int half = warp >> 2, ch = (warp & 3) + 4 * half, tr = lane + 32 * half;
+                const float4 x0 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch);
+                const float4 x1 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch + 4);
+                const float4 b0 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[0];
+                const float4 b1 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[1];
+                const float v[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
+                                    x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
+                store_split8(sm + SM_T, sm + SM_T + 8192, tr, ch, v);
+                const uint32_t zoff = chunk_off(lane, 4 + (warp & 3)) + (uint32_t)half * 8192u;
+                *reinterpret_cast<uint4*>(sm + SM_T + zoff) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncthreads();
+            // X[32:64, 0:32]: thread -> row 32 + r2, columns 4 c4 .. 4 c4 + 3, straight into T.
+            // X[32 + r2][32 + mm] is zero for mm > r2: warps 0-3 hold rows r2 < 16.
+            const int r2 = tid >> 3, c4 = tid & 7;
+            const int mmax = (warp < 4) ? 16 : 32;
+            float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int mm = 0; mm < mmax; ++mm) {
+                const float xd = xs[(32 + r2) * XS_LD + 32 + mm];
+                const float4 rv = *reinterpret_cast<const float4*>(rs + mm * 36 + 4 * c4);
+                xo.x = fmaf(xd, rv.x, xo.x);
+                xo.y = fmaf(xd, rv.y, xo.y);
+                xo.z = fmaf(xd, rv.z, xo.z);
+                xo.w = fmaf(xd, rv.w, xo.w);
+            }
+            const float4 b4 = reinterpret_cast<const float4*>(sh_beta)[c4];
+            uint32_t h0, l0, h1, l1;
+            split2(-xo.x * b4.x, -xo.y * b4.y, h0, l0);
+            split2(-xo.z * b4.z, -xo.w * b4.w, h1, l1);
+            const uint32_t off = chunk_off(32 + r2, c4 >> 1) + (uint32_t)(c4 & 1) * 8u;
+            *reinterpret_cast<uint2*>(sm + SM_T + off) = make_uint2(h0, h1);
+            *reinterpret_cast<uint2*>(sm + SM_T + 8192 + off) = make_uint2(l0, l1);
         }
         sync_for_mma();
 
