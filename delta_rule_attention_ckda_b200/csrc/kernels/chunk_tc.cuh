@@ -10,7 +10,7 @@
 //   A_rs    = b_r k_r^T Diag(Gamma_r/Gamma_s) k_s   (s < r),
 //   P_rs    =     q_r^T Diag(Gamma_r/Gamma_s) k_s   (s <= r),
 //   T       = (I + A)^{-1} Diag(b)                   (UT transform, forward solve),
-//   U~ = T V,  W = T (Gamma (.) K),  U = U~ - W S0,
+//   U  = T V - T (Gamma (.) K) S0 = T (V - Z),  Z = (Gamma (.) K) S0,
 //   O  = (Gamma (.) Q) S0 + P U,
 //   S_C = Diag(Gamma_C) S0 + ((Gamma_C/Gamma) (.) K)^T U.
 // In exact arithmetic this equals the token loop; the WY/UT evaluation is the
@@ -24,8 +24,10 @@
 //   Gamma_C = g_ref kappa,
 // and every factor lies in [2^{L_C/2}, 2^{-L_C/2}].
 // So one pair of token tiles X = [k e1 ; q e1] and Y = k e2 serves every product:
-//   [A ; P] from X Y^T;  W / g_ref from (k e1) T^T;  O from S0 Diag(g_ref) and q e1;
+//   [A ; P] from X Y^T;  [Z | O_inter] from (S0 Diag g_ref)^T X^T;  U from T (V - Z);
 //   the state update from S0 Diag(g_ref) + U^T (k e2), which is S_C Diag(1/kappa).
+// Z and O_inter depend only on the gate and the state entering the chunk, so their MMA
+// runs on the tensor cores while the CUDA cores solve for T.
 // The TMEM accumulator therefore holds S Diag(1/kappa_prev); each chunk rescales it
 // by kappa_prev * g_ref (a per-column factor, folded into the pass that copies the
 // state into the MMA operand), and the final write multiplies by the last kappa.
@@ -56,7 +58,13 @@ namespace ctc {
 
 constexpr int C = 64;        // chunk length
 constexpr int D = 128;       // d_k = d_v
-constexpr int NT = 256;      // threads per CTA
+constexpr int NT = 256;      // compute threads (warpgroups 0 and 1)
+constexpr int NT_ALL = 384;  // + warpgroup 2, whose first warp issues every MMA, TMA load and o store
+// Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64512); the
+// issuer warpgroup drops to 56 and the compute warpgroups rise to 224 (256 x 224 + 128 x 56).
+constexpr uint32_t kRegCompute = 224;
+constexpr uint32_t kRegIssuer = 56;
+static_assert(NT * kRegCompute + (NT_ALL - NT) * kRegIssuer <= NT_ALL * 168, "register split exceeds the launch");
 
 // log2-domain limits of the single-reference factorisation
 constexpr float kLgFloor = -100.f;    // floor of log2|a| per token (a = 0 allowed)
@@ -89,15 +97,17 @@ static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
 constexpr uint32_t TM_S = 0;          // state accumulator S^T Diag(1/kappa) [d_v lanes][d_k cols]
 constexpr uint32_t TM_SAHI = 128;     // (S0 Diag g)^T hi / lo, packed bf16 (A operand of C1)
 constexpr uint32_t TM_SALO = 192;
-constexpr uint32_t TM_UAHI = 128;     // U^T hi / lo, packed bf16 (A operand of the O / S MMAs)
-constexpr uint32_t TM_UALO = 160;
-constexpr uint32_t TM_DU = 256;       // V^T [T_hi^T | T_lo^T]
+constexpr uint32_t TM_ZAHI = 128;     //   after C1: -Z^T hi / lo, packed bf16 (A operand of the U MMA)
+constexpr uint32_t TM_ZALO = 160;
+constexpr uint32_t TM_UAHI = 192;     //   after the U MMA: U^T hi / lo, packed bf16 (A of the O / S MMAs)
+constexpr uint32_t TM_UALO = 224;
+constexpr uint32_t TM_Z = 256;        // C1 result: Z^T [d_v][64 tok] ...
+constexpr uint32_t TM_O = 320;        //   ... and O^T, which the P U MMA accumulates into
 constexpr uint32_t TM_D1 = 384;       // [A ; P] 128 x 64
-constexpr uint32_t TM_DW = 384;       // (k e1)^T [T_hi^T | T_lo^T] + lo part
-constexpr uint32_t TM_DR = 384;       // (S0 Diag g)^T [W^T/g | (q e1)^T] 128 x 128
-constexpr uint32_t TM_O = 448;        //   its second half accumulates O^T (read in the next chunk)
+constexpr uint32_t TM_DU = 448;       // U^T = V^T T^T - Z^T T^T, 128 x 64
 
-constexpr uint32_t kTmaBytes = 10 * 8192;    // 6 bf16 boxes + 4 fp32 boxes
+constexpr uint32_t kTmaBytes1 = 6 * 8192;   // k (2 bf16 boxes) + alpha (4 fp32 boxes)
+constexpr uint32_t kTmaBytes2 = 4 * 8192;   // q + v (2 bf16 boxes each)
 
 // Byte address (from tile base) of the 16-byte chunk `ch` (0..7) of row `row` in a
 // tile of 128-byte rows with 128-byte swizzle.
@@ -153,32 +163,67 @@ __device__ __forceinline__ void tmem_st_f32x32(uint32_t taddr, const float (&x)[
     tc::tmem_st32<16>(taddr + 16, b);
 }
 
-// Every thread waits on the barrier; returns true if any thread of the CTA timed out.
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
-    const bool ok = tc::mbar_wait(bar, parity);
-    return __syncthreads_or(!ok) != 0;
+// Barrier among the 256 compute threads only (named barrier 1; the issuer warp never joins).
+__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Same barrier with an OR over the threads' predicates.
+__device__ __forceinline__ bool csync_or(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred a, q;\n\t"
+        "setp.ne.u32 a, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 256, a;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p)
+        : "memory");
+    return r != 0;
 }
 
-// Make generic-proxy shared-memory writes and tcgen05.st visible to the MMA issuer.
-__device__ __forceinline__ void sync_for_mma() {
+// Every compute thread waits on the barrier; true if any of them timed out.
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
+    const bool ok = tc::mbar_wait(bar, parity);
+    return csync_or(!ok);
+}
+
+// Hand this thread's shared-memory writes and tcgen05.st to the issuer warp: complete
+// the stores, order them before the async proxy and the thread sync, then arrive.
+__device__ __forceinline__ void handoff(uint64_t* bar) {
     tc::tmem_st_wait();
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
+    tc::mbar_arrive(bar);
+}
+
+// A copy of x the compiler cannot see through: keeps loop-invariant MMA descriptors from
+// being hoisted out of the chunk loop into (scarce) issuer registers.
+__device__ __forceinline__ uint32_t opaque(uint32_t x) {
+    asm volatile("mov.b32 %0, %0;" : "+r"(x));
+    return x;
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 }  // namespace ctc
 
 // ------------------------------------------------------------------------------ kernel
 
-// Per-chunk schedule (one CTA per (batch, head), 8 warps). Each tcgen05 group commits to
-// its own mbarrier, so work that does not depend on an MMA runs while it executes:
-//   gate cumulation of chunk c          ||  O / state MMAs of chunk c-1
-//   o store of chunk c-1, state copy     ||  [A ; P] MMA of chunk c
-//   W^T epilogue                         ||  U~ MMA
-// and the next chunk's inputs are fetched by TMA once the U~ MMA has consumed V and T.
-__global__ void __launch_bounds__(ctc::NT, 1)
+// Per-chunk schedule (one CTA per (batch, head)). Eight compute warps do the CUDA-core
+// work; one issuer warp issues every tcgen05 MMA group, TMA load and o store, so that the
+// compute warps never stall while an MMA group drains (an issuing thread blocks for about
+// the duration of the MMAs it issues). The compute warps hand their operands over through
+// mbarriers; each MMA group commits to its own mbarrier. What overlaps:
+//   gate cumulation of chunk c           ||  O / state MMAs of chunk c-1
+//   o tile of chunk c-1, state copy       ||  [A ; P] MMA of chunk c
+//   [A ; P] epilogue, solve for T         ||  C1 MMA ([Z | O_inter]), k / alpha of chunk c+1
+__global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
                 const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta, const float* S0,
@@ -186,8 +231,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tma, bar_ap, bar_w, bar_u, bar_c1, bar_c2;
-    __shared__ uint32_t tmem_base_s;
+    __shared__ uint64_t bar_tma1, bar_tma2, bar_ap, bar_c1, bar_u, bar_c2;    // TMA / MMA completion
+    __shared__ uint64_t bar_hap, bar_hc1, bar_hl2, bar_hu, bar_hc2, bar_hfin;  // compute -> issuer
+    __shared__ uint64_t bar_ofree;                                              // issuer -> compute
+    __shared__ uint32_t tmem_base_s, slow_flag_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
     float* sh_fa = sh_beta + 64;            // [128] g_ref (operand copy = S g_ref)
@@ -212,12 +259,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
     if (tid == 0) {
-        tc::mbar_init(&bar_tma, 1);
+        tc::mbar_init(&bar_tma1, 1);
+        tc::mbar_init(&bar_tma2, 1);
         tc::mbar_init(&bar_ap, 1);
-        tc::mbar_init(&bar_w, 1);
-        tc::mbar_init(&bar_u, 1);
         tc::mbar_init(&bar_c1, 1);
+        tc::mbar_init(&bar_u, 1);
         tc::mbar_init(&bar_c2, 1);
+        tc::mbar_init(&bar_hap, NT);
+        tc::mbar_init(&bar_hc1, NT);
+        tc::mbar_init(&bar_hl2, NT);
+        tc::mbar_init(&bar_hu, NT);
+        tc::mbar_init(&bar_hc2, NT);
+        tc::mbar_init(&bar_hfin, NT);
+        tc::mbar_init(&bar_ofree, 1);
         tc::fence_mbar_init();
         tc::prefetch_tensormap(&map_k);
         tc::prefetch_tensormap(&map_q);
@@ -227,7 +281,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     }
     if (tid < D) sh_kref[tid] = 1.f;
     // blocks of (I + A)^{-1} above the 16 x 16 block diagonal: zero once, never written again
-    for (int e = tid; e < 384; e += NT) {
+    for (int e = tid; e < 384; e += NT_ALL) {
         int r, g;
         if (e < 192) { r = e / 12; g = 4 + e % 12; }
         else if (e < 320) { r = 16 + (e - 192) / 8; g = 8 + (e - 192) % 8; }
@@ -240,23 +294,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const uint32_t tm = tmem_base_s;
     const uint32_t tl = tm + lane_base;           // this warp's lane quarter
 
-    auto issue_loads = [&](int t0) {
-        tc::mbar_arrive_expect_tx(&bar_tma, kTmaBytes);
-        for (int i = 0; i < 2; ++i) {
-            tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma, 64 * i, h, t0, b);
-            tc::tma_load_4d(sm + SM_Q + i * 8192, &map_q, &bar_tma, 64 * i, h, t0, b);
-            tc::tma_load_4d(sm + SM_V + i * 8192, &map_v, &bar_tma, 64 * i, h, t0, b);
-        }
-        for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma, 32 * i, h, t0, b);
+    // inputs of a chunk arrive in two groups: k and alpha (their space frees up during the
+    // solve), then q and v (read by the U MMA)
+    auto issue_loads1 = [&](int t0) {
+        tc::mbar_arrive_expect_tx(&bar_tma1, kTmaBytes1);
+        for (int i = 0; i < 2; ++i) tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma1, 64 * i, h, t0, b);
+        for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma1, 32 * i, h, t0, b);
     };
-    if (tid == 0) issue_loads(0);
+    auto issue_loads2 = [&](int t0) {
+        tc::mbar_arrive_expect_tx(&bar_tma2, kTmaBytes2);
+        for (int i = 0; i < 2; ++i) {
+            tc::tma_load_4d(sm + SM_Q + i * 8192, &map_q, &bar_tma2, 64 * i, h, t0, b);
+            tc::tma_load_4d(sm + SM_V + i * 8192, &map_v, &bar_tma2, 64 * i, h, t0, b);
+        }
+    };
     auto load_beta = [&](int t0) -> float {
         return (tid < C && t0 + tid < T) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
     };
     float beta_next = load_beta(0);
 
     // o rows of a finished chunk: TMEM -> shared tile [64 tok][128] fp32 in the alpha space.
-    // The TMA store itself is issued by thread 0 after the next CTA barrier.
+    // The issuer warp stores the tile by TMA once the compute threads have handed it over.
     auto stage_o = [&]() {
         float ov[32];
         tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
@@ -313,460 +371,532 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
     };
 
-    // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
-    {
-        const size_t sb = (size_t)bh * D * D;
-        for (int cb = 0; cb < 2; ++cb) {
-            float x[32];
-            const int c0 = 64 * hh + 32 * cb;
+    // C1: [Z^T | O^T] = (S0 Diag g)^T [(k e1)^T | (q e1)^T]  (3 passes), after the state copy
+    auto issue_c1 = [&](uint32_t sb_) {
+        const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
+        const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = S0 ? S0[sb + (size_t)(c0 + i) * D + m] : 0.f;
-            tmem_st_f32x32(tl + TM_S + c0, x);
+        for (int ps = 0; ps < 3; ++ps) {
+            const uint32_t aa = tm0 + (ps == 2 ? TM_SALO : TM_SAHI);
+            const uint32_t bb = sb0 + (ps == 1 ? SM_XLO : SM_XHI);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                tc::mma_ts(tm0 + TM_Z, aa + ks * 8, tc::sdesc(bb + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
         }
-        tc::tmem_st_wait();
-    }
+        tc::mma_commit(&bar_c1);
+    };
+    // [A ; P] = X Y  (3 passes)
+    auto issue_ap = [&](uint32_t sb_) {
+        const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
+        const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+        for (int ps = 0; ps < 3; ++ps) {
+            const uint32_t xa = sb0 + (ps == 2 ? SM_XLO : SM_XHI);
+            const uint32_t yb = sb0 + (ps == 1 ? SM_YLO : SM_YHI);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                tc::mma_ss(tm0 + TM_D1, tc::sdesc(xa + ks * 2048, 16384, 1024), tc::sdesc(yb + ks * 2048, 16384, 1024),
+                           idesc, (ps | ks) != 0);
+        }
+        tc::mma_commit(&bar_ap);
+    };
+    // U^T = V^T [T_hi ; T_lo]^T  +  (-Z^T)_hi T_hi^T + (-Z^T)_hi T_lo^T + (-Z^T)_lo T_hi^T
+    auto issue_u = [&](uint32_t sb_) {
+        const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
+        const uint32_t iv = tc::idesc_bf16(128, 64, 1, 0);    // A = V^T (MN-major), B = T (K-major)
+        const uint32_t iz = tc::idesc_bf16(128, 64, 0, 0);    // A = -Z^T (TMEM)
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_ss(tm0 + TM_DU, tc::sdesc(sb0 + SM_V + ks * 2048, 8192, 1024),
+                           tc::sdesc(sb0 + SM_T + ps * 8192 + ks * 32, 16, 1024), iv, (ps | ks) != 0);
+#pragma unroll
+        for (int ps = 0; ps < 3; ++ps) {
+            const uint32_t aa = tm0 + (ps == 2 ? TM_ZALO : TM_ZAHI);
+            const uint32_t tb = sb0 + SM_T + (ps == 1 ? 8192 : 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) tc::mma_ts(tm0 + TM_DU, aa + ks * 8, tc::sdesc(tb + ks * 32, 16, 1024), iz, 1);
+        }
+        tc::mma_commit(&bar_u);
+    };
+    // O^T += U^T P^T ;  acc += U^T (k e2)  (3 passes each)
+    auto issue_c2 = [&](uint32_t sb_) {
+        const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
+        const uint32_t io = tc::idesc_bf16(128, 64, 0, 0);
+        const uint32_t is = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+        for (int ps = 0; ps < 3; ++ps) {
+            const uint32_t aa = tm0 + (ps == 2 ? TM_UALO : TM_UAHI);
+            const uint32_t pb = sb0 + (ps == 1 ? SM_PLO : SM_PHI);
+            const uint32_t kb = sb0 + (ps == 1 ? SM_YLO : SM_YHI);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                tc::mma_ts(tm0 + TM_O, aa + ks * 8, tc::sdesc(pb + ks * 32, 16, 1024), io, 1);
+                tc::mma_ts(tm0 + TM_S, aa + ks * 8, tc::sdesc(kb + ks * 32, 16, 1024), is, 1);
+            }
+        }
+        tc::mma_commit(&bar_c2);
+    };
 
     const uint32_t sbase = tc::smem_u32(sm);
-    uint32_t ph_ap = 0, ph_w = 0, ph_u = 0, ph_c1 = 0, ph_c2 = 0;
-    bool failed = false;
     const int nchunks = (T + C - 1) / C;
 
-    for (int ck = 0; ck < nchunks && !failed; ++ck) {
-        const int t0 = ck * C;
-        const int nvalid = min(C, T - t0);
-        if (tid < C) sh_beta[tid] = beta_next;
-        if (wait_all(&bar_tma, ck & 1)) { failed = true; break; }
-
-        // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
-        bool slow;
-        {
-            float L[32];
-            uint32_t par = 0;
-            float run = 0.f;
-            uint32_t p = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = 32 * hh + i;
-                const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
-                run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
-                p ^= (a < 0.f) ? 1u : 0u;
-                L[i] = run;
-                par |= p << i;
+    if (warp >= NT / 32) {
+        // ================================================================ issuer warpgroup
+        setmaxnreg_dec<kRegIssuer>();
+        if (warp == NT / 32) {
+            const bool leader = (lane == 0);
+            // one thread polls, the whole warp learns the outcome (the warp stays converged)
+            auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
+                bool ok = true;
+                if (leader) ok = tc::mbar_wait(bar, parity);
+                return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            };
+            if (leader && nchunks > 0) {
+                issue_loads1(0);
+                issue_loads2(0);
             }
-            if (hh == 0) { sh_Lx[m] = run; sh_px[m] = p; }
-            __syncthreads();
-            float Lref, LC;
-            uint32_t pref, pC;
-            int bad = 0;
-            if (hh == 1) {
-                Lref = sh_Lx[m];
-                pref = sh_px[m];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) L[i] += Lref;
-                if (pref) par = ~par;
-                LC = L[31];
-                pC = par >> 31;
-                sh_LC[m] = LC;
-                sh_pC[m] = pC;
-                bad = (-LC > kChunkRange);
-            }
-            slow = __syncthreads_or(bad) != 0;
-            if (hh == 0) {
-                Lref = L[31];
-                pref = par >> 31;
-                LC = sh_LC[m];
-                pC = sh_pC[m];
-                sh_kp[m] = sh_kref[m];
-                const float gC = (pC ? -1.f : 1.f) * exp2f(LC);
-                if (!slow) {
-                    const float gref = exp2f(0.5f * LC);
-                    const float kappa = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
-                    sh_fa[m] = gref;
-                    sh_fs[m] = gref;
-                    sh_kref[m] = kappa;
-                } else {
-                    sh_fa[m] = 1.f;
-                    sh_fs[m] = gC;
-                    sh_kref[m] = 1.f;
+            __syncwarp();
+            for (int ck = 0; ck < nchunks; ++ck) {
+                const uint32_t par = (uint32_t)ck & 1u;
+                const int t0 = ck * C;
+                // X, Y tiles written: [A ; P], unless the chunk takes the exact path
+                if (!wait1(&bar_hap, par)) break;
+                if (leader && slow_flag_s == 0u) {
+                    tc::tc_fence_after();
+                    issue_ap(sbase);
                 }
-            }
-            // per-token factors: fast path e1 = Gamma_r/Gamma_ref, e2 = Gamma_ref/Gamma_r;
-            // slow path e1 = Gamma_r, e2 = Gamma_C/Gamma_r
-            const float Rm = 0.5f * LC;                 // reference: middle of the chunk's log range
-            const float lo1 = slow ? 0.f : Rm;
-            const float lo2 = slow ? LC : Rm;
-            const uint32_t ps1 = 0u;
-            const uint32_t ps2 = slow ? pC : 0u;
-            if (slow) {
-                float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i];
-            }
-            // the previous chunk's O / S MMAs read Y and P: wait for them before overwriting
-            if (ck > 0) {
-                if (wait_all(&bar_c2, ph_c2)) { failed = true; break; }
-                ph_c2 ^= 1u;
-                tc::tc_fence_after();
-            }
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                float xk[8], xq[8], yk[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = 8 * q8 + e, r = 32 * hh + i;
-                    const uint32_t pr = (par >> i) & 1u;
-                    const float e1 = ((pr ^ ps1) ? -1.f : 1.f) * tc::ex2_approx(L[i] - lo1);
-                    const float e2 = ((pr ^ ps2) ? -1.f : 1.f) * tc::ex2_approx(lo2 - L[i]);
-                    const float kv = ld_bf16_tile(sm + SM_K, r, m);
-                    const float qv = ld_bf16_tile(sm + SM_Q, r, m);
-                    xk[e] = kv * e1;
-                    xq[e] = qv * e1;
-                    yk[e] = kv * e2;
-                }
-                store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xk);
-                store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xq);
-                store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
-            }
-            if (slow) {
-                // sign bits of Gamma per (token, channel): word [r][m/32], bit m%32
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const unsigned bits = __ballot_sync(0xffffffffu, (par >> i) & 1u);
-                    if (lane == 0) sh_sign[(32 * hh + i) * 4 + quarter] = bits;
-                }
-            }
-        }
-        sync_for_mma();
-
-        // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact pairwise path
-        if (!slow) {
-            if (tid == 0) {
-                const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
-#pragma unroll
-                for (int ps = 0; ps < 3; ++ps) {
-                    const uint32_t xa = sbase + (ps == 2 ? SM_XLO : SM_XHI);
-                    const uint32_t yb = sbase + (ps == 1 ? SM_YLO : SM_YHI);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        tc::mma_ss(tm + TM_D1, tc::sdesc(xa + ks * 2048, 16384, 1024),
-                                   tc::sdesc(yb + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
-                }
-                tc::mma_commit(&bar_ap);
-            }
-            // while the MMA runs: the previous chunk's o tile and this chunk's state copy
-            if (ck > 0) stage_o();
-            state_copy(slow);
-            if (wait_all(&bar_ap, ph_ap)) { failed = true; break; }
-            ph_ap ^= 1u;
-            tc::tc_fence_after();
-            if (tid == 0 && ck > 0) {
-                tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
-                tc::bulk_commit();
-            }
-            // ---------------- P3: A (fp32, column-major) and P (hi/lo) out of TMEM
-            float d1[32];
-            tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
-            tc::tmem_ld_wait();
-            if (m < C) {
-                const int r = m;
-                const float br = sh_beta[r];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int s = 32 * hh + i;
-                    at[s * 64 + r] = (s < r) ? br * d1[i] : 0.f;
-                }
-            } else {
-                const int r = m - C;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) d1[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_PHI, sm + SM_PLO, r, 4 * hh + q8, d1 + 8 * q8);
-            }
-        } else {
-            // exact pairwise evaluation: thread (row r, columns s = sq + 4 j), 128 channels each;
-            // row data is loaded once per channel and reused for the 16 columns
-            const float* Ls = reinterpret_cast<const float*>(sm + SM_SLOWL);
-            const int r = tid >> 2, sq = tid & 3;
-            float va[16], vp[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) va[j] = vp[j] = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < D; ++c) {
-                const float Lr = Ls[r * D + c];
-                const uint32_t sr = (sh_sign[r * 4 + (c >> 5)] >> (c & 31)) & 1u;
-                const float kr = ld_bf16_tile(sm + SM_K, r, c), qr = ld_bf16_tile(sm + SM_Q, r, c);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int sc = sq + 4 * j;
-                    if (sc <= r) {
-                        const uint32_t ss = (sh_sign[sc * 4 + (c >> 5)] >> (c & 31)) & 1u;
-                        const float w = ((sr ^ ss) ? -1.f : 1.f) * tc::ex2_approx(Lr - Ls[sc * D + c]);
-                        const float ksw = ld_bf16_tile(sm + SM_K, sc, c) * w;
-                        va[j] = fmaf(kr, ksw, va[j]);
-                        vp[j] = fmaf(qr, ksw, vp[j]);
+                __syncwarp();
+                // previous chunk's o tile staged and state copied: store o, then C1
+                if (!wait1(&bar_hc1, par)) break;
+                if (leader) {
+                    tc::tc_fence_after();
+                    if (ck > 0) {
+                        tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
+                        tc::bulk_commit();
                     }
+                    issue_c1(sbase);
                 }
-            }
-            __syncthreads();      // k, q tiles fully read before A overwrites them
-            {
-                const float br = sh_beta[r];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int sc = sq + 4 * j;
-                    at[sc * 64 + r] = (sc < r) ? br * va[j] : 0.f;
-                    uint32_t hpair, lpair;
-                    split2((sc <= r) ? vp[j] : 0.f, 0.f, hpair, lpair);
-                    const uint32_t offp = chunk_off(r, sc >> 3) + (uint32_t)(sc & 7) * 2u;
-                    *reinterpret_cast<uint16_t*>(sm + SM_PHI + offp) = (uint16_t)(hpair & 0xffffu);
-                    *reinterpret_cast<uint16_t*>(sm + SM_PLO + offp) = (uint16_t)(lpair & 0xffffu);
+                __syncwarp();
+                // A consumed: the next chunk's k and alpha, once the o tile has left the alpha space
+                if (!wait1(&bar_hl2, par)) break;
+                if (leader && ck + 1 < nchunks) {
+                    tc::bulk_wait_read0();
+                    issue_loads1(t0 + C);
                 }
-            }
-            if (ck > 0) stage_o();
-            state_copy(slow);
-            __syncthreads();
-            if (tid == 0 && ck > 0) {
-                tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);
-                tc::bulk_commit();
-            }
-        }
-        tc::tmem_ld_wait();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ---------------- P4: T = (I + A)^{-1} Diag(beta): 16 x 16 diagonal blocks, then two
-        // doubling levels. With L = I + A split into 2 x 2 blocks, L^{-1} has the lower-left
-        // block -X_22 A_21 X_11 (X_ii the inverses of the diagonal blocks).
-        if (warp < 4 && lane < 16) {
-            // diagonal block I, column j: right-looking forward substitution; column ss of
-            // A_II is contiguous in the column-major A, so each step is 4 broadcast loads
-            const int I = warp, j = lane;
-            const float* acol = at + (16 * I) * 64 + 16 * I;
-            float acc[16];
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) acc[rr] = (rr == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int ss = 0; ss < 15; ++ss) {
-                const float xv = acc[ss];             // final value of x_ss (0 above the diagonal)
-                float a[16];
-#pragma unroll
-                for (int g = (ss + 1) >> 2; g < 4; ++g) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(acol + ss * 64 + 4 * g);
-                    a[4 * g] = t4.x; a[4 * g + 1] = t4.y; a[4 * g + 2] = t4.z; a[4 * g + 3] = t4.w;
+                __syncwarp();
+                // T and -Z^T ready: U
+                if (!wait1(&bar_hu, par)) break;
+                if (leader) {
+                    tc::tc_fence_after();
+                    issue_u(sbase);
                 }
-#pragma unroll
-                for (int rr = ss + 1; rr < 16; ++rr) acc[rr] = fmaf(-a[rr], xv, acc[rr]);
-            }
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) xs[(16 * I + rr) * XS_LD + 16 * I + j] = acc[rr];
-        }
-        __syncthreads();
-        // level 1 (blocks of 16 -> 32), pairs (0,1) and (2,3): R = A_10 X_00, X_10 = -X_11 R.
-        // Thread: pair pb, row r, columns 2 c2, 2 c2 + 1.
-        {
-            const int pb = tid >> 7, r = (tid >> 3) & 15, c2 = tid & 7, o = 32 * pb;
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float a = at[(o + k) * 64 + o + 16 + r];
-                const float2 xv = *reinterpret_cast<const float2*>(xs + (o + k) * XS_LD + o + 2 * c2);
-                acc.x = fmaf(a, xv.x, acc.x);
-                acc.y = fmaf(a, xv.y, acc.y);
-            }
-            *reinterpret_cast<float2*>(rs + pb * 320 + r * 20 + 2 * c2) = acc;
-            __syncthreads();
-            float2 xo = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int mm = 0; mm < 16; ++mm) {
-                const float xd = xs[(o + 16 + r) * XS_LD + o + 16 + mm];   // X_11, zero above the diagonal
-                const float2 rv = *reinterpret_cast<const float2*>(rs + pb * 320 + mm * 20 + 2 * c2);
-                xo.x = fmaf(xd, rv.x, xo.x);
-                xo.y = fmaf(xd, rv.y, xo.y);
-            }
-            *reinterpret_cast<float2*>(xs + (o + 16 + r) * XS_LD + o + 2 * c2) = make_float2(-xo.x, -xo.y);
-        }
-        __syncthreads();
-        // level 2 (32 -> 64): R = A[32:64, 0:32] X[0:32, 0:32], X[32:64, 0:32] = -X[32:64, 32:64] R.
-        // T = X Diag(beta) is split into the MMA operand as soon as a block of X is final.
-        {
-            // R: warp -> columns 4 w .. 4 w + 3, lane -> row; X[k][c] = 0 for k < c
-            const int cg = warp, r = lane;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-            for (int k = 4 * cg; k < 32; ++k) {
-                const float a = at[k * 64 + 32 + r];
-                const float4 xv = *reinterpret_cast<const float4*>(xs + k * XS_LD + 4 * cg);
-                acc.x = fmaf(a, xv.x, acc.x);
-                acc.y = fmaf(a, xv.y, acc.y);
-                acc.z = fmaf(a, xv.z, acc.z);
-                acc.w = fmaf(a, xv.w, acc.w);
-            }
-            *reinterpret_cast<float4*>(rs + r * 36 + 4 * cg) = acc;
-            // final blocks of T: rows 0..31 x columns 0..31 and rows 32..63 x columns 32..63
-            // (16-byte chunk ch of row tr), and the zero block rows 0..31 x columns 32..63
-            {
-                const int half = warp >> 2, ch = (warp & 3) + 4 * half, tr = lane + 32 * half;
-                const float4 x0 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch);
-                const float4 x1 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch + 4);
-                const float4 b0 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[0];
-                const float4 b1 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[1];
-                const float v[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
-                                    x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
-                store_split8(sm + SM_T, sm + SM_T + 8192, tr, ch, v);
-                const uint32_t zoff = chunk_off(lane, 4 + (warp & 3)) + (uint32_t)half * 8192u;
-                *reinterpret_cast<uint4*>(sm + SM_T + zoff) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            __syncthreads();
-            // X[32:64, 0:32]: thread -> row 32 + r2, columns 4 c4 .. 4 c4 + 3, straight into T.
-            // X[32 + r2][32 + mm] is zero for mm > r2: warps 0-3 hold rows r2 < 16.
-            const int r2 = tid >> 3, c4 = tid & 7;
-            const int mmax = (warp < 4) ? 16 : 32;
-            float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-            for (int mm = 0; mm < mmax; ++mm) {
-                const float xd = xs[(32 + r2) * XS_LD + 32 + mm];
-                const float4 rv = *reinterpret_cast<const float4*>(rs + mm * 36 + 4 * c4);
-                xo.x = fmaf(xd, rv.x, xo.x);
-                xo.y = fmaf(xd, rv.y, xo.y);
-                xo.z = fmaf(xd, rv.z, xo.z);
-                xo.w = fmaf(xd, rv.w, xo.w);
-            }
-            const float4 b4 = reinterpret_cast<const float4*>(sh_beta)[c4];
-            uint32_t h0, l0, h1, l1;
-            split2(-xo.x * b4.x, -xo.y * b4.y, h0, l0);
-            split2(-xo.z * b4.z, -xo.w * b4.w, h1, l1);
-            const uint32_t off = chunk_off(32 + r2, c4 >> 1) + (uint32_t)(c4 & 1) * 8u;
-            *reinterpret_cast<uint2*>(sm + SM_T + off) = make_uint2(h0, h1);
-            *reinterpret_cast<uint2*>(sm + SM_T + 8192 + off) = make_uint2(l0, l1);
-        }
-        sync_for_mma();
-
-        // ---------------- P5: W^T/g = (k e1)^T [T_hi^T | T_lo^T] + lo part;  U~^T = V^T [..]
-        if (tid == 0) {
-            const uint32_t iw = tc::idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(tm + TM_DW, tc::sdesc(sbase + SM_XHI + ks * 32, 16, 1024),
-                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw, ks != 0);
-            const uint32_t iw2 = tc::idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(tm + TM_DW, tc::sdesc(sbase + SM_XLO + ks * 32, 16, 1024),
-                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iw2, 1);
-            tc::mma_commit(&bar_w);
-            const uint32_t iu = tc::idesc_bf16(128, 128, 1, 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(tm + TM_DU, tc::sdesc(sbase + SM_V + ks * 2048, 8192, 1024),
-                           tc::sdesc(sbase + SM_T + ks * 32, 16, 1024), iu, ks != 0);
-            tc::mma_commit(&bar_u);
-        }
-        if (wait_all(&bar_w, ph_w)) { failed = true; break; }
-        ph_w ^= 1u;
-        tc::tc_fence_after();
-
-        // ---------------- P6: W^T/g -> X block 0, while the U~ MMA runs
-        {
-            float w0[32], w1[32];
-            tc::tmem_ld32<32>(tl + TM_DW + 32 * hh, w0);
-            tc::tmem_ld32<32>(tl + TM_DW + 64 + 32 * hh, w1);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w0[i] += w1[i];
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, w0 + 8 * q8);
-        }
-        if (wait_all(&bar_u, ph_u)) { failed = true; break; }
-        ph_u ^= 1u;
-        tc::tc_fence_after();
-        // this chunk's k, q, v, alpha and the solve scratch are consumed: prefetch the next chunk
-        if (tid == 0 && ck + 1 < nchunks) {
-            tc::bulk_wait_read0();               // the o tile in the alpha space has been read
-            issue_loads(t0 + C);
-        }
-        if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
-        sync_for_mma();
-
-        // ---------------- P7: D_R = (S0 Diag g)^T [W^T/g | (q e1)^T]  (3 passes)
-        if (tid == 0) {
-            const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
-#pragma unroll
-            for (int ps = 0; ps < 3; ++ps) {
-                const uint32_t aa = tm + (ps == 2 ? TM_SALO : TM_SAHI);
-                const uint32_t bb = sbase + (ps == 1 ? SM_XLO : SM_XHI);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_ts(tm + TM_DR, aa + ks * 8, tc::sdesc(bb + ks * 2048, 16384, 1024), idesc,
-                               (ps | ks) != 0);
-            }
-            tc::mma_commit(&bar_c1);
-        }
-        if (wait_all(&bar_c1, ph_c1)) { failed = true; break; }
-        ph_c1 ^= 1u;
-        tc::tc_fence_after();
-
-        // ---------------- P8: U^T = U~^T - (S0^T W^T) -> TMEM A operand
-        {
-            float ua[32], ub[32], ws[32];
-            tc::tmem_ld32<32>(tl + TM_DU + 32 * hh, ua);
-            tc::tmem_ld32<32>(tl + TM_DU + 64 + 32 * hh, ub);
-            tc::tmem_ld32<32>(tl + TM_DR + 32 * hh, ws);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ua[i] = (ua[i] + ub[i]) - ws[i];
-            uint32_t hi[16], lo[16];
-            split_pack32(ua, hi, lo);
-            tc::tmem_st32<16>(tl + TM_UAHI + 16 * hh, hi);
-            tc::tmem_st32<16>(tl + TM_UALO + 16 * hh, lo);
-        }
-        sync_for_mma();
-
-        // ---------------- P9: O^T += U^T P^T ;  acc += U^T (k e2)  (3 passes each, waited in the next chunk)
-        if (tid == 0) {
-            const uint32_t io = tc::idesc_bf16(128, 64, 0, 0);
-            const uint32_t is = tc::idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-            for (int ps = 0; ps < 3; ++ps) {
-                const uint32_t aa = tm + (ps == 2 ? TM_UALO : TM_UAHI);
-                const uint32_t pb = sbase + (ps == 1 ? SM_PLO : SM_PHI);
-                const uint32_t kb = sbase + (ps == 1 ? SM_YLO : SM_YHI);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    tc::mma_ts(tm + TM_O, aa + ks * 8, tc::sdesc(pb + ks * 32, 16, 1024), io, 1);
-                    tc::mma_ts(tm + TM_S, aa + ks * 8, tc::sdesc(kb + ks * 32, 16, 1024), is, 1);
+                __syncwarp();
+                // V and T consumed: the next chunk's q and v
+                if (!wait1(&bar_u, par)) break;
+                if (leader && ck + 1 < nchunks) issue_loads2(t0 + C);
+                __syncwarp();
+                // U^T ready: O and state MMAs
+                if (!wait1(&bar_hc2, par)) break;
+                if (leader) {
+                    tc::tc_fence_after();
+                    issue_c2(sbase);
                 }
+                __syncwarp();
             }
-            tc::mma_commit(&bar_c2);
-        }
-    }
-
-    // last chunk: its O / state MMAs, then its o tile
-    if (!failed && nchunks > 0) {
-        if (wait_all(&bar_c2, ph_c2)) {
-            failed = true;
-        } else {
-            tc::tc_fence_after();
-            if (tid == 0) tc::bulk_wait_read0();
-            __syncthreads();
-            stage_o();
-            __syncthreads();
-            if (tid == 0) {
+            // last o tile: free the staging space, then store what the compute warps stage
+            if (leader) {
+                tc::bulk_wait_read0();
+                tc::mbar_arrive(&bar_ofree);
+            }
+            __syncwarp();
+            if (nchunks > 0 && wait1(&bar_hfin, 0) && leader) {
                 tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, (nchunks - 1) * C, b);
                 tc::bulk_commit();
             }
+            if (leader) tc::bulk_wait0();
+            __syncwarp();
         }
-    }
-    if (tid == 0) tc::bulk_wait0();
-
-    // final state: S = acc Diag(kappa_last)
-    if (!failed && ST != nullptr) {
-        const size_t sb = (size_t)bh * D * D;
-        for (int cb = 0; cb < 2; ++cb) {
-            const int c0 = 64 * hh + 32 * cb;
-            float x[32];
-            tc::tmem_ld32<32>(tl + TM_S + c0, x);
-            tc::tmem_ld_wait();
+    } else {
+        // ================================================================ compute warpgroups
+        setmaxnreg_inc<kRegCompute>();
+        // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
+        {
+            const size_t sb = (size_t)bh * D * D;
+            for (int cb = 0; cb < 2; ++cb) {
+                float x[32];
+                const int c0 = 64 * hh + 32 * cb;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ST[sb + (size_t)(c0 + i) * D + m] = x[i] * sh_kref[c0 + i];
+                for (int i = 0; i < 32; ++i) x[i] = S0 ? S0[sb + (size_t)(c0 + i) * D + m] : 0.f;
+                tmem_st_f32x32(tl + TM_S + c0, x);
+            }
+            tc::tmem_st_wait();
+        }
+
+        uint32_t ph_ap = 0, ph_c1 = 0, ph_u = 0, ph_c2 = 0;
+        bool failed = false;
+
+        for (int ck = 0; ck < nchunks && !failed; ++ck) {
+            const int t0 = ck * C;
+            const int nvalid = min(C, T - t0);
+            if (tid < C) sh_beta[tid] = beta_next;
+            if (wait_all(&bar_tma1, ck & 1)) { failed = true; break; }
+
+            // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
+            bool slow;
+            {
+                float L[32];
+                uint32_t par = 0;
+                float run = 0.f;
+                uint32_t p = 0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int r = 32 * hh + i;
+                    const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
+                    run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+                    p ^= (a < 0.f) ? 1u : 0u;
+                    L[i] = run;
+                    par |= p << i;
+                }
+                if (hh == 0) { sh_Lx[m] = run; sh_px[m] = p; }
+                csync();
+                float Lref, LC;
+                uint32_t pref, pC;
+                int bad = 0;
+                if (hh == 1) {
+                    Lref = sh_Lx[m];
+                    pref = sh_px[m];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) L[i] += Lref;
+                    if (pref) par = ~par;
+                    LC = L[31];
+                    pC = par >> 31;
+                    sh_LC[m] = LC;
+                    sh_pC[m] = pC;
+                    bad = (-LC > kChunkRange);
+                }
+                slow = csync_or(bad);
+                if (hh == 0) {
+                    Lref = L[31];
+                    pref = par >> 31;
+                    LC = sh_LC[m];
+                    pC = sh_pC[m];
+                    sh_kp[m] = sh_kref[m];
+                    const float gC = (pC ? -1.f : 1.f) * exp2f(LC);
+                    if (!slow) {
+                        const float gref = exp2f(0.5f * LC);
+                        const float kappa = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
+                        sh_fa[m] = gref;
+                        sh_fs[m] = gref;
+                        sh_kref[m] = kappa;
+                    } else {
+                        sh_fa[m] = 1.f;
+                        sh_fs[m] = gC;
+                        sh_kref[m] = 1.f;
+                    }
+                }
+                // per-token factors: fast path e1 = Gamma_r/Gamma_ref, e2 = Gamma_ref/Gamma_r;
+                // slow path e1 = Gamma_r, e2 = Gamma_C/Gamma_r
+                const float Rm = 0.5f * LC;                 // reference: middle of the chunk's log range
+                const float lo1 = slow ? 0.f : Rm;
+                const float lo2 = slow ? LC : Rm;
+                const uint32_t ps1 = 0u;
+                const uint32_t ps2 = slow ? pC : 0u;
+                if (slow) {
+                    float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i];
+                }
+                // q and v of this chunk; the previous chunk's O / S MMAs read Y and P: wait for
+                // them before overwriting
+                if (wait_all(&bar_tma2, ck & 1)) { failed = true; break; }
+                if (ck > 0) {
+                    if (wait_all(&bar_c2, ph_c2)) { failed = true; break; }
+                    ph_c2 ^= 1u;
+                    tc::tc_fence_after();
+                }
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float xk[8], xq[8], yk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 8 * q8 + e, r = 32 * hh + i;
+                        const uint32_t pr = (par >> i) & 1u;
+                        const float e1 = ((pr ^ ps1) ? -1.f : 1.f) * tc::ex2_approx(L[i] - lo1);
+                        const float e2 = ((pr ^ ps2) ? -1.f : 1.f) * tc::ex2_approx(lo2 - L[i]);
+                        const float kv = ld_bf16_tile(sm + SM_K, r, m);
+                        const float qv = ld_bf16_tile(sm + SM_Q, r, m);
+                        xk[e] = kv * e1;
+                        xq[e] = qv * e1;
+                        yk[e] = kv * e2;
+                    }
+                    store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xk);
+                    store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xq);
+                    store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
+                }
+                if (slow) {
+                    // sign bits of Gamma per (token, channel): word [r][m/32], bit m%32
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const unsigned bits = __ballot_sync(0xffffffffu, (par >> i) & 1u);
+                        if (lane == 0) sh_sign[(32 * hh + i) * 4 + quarter] = bits;
+                    }
+                }
+            }
+            // hand the tiles to the issuer; the barrier also publishes the per-channel constants
+            if (tid == 0) slow_flag_s = slow ? 1u : 0u;
+            handoff(&bar_hap);
+            csync();
+
+            // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact pairwise path
+            if (!slow) {
+                // while the MMA runs: the previous chunk's o tile and this chunk's state copy, then
+                // C1, which overwrites the o accumulator and runs during the solve
+                if (ck > 0) stage_o();
+                state_copy(slow);
+                handoff(&bar_hc1);             // issuer: o store of chunk c-1, then C1
+                if (wait_all(&bar_ap, ph_ap)) { failed = true; break; }
+                ph_ap ^= 1u;
+                tc::tc_fence_after();
+                // ---------------- P3: A (fp32, column-major) and P (hi/lo) out of TMEM
+                float d1[32];
+                tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
+                tc::tmem_ld_wait();
+                if (m < C) {
+                    const int r = m;
+                    const float br = sh_beta[r];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int s = 32 * hh + i;
+                        at[s * 64 + r] = (s < r) ? br * d1[i] : 0.f;
+                    }
+                } else {
+                    const int r = m - C;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) d1[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_PHI, sm + SM_PLO, r, 4 * hh + q8, d1 + 8 * q8);
+                }
+            } else {
+                // exact pairwise evaluation: thread (row r, columns s = sq + 4 j), 128 channels each;
+                // row data is loaded once per channel and reused for the 16 columns
+                const float* Ls = reinterpret_cast<const float*>(sm + SM_SLOWL);
+                const int r = tid >> 2, sq = tid & 3;
+                float va[16], vp[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) va[j] = vp[j] = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < D; ++c) {
+                    const float Lr = Ls[r * D + c];
+                    const uint32_t sr = (sh_sign[r * 4 + (c >> 5)] >> (c & 31)) & 1u;
+                    const float kr = ld_bf16_tile(sm + SM_K, r, c), qr = ld_bf16_tile(sm + SM_Q, r, c);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int sc = sq + 4 * j;
+                        if (sc <= r) {
+                            const uint32_t ss = (sh_sign[sc * 4 + (c >> 5)] >> (c & 31)) & 1u;
+                            const float w = ((sr ^ ss) ? -1.f : 1.f) * tc::ex2_approx(Lr - Ls[sc * D + c]);
+                            const float ksw = ld_bf16_tile(sm + SM_K, sc, c) * w;
+                            va[j] = fmaf(kr, ksw, va[j]);
+                            vp[j] = fmaf(qr, ksw, vp[j]);
+                        }
+                    }
+                }
+                csync();              // k, q tiles fully read before A overwrites them
+                {
+                    const float br = sh_beta[r];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int sc = sq + 4 * j;
+                        at[sc * 64 + r] = (sc < r) ? br * va[j] : 0.f;
+                        uint32_t hpair, lpair;
+                        split2((sc <= r) ? vp[j] : 0.f, 0.f, hpair, lpair);
+                        const uint32_t offp = chunk_off(r, sc >> 3) + (uint32_t)(sc & 7) * 2u;
+                        *reinterpret_cast<uint16_t*>(sm + SM_PHI + offp) = (uint16_t)(hpair & 0xffffu);
+                        *reinterpret_cast<uint16_t*>(sm + SM_PLO + offp) = (uint16_t)(lpair & 0xffffu);
+                    }
+                }
+                if (ck > 0) stage_o();
+                state_copy(slow);
+                handoff(&bar_hc1);
+            }
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            csync();
+
+            // ---------------- P4: T = (I + A)^{-1} Diag(beta): 16 x 16 diagonal blocks, then two
+            // doubling levels. With L = I + A split into 2 x 2 blocks, L^{-1} has the lower-left
+            // block -X_22 A_21 X_11 (X_ii the inverses of the diagonal blocks).
+            if (warp < 4 && lane < 16) {
+                // diagonal block I, column j: right-looking forward substitution; column ss of
+                // A_II is contiguous in the column-major A, so each step is 4 broadcast loads
+                const int I = warp, j = lane;
+                const float* acol = at + (16 * I) * 64 + 16 * I;
+                float acc[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) acc[rr] = (rr == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int ss = 0; ss < 15; ++ss) {
+                    const float xv = acc[ss];             // final value of x_ss (0 above the diagonal)
+                    float a[16];
+#pragma unroll
+                    for (int g = (ss + 1) >> 2; g < 4; ++g) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(acol + ss * 64 + 4 * g);
+                        a[4 * g] = t4.x; a[4 * g + 1] = t4.y; a[4 * g + 2] = t4.z; a[4 * g + 3] = t4.w;
+                    }
+#pragma unroll
+                    for (int rr = ss + 1; rr < 16; ++rr) acc[rr] = fmaf(-a[rr], xv, acc[rr]);
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) xs[(16 * I + rr) * XS_LD + 16 * I + j] = acc[rr];
+            }
+            csync();
+            // level 1 (blocks of 16 -> 32), pairs (0,1) and (2,3): R = A_10 X_00, X_10 = -X_11 R.
+            // Thread: pair pb, row r, columns 2 c2, 2 c2 + 1.
+            {
+                const int pb = tid >> 7, r = (tid >> 3) & 15, c2 = tid & 7, o = 32 * pb;
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float a = at[(o + k) * 64 + o + 16 + r];
+                    const float2 xv = *reinterpret_cast<const float2*>(xs + (o + k) * XS_LD + o + 2 * c2);
+                    acc.x = fmaf(a, xv.x, acc.x);
+                    acc.y = fmaf(a, xv.y, acc.y);
+                }
+                *reinterpret_cast<float2*>(rs + pb * 320 + r * 20 + 2 * c2) = acc;
+                csync();
+                float2 xo = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int mm = 0; mm < 16; ++mm) {
+                    const float xd = xs[(o + 16 + r) * XS_LD + o + 16 + mm];   // X_11, zero above the diagonal
+                    const float2 rv = *reinterpret_cast<const float2*>(rs + pb * 320 + mm * 20 + 2 * c2);
+                    xo.x = fmaf(xd, rv.x, xo.x);
+                    xo.y = fmaf(xd, rv.y, xo.y);
+                }
+                *reinterpret_cast<float2*>(xs + (o + 16 + r) * XS_LD + o + 2 * c2) = make_float2(-xo.x, -xo.y);
+            }
+            csync();
+            // level 2 (32 -> 64): R = A[32:64, 0:32] X[0:32, 0:32], X[32:64, 0:32] = -X[32:64, 32:64] R.
+            // T = X Diag(beta) is split into the MMA operand as soon as a block of X is final.
+            {
+                // R: warp -> columns 4 w .. 4 w + 3, lane -> row; X[k][c] = 0 for k < c
+                const int cg = warp, r = lane;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+                for (int k = 4 * cg; k < 32; ++k) {
+                    const float a = at[k * 64 + 32 + r];
+                    const float4 xv = *reinterpret_cast<const float4*>(xs + k * XS_LD + 4 * cg);
+                    acc.x = fmaf(a, xv.x, acc.x);
+                    acc.y = fmaf(a, xv.y, acc.y);
+                    acc.z = fmaf(a, xv.z, acc.z);
+                    acc.w = fmaf(a, xv.w, acc.w);
+                }
+                *reinterpret_cast<float4*>(rs + r * 36 + 4 * cg) = acc;
+                // final blocks of T: rows 0..31 x columns 0..31 and rows 32..63 x columns 32..63
+                // (16-byte chunk ch of row tr), and the zero block rows 0..31 x columns 32..63
+                {
+                    const int half = warp >> 2, ch = (warp & 3) + 4 * half, tr = lane + 32 * half;
+                    const float4 x0 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch);
+                    const float4 x1 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch + 4);
+                    const float4 b0 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[0];
+                    const float4 b1 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[1];
+                    const float v[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
+                                        x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
+                    store_split8(sm + SM_T, sm + SM_T + 8192, tr, ch, v);
+                    const uint32_t zoff = chunk_off(lane, 4 + (warp & 3)) + (uint32_t)half * 8192u;
+                    *reinterpret_cast<uint4*>(sm + SM_T + zoff) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                // A (k-tile space) is consumed: the issuer loads the next chunk's k and alpha
+                // once the o tile has left the alpha space
+                tc::mbar_arrive(&bar_hl2);
+                csync();
+                // X[32:64, 0:32]: thread -> row 32 + r2, columns 4 c4 .. 4 c4 + 3, straight into T.
+                // X[32 + r2][32 + mm] is zero for mm > r2: warps 0-3 hold rows r2 < 16.
+                const int r2 = tid >> 3, c4 = tid & 7;
+                const int mmax = (warp < 4) ? 16 : 32;
+                float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+                for (int mm = 0; mm < mmax; ++mm) {
+                    const float xd = xs[(32 + r2) * XS_LD + 32 + mm];
+                    const float4 rv = *reinterpret_cast<const float4*>(rs + mm * 36 + 4 * c4);
+                    xo.x = fmaf(xd, rv.x, xo.x);
+                    xo.y = fmaf(xd, rv.y, xo.y);
+                    xo.z = fmaf(xd, rv.z, xo.z);
+                    xo.w = fmaf(xd, rv.w, xo.w);
+                }
+                const float4 b4 = reinterpret_cast<const float4*>(sh_beta)[c4];
+                uint32_t h0, l0, h1, l1;
+                split2(-xo.x * b4.x, -xo.y * b4.y, h0, l0);
+                split2(-xo.z * b4.z, -xo.w * b4.w, h1, l1);
+                const uint32_t off = chunk_off(32 + r2, c4 >> 1) + (uint32_t)(c4 & 1) * 8u;
+                *reinterpret_cast<uint2*>(sm + SM_T + off) = make_uint2(h0, h1);
+                *reinterpret_cast<uint2*>(sm + SM_T + 8192 + off) = make_uint2(l0, l1);
+            }
+
+            if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
+
+            // ---------------- P5: -Z^T (from C1) -> TMEM A operand; U^T = V^T T^T - Z^T T^T
+            if (wait_all(&bar_c1, ph_c1)) { failed = true; break; }
+            ph_c1 ^= 1u;
+            tc::tc_fence_after();
+            {
+                float z[32];
+                tc::tmem_ld32<32>(tl + TM_Z + 32 * hh, z);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) z[i] = -z[i];
+                uint32_t hi[16], lo[16];
+                split_pack32(z, hi, lo);
+                tc::tmem_st32<16>(tl + TM_ZAHI + 16 * hh, hi);
+                tc::tmem_st32<16>(tl + TM_ZALO + 16 * hh, lo);
+            }
+            handoff(&bar_hu);                  // T tiles and -Z^T: the issuer starts the U MMA
+            if (wait_all(&bar_u, ph_u)) { failed = true; break; }
+            ph_u ^= 1u;
+            tc::tc_fence_after();
+
+            // ---------------- P8: U^T -> TMEM A operand (hi / lo)
+            {
+                float u[32];
+                tc::tmem_ld32<32>(tl + TM_DU + 32 * hh, u);
+                tc::tmem_ld_wait();
+                uint32_t hi[16], lo[16];
+                split_pack32(u, hi, lo);
+                tc::tmem_st32<16>(tl + TM_UAHI + 16 * hh, hi);
+                tc::tmem_st32<16>(tl + TM_UALO + 16 * hh, lo);
+            }
+
+            // ---------------- P9: O^T += U^T P^T ;  acc += U^T (k e2), issued by the issuer warp
+            handoff(&bar_hc2);
+        }
+
+        // last chunk: its O / state MMAs, then its o tile (stored by the issuer)
+        if (!failed && nchunks > 0) {
+            if (wait_all(&bar_c2, ph_c2)) {
+                failed = true;
+            } else {
+                tc::tc_fence_after();
+                if (wait_all(&bar_ofree, 0)) {          // the previous o tile has left the staging space
+                    failed = true;
+                } else {
+                    stage_o();
+                    handoff(&bar_hfin);
+                }
+            }
+        }
+
+        // final state: S = acc Diag(kappa_last)
+        if (!failed && ST != nullptr) {
+            const size_t sb = (size_t)bh * D * D;
+            for (int cb = 0; cb < 2; ++cb) {
+                const int c0 = 64 * hh + 32 * cb;
+                float x[32];
+                tc::tmem_ld32<32>(tl + TM_S + c0, x);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ST[sb + (size_t)(c0 + i) * D + m] = x[i] * sh_kref[c0 + i];
+            }
         }
     }
     tc::tc_fence_before();
@@ -807,7 +937,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    chunk_tc_kernel<<<(unsigned)(B * H), ctc::NT, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H);
+    chunk_tc_kernel<<<(unsigned)(B * H), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H);
     return cudaGetLastError();
 }
 
