@@ -23,8 +23,8 @@
 //   Gamma_r/Gamma_s = e1_r e2_s,  Gamma_r = e1_r g_ref,  Gamma_C/Gamma_s = e2_s kappa,
 //   Gamma_C = g_ref kappa,
 // and every factor lies in [2^{L_C/2}, 2^{-L_C/2}].
-// So one pair of token tiles X = [k e1 ; q e1] and Y = k e2 serves every product:
-//   [A ; P] from X Y^T;  [Z | O_inter] from (S0 Diag g_ref)^T X^T;  U from T (V - Z);
+// So one pair of token tiles X = [q e1 ; k e1] and Y = k e2 serves every product:
+//   [P ; A] from X Y^T;  [O_inter | Z] from (S0 Diag g_ref)^T X^T;  U from T (V - Z);
 //   the state update from S0 Diag(g_ref) + U^T (k e2), which is S_C Diag(1/kappa).
 // Z and O_inter depend only on the gate and the state entering the chunk, so their MMA
 // runs on the tensor cores while the CUDA cores solve for T.
@@ -79,11 +79,11 @@ constexpr uint32_t SM_V = 32768;        // v tile (MN-major A operand of V^T T^T
 constexpr uint32_t SM_AL = 49152;       // alpha tile: 4 boxes [64 tok][32 ch] fp32
 constexpr uint32_t SM_SLOWL = 49152;    //   slow path only: L fp32 [64][128]
 constexpr uint32_t SM_OT = 49152;       //   after the gate: o tile fp32 [64 tok][128], TMA-stored
-constexpr uint32_t SM_XHI = 81920;      // X hi: block 0 = k e1 (later W^T), block 1 = q e1, [128 c][64 r]
+constexpr uint32_t SM_XHI = 81920;      // X hi: block 0 = q e1, block 1 = k e1, [128 c][64 r]
 constexpr uint32_t SM_XLO = 114688;     // X lo
-constexpr uint32_t SM_YHI = 147456;     // Y = k e2, [128 c][64 s] (MN-major for A/P, K-major for S)
-constexpr uint32_t SM_YLO = 163840;
-constexpr uint32_t SM_PHI = 180224;     // P K-major [64 r][64 s]
+constexpr uint32_t SM_YHI = 147456;     // Y = k e2, [128 c][64 s] (MN-major for A/P, K-major for S) ...
+constexpr uint32_t SM_PHI = 163840;     //   ... followed by P K-major [64 r][64 s]: [Y ; P] is one
+constexpr uint32_t SM_YLO = 172032;     //   K-major B operand of 192 rows for the O / state MMA
 constexpr uint32_t SM_PLO = 188416;
 constexpr uint32_t SM_XS = 196608;      // (I + A)^{-1}, fp32 row-major [64][XS_LD]; blocks above the
 constexpr int XS_LD = 68;               //   16 x 16 block diagonal stay zero for the whole kernel
@@ -94,17 +94,18 @@ constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;       // + alignment slack
 static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
 
 // TMEM column map (512 columns allocated)
-constexpr uint32_t TM_S = 0;          // state accumulator S^T Diag(1/kappa) [d_v lanes][d_k cols]
-constexpr uint32_t TM_SAHI = 128;     // (S0 Diag g)^T hi / lo, packed bf16 (A operand of C1)
-constexpr uint32_t TM_SALO = 192;
-constexpr uint32_t TM_ZAHI = 128;     //   after C1: -Z^T hi / lo, packed bf16 (A operand of the U MMA)
-constexpr uint32_t TM_ZALO = 160;
-constexpr uint32_t TM_UAHI = 192;     //   after the U MMA: U^T hi / lo, packed bf16 (A of the O / S MMAs)
-constexpr uint32_t TM_UALO = 224;
-constexpr uint32_t TM_Z = 256;        // C1 result: Z^T [d_v][64 tok] ...
-constexpr uint32_t TM_O = 320;        //   ... and O^T, which the P U MMA accumulates into
-constexpr uint32_t TM_D1 = 384;       // [A ; P] 128 x 64
-constexpr uint32_t TM_DU = 448;       // U^T = V^T T^T - Z^T T^T, 128 x 64
+constexpr uint32_t TM_S = 0;          // state accumulator S^T Diag(1/kappa) [d_v lanes][d_k cols] ...
+constexpr uint32_t TM_O = 128;        //   ... then O^T [d_v][64 tok]: one 192-column accumulator for C2
+constexpr uint32_t TM_Z = 192;        // Z^T [d_v][64 tok]; C1 writes [O^T | Z^T]
+constexpr uint32_t TM_SAHI = 256;     // (S0 Diag g)^T hi / lo, packed bf16 (A operand of C1)
+constexpr uint32_t TM_SALO = 320;
+constexpr uint32_t TM_ZAHI = 256;     //   after C1: -Z^T hi / lo, packed bf16 (A operand of the U MMA)
+constexpr uint32_t TM_ZALO = 288;
+constexpr uint32_t TM_UAHI = 320;     //   after the U MMA: U^T hi / lo, packed bf16 (A of C2)
+constexpr uint32_t TM_UALO = 352;
+constexpr uint32_t TM_D1 = 384;       // [A ; P] as two partial sums: X_hi Y_hi + X_lo Y_hi | X_hi Y_lo
+constexpr uint32_t TM_DU = 384;       //   after the [A ; P] epilogue: U^T as two partial sums,
+                                      //   (V^T - Z^T) T_hi^T | (V^T - Z^T) T_lo^T
 
 constexpr uint32_t kTmaBytes1 = 6 * 8192;   // k (2 bf16 boxes) + alpha (4 fp32 boxes)
 constexpr uint32_t kTmaBytes2 = 4 * 8192;   // q + v (2 bf16 boxes each)
@@ -232,7 +233,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar_tma1, bar_tma2, bar_ap, bar_c1, bar_u, bar_c2;    // TMA / MMA completion
-    __shared__ uint64_t bar_hap, bar_hc1, bar_hl2, bar_hu, bar_hc2, bar_hfin;  // compute -> issuer
+    __shared__ uint64_t bar_hap, bar_hc1, bar_hl2, bar_ht, bar_hu, bar_hc2, bar_hfin;  // compute -> issuer
     __shared__ uint64_t bar_ofree;                                              // issuer -> compute
     __shared__ uint32_t tmem_base_s, slow_flag_s;
 
@@ -268,6 +269,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::mbar_init(&bar_hap, NT);
         tc::mbar_init(&bar_hc1, NT);
         tc::mbar_init(&bar_hl2, NT);
+        tc::mbar_init(&bar_ht, NT);
         tc::mbar_init(&bar_hu, NT);
         tc::mbar_init(&bar_hc2, NT);
         tc::mbar_init(&bar_hfin, NT);
@@ -324,31 +326,43 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
         tc::fence_proxy_async_smem();
     };
-    // state copy into the C1 operand and rescale of the accumulator. The accumulator holds
-    // S Diag(1/kappa_prev): first S = acc kappa_prev, then the operand S g_ref and the new
-    // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
+    // state copy into the C1 operand and rescale of the accumulator, with the previous
+    // chunk's o tile staged first (the next TMEM load is in flight while the previous block
+    // is processed). The accumulator
+    // holds S Diag(1/kappa_prev): first S = acc kappa_prev, then the operand S g_ref and the
+    // new accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
     // for fast-decaying channels although each factor and each result is in range.
-    auto state_copy = [&](bool slow_chunk) {
+    auto stage_and_copy = [&](bool with_o, bool slow_chunk) {
+        float sv[2][32];
+        tc::tmem_ld32<32>(tl + TM_S + 64 * hh, sv[0]);
+        if (with_o) {
+            float ov[32];
+            tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
+            tc::tmem_ld_wait();
+            float* ot = reinterpret_cast<float*>(sm + SM_OT);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
+        }
 #pragma unroll
         for (int cb = 0; cb < 2; ++cb) {
             const int c0 = 64 * hh + 32 * cb;
-            float sv[32], z[32];
-            tc::tmem_ld32<32>(tl + TM_S + c0, sv);
             tc::tmem_ld_wait();
+            if (cb == 0) tc::tmem_ld32<32>(tl + TM_S + 64 * hh + 32, sv[1]);
+            float z[32];
             const float4* kp4 = reinterpret_cast<const float4*>(sh_kp + c0);
             const float4* fa4 = reinterpret_cast<const float4*>(sh_fa + c0);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 kk = kp4[i];
                 const float4 f = fa4[i];
-                sv[4 * i] *= kk.x;
-                sv[4 * i + 1] *= kk.y;
-                sv[4 * i + 2] *= kk.z;
-                sv[4 * i + 3] *= kk.w;
-                z[4 * i] = sv[4 * i] * f.x;
-                z[4 * i + 1] = sv[4 * i + 1] * f.y;
-                z[4 * i + 2] = sv[4 * i + 2] * f.z;
-                z[4 * i + 3] = sv[4 * i + 3] * f.w;
+                sv[cb][4 * i] *= kk.x;
+                sv[cb][4 * i + 1] *= kk.y;
+                sv[cb][4 * i + 2] *= kk.z;
+                sv[cb][4 * i + 3] *= kk.w;
+                z[4 * i] = sv[cb][4 * i] * f.x;
+                z[4 * i + 1] = sv[cb][4 * i + 1] * f.y;
+                z[4 * i + 2] = sv[cb][4 * i + 2] * f.z;
+                z[4 * i + 3] = sv[cb][4 * i + 3] * f.w;
             }
             uint32_t hi[16], lo[16];
             split_pack32(z, hi, lo);
@@ -361,17 +375,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 f = fs4[i];
-                    sv[4 * i] *= f.x;
-                    sv[4 * i + 1] *= f.y;
-                    sv[4 * i + 2] *= f.z;
-                    sv[4 * i + 3] *= f.w;
+                    sv[cb][4 * i] *= f.x;
+                    sv[cb][4 * i + 1] *= f.y;
+                    sv[cb][4 * i + 2] *= f.z;
+                    sv[cb][4 * i + 3] *= f.w;
                 }
-                tmem_st_f32x32(tl + TM_S + c0, sv);
+                tmem_st_f32x32(tl + TM_S + c0, sv[cb]);
             }
         }
     };
 
-    // C1: [Z^T | O^T] = (S0 Diag g)^T [(k e1)^T | (q e1)^T]  (3 passes), after the state copy
+    // C1: [O^T | Z^T] = (S0 Diag g)^T [(q e1)^T | (k e1)^T]  (3 passes), after the state copy
     auto issue_c1 = [&](uint32_t sb_) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
         const uint32_t idesc = tc::idesc_bf16(128, 128, 0, 1);
@@ -381,60 +395,57 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             const uint32_t bb = sb0 + (ps == 1 ? SM_XLO : SM_XHI);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                tc::mma_ts(tm0 + TM_Z, aa + ks * 8, tc::sdesc(bb + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
+                tc::mma_ts(tm0 + TM_O, aa + ks * 8, tc::sdesc(bb + ks * 2048, 16384, 1024), idesc, (ps | ks) != 0);
         }
         tc::mma_commit(&bar_c1);
     };
-    // [A ; P] = X Y  (3 passes)
+    // [P ; A] = X Y  (3 passes as X_hi [Y_hi | Y_lo] with N = 128, then X_lo Y_hi)
     auto issue_ap = [&](uint32_t sb_) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
-        const uint32_t idesc = tc::idesc_bf16(128, 64, 1, 1);
+        const uint32_t i128 = tc::idesc_bf16(128, 128, 1, 1), i64 = tc::idesc_bf16(128, 64, 1, 1);
 #pragma unroll
-        for (int ps = 0; ps < 3; ++ps) {
-            const uint32_t xa = sb0 + (ps == 2 ? SM_XLO : SM_XHI);
-            const uint32_t yb = sb0 + (ps == 1 ? SM_YLO : SM_YHI);
+        for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ss(tm0 + TM_D1, tc::sdesc(sb0 + SM_XHI + ks * 2048, 16384, 1024),
+                       tc::sdesc(sb0 + SM_YHI + ks * 2048, SM_YLO - SM_YHI, 1024), i128, ks != 0);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                tc::mma_ss(tm0 + TM_D1, tc::sdesc(xa + ks * 2048, 16384, 1024), tc::sdesc(yb + ks * 2048, 16384, 1024),
-                           idesc, (ps | ks) != 0);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ss(tm0 + TM_D1, tc::sdesc(sb0 + SM_XLO + ks * 2048, 16384, 1024),
+                       tc::sdesc(sb0 + SM_YHI + ks * 2048, SM_YLO - SM_YHI, 1024), i64, 1);
         tc::mma_commit(&bar_ap);
     };
-    // U^T = V^T [T_hi ; T_lo]^T  +  (-Z^T)_hi T_hi^T + (-Z^T)_hi T_lo^T + (-Z^T)_lo T_hi^T
-    auto issue_u = [&](uint32_t sb_) {
+    // U^T = V^T [T_hi ; T_lo]^T, issued as soon as T is ready (N = 128: both halves at once)
+    auto issue_uv = [&](uint32_t sb_) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
-        const uint32_t iv = tc::idesc_bf16(128, 64, 1, 0);    // A = V^T (MN-major), B = T (K-major)
-        const uint32_t iz = tc::idesc_bf16(128, 64, 0, 0);    // A = -Z^T (TMEM)
+        const uint32_t iv = tc::idesc_bf16(128, 128, 1, 0);   // A = V^T (MN-major), B = T (K-major)
 #pragma unroll
-        for (int ps = 0; ps < 2; ++ps)
+        for (int ks = 0; ks < 4; ++ks)
+            tc::mma_ss(tm0 + TM_DU, tc::sdesc(sb0 + SM_V + ks * 2048, 8192, 1024),
+                       tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iv, ks != 0);
+    };
+    //   += (-Z^T)_hi [T_hi ; T_lo]^T + (-Z^T)_lo [T_hi ; T_lo]^T once -Z^T is in TMEM
+    auto issue_uz = [&](uint32_t sb_) {
+        const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
+        const uint32_t iz = tc::idesc_bf16(128, 128, 0, 0);   // A = -Z^T (TMEM)
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps) {
+            const uint32_t aa = tm0 + (ps == 1 ? TM_ZALO : TM_ZAHI);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(tm0 + TM_DU, tc::sdesc(sb0 + SM_V + ks * 2048, 8192, 1024),
-                           tc::sdesc(sb0 + SM_T + ps * 8192 + ks * 32, 16, 1024), iv, (ps | ks) != 0);
-#pragma unroll
-        for (int ps = 0; ps < 3; ++ps) {
-            const uint32_t aa = tm0 + (ps == 2 ? TM_ZALO : TM_ZAHI);
-            const uint32_t tb = sb0 + SM_T + (ps == 1 ? 8192 : 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) tc::mma_ts(tm0 + TM_DU, aa + ks * 8, tc::sdesc(tb + ks * 32, 16, 1024), iz, 1);
+                tc::mma_ts(tm0 + TM_DU, aa + ks * 8, tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iz, 1);
         }
         tc::mma_commit(&bar_u);
     };
-    // O^T += U^T P^T ;  acc += U^T (k e2)  (3 passes each)
+    // [acc | O^T] += U^T [(k e2) | P^T]  (3 passes, N = 192: state and output in one MMA)
     auto issue_c2 = [&](uint32_t sb_) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
-        const uint32_t io = tc::idesc_bf16(128, 64, 0, 0);
-        const uint32_t is = tc::idesc_bf16(128, 128, 0, 0);
+        const uint32_t idesc = tc::idesc_bf16(128, 192, 0, 0);
 #pragma unroll
         for (int ps = 0; ps < 3; ++ps) {
             const uint32_t aa = tm0 + (ps == 2 ? TM_UALO : TM_UAHI);
-            const uint32_t pb = sb0 + (ps == 1 ? SM_PLO : SM_PHI);
-            const uint32_t kb = sb0 + (ps == 1 ? SM_YLO : SM_YHI);
+            const uint32_t yb = sb0 + (ps == 1 ? SM_YLO : SM_YHI);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                tc::mma_ts(tm0 + TM_O, aa + ks * 8, tc::sdesc(pb + ks * 32, 16, 1024), io, 1);
-                tc::mma_ts(tm0 + TM_S, aa + ks * 8, tc::sdesc(kb + ks * 32, 16, 1024), is, 1);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_ts(tm0 + TM_S, aa + ks * 8, tc::sdesc(yb + ks * 32, 16, 1024), idesc, 1);
         }
         tc::mma_commit(&bar_c2);
     };
@@ -486,11 +497,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     issue_loads1(t0 + C);
                 }
                 __syncwarp();
-                // T and -Z^T ready: U
+                // T ready: the V part of U
+                if (!wait1(&bar_ht, par)) break;
+                if (leader) {
+                    tc::tc_fence_after();
+                    issue_uv(sbase);
+                }
+                __syncwarp();
+                // -Z^T ready: the Z part
                 if (!wait1(&bar_hu, par)) break;
                 if (leader) {
                     tc::tc_fence_after();
-                    issue_u(sbase);
+                    issue_uz(sbase);
                 }
                 __syncwarp();
                 // V and T consumed: the next chunk's q and v
@@ -546,31 +564,34 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
             bool slow;
             {
+                // L[i]: log2 |prod a| from the start of this thread's half of the chunk;
+                // par bit i: sign of the same product (prefix XOR of the gates' sign bits)
                 float L[32];
                 uint32_t par = 0;
                 float run = 0.f;
-                uint32_t p = 0;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int r = 32 * hh + i;
                     const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
                     run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
-                    p ^= (a < 0.f) ? 1u : 0u;
+                    par |= (__float_as_uint(a) >> 31) << i;
                     L[i] = run;
-                    par |= p << i;
                 }
-                if (hh == 0) { sh_Lx[m] = run; sh_px[m] = p; }
+                par ^= par << 1;
+                par ^= par << 2;
+                par ^= par << 4;
+                par ^= par << 8;
+                par ^= par << 16;
+                if (hh == 0) { sh_Lx[m] = run; sh_px[m] = par >> 31; }
                 csync();
-                float Lref, LC;
-                uint32_t pref, pC;
+                // second half: offset by the first half's totals (kept apart from L[])
+                float Lofs = 0.f, LC = 0.f;
+                uint32_t pC = 0;
                 int bad = 0;
                 if (hh == 1) {
-                    Lref = sh_Lx[m];
-                    pref = sh_px[m];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) L[i] += Lref;
-                    if (pref) par = ~par;
-                    LC = L[31];
+                    Lofs = sh_Lx[m];
+                    if (sh_px[m]) par = ~par;
+                    LC = L[31] + Lofs;
                     pC = par >> 31;
                     sh_LC[m] = LC;
                     sh_pC[m] = pC;
@@ -578,39 +599,57 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
                 slow = csync_or(bad);
                 if (hh == 0) {
-                    Lref = L[31];
-                    pref = par >> 31;
                     LC = sh_LC[m];
                     pC = sh_pC[m];
                     sh_kp[m] = sh_kref[m];
-                    const float gC = (pC ? -1.f : 1.f) * exp2f(LC);
                     if (!slow) {
                         const float gref = exp2f(0.5f * LC);
-                        const float kappa = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
                         sh_fa[m] = gref;
                         sh_fs[m] = gref;
-                        sh_kref[m] = kappa;
+                        sh_kref[m] = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
                     } else {
                         sh_fa[m] = 1.f;
-                        sh_fs[m] = gC;
+                        sh_fs[m] = (pC ? -1.f : 1.f) * exp2f(LC);
                         sh_kref[m] = 1.f;
                     }
                 }
-                // per-token factors: fast path e1 = Gamma_r/Gamma_ref, e2 = Gamma_ref/Gamma_r;
-                // slow path e1 = Gamma_r, e2 = Gamma_C/Gamma_r
-                const float Rm = 0.5f * LC;                 // reference: middle of the chunk's log range
-                const float lo1 = slow ? 0.f : Rm;
-                const float lo2 = slow ? LC : Rm;
-                const uint32_t ps1 = 0u;
-                const uint32_t ps2 = slow ? pC : 0u;
                 if (slow) {
                     float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i];
+                    for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
                 }
-                // q and v of this chunk; the previous chunk's O / S MMAs read Y and P: wait for
-                // them before overwriting
+                // q and v of this chunk
                 if (wait_all(&bar_tma2, ck & 1)) { failed = true; break; }
+                // per-token factors (the sign of Gamma_r is XORed into the factor's sign bit):
+                //   fast path  e1 = Gamma_r / 2^R,  e2 = 2^R / Gamma_r  (R = L_C / 2: middle of the range)
+                //   exact path e1 = Gamma_r,        e2 = Gamma_C / Gamma_r
+                const float c1 = slow ? -Lofs : 0.5f * LC - Lofs;     // t = L_r - R, or L_r
+                const uint32_t sC = slow ? (pC << 31) : 0u;
+                const float d2 = slow ? LC : 0.f;                       // e2 = 2^(d2 - t)
+                uint32_t yh[4][4], yl[4][4];      // Y = k e2 split, held until the tile is free
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float xk[8], xq[8], yk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 8 * q8 + e, r = 32 * hh + i;
+                        const uint32_t sg = (par << (31 - i)) & 0x80000000u;
+                        const float t = L[i] - c1;
+                        const float m2 = tc::ex2_approx(d2 - t);
+                        const float e1 = __uint_as_float(__float_as_uint(tc::ex2_approx(t)) ^ sg);
+                        const float e2 = __uint_as_float(__float_as_uint(m2) ^ sg ^ sC);
+                        const float kv = ld_bf16_tile(sm + SM_K, r, m);
+                        const float qv = ld_bf16_tile(sm + SM_Q, r, m);
+                        xk[e] = kv * e1;
+                        xq[e] = qv * e1;
+                        yk[e] = kv * e2;
+                    }
+                    store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xq);
+                    store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xk);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) split2(yk[2 * e], yk[2 * e + 1], yh[q8][e], yl[q8][e]);
+                }
+                // the previous chunk's O / state MMA reads Y and P: wait for it before writing Y
                 if (ck > 0) {
                     if (wait_all(&bar_c2, ph_c2)) { failed = true; break; }
                     ph_c2 ^= 1u;
@@ -618,22 +657,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
-                    float xk[8], xq[8], yk[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = 8 * q8 + e, r = 32 * hh + i;
-                        const uint32_t pr = (par >> i) & 1u;
-                        const float e1 = ((pr ^ ps1) ? -1.f : 1.f) * tc::ex2_approx(L[i] - lo1);
-                        const float e2 = ((pr ^ ps2) ? -1.f : 1.f) * tc::ex2_approx(lo2 - L[i]);
-                        const float kv = ld_bf16_tile(sm + SM_K, r, m);
-                        const float qv = ld_bf16_tile(sm + SM_Q, r, m);
-                        xk[e] = kv * e1;
-                        xq[e] = qv * e1;
-                        yk[e] = kv * e2;
-                    }
-                    store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xk);
-                    store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xq);
-                    store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
+                    const uint32_t off = chunk_off(m, 4 * hh + q8);
+                    *reinterpret_cast<uint4*>(sm + SM_YHI + off) = make_uint4(yh[q8][0], yh[q8][1], yh[q8][2], yh[q8][3]);
+                    *reinterpret_cast<uint4*>(sm + SM_YLO + off) = make_uint4(yl[q8][0], yl[q8][1], yl[q8][2], yl[q8][3]);
                 }
                 if (slow) {
                     // sign bits of Gamma per (token, channel): word [r][m/32], bit m%32
@@ -653,18 +679,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             if (!slow) {
                 // while the MMA runs: the previous chunk's o tile and this chunk's state copy, then
                 // C1, which overwrites the o accumulator and runs during the solve
-                if (ck > 0) stage_o();
-                state_copy(slow);
+                stage_and_copy(ck > 0, slow);
                 handoff(&bar_hc1);             // issuer: o store of chunk c-1, then C1
                 if (wait_all(&bar_ap, ph_ap)) { failed = true; break; }
                 ph_ap ^= 1u;
                 tc::tc_fence_after();
                 // ---------------- P3: A (fp32, column-major) and P (hi/lo) out of TMEM
-                float d1[32];
+                float d1[32], d2[32];
                 tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
+                tc::tmem_ld32<32>(tl + TM_D1 + 64 + 32 * hh, d2);
                 tc::tmem_ld_wait();
-                if (m < C) {
-                    const int r = m;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) d1[i] += d2[i];
+                if (m >= C) {
+                    const int r = m - C;
                     const float br = sh_beta[r];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -672,7 +700,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         at[s * 64 + r] = (s < r) ? br * d1[i] : 0.f;
                     }
                 } else {
-                    const int r = m - C;
+                    const int r = m;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) d1[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
 #pragma unroll
@@ -717,8 +745,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         *reinterpret_cast<uint16_t*>(sm + SM_PLO + offp) = (uint16_t)(lpair & 0xffffu);
                     }
                 }
-                if (ck > 0) stage_o();
-                state_copy(slow);
+                stage_and_copy(ck > 0, slow);
                 handoff(&bar_hc1);
             }
             tc::tmem_ld_wait();
@@ -833,6 +860,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 *reinterpret_cast<uint2*>(sm + SM_T + off) = make_uint2(h0, h1);
                 *reinterpret_cast<uint2*>(sm + SM_T + 8192 + off) = make_uint2(l0, l1);
             }
+            handoff(&bar_ht);                      // T tiles complete: the issuer starts V T^T
 
             if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
 
@@ -851,16 +879,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 tc::tmem_st32<16>(tl + TM_ZAHI + 16 * hh, hi);
                 tc::tmem_st32<16>(tl + TM_ZALO + 16 * hh, lo);
             }
-            handoff(&bar_hu);                  // T tiles and -Z^T: the issuer starts the U MMA
+            handoff(&bar_hu);                  // -Z^T: the issuer adds Z T^T
             if (wait_all(&bar_u, ph_u)) { failed = true; break; }
             ph_u ^= 1u;
             tc::tc_fence_after();
 
             // ---------------- P8: U^T -> TMEM A operand (hi / lo)
             {
-                float u[32];
+                float u[32], u2[32];
                 tc::tmem_ld32<32>(tl + TM_DU + 32 * hh, u);
+                tc::tmem_ld32<32>(tl + TM_DU + 64 + 32 * hh, u2);
                 tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) u[i] += u2[i];
                 uint32_t hi[16], lo[16];
                 split_pack32(u, hi, lo);
                 tc::tmem_st32<16>(tl + TM_UAHI + 16 * hh, hi);
