@@ -554,12 +554,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
         uint32_t ph_ap = 0, ph_c1 = 0, ph_u = 0, ph_c2 = 0;
         bool failed = false;
+        // a bounded mbarrier wait that gave up: every thread waits for itself (the wait
+        // acquires what the TMA or MMA wrote) and the flag is OR-reduced at the next barrier
+        // the schedule needs anyway, where all compute warps leave the loop together
+        bool wfail = false;
 
         for (int ck = 0; ck < nchunks && !failed; ++ck) {
             const int t0 = ck * C;
             const int nvalid = min(C, T - t0);
             if (tid < C) sh_beta[tid] = beta_next;
-            if (wait_all(&bar_tma1, ck & 1)) { failed = true; break; }
+            wfail |= !tc::mbar_wait(&bar_tma1, ck & 1);
 
             // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
             bool slow;
@@ -583,7 +587,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 par ^= par << 8;
                 par ^= par << 16;
                 if (hh == 0) { sh_Lx[m] = run; sh_px[m] = par >> 31; }
-                csync();
+                if (csync_or(wfail)) { failed = true; break; }
                 // second half: offset by the first half's totals (kept apart from L[])
                 float Lofs = 0.f, LC = 0.f;
                 uint32_t pC = 0;
@@ -619,7 +623,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
                 }
                 // q and v of this chunk
-                if (wait_all(&bar_tma2, ck & 1)) { failed = true; break; }
+                wfail |= !tc::mbar_wait(&bar_tma2, ck & 1);
                 // per-token factors (the sign of Gamma_r is XORed into the factor's sign bit):
                 //   fast path  e1 = Gamma_r / 2^R,  e2 = 2^R / Gamma_r  (R = L_C / 2: middle of the range)
                 //   exact path e1 = Gamma_r,        e2 = Gamma_C / Gamma_r
@@ -651,7 +655,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
                 // the previous chunk's O / state MMA reads Y and P: wait for it before writing Y
                 if (ck > 0) {
-                    if (wait_all(&bar_c2, ph_c2)) { failed = true; break; }
+                    wfail |= !tc::mbar_wait(&bar_c2, ph_c2);
                     ph_c2 ^= 1u;
                     tc::tc_fence_after();
                 }
@@ -673,7 +677,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // hand the tiles to the issuer; the barrier also publishes the per-channel constants
             if (tid == 0) slow_flag_s = slow ? 1u : 0u;
             handoff(&bar_hap);
-            csync();
+            if (csync_or(wfail)) { failed = true; break; }
 
             // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact pairwise path
             if (!slow) {
@@ -681,7 +685,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 // C1, which overwrites the o accumulator and runs during the solve
                 stage_and_copy(ck > 0, slow);
                 handoff(&bar_hc1);             // issuer: o store of chunk c-1, then C1
-                if (wait_all(&bar_ap, ph_ap)) { failed = true; break; }
+                wfail |= !tc::mbar_wait(&bar_ap, ph_ap);
                 ph_ap ^= 1u;
                 tc::tc_fence_after();
                 // ---------------- P3: A (fp32, column-major) and P (hi/lo) out of TMEM
@@ -750,7 +754,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             }
             tc::tmem_ld_wait();
             tc::tc_fence_before();
-            csync();
+            if (csync_or(wfail)) { failed = true; break; }
 
             // ---------------- P4: T = (I + A)^{-1} Diag(beta): 16 x 16 diagonal blocks, then two
             // doubling levels. With L = I + A split into 2 x 2 blocks, L^{-1} has the lower-left
@@ -865,7 +869,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
 
             // ---------------- P5: -Z^T (from C1) -> TMEM A operand; U^T = V^T T^T - Z^T T^T
-            if (wait_all(&bar_c1, ph_c1)) { failed = true; break; }
+            wfail |= !tc::mbar_wait(&bar_c1, ph_c1);
             ph_c1 ^= 1u;
             tc::tc_fence_after();
             {
@@ -880,7 +884,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 tc::tmem_st32<16>(tl + TM_ZALO + 16 * hh, lo);
             }
             handoff(&bar_hu);                  // -Z^T: the issuer adds Z T^T
-            if (wait_all(&bar_u, ph_u)) { failed = true; break; }
+            wfail |= !tc::mbar_wait(&bar_u, ph_u);
             ph_u ^= 1u;
             tc::tc_fence_after();
 
@@ -902,6 +906,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             handoff(&bar_hc2);
         }
 
+        if (!failed && csync_or(wfail)) failed = true;
         // last chunk: its O / state MMAs, then its o tile (stored by the issuer)
         if (!failed && nchunks > 0) {
             if (wait_all(&bar_c2, ph_c2)) {
