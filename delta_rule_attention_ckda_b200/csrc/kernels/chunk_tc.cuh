@@ -811,8 +811,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // level 2 (32 -> 64): R = A[32:64, 0:32] X[0:32, 0:32], X[32:64, 0:32] = -X[32:64, 32:64] R.
             // T = X Diag(beta) is split into the MMA operand as soon as a block of X is final.
             {
-                // R: warp -> columns 4 w .. 4 w + 3, lane -> row; X[k][c] = 0 for k < c
-                const int cg = warp, r = lane;
+                // R: warp -> column group cg (columns 4 cg .. 4 cg + 3), lane -> row; X[k][c] = 0
+                // for k < c, so group cg runs 32 - 4 cg steps. Warps w and w + 4 share a
+                // scheduler: they take groups w and 7 - w (36 steps per scheduler).
+                const int cg = (warp < 4) ? warp : 11 - warp, r = lane;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
                 for (int k = 4 * cg; k < 32; ++k) {
