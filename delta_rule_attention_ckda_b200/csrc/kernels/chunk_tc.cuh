@@ -38,7 +38,7 @@
 // TMEM lanes: the fp32 state lives in TMEM for the whole sequence and never
 // round-trips HBM. Every product runs on tcgen05 with bf16 operands; operands that
 // are not raw bf16 inputs are split x = hi + lo (two bf16) and each product is the
-// three passes hi*hi + hi*lo + lo*hi (about 16 significant bits), which the fp32-state
+// three passes hi*hi + hi*lo + lo*hi (relative error about 2^-17), which the fp32-state
 // tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by TMA (no
 // multicast) with 128-byte swizzle; tokens past the end read as zero and get gate 1.
 //
@@ -128,13 +128,15 @@ __device__ __forceinline__ float ld_alpha_tile(const uint8_t* tile, int r, int c
     return *reinterpret_cast<const float*>(tile + off);
 }
 
-// (a, b) -> packed bf16 hi pair and packed bf16 lo pair, a + b exact to ~16 bits each.
+// (a, b) -> packed bf16 hi pair and packed bf16 lo pair with hi + lo = x to within
+// 2^-17 |x|: hi is x rounded to nearest, the remainder x - hi (exact in fp32) is truncated
+// to bf16 by taking its upper half. One conversion per pair; the conversion unit is the
+// scarce resource in the operand-splitting epilogues.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    const float2 hf = __bfloat1622float2(h);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
     hi = *reinterpret_cast<const uint32_t*>(&h);
-    lo = *reinterpret_cast<const uint32_t*>(&l);
+    const float la = a - __uint_as_float(hi << 16), lb = b - __uint_as_float(hi & 0xFFFF0000u);
+    lo = __byte_perm(__float_as_uint(la), __float_as_uint(lb), 0x7632);
 }
 
 // Split 8 fp32 values and store them as 16-byte chunk `ch` of row `row` (hi and lo tiles).

@@ -4,6 +4,8 @@ workloads fix (max-abs error <= tau * RMS of the oracle tensor; tau = 1e-4 for f
 q/k/v, 3e-3 for bf16 q/k/v with fp32 alpha, beta and state)."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -56,5 +58,7 @@ def check(name, got, ref, tau):
     scale = oracle.rms(ref)
     err = float(np.abs(got - ref).max()) if ref.size else 0.0
     bound = tau * scale
+    if os.environ.get("CKDA_PARITY_REPORT"):
+        print(f"[parity] {name}: max|err|/RMS = {err / scale if scale > 0 else 0.0:.3e} (bound {tau:g})")
     assert err <= bound, f"{name}: max|err| = {err:.3e} > {tau:g} * RMS ({scale:.3e}) = {bound:.3e}"
     return err / scale if scale > 0 else 0.0
