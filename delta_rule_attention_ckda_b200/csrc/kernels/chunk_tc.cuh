@@ -580,7 +580,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     const int r = 32 * hh + i;
                     const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
                     run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
-                    par |= (__float_as_uint(a) >> 31) << i;
+                    par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
                     L[i] = run;
                 }
                 par ^= par << 1;

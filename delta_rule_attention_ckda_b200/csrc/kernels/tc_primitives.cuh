@@ -62,38 +62,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
     return ok != 0;
 }
 
-// try_wait with a suspend-time hint: the thread sleeps up to `hint_ns` nanoseconds unless
-// the phase completes first (fewer polls from a thread that only waits).
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t phase, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.b32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
 // Wait until the barrier's phase with the given parity has completed. Gives up after
 // `limit` polls (each try_wait itself blocks for a hardware-defined time slice),
 // records kErrTimeout and returns false.
 constexpr uint32_t kSpinLimit = 1u << 22;
-constexpr uint32_t kSleepHintNs = 1000;          // waits of the MMA-issuer warp
-constexpr uint32_t kSleepLimit = 1u << 22;       // at most ~4 s at the hint
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = kSpinLimit) {
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, phase)) return true;
-    report_error(kErrTimeout);
-    return false;
-}
-
-// Same, sleeping between polls (for a thread with nothing else to do).
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t phase) {
-    for (uint32_t i = 0; i < kSleepLimit; ++i)
-        if (mbar_try_wait_sleep(bar, phase, kSleepHintNs)) return true;
     report_error(kErrTimeout);
     return false;
 }

@@ -61,6 +61,7 @@ def test_extreme_decay_takes_exact_path(ck):
     inp.alpha[0, 70:75, :, :40] = 1e-20         # chunk 1: L drops by ~330 in log2
     inp.alpha[0, 130, 0, :] = 0.0               # chunk 2: exact zeros (floored)
     inp.alpha[0, 131, 0, :] = -1e-35
+    inp.alpha[0, 140, 1, :8] = -0.0             # negative zero: sign taken as +
     inp.alpha[0, 200:230, 1, 5:9] = -0.02       # chunk 3: long fast decay, signed
     o, ST = run_chunk(ck, inp)
     assert torch.isfinite(o).all() and torch.isfinite(ST).all()
