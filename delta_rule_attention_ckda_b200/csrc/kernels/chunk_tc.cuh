@@ -107,7 +107,8 @@ constexpr uint32_t TM_D1 = 384;       // [A ; P] as two partial sums: X_hi Y_hi 
 constexpr uint32_t TM_DU = 384;       //   after the [A ; P] epilogue: U^T as two partial sums,
                                       //   (V^T - Z^T) T_hi^T | (V^T - Z^T) T_lo^T
 
-constexpr uint32_t kTmaBytes1 = 6 * 8192;   // k (2 bf16 boxes) + alpha (4 fp32 boxes)
+constexpr uint32_t kTmaBytes1a = 4 * 8192;  // alpha (4 fp32 boxes)
+constexpr uint32_t kTmaBytes1b = 2 * 8192;  // k (2 bf16 boxes)
 constexpr uint32_t kTmaBytes2 = 4 * 8192;   // q + v (2 bf16 boxes each)
 
 // Byte address (from tile base) of the 16-byte chunk `ch` (0..7) of row `row` in a
@@ -234,7 +235,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tma1, bar_tma2, bar_ap, bar_c1, bar_u, bar_c2;    // TMA / MMA completion
+    __shared__ uint64_t bar_tma1a, bar_tma1b, bar_tma2, bar_ap, bar_c1, bar_u, bar_c2;   // TMA / MMA completion
     __shared__ uint64_t bar_hap, bar_hc1, bar_hl2, bar_ht, bar_hu, bar_hc2, bar_hfin;  // compute -> issuer
     __shared__ uint64_t bar_ofree;                                              // issuer -> compute
     __shared__ uint32_t tmem_base_s, slow_flag_s;
@@ -262,7 +263,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
     if (tid == 0) {
-        tc::mbar_init(&bar_tma1, 1);
+        tc::mbar_init(&bar_tma1a, 1);
+        tc::mbar_init(&bar_tma1b, 1);
         tc::mbar_init(&bar_tma2, 1);
         tc::mbar_init(&bar_ap, 1);
         tc::mbar_init(&bar_c1, 1);
@@ -298,12 +300,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const uint32_t tm = tmem_base_s;
     const uint32_t tl = tm + lane_base;           // this warp's lane quarter
 
-    // inputs of a chunk arrive in two groups: k and alpha (their space frees up during the
-    // solve), then q and v (read by the U MMA)
-    auto issue_loads1 = [&](int t0) {
-        tc::mbar_arrive_expect_tx(&bar_tma1, kTmaBytes1);
-        for (int i = 0; i < 2; ++i) tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma1, 64 * i, h, t0, b);
-        for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma1, 32 * i, h, t0, b);
+    // inputs of a chunk arrive in three groups: alpha (its space frees up once the previous
+    // o tile is stored, early in the chunk before), k (its space holds A until the solve's
+    // second level), then q and v (read by the U MMA)
+    auto issue_loads1a = [&](int t0) {
+        tc::mbar_arrive_expect_tx(&bar_tma1a, kTmaBytes1a);
+        for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma1a, 32 * i, h, t0, b);
+    };
+    auto issue_loads1b = [&](int t0) {
+        tc::mbar_arrive_expect_tx(&bar_tma1b, kTmaBytes1b);
+        for (int i = 0; i < 2; ++i) tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma1b, 64 * i, h, t0, b);
     };
     auto issue_loads2 = [&](int t0) {
         tc::mbar_arrive_expect_tx(&bar_tma2, kTmaBytes2);
@@ -467,7 +473,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             };
             if (leader && nchunks > 0) {
-                issue_loads1(0);
+                issue_loads1a(0);
+                issue_loads1b(0);
                 issue_loads2(0);
             }
             __syncwarp();
@@ -490,14 +497,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         tc::bulk_commit();
                     }
                     issue_c1(sbase);
+                    // the next chunk's alpha, once the o tile has left the alpha space (its gate
+                    // cumulation runs while this chunk's U MMA does)
+                    if (ck + 1 < nchunks) {
+                        tc::bulk_wait_read0();
+                        issue_loads1a(t0 + C);
+                    }
                 }
                 __syncwarp();
-                // A consumed: the next chunk's k and alpha, once the o tile has left the alpha space
+                // A consumed: the next chunk's k
                 if (!wait1(&bar_hl2, par)) break;
-                if (leader && ck + 1 < nchunks) {
-                    tc::bulk_wait_read0();
-                    issue_loads1(t0 + C);
-                }
+                if (leader && ck + 1 < nchunks) issue_loads1b(t0 + C);
                 __syncwarp();
                 // T ready: the V part of U
                 if (!wait1(&bar_ht, par)) break;
@@ -561,70 +571,83 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // the schedule needs anyway, where all compute warps leave the loop together
         bool wfail = false;
 
+        // gate state of a chunk, computed one chunk ahead (while the previous chunk's U MMA runs):
+        // L[i] = log2 |prod a| from the start of this thread's half of the chunk, par bit i = the
+        // sign of the same product, Lofs = the first half's total (second-half threads), L_C and
+        // its sign over the whole chunk, and the exact-path decision
+        float L[32];
+        uint32_t par = 0, pC = 0;
+        float Lofs = 0.f, LC = 0.f;
+        bool slow = false;
+        // ---------------- P0: gate cumulation of chunk ckn (thread = channel m, tokens 32hh .. 32hh+31),
+        // the per-channel constants and the exact-path decision. True if a wait gave up.
+        auto gate_logs = [&](int ckn) -> bool {
+            const int nvalid = min(C, T - ckn * C);
+            wfail |= !tc::mbar_wait(&bar_tma1a, ckn & 1);
+            float run = 0.f;
+            par = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int r = 32 * hh + i;
+                const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
+                run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+                par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
+                L[i] = run;
+            }
+            par ^= par << 1;                      // prefix XOR of the sign bits
+            par ^= par << 2;
+            par ^= par << 4;
+            par ^= par << 8;
+            par ^= par << 16;
+            if (hh == 0) { sh_Lx[m] = run; sh_px[m] = par >> 31; }
+            if (csync_or(wfail)) return true;
+            // second half: offset by the first half's totals (kept apart from L[])
+            Lofs = 0.f;
+            LC = 0.f;
+            pC = 0;
+            int bad = 0;
+            if (hh == 1) {
+                Lofs = sh_Lx[m];
+                if (sh_px[m]) par = ~par;
+                LC = L[31] + Lofs;
+                pC = par >> 31;
+                sh_LC[m] = LC;
+                sh_pC[m] = pC;
+                bad = (-LC > kChunkRange);
+            }
+            slow = csync_or(bad);
+            if (hh == 0) {
+                LC = sh_LC[m];
+                pC = sh_pC[m];
+                sh_kp[m] = sh_kref[m];
+                if (!slow) {
+                    const float gref = exp2f(0.5f * LC);
+                    sh_fa[m] = gref;
+                    sh_fs[m] = gref;
+                    sh_kref[m] = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
+                } else {
+                    sh_fa[m] = 1.f;
+                    sh_fs[m] = (pC ? -1.f : 1.f) * exp2f(LC);
+                    sh_kref[m] = 1.f;
+                }
+            }
+            if (slow) {
+                float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
+            }
+            return false;
+        };
+
+        if (nchunks > 0 && gate_logs(0)) failed = true;
         for (int ck = 0; ck < nchunks && !failed; ++ck) {
             const int t0 = ck * C;
-            const int nvalid = min(C, T - t0);
             if (tid < C) sh_beta[tid] = beta_next;
-            wfail |= !tc::mbar_wait(&bar_tma1, ck & 1);
 
-            // ---------------- P1: gate cumulation (thread = channel m, tokens 32hh .. 32hh+31)
-            bool slow;
+            // ---------------- P1: gate factors (thread = channel m, tokens 32hh .. 32hh+31)
             {
-                // L[i]: log2 |prod a| from the start of this thread's half of the chunk;
-                // par bit i: sign of the same product (prefix XOR of the gates' sign bits)
-                float L[32];
-                uint32_t par = 0;
-                float run = 0.f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = 32 * hh + i;
-                    const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
-                    run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
-                    par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
-                    L[i] = run;
-                }
-                par ^= par << 1;
-                par ^= par << 2;
-                par ^= par << 4;
-                par ^= par << 8;
-                par ^= par << 16;
-                if (hh == 0) { sh_Lx[m] = run; sh_px[m] = par >> 31; }
-                if (csync_or(wfail)) { failed = true; break; }
-                // second half: offset by the first half's totals (kept apart from L[])
-                float Lofs = 0.f, LC = 0.f;
-                uint32_t pC = 0;
-                int bad = 0;
-                if (hh == 1) {
-                    Lofs = sh_Lx[m];
-                    if (sh_px[m]) par = ~par;
-                    LC = L[31] + Lofs;
-                    pC = par >> 31;
-                    sh_LC[m] = LC;
-                    sh_pC[m] = pC;
-                    bad = (-LC > kChunkRange);
-                }
-                slow = csync_or(bad);
-                if (hh == 0) {
-                    LC = sh_LC[m];
-                    pC = sh_pC[m];
-                    sh_kp[m] = sh_kref[m];
-                    if (!slow) {
-                        const float gref = exp2f(0.5f * LC);
-                        sh_fa[m] = gref;
-                        sh_fs[m] = gref;
-                        sh_kref[m] = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
-                    } else {
-                        sh_fa[m] = 1.f;
-                        sh_fs[m] = (pC ? -1.f : 1.f) * exp2f(LC);
-                        sh_kref[m] = 1.f;
-                    }
-                }
-                if (slow) {
-                    float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
-                }
-                // q and v of this chunk
+                // k, q and v of this chunk
+                wfail |= !tc::mbar_wait(&bar_tma1b, ck & 1);
                 wfail |= !tc::mbar_wait(&bar_tma2, ck & 1);
                 // per-token factors (the sign of Gamma_r is XORed into the factor's sign bit):
                 //   fast path  e1 = Gamma_r / 2^R,  e2 = 2^R / Gamma_r  (R = L_C / 2: middle of the range)
@@ -888,6 +911,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 tc::tmem_st32<16>(tl + TM_ZALO + 16 * hh, lo);
             }
             handoff(&bar_hu);                  // -Z^T: the issuer adds Z T^T
+            // the next chunk's gate cumulation runs while the U MMA does
+            if (ck + 1 < nchunks && gate_logs(ck + 1)) { failed = true; break; }
             wfail |= !tc::mbar_wait(&bar_u, ph_u);
             ph_u ^= 1u;
             tc::tc_fence_after();
