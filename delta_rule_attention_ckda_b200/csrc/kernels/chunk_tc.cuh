@@ -59,12 +59,15 @@ namespace ctc {
 constexpr int C = 64;        // chunk length
 constexpr int D = 128;       // d_k = d_v
 constexpr int NT = 256;      // compute threads (warpgroups 0 and 1)
-constexpr int NT_ALL = 384;  // + warpgroup 2, whose first warp issues every MMA, TMA load and o store
+constexpr int NT_ALL = 384;  // + warpgroup 2: TMEM epilogue warps, one per lane quarter; the
+                             //   first lane of its first warp issues C1, U, the state MMA and TMA
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64512); the
-// issuer warpgroup drops to 56 and the compute warpgroups rise to 224 (256 x 224 + 128 x 56).
-constexpr uint32_t kRegCompute = 224;
-constexpr uint32_t kRegIssuer = 56;
-static_assert(NT * kRegCompute + (NT_ALL - NT) * kRegIssuer <= NT_ALL * 168, "register split exceeds the launch");
+// epilogue warpgroup drops to 104 and the compute warpgroups rise to 200
+// (256 x 200 + 128 x 104 = 64512; per scheduler 2 x 200 + 104 <= 512).
+constexpr uint32_t kRegCompute = 200;
+constexpr uint32_t kRegEpi = 104;
+static_assert(NT * kRegCompute + (NT_ALL - NT) * kRegEpi <= NT_ALL * 168, "register split exceeds the launch");
+static_assert(2 * kRegCompute + kRegEpi <= 512, "register split exceeds a scheduler's file");
 
 // log2-domain limits of the single-reference factorisation
 constexpr float kLgFloor = -100.f;    // floor of log2|a| per token (a = 0 allowed)
@@ -184,6 +187,26 @@ __device__ __forceinline__ bool csync_or(bool p) {
     return r != 0;
 }
 
+// Barrier among the 128 threads of the epilogue warpgroup (named barrier 2), with an OR.
+__device__ __forceinline__ bool esync_or(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred a, q;\n\t"
+        "setp.ne.u32 a, %1, 0;\n\t"
+        "bar.red.or.pred q, 2, 128, a;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p)
+        : "memory");
+    return r != 0;
+}
+
+// Split 16 fp32 values (consecutive K positions) into packed bf16 pairs (TMEM A operand).
+__device__ __forceinline__ void split_pack16(const float (&x)[16], uint32_t (&hi)[8], uint32_t (&lo)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) split2(x[2 * e], x[2 * e + 1], hi[e], lo[e]);
+}
+
 // Every compute thread waits on the barrier; true if any of them timed out.
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
     const bool ok = tc::mbar_wait(bar, parity);
@@ -236,9 +259,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar_tma1a, bar_tma1b, bar_tma2, bar_ap, bar_c1, bar_u, bar_c2;   // TMA / MMA completion
-    __shared__ uint64_t bar_hap, bar_hc1, bar_hl2, bar_ht, bar_hu, bar_hc2, bar_hfin;  // compute -> issuer
-    __shared__ uint64_t bar_ofree;                                              // issuer -> compute
-    __shared__ uint32_t tmem_base_s, slow_flag_s;
+    // compute -> epilogue group: per-channel constants of the chunk (hk), X / Y tiles written and
+    // the alpha space free (hap), T written and A consumed (ht)
+    __shared__ uint64_t bar_hk, bar_hap, bar_ht;
+    __shared__ uint32_t tmem_base_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
     float* sh_fa = sh_beta + 64;            // [128] g_ref (operand copy = S g_ref)
@@ -270,14 +294,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::mbar_init(&bar_c1, 1);
         tc::mbar_init(&bar_u, 1);
         tc::mbar_init(&bar_c2, 1);
+        tc::mbar_init(&bar_hk, NT);
         tc::mbar_init(&bar_hap, NT);
-        tc::mbar_init(&bar_hc1, NT);
-        tc::mbar_init(&bar_hl2, NT);
         tc::mbar_init(&bar_ht, NT);
-        tc::mbar_init(&bar_hu, NT);
-        tc::mbar_init(&bar_hc2, NT);
-        tc::mbar_init(&bar_hfin, NT);
-        tc::mbar_init(&bar_ofree, 1);
         tc::fence_mbar_init();
         tc::prefetch_tensormap(&map_k);
         tc::prefetch_tensormap(&map_q);
@@ -322,76 +341,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         return (tid < C && t0 + tid < T) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
     };
     float beta_next = load_beta(0);
-
-    // o rows of a finished chunk: TMEM -> shared tile [64 tok][128] fp32 in the alpha space.
-    // The issuer warp stores the tile by TMA once the compute threads have handed it over.
-    auto stage_o = [&]() {
-        float ov[32];
-        tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
-        tc::tmem_ld_wait();
-        float* ot = reinterpret_cast<float*>(sm + SM_OT);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
-        tc::fence_proxy_async_smem();
-    };
-    // state copy into the C1 operand and rescale of the accumulator, with the previous
-    // chunk's o tile staged first (the next TMEM load is in flight while the previous block
-    // is processed). The accumulator
-    // holds S Diag(1/kappa_prev): first S = acc kappa_prev, then the operand S g_ref and the
-    // new accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
-    // for fast-decaying channels although each factor and each result is in range.
-    auto stage_and_copy = [&](bool with_o, bool slow_chunk) {
-        float sv[2][32];
-        tc::tmem_ld32<32>(tl + TM_S + 64 * hh, sv[0]);
-        if (with_o) {
-            float ov[32];
-            tc::tmem_ld32<32>(tl + TM_O + 32 * hh, ov);
-            tc::tmem_ld_wait();
-            float* ot = reinterpret_cast<float*>(sm + SM_OT);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ot[(32 * hh + i) * D + m] = ov[i];
-        }
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-            const int c0 = 64 * hh + 32 * cb;
-            tc::tmem_ld_wait();
-            if (cb == 0) tc::tmem_ld32<32>(tl + TM_S + 64 * hh + 32, sv[1]);
-            float z[32];
-            const float4* kp4 = reinterpret_cast<const float4*>(sh_kp + c0);
-            const float4* fa4 = reinterpret_cast<const float4*>(sh_fa + c0);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 kk = kp4[i];
-                const float4 f = fa4[i];
-                sv[cb][4 * i] *= kk.x;
-                sv[cb][4 * i + 1] *= kk.y;
-                sv[cb][4 * i + 2] *= kk.z;
-                sv[cb][4 * i + 3] *= kk.w;
-                z[4 * i] = sv[cb][4 * i] * f.x;
-                z[4 * i + 1] = sv[cb][4 * i + 1] * f.y;
-                z[4 * i + 2] = sv[cb][4 * i + 2] * f.z;
-                z[4 * i + 3] = sv[cb][4 * i + 3] * f.w;
-            }
-            uint32_t hi[16], lo[16];
-            split_pack32(z, hi, lo);
-            tc::tmem_st32<16>(tl + TM_SAHI + c0 / 2, hi);
-            tc::tmem_st32<16>(tl + TM_SALO + c0 / 2, lo);
-            if (!slow_chunk) {
-                tmem_st_f32x32(tl + TM_S + c0, z);        // fast path: fs == fa
-            } else {
-                const float4* fs4 = reinterpret_cast<const float4*>(sh_fs + c0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 f = fs4[i];
-                    sv[cb][4 * i] *= f.x;
-                    sv[cb][4 * i + 1] *= f.y;
-                    sv[cb][4 * i + 2] *= f.z;
-                    sv[cb][4 * i + 3] *= f.w;
-                }
-                tmem_st_f32x32(tl + TM_S + c0, sv[cb]);
-            }
-        }
-    };
 
     // C1: [O^T | Z^T] = (S0 Diag g)^T [(q e1)^T | (k e1)^T]  (3 passes), after the state copy
     auto issue_c1 = [&](uint32_t sb_) {
@@ -462,109 +411,185 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const int nchunks = (T + C - 1) / C;
 
     if (warp >= NT / 32) {
-        // ================================================================ issuer warpgroup
-        setmaxnreg_dec<kRegIssuer>();
-        if (warp == NT / 32) {
-            const bool leader = (lane == 0);
-            // one thread polls, the whole warp learns the outcome (the warp stays converged)
-            auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
-                bool ok = true;
-                if (leader) ok = tc::mbar_wait(bar, parity);
-                return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            };
-            if (leader && nchunks > 0) {
-                issue_loads1a(0);
-                issue_loads1b(0);
-                issue_loads2(0);
+        // ================================================================ epilogue warpgroup
+        // Warp 8 + q owns TMEM lane quarter q (d_v rows 32q .. 32q + 31) for all TMEM epilogues
+        // of the state chain: the state copy, the o tile, -Z^T and U^T. Lane 0 of warp 8 also
+        // issues C1, U, the O / state MMA, every TMA load and the o store. Each thread waits on
+        // the mbarriers for itself (bounded); the group synchronises on named barrier 2, where
+        // a timeout anywhere stops every epilogue warp together.
+        setmaxnreg_dec<kRegEpi>();
+        const int qe = warp & 3;
+        const int me = qe * 32 + lane;
+        const uint32_t te = tm + ((uint32_t)(qe * 32) << 16);
+        const bool leader = (warp == NT / 32) && (lane == 0);
+        bool efail = false;
+        // before the leader issues an MMA that reads what the group wrote (TMEM and shared)
+        auto epi_publish = [&]() {
+            tc::tmem_st_wait();
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+        };
+        // o rows of a finished chunk: TMEM -> shared tile [64 tok][128] fp32 in the alpha space
+        auto stage_o = [&]() {
+            float* ot = reinterpret_cast<float*>(sm + SM_OT);
+#pragma unroll
+            for (int b16 = 0; b16 < 4; ++b16) {
+                float ov[16];
+                tc::tmem_ld32<16>(te + TM_O + 16 * b16, ov);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ot[(16 * b16 + i) * D + me] = ov[i];
             }
-            __syncwarp();
-            for (int ck = 0; ck < nchunks; ++ck) {
-                const uint32_t par = (uint32_t)ck & 1u;
-                const int t0 = ck * C;
-                // X, Y tiles written: [A ; P], unless the chunk takes the exact path
-                if (!wait1(&bar_hap, par)) break;
-                if (leader && slow_flag_s == 0u) {
-                    tc::tc_fence_after();
-                    issue_ap(sbase);
-                }
-                __syncwarp();
-                // previous chunk's o tile staged and state copied: store o, then C1
-                if (!wait1(&bar_hc1, par)) break;
-                if (leader) {
-                    tc::tc_fence_after();
-                    if (ck > 0) {
-                        tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
-                        tc::bulk_commit();
-                    }
-                    issue_c1(sbase);
-                    // the next chunk's alpha, once the o tile has left the alpha space (its gate
-                    // cumulation runs while this chunk's U MMA does)
-                    if (ck + 1 < nchunks) {
-                        tc::bulk_wait_read0();
-                        issue_loads1a(t0 + C);
-                    }
-                }
-                __syncwarp();
-                // A consumed: the next chunk's k
-                if (!wait1(&bar_hl2, par)) break;
-                if (leader && ck + 1 < nchunks) issue_loads1b(t0 + C);
-                __syncwarp();
-                // T ready: the V part of U
-                if (!wait1(&bar_ht, par)) break;
-                if (leader) {
-                    tc::tc_fence_after();
-                    issue_uv(sbase);
-                }
-                __syncwarp();
-                // -Z^T ready: the Z part
-                if (!wait1(&bar_hu, par)) break;
-                if (leader) {
-                    tc::tc_fence_after();
-                    issue_uz(sbase);
-                }
-                __syncwarp();
-                // V and T consumed: the next chunk's q and v
-                if (!wait1(&bar_u, par)) break;
-                if (leader && ck + 1 < nchunks) issue_loads2(t0 + C);
-                __syncwarp();
-                // U^T ready: O and state MMAs
-                if (!wait1(&bar_hc2, par)) break;
-                if (leader) {
-                    tc::tc_fence_after();
-                    issue_c2(sbase);
-                }
-                __syncwarp();
-            }
-            // last o tile: free the staging space, then store what the compute warps stage
-            if (leader) {
-                tc::bulk_wait_read0();
-                tc::mbar_arrive(&bar_ofree);
-            }
-            __syncwarp();
-            if (nchunks > 0 && wait1(&bar_hfin, 0) && leader) {
-                tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, (nchunks - 1) * C, b);
-                tc::bulk_commit();
-            }
-            if (leader) tc::bulk_wait0();
-            __syncwarp();
-        }
-    } else {
-        // ================================================================ compute warpgroups
-        setmaxnreg_inc<kRegCompute>();
+        };
+
         // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
         {
             const size_t sb = (size_t)bh * D * D;
-            for (int cb = 0; cb < 2; ++cb) {
-                float x[32];
-                const int c0 = 64 * hh + 32 * cb;
+#pragma unroll 1
+            for (int cb = 0; cb < 8; ++cb) {
+                uint32_t x[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = S0 ? S0[sb + (size_t)(c0 + i) * D + m] : 0.f;
-                tmem_st_f32x32(tl + TM_S + c0, x);
+                for (int i = 0; i < 16; ++i) x[i] = __float_as_uint(S0 ? S0[sb + (size_t)(16 * cb + i) * D + me] : 0.f);
+                tc::tmem_st32<16>(te + TM_S + 16 * cb, x);
             }
             tc::tmem_st_wait();
         }
-
-        uint32_t ph_ap = 0, ph_c1 = 0, ph_u = 0, ph_c2 = 0;
+        if (leader && nchunks > 0) {
+            issue_loads1a(0);
+            issue_loads1b(0);
+            issue_loads2(0);
+        }
+        int ck = 0;
+        for (; ck < nchunks; ++ck) {
+            const uint32_t par = (uint32_t)ck & 1u;
+            const int t0 = ck * C;
+            // ---------------- E1: state copy. The accumulator holds S Diag(1/kappa_prev):
+            // S = acc kappa_prev, then the operand S g_ref (split into TMEM) and the new
+            // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
+            // for fast-decaying channels although each factor and each result is in range.
+            efail |= !tc::mbar_wait(&bar_hk, par);             // this chunk's constants
+            if (ck > 0) efail |= !tc::mbar_wait(&bar_c2, par ^ 1u);
+            tc::tc_fence_after();
+            {
+                float sv[2][16];
+                tc::tmem_ld32<16>(te + TM_S, sv[0]);
+#pragma unroll
+                for (int cb = 0; cb < 8; ++cb) {
+                    float (&cur)[16] = sv[cb & 1];
+                    tc::tmem_ld_wait();
+                    if (cb + 1 < 8) tc::tmem_ld32<16>(te + TM_S + 16 * (cb + 1), sv[(cb + 1) & 1]);
+                    float z[16];
+                    uint32_t snew[16];
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const float4 kk = reinterpret_cast<const float4*>(sh_kp + 16 * cb)[i4];
+                        const float4 fa = reinterpret_cast<const float4*>(sh_fa + 16 * cb)[i4];
+                        const float4 fs = reinterpret_cast<const float4*>(sh_fs + 16 * cb)[i4];
+                        const float s0 = cur[4 * i4] * kk.x, s1 = cur[4 * i4 + 1] * kk.y;
+                        const float s2 = cur[4 * i4 + 2] * kk.z, s3 = cur[4 * i4 + 3] * kk.w;
+                        z[4 * i4] = s0 * fa.x;
+                        z[4 * i4 + 1] = s1 * fa.y;
+                        z[4 * i4 + 2] = s2 * fa.z;
+                        z[4 * i4 + 3] = s3 * fa.w;
+                        snew[4 * i4] = __float_as_uint(s0 * fs.x);
+                        snew[4 * i4 + 1] = __float_as_uint(s1 * fs.y);
+                        snew[4 * i4 + 2] = __float_as_uint(s2 * fs.z);
+                        snew[4 * i4 + 3] = __float_as_uint(s3 * fs.w);
+                    }
+                    uint32_t hi[8], lo[8];
+                    split_pack16(z, hi, lo);
+                    tc::tmem_st32<8>(te + TM_SAHI + 8 * cb, hi);
+                    tc::tmem_st32<8>(te + TM_SALO + 8 * cb, lo);
+                    tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
+                }
+            }
+            // the previous chunk's o rows, once the gate (or the exact path) is done with the
+            // alpha space
+            efail |= !tc::mbar_wait(&bar_hap, par);
+            if (ck > 0) stage_o();
+            epi_publish();
+            if (esync_or(efail)) break;
+            // leader: o store, C1 (runs while the compute warps solve), the next chunk's alpha
+            if (leader) {
+                tc::tc_fence_after();
+                if (ck > 0) {
+                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
+                    tc::bulk_commit();
+                }
+                issue_c1(sbase);
+                if (ck + 1 < nchunks) {
+                    tc::bulk_wait_read0();
+                    issue_loads1a(t0 + C);
+                }
+            }
+            // ---------------- E2: -Z^T -> TMEM operand of the U MMA
+            efail |= !tc::mbar_wait(&bar_c1, par);
+            tc::tc_fence_after();
+#pragma unroll
+            for (int b16 = 0; b16 < 4; ++b16) {
+                float z[16];
+                tc::tmem_ld32<16>(te + TM_Z + 16 * b16, z);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) z[i] = -z[i];
+                uint32_t hi[8], lo[8];
+                split_pack16(z, hi, lo);
+                tc::tmem_st32<8>(te + TM_ZAHI + 8 * b16, hi);
+                tc::tmem_st32<8>(te + TM_ZALO + 8 * b16, lo);
+            }
+            epi_publish();
+            if (esync_or(efail)) break;
+            // leader: once T is written (and A consumed): the next chunk's k, then U
+            if (leader) {
+                efail |= !tc::mbar_wait(&bar_ht, par);
+                tc::tc_fence_after();
+                if (ck + 1 < nchunks) issue_loads1b(t0 + C);
+                issue_uv(sbase);
+                issue_uz(sbase);
+            }
+            // ---------------- E3: U^T -> TMEM operand of the O / state MMA
+            efail |= !tc::mbar_wait(&bar_u, par);
+            tc::tc_fence_after();
+            if (leader && ck + 1 < nchunks) issue_loads2(t0 + C);      // V and T consumed
+#pragma unroll
+            for (int b16 = 0; b16 < 4; ++b16) {
+                float u[16], u2[16];
+                tc::tmem_ld32<16>(te + TM_DU + 16 * b16, u);
+                tc::tmem_ld32<16>(te + TM_DU + 64 + 16 * b16, u2);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) u[i] += u2[i];
+                uint32_t hi[8], lo[8];
+                split_pack16(u, hi, lo);
+                tc::tmem_st32<8>(te + TM_UAHI + 8 * b16, hi);
+                tc::tmem_st32<8>(te + TM_UALO + 8 * b16, lo);
+            }
+            epi_publish();
+            if (esync_or(efail)) break;
+            if (leader) {
+                tc::tc_fence_after();
+                issue_c2(sbase);
+            }
+        }
+        // last chunk's o rows, once its O MMA is done and the previous o tile has been stored
+        if (ck == nchunks && nchunks > 0) {
+            efail |= !tc::mbar_wait(&bar_c2, (uint32_t)(nchunks - 1) & 1u);
+            tc::tc_fence_after();
+            if (leader) tc::bulk_wait_read0();
+            if (!esync_or(efail)) {
+                stage_o();
+                epi_publish();
+                if (!esync_or(false) && leader) {
+                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, (nchunks - 1) * C, b);
+                    tc::bulk_commit();
+                }
+            }
+        }
+        if (leader) tc::bulk_wait0();
+    } else {
+        // ================================================================ compute warpgroups
+        setmaxnreg_inc<kRegCompute>();
+        uint32_t ph_ap = 0, ph_c1 = 0, ph_c2 = 0;
         bool failed = false;
         // a bounded mbarrier wait that gave up: every thread waits for itself (the wait
         // acquires what the TMA or MMA wrote) and the flag is OR-reduced at the next barrier
@@ -636,6 +661,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
             }
+            handoff(&bar_hk);                     // the epilogue group copies the state with them
             return false;
         };
 
@@ -649,6 +675,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 // k, q and v of this chunk
                 wfail |= !tc::mbar_wait(&bar_tma1b, ck & 1);
                 wfail |= !tc::mbar_wait(&bar_tma2, ck & 1);
+                // the previous chunk's C1 reads X: wait for it before overwriting
+                if (ck > 0) {
+                    wfail |= !tc::mbar_wait(&bar_c1, ph_c1);
+                    ph_c1 ^= 1u;
+                }
                 // per-token factors (the sign of Gamma_r is XORed into the factor's sign bit):
                 //   fast path  e1 = Gamma_r / 2^R,  e2 = 2^R / Gamma_r  (R = L_C / 2: middle of the range)
                 //   exact path e1 = Gamma_r,        e2 = Gamma_C / Gamma_r
@@ -699,17 +730,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     }
                 }
             }
-            // hand the tiles to the issuer; the barrier also publishes the per-channel constants
-            if (tid == 0) slow_flag_s = slow ? 1u : 0u;
-            handoff(&bar_hap);
+            // X, Y tiles written and the alpha space free (exact path: after its pairwise
+            // evaluation): the epilogue group stages the previous o tile and issues C1
+            if (!slow) handoff(&bar_hap);
+            else {
+                tc::fence_proxy_async_smem();
+                tc::tc_fence_before();
+            }
             if (csync_or(wfail)) { failed = true; break; }
 
             // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact pairwise path
             if (!slow) {
-                // while the MMA runs: the previous chunk's o tile and this chunk's state copy, then
-                // C1, which overwrites the o accumulator and runs during the solve
-                stage_and_copy(ck > 0, slow);
-                handoff(&bar_hc1);             // issuer: o store of chunk c-1, then C1
+                // one compute thread issues the [P ; A] MMA; every compute warp waits for it
+                if (tid == 0) {
+                    tc::tc_fence_after();
+                    issue_ap(sbase);
+                }
                 wfail |= !tc::mbar_wait(&bar_ap, ph_ap);
                 ph_ap ^= 1u;
                 tc::tc_fence_after();
@@ -774,8 +810,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         *reinterpret_cast<uint16_t*>(sm + SM_PLO + offp) = (uint16_t)(lpair & 0xffffu);
                     }
                 }
-                stage_and_copy(ck > 0, slow);
-                handoff(&bar_hc1);
+                handoff(&bar_hap);
             }
             tc::tmem_ld_wait();
             tc::tc_fence_before();
@@ -867,7 +902,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
                 // A (k-tile space) is consumed: the issuer loads the next chunk's k and alpha
                 // once the o tile has left the alpha space
-                tc::mbar_arrive(&bar_hl2);
                 csync();
                 // X[32:64, 0:32]: thread -> row 32 + r2, columns 4 c4 .. 4 c4 + 3, straight into T.
                 // X[32 + r2][32 + mm] is zero for mm > r2: warps 0-3 hold rows r2 < 16.
@@ -895,60 +929,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
             if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
 
-            // ---------------- P5: -Z^T (from C1) -> TMEM A operand; U^T = V^T T^T - Z^T T^T
-            wfail |= !tc::mbar_wait(&bar_c1, ph_c1);
-            ph_c1 ^= 1u;
-            tc::tc_fence_after();
-            {
-                float z[32];
-                tc::tmem_ld32<32>(tl + TM_Z + 32 * hh, z);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) z[i] = -z[i];
-                uint32_t hi[16], lo[16];
-                split_pack32(z, hi, lo);
-                tc::tmem_st32<16>(tl + TM_ZAHI + 16 * hh, hi);
-                tc::tmem_st32<16>(tl + TM_ZALO + 16 * hh, lo);
-            }
-            handoff(&bar_hu);                  // -Z^T: the issuer adds Z T^T
-            // the next chunk's gate cumulation runs while the U MMA does
+            // the next chunk's gate cumulation, while the epilogue group and the tensor cores
+            // finish this chunk's state chain
             if (ck + 1 < nchunks && gate_logs(ck + 1)) { failed = true; break; }
-            wfail |= !tc::mbar_wait(&bar_u, ph_u);
-            ph_u ^= 1u;
-            tc::tc_fence_after();
-
-            // ---------------- P8: U^T -> TMEM A operand (hi / lo)
-            {
-                float u[32], u2[32];
-                tc::tmem_ld32<32>(tl + TM_DU + 32 * hh, u);
-                tc::tmem_ld32<32>(tl + TM_DU + 64 + 32 * hh, u2);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) u[i] += u2[i];
-                uint32_t hi[16], lo[16];
-                split_pack32(u, hi, lo);
-                tc::tmem_st32<16>(tl + TM_UAHI + 16 * hh, hi);
-                tc::tmem_st32<16>(tl + TM_UALO + 16 * hh, lo);
-            }
-
-            // ---------------- P9: O^T += U^T P^T ;  acc += U^T (k e2), issued by the issuer warp
-            handoff(&bar_hc2);
         }
 
         if (!failed && csync_or(wfail)) failed = true;
-        // last chunk: its O / state MMAs, then its o tile (stored by the issuer)
+        // last chunk's state MMA
         if (!failed && nchunks > 0) {
-            if (wait_all(&bar_c2, ph_c2)) {
-                failed = true;
-            } else {
-                tc::tc_fence_after();
-                if (wait_all(&bar_ofree, 0)) {          // the previous o tile has left the staging space
-                    failed = true;
-                } else {
-                    stage_o();
-                    handoff(&bar_hfin);
-                }
-            }
+            if (wait_all(&bar_c2, ph_c2)) failed = true;
+            else tc::tc_fence_after();
         }
 
         // final state: S = acc Diag(kappa_last)
