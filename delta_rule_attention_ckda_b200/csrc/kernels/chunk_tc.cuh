@@ -62,10 +62,10 @@ constexpr int NT = 256;      // compute threads (warpgroups 0 and 1)
 constexpr int NT_ALL = 384;  // + warpgroup 2: TMEM epilogue warps, one per lane quarter; the
                              //   first lane of its first warp issues C1, U, the state MMA and TMA
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 = 64512); the
-// epilogue warpgroup drops to 104 and the compute warpgroups rise to 200
-// (256 x 200 + 128 x 104 = 64512; per scheduler 2 x 200 + 104 <= 512).
-constexpr uint32_t kRegCompute = 200;
-constexpr uint32_t kRegEpi = 104;
+// epilogue warpgroup drops to 120 and the compute warpgroups rise to 192
+// (256 x 192 + 128 x 120 = 64512; per scheduler 2 x 192 + 120 <= 512).
+constexpr uint32_t kRegCompute = 192;
+constexpr uint32_t kRegEpi = 120;
 static_assert(NT * kRegCompute + (NT_ALL - NT) * kRegEpi <= NT_ALL * 168, "register split exceeds the launch");
 static_assert(2 * kRegCompute + kRegEpi <= 512, "register split exceeds a scheduler's file");
 
