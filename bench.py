@@ -26,6 +26,7 @@ import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+from delta_rule_attention_ckda_b200.replicas import aggregate_throughput  # noqa: E402
 
 METRIC = "CKDA fwd tokens/s at H=16,d=128,T=4096; % of tensor-core/HBM roofline"
 WORKLOAD = dict(B=8, T=4096, H=16, dk=128, dv=128)
@@ -172,16 +173,6 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x, world):
-    import torch
-    import torch.distributed as dist
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 # ----------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(inp, n_seq, threads=None):
@@ -319,9 +310,8 @@ def ours_arm(args):
     clocks = sampler.stop()
     if ck.get_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
-    secs = max_over_ranks(secs, world)
-    tokens = B * T * world * args.steps
-    value = tokens / secs
+    # replicas: every rank ran its own batch; whole-job tokens over the slowest rank's time
+    value, secs = aggregate_throughput(B * T * args.steps, secs, world, device="cuda")
     per_launch = secs / args.steps
     alg_bytes = B * T * H * BYTES_PER_TOKEN_HEAD + B * H * dk * dv * 4
     hbm, src = peaks()
@@ -378,10 +368,10 @@ def e2e_measure(ck, inp, dev, stream, world, args):
     n = max(3, min(args.steps, 5))
     barrier(world)
     secs = time_launches(step, n, stream)
-    secs = max_over_ranks(secs, world)
+    value, secs = aggregate_throughput(B * T * n, secs, world, device="cuda")
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, hb))
     d2h = ho.numel() * 4 + hS.numel() * 4
-    return {"value": B * T * world * n / secs, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n}
 
 
@@ -407,13 +397,13 @@ def decode_measure(ck, dev, stream, world):
 
     secs = time_launches(one, calls, stream)
     assert ck.get_device_error() == 0
-    secs = max_over_ranks(secs, world)
+    tok_s, secs = aggregate_throughput(N * calls, secs, world, device="cuda")
     per = secs / calls
     bytes_call = N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4)
     hbm, src = peaks()
     gbs = bytes_call / per / 1e9
     return {"workload": "decode N=256 H=16 d=128 fp32 state, 1024 calls", "us_per_call": per * 1e6,
-            "tokens_per_s": N * world / per, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
+            "tokens_per_s": tok_s, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
                                                          "unit": "GB/s", "frac": gbs / hbm,
                                                          "alg_bytes_per_launch": bytes_call,
                                                          "kernel": "decode128", "traffic": committed_traffic("decode128")},
