@@ -333,6 +333,8 @@ def ours_arm(args):
                        "state": "S0 = 0 (not read), S_T written"},
             "roofline": roof, "gpu_launches": args.steps, "clocks": clocks}
 
+    if not args.no_extras:
+        line["kda"] = kda_measure(ck, q, k, v, a, b, o, ST, stream, world, args.steps, value)
     if not args.no_e2e:
         line["e2e"] = e2e_measure(ck, inp, dev, stream, world, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -345,6 +347,29 @@ def ours_arm(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def kda_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, ckda_value):
+    """The same layer step with the gate in KDA's form: g = ln |alpha| (the same
+    magnitudes, never negative), through the log-gate mode of the same kernels. Reports
+    CKDA's throughput over KDA's, the comparison the pages make for the signed gate."""
+    import torch
+    B, T, H, dk = q.shape
+    g = torch.log(a.abs())
+
+    def step():
+        ck.chunk_fwd(q, k, v, g, b, None, o=o, S_T=ST, gate="log")
+
+    for _ in range(3):
+        step()
+    assert ck.get_device_error() == 0
+    barrier(world)
+    secs = time_launches(step, steps, stream)
+    assert ck.get_device_error() == 0
+    value, secs = aggregate_throughput(B * T * steps, secs, world, device="cuda")
+    return {"workload": "layer, gate given as g = ln|alpha| (non-negative gate, KDA form)",
+            "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * secs / steps,
+            "ckda_over_kda": ckda_value / value, "gpu_launches": steps}
 
 
 def e2e_measure(ck, inp, dev, stream, world, args):

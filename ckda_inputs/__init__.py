@@ -91,6 +91,10 @@ def _gate(kind: str, shape, g: torch.Generator) -> torch.Tensor:
         return torch.tanh(1.5 * noise)
     if kind == "tanh15":
         return torch.tanh(1.5 + noise)
+    if kind == "log15":
+        # the layer gate's magnitudes in the log form a non-negative (KDA) gate takes:
+        # this tensor holds g = ln |tanh(1.5 + N)| <= 0, the input of the log-gate mode
+        return torch.log(torch.tanh(1.5 + noise).abs())
     if kind == "signmag":
         # the noise draw is kept so the draw order matches the other kinds
         sign = torch.where(torch.rand(shape, generator=g) < 0.5, -1.0, 1.0)

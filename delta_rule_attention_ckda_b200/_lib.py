@@ -52,6 +52,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_chunk_fwd.restype = i
     lib.ckda_recurrent_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 6 + [vp]
     lib.ckda_recurrent_fwd.restype = i
+    lib.ckda_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp, sz, vp]
+    lib.ckda_chunk_fwd_ex.restype = i
+    lib.ckda_recurrent_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp]
+    lib.ckda_recurrent_fwd_ex.restype = i
     lib.ckda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 5 + [vp]
     lib.ckda_decode_step.restype = i
     lib.ckda_get_device_error.argtypes = [vp]
@@ -123,10 +127,20 @@ def _fwd_common(q, k, v, alpha, beta, S0, o, S_T):
     return B, T, H, dk, dv, _dt(q), o
 
 
+GATES = {"signed": 0, "log": 1}       # ckda_gate_t: alpha in [-1,1], or g = ln(alpha) (KDA form)
+
+
+def _gate(gate: str) -> int:
+    if gate not in GATES:
+        raise ValueError(f"gate must be one of {sorted(GATES)}, got {gate!r}")
+    return GATES[gate]
+
+
 def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
-              workspace=None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """ckda_chunk_fwd. Returns (o, S_T). Allocates o / S_T / workspace with torch when
-    not given (the library itself never allocates)."""
+              workspace=None, stream=None, gate="signed") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """ckda_chunk_fwd_ex. Returns (o, S_T). `alpha` is the gate in the form `gate` names:
+    "signed" (alpha in [-1,1], CKDA) or "log" (g = ln(alpha) of a non-negative gate, KDA).
+    Allocates o / S_T / workspace with torch when not given (the library never allocates)."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
     if S_T is None and want_state:
         S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
@@ -135,21 +149,22 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=Tru
     if need and workspace is None:
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.ckda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o),
-                            _ptr(S_T), B, T, H, dk, dv, dt, _ptr(workspace), wbytes, _stream(stream))
-    _raise(st, "ckda_chunk_fwd")
+    st = lib.ckda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o),
+                               _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate), _ptr(workspace), wbytes,
+                               _stream(stream))
+    _raise(st, "ckda_chunk_fwd_ex")
     return o, S_T
 
 
 def recurrent_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
-                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """ckda_recurrent_fwd (fp32 SIMT token-by-token kernel). Returns (o, S_T)."""
+                  stream=None, gate="signed") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """ckda_recurrent_fwd_ex (fp32 SIMT token-by-token kernel). Returns (o, S_T)."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
     if S_T is None and want_state:
         S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
-    st = load().ckda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
-                                   _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _stream(stream))
-    _raise(st, "ckda_recurrent_fwd")
+    st = load().ckda_recurrent_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                      _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate), _stream(stream))
+    _raise(st, "ckda_recurrent_fwd_ex")
     return o, S_T
 
 

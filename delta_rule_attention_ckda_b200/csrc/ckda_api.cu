@@ -35,7 +35,7 @@ ckda_status_t copy_state(const float* S0, float* S_T, size_t n, cudaStream_t st)
     return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
-template <typename TIn>
+template <typename TIn, bool kLogGate>
 ckda_status_t launch_recurrent(const TIn* q, const TIn* k, const TIn* v, const float* alpha,
                                const float* beta, const float* S0, float* o, float* S_T,
                                int B, int T, int H, int dk, int dv, cudaStream_t st) {
@@ -46,7 +46,7 @@ ckda_status_t launch_recurrent(const TIn* q, const TIn* k, const TIn* v, const f
     dim3 grid((unsigned)seqs, (unsigned)((dv + cols_per_cta - 1) / cols_per_cta));
     dim3 block((unsigned)cols_per_cta);
 #define CKDA_LAUNCH_REC(DKT)                                                                  \
-    ckda::recurrent_fwd_kernel<DKT, TIn><<<grid, block, 0, st>>>(q, k, v, alpha, beta, S0, o, \
+    ckda::recurrent_fwd_kernel<DKT, TIn, kLogGate><<<grid, block, 0, st>>>(q, k, v, alpha, beta, S0, o, \
                                                                   S_T, T, H, dk, dv, cols_per_cta)
     if (dk <= 16) CKDA_LAUNCH_REC(16);
     else if (dk <= 32) CKDA_LAUNCH_REC(32);
@@ -101,28 +101,45 @@ size_t ckda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_
     return ckda::chunk_tc_workspace_bytes(B, T, H, dk, dv);
 }
 
-ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const void* v,
-                                 const float* alpha, const float* beta, const float* S0,
-                                 float* o, float* S_T, int B, int T, int H, int dk, int dv,
-                                 ckda_dtype_t dt, void* stream) {
-    ckda_status_t s = check_fwd_args(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt);
+ckda_status_t ckda_recurrent_fwd_ex(const void* q, const void* k, const void* v,
+                                    const float* gate, const float* beta, const float* S0,
+                                    float* o, float* S_T, int B, int T, int H, int dk, int dv,
+                                    ckda_dtype_t dt, ckda_gate_t gate_mode, void* stream) {
+    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+    ckda_status_t s = check_fwd_args(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt);
     if (s != CKDA_OK) return s;
     cudaStream_t st = as_stream(stream);
     if ((long long)B * H == 0) return CKDA_OK;
     if (T == 0) return copy_state(S0, S_T, (size_t)B * H * dk * dv, st);
-    if (dt == CKDA_BF16)
-        return launch_recurrent(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                static_cast<const __nv_bfloat16*>(v), alpha, beta, S0, o, S_T, B, T, H,
-                                dk, dv, st);
-    return launch_recurrent(static_cast<const float*>(q), static_cast<const float*>(k),
-                            static_cast<const float*>(v), alpha, beta, S0, o, S_T, B, T, H, dk, dv, st);
+    const bool lg = gate_mode == CKDA_GATE_LOG;
+    if (dt == CKDA_BF16) {
+        const auto* qb = static_cast<const __nv_bfloat16*>(q);
+        const auto* kb = static_cast<const __nv_bfloat16*>(k);
+        const auto* vb = static_cast<const __nv_bfloat16*>(v);
+        return lg ? launch_recurrent<__nv_bfloat16, true>(qb, kb, vb, gate, beta, S0, o, S_T, B, T, H, dk, dv, st)
+                  : launch_recurrent<__nv_bfloat16, false>(qb, kb, vb, gate, beta, S0, o, S_T, B, T, H, dk, dv, st);
+    }
+    const auto* qf = static_cast<const float*>(q);
+    const auto* kf = static_cast<const float*>(k);
+    const auto* vf = static_cast<const float*>(v);
+    return lg ? launch_recurrent<float, true>(qf, kf, vf, gate, beta, S0, o, S_T, B, T, H, dk, dv, st)
+              : launch_recurrent<float, false>(qf, kf, vf, gate, beta, S0, o, S_T, B, T, H, dk, dv, st);
 }
 
-ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
-                             const float* beta, const float* S0, float* o, float* S_T, int B,
-                             int T, int H, int dk, int dv, ckda_dtype_t dt, void* workspace,
-                             size_t workspace_bytes, void* stream) {
-    ckda_status_t s = check_fwd_args(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt);
+ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, const float* S0,
+                                 float* o, float* S_T, int B, int T, int H, int dk, int dv,
+                                 ckda_dtype_t dt, void* stream) {
+    return ckda_recurrent_fwd_ex(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt, CKDA_GATE_SIGNED,
+                                 stream);
+}
+
+ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* gate,
+                                const float* beta, const float* S0, float* o, float* S_T, int B,
+                                int T, int H, int dk, int dv, ckda_dtype_t dt, ckda_gate_t gate_mode,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+    ckda_status_t s = check_fwd_args(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt);
     if (s != CKDA_OK) return s;
     const size_t need = ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
@@ -133,11 +150,20 @@ ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const 
     if (ckda_chunk_fwd_path(B, T, H, dk, dv, dt) == CKDA_PATH_CHUNK_TC) {
         cudaError_t e = ckda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
                                               static_cast<const __nv_bfloat16*>(k),
-                                              static_cast<const __nv_bfloat16*>(v), alpha, beta,
-                                              S0, o, S_T, B, T, H, dk, dv, workspace, st);
+                                              static_cast<const __nv_bfloat16*>(v), gate, beta,
+                                              S0, o, S_T, B, T, H, dk, dv, gate_mode == CKDA_GATE_LOG,
+                                              workspace, st);
         return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
     }
-    return ckda_recurrent_fwd(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt, stream);
+    return ckda_recurrent_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, gate_mode, stream);
+}
+
+ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, float* o, float* S_T, int B,
+                             int T, int H, int dk, int dv, ckda_dtype_t dt, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    return ckda_chunk_fwd_ex(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt, CKDA_GATE_SIGNED,
+                             workspace, workspace_bytes, stream);
 }
 
 ckda_status_t ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,

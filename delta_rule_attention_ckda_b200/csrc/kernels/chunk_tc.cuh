@@ -71,6 +71,7 @@ static_assert(2 * kRegCompute + kRegEpi <= 512, "register split exceeds a schedu
 
 // log2-domain limits of the single-reference factorisation
 constexpr float kLgFloor = -100.f;    // floor of log2|a| per token (a = 0 allowed)
+constexpr float kLog2e = 1.4426950408889634f;   // log2(e): a log gate g = ln a gives log2 a = g log2(e)
 constexpr float kChunkRange = 192.f;  // -L_C bound for the fast path (factors within 2^{+-96})
 
 // shared-memory map (bytes from a 1024-aligned base)
@@ -250,6 +251,10 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 //   gate cumulation of chunk c           ||  O / state MMAs of chunk c-1
 //   o tile of chunk c-1, state copy       ||  [A ; P] MMA of chunk c
 //   [A ; P] epilogue, solve for T         ||  C1 MMA ([Z | O_inter]), k / alpha of chunk c+1
+//
+// kLogGate: the gate input holds g = ln a of a non-negative gate (KDA) instead of a signed
+// a; the cumulation then needs no logarithm and no sign parity.
+template <bool kLogGate>
 __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
@@ -614,9 +619,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int r = 32 * hh + i;
-                const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
-                run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
-                par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
+                if constexpr (kLogGate) {
+                    const float g = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 0.f;
+                    run += fmaxf(g * kLog2e, kLgFloor);
+                } else {
+                    const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
+                    run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+                    par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
+                }
                 L[i] = run;
             }
             par ^= par << 1;                      // prefix XOR of the sign bits
@@ -974,7 +984,8 @@ inline size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv) {
 
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const float* alpha, const float* beta, const float* S0, float* o, float* ST,
-                                   int B, int T, int H, int dk, int dv, void* workspace, cudaStream_t st) {
+                                   int B, int T, int H, int dk, int dv, bool log_gate, void* workspace,
+                                   cudaStream_t st) {
     (void)workspace;
     if (dk != 128 || dv != 128) return cudaErrorNotSupported;
     CUtensorMap mk, mq, mv, ma, mo;
@@ -985,14 +996,14 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         !tc::make_map_bthd(&mo, o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dv, 128, 64,
                            CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)ctc::SMEM_ALLOC);
+    static bool attr_set[2] = {false, false};
+    auto* kern = log_gate ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+    if (!attr_set[log_gate ? 1 : 0]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ctc::SMEM_ALLOC);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[log_gate ? 1 : 0] = true;
     }
-    chunk_tc_kernel<<<(unsigned)(B * H), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H);
+    kern<<<(unsigned)(B * H), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H);
     return cudaGetLastError();
 }
 

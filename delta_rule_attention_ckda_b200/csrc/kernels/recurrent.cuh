@@ -11,12 +11,14 @@
 // to 128 columns of one (b, h) and stages TB tokens of k, q, alpha in shared memory
 // (broadcast reads). Rows beyond d_k are padded with k = q = alpha = 0, which keeps
 // them exactly zero.
+//
+// kLogGate: the gate input holds g = ln a (a non-negative gate, a = e^g <= 1) instead of a.
 #pragma once
 #include "common.cuh"
 
 namespace ckda {
 
-template <int DK, typename TIn>
+template <int DK, typename TIn, bool kLogGate>
 __global__ void __launch_bounds__(128)
 recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                      const TIn* __restrict__ v, const float* __restrict__ alpha,
@@ -48,7 +50,8 @@ recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
             const bool in = i < dk;
             sk[tt][i] = in ? ld_in(k + tok * dk + i) : 0.f;
             sq[tt][i] = in ? ld_in(q + tok * dk + i) : 0.f;
-            sa[tt][i] = in ? __ldg(alpha + tok * dk + i) : 0.f;
+            const float ga = in ? __ldg(alpha + tok * dk + i) : 0.f;
+            sa[tt][i] = in ? (kLogGate ? expf(ga) : ga) : 0.f;
         }
         if (threadIdx.x < nt) sb[threadIdx.x] = __ldg(beta + ((size_t)b * T + t0 + threadIdx.x) * H + h);
         for (int tt = 0; tt < nt; ++tt) {

@@ -52,7 +52,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 1
+#define CKDA_ABI_VERSION 2
 
 typedef enum {
     CKDA_OK = 0,
@@ -74,6 +74,12 @@ typedef enum {
     CKDA_PATH_RECURRENT = 0,    /* fp32 SIMT token-by-token kernel (any d <= 128)    */
     CKDA_PATH_CHUNK_TC = 1      /* chunked WY/UT kernel on tcgen05 tensor cores      */
 } ckda_path_t;
+
+/* How the gate argument of the _ex forward calls is given. */
+typedef enum {
+    CKDA_GATE_SIGNED = 0,       /* alpha in [-1,1]^dk: the CKDA gate, sign and magnitude   */
+    CKDA_GATE_LOG = 1           /* g = ln(alpha) <= 0 of a non-negative gate (the KDA form) */
+} ckda_gate_t;
 
 /* Version of this ABI (CKDA_ABI_VERSION). */
 CKDA_API int ckda_abi_version(void);
@@ -117,6 +123,23 @@ CKDA_API ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* 
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * ckda_chunk_fwd with the gate in the form gate_mode selects. CKDA_GATE_SIGNED is
+ * ckda_chunk_fwd itself. CKDA_GATE_LOG reads g = ln(alpha), fp32, in alpha's
+ * [B,T,H,dk] layout, for a gate that never changes sign: the parameterisation of KDA,
+ * whose gate CKDA extends from [0,1] to [-1,1] (ai.info summary of the Complex KDA paper,
+ * "What This Paper Is About"). The map is the same recurrence with alpha = e^g
+ * (g = -inf gives alpha = 0). It runs on the same kernels, so that CKDA's cost over KDA
+ * can be measured (ai.info summary, "Main Findings": the throughput cost of the signed
+ * gate). An unknown gate_mode returns CKDA_ERR_INVALID_ARG.
+ */
+CKDA_API ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                                const float* gate, const float* beta, const float* S0,
+                                float* o, float* S_T,
+                                int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                ckda_gate_t gate_mode,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Token-by-token forward on CUDA cores in fp32 (the recurrent path of
  * ckda_chunk_fwd, callable directly). Same arguments and semantics as
  * ckda_chunk_fwd, no workspace. Each thread keeps one state column resident in
@@ -127,6 +150,13 @@ CKDA_API ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const vo
                                  float* o, float* S_T,
                                  int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
                                  void* stream);
+
+/* ckda_recurrent_fwd with the gate in the form gate_mode selects (see ckda_chunk_fwd_ex). */
+CKDA_API ckda_status_t ckda_recurrent_fwd_ex(const void* q, const void* k, const void* v,
+                                    const float* gate, const float* beta, const float* S0,
+                                    float* o, float* S_T,
+                                    int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                    ckda_gate_t gate_mode, void* stream);
 
 /*
  * One recurrent decode step for N independent sequences (blog post "One update,

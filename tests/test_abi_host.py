@@ -49,7 +49,7 @@ def test_status_strings(lib):
         s = lib.ckda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.ckda_status_string(99) == b"unknown status"
-    assert lib.ckda_abi_version() == 1
+    assert lib.ckda_abi_version() == 2
 
 
 NULL = None
@@ -116,3 +116,13 @@ def test_python_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 16)
     with pytest.raises(ValueError):
         ck.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def test_gate_mode_names():
+    """The binding maps gate names onto ckda_gate_t and rejects unknown ones (host only)."""
+    from delta_rule_attention_ckda_b200 import _lib
+    assert _lib.GATES == {"signed": 0, "log": 1}
+    with pytest.raises(ValueError):
+        _lib._gate("exp")
+    text = open(os.path.join(ROOT, "include", "ckda.h")).read()
+    assert "CKDA_GATE_SIGNED = 0" in text and "CKDA_GATE_LOG = 1" in text

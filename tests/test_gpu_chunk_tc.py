@@ -121,3 +121,21 @@ def test_long_workload_full_size(ck):
     # late tokens are as accurate as early ones (no drift over 1024 chunks)
     for sl in (slice(0, 4096), slice(61440, 65536)):
         check(f"long/o[{sl.start}:]", got_o[:, sl], o_ref[:, sl], TAU_BF16)
+
+
+@pytest.mark.parametrize("T", [64, 300])
+def test_log_gate_mode(ck, T):
+    """KDA form: the gate tensor holds g = ln(alpha) of a non-negative gate; the map is
+    the same recurrence with alpha = e^g (evaluated in fp64 for the oracle)."""
+    inp = make_inputs(2, T, 2, 128, 128, torch.bfloat16, seed=40 + T, gate="log15", s0_std=0.05)
+    g = inp.alpha
+    g[0, 10:12, 1, :4] = -float("inf")          # alpha = 0
+    g[1, 20:40, 0, 8:16] = -20.0                 # fast decay: the chunk takes the exact path
+    q, k, v, _, b, s0 = to_dev(inp)
+    o, ST = ck.chunk_fwd(q, k, v, g.cuda(), b, s0, gate="log")
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    alpha = np.exp(g.double().numpy())
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, alpha, inp.beta, inp.S0)
+    check(f"loggate T={T}/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check(f"loggate T={T}/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)

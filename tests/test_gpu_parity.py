@@ -262,3 +262,21 @@ def test_decode_full_size_sampled(ck):
         check(f"decode call {t}", got[t], o_ref[:, t, 0], TAU_BF16)
     got_S = np.stack([S[n, h].double().cpu().numpy() for n, h in pairs])
     check("decode final state", got_S, S_ref[:, 0], TAU_BF16)
+
+
+# ------------------------------------------------------------------ log-gate (KDA) form
+
+@pytest.mark.parametrize("fn", ["chunk", "recurrent"])
+@pytest.mark.parametrize("dims,dtype", [((16, 16), torch.float32), ((64, 64), torch.bfloat16),
+                                        ((32, 48), torch.float32)])
+def test_log_gate_mode_recurrent_shapes(ck, fn, dims, dtype):
+    """g = ln(alpha) of a non-negative gate on the SIMT path (shapes the tensor-core path
+    does not take); the oracle runs the same recurrence with alpha = e^g in fp64."""
+    dk, dv = dims
+    inp = make_inputs(2, 150, 3, dk, dv, dtype, seed=dk + dv, gate="log15", s0_std=0.05)
+    o, ST = run_fwd(ck, fn, inp, gate="log")
+    alpha = np.exp(inp.alpha.double().numpy())
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, alpha, inp.beta, inp.S0)
+    tau = tau_for(dtype)
+    check(f"loggate/{fn}/{dk}x{dv}/o", o.double().cpu().numpy(), o_ref, tau)
+    check(f"loggate/{fn}/{dk}x{dv}/S", ST.double().cpu().numpy(), S_ref, tau)
