@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
                 const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta, const float* S0,
-                float* ST, int T, int H) {
+                float* ST, int T, int H, int dk, int dv) {
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -449,12 +449,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
         // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
         {
-            const size_t sb = (size_t)bh * D * D;
+            const size_t sb = (size_t)bh * dk * dv;
 #pragma unroll 1
             for (int cb = 0; cb < 8; ++cb) {
                 uint32_t x[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = __float_as_uint(S0 ? S0[sb + (size_t)(16 * cb + i) * D + me] : 0.f);
+                for (int i = 0; i < 16; ++i) {
+                    const int c = 16 * cb + i;
+                    x[i] = __float_as_uint((S0 && c < dk && me < dv) ? S0[sb + (size_t)c * dv + me] : 0.f);
+                }
                 tc::tmem_st32<16>(te + TM_S + 16 * cb, x);
             }
             tc::tmem_st_wait();
@@ -620,10 +623,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             for (int i = 0; i < 32; ++i) {
                 const int r = 32 * hh + i;
                 if constexpr (kLogGate) {
-                    const float g = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 0.f;
+                    const float g = (r < nvalid && m < dk) ? ld_alpha_tile(sm + SM_AL, r, m) : 0.f;
                     run += fmaxf(g * kLog2e, kLgFloor);
                 } else {
-                    const float a = (r < nvalid) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
+                    const float a = (r < nvalid && m < dk) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
                     run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
                     par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
                 }
@@ -953,14 +956,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
         // final state: S = acc Diag(kappa_last)
         if (!failed && ST != nullptr) {
-            const size_t sb = (size_t)bh * D * D;
+            const size_t sb = (size_t)bh * dk * dv;
             for (int cb = 0; cb < 2; ++cb) {
                 const int c0 = 64 * hh + 32 * cb;
                 float x[32];
                 tc::tmem_ld32<32>(tl + TM_S + c0, x);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ST[sb + (size_t)(c0 + i) * D + m] = x[i] * sh_kref[c0 + i];
+                for (int i = 0; i < 32; ++i)
+                    if (c0 + i < dk && m < dv) ST[sb + (size_t)(c0 + i) * dv + m] = x[i] * sh_kref[c0 + i];
             }
         }
     }
@@ -975,7 +979,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
 // ------------------------------------------------------------------------------ host
 
-inline bool chunk_tc_supported(int dk, int dv, int dt) { return dt == 1 && dk == 128 && dv == 128; }
+// d_k, d_v in {64, 128}: a 64-wide problem runs as the 128-wide one with zero padding,
+// which the TMA supplies (boxes past the tensor's d read as zero; o columns past d_v are
+// not stored) and which leaves the padded state rows and columns exactly zero (pad
+// channels get gate 1, and their k, q and initial state are zero).
+inline bool chunk_tc_supported(int dk, int dv, int dt) {
+    return dt == 1 && (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+}
 
 inline size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv) {
     (void)B; (void)T; (void)H; (void)dk; (void)dv;
@@ -987,7 +997,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
                                    int B, int T, int H, int dk, int dv, bool log_gate, void* workspace,
                                    cudaStream_t st) {
     (void)workspace;
-    if (dk != 128 || dv != 128) return cudaErrorNotSupported;
+    if (!chunk_tc_supported(dk, dv, 1)) return cudaErrorNotSupported;
     CUtensorMap mk, mq, mv, ma, mo;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!tc::make_map_bthd(&mk, k, bf, 2, B, T, H, dk, 64, 64) || !tc::make_map_bthd(&mq, q, bf, 2, B, T, H, dk, 64, 64) ||
@@ -1003,7 +1013,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         if (e != cudaSuccess) return e;
         attr_set[log_gate ? 1 : 0] = true;
     }
-    kern<<<(unsigned)(B * H), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H);
+    kern<<<(unsigned)(B * H), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H, dk, dv);
     return cudaGetLastError();
 }
 

@@ -34,6 +34,23 @@ def run_chunk(ck, inp, S0=True):
 def test_tc_path_is_selected(ck):
     assert ck.chunk_path(8, 4096, 16, 128, 128, torch.bfloat16) == ck.PATH_CHUNK_TC
     assert ck.chunk_path(8, 4096, 16, 128, 128, torch.float32) == ck.PATH_RECURRENT
+    for dk, dv in [(64, 64), (64, 128), (128, 64)]:
+        assert ck.chunk_path(2, 512, 4, dk, dv, torch.bfloat16) == ck.PATH_CHUNK_TC
+    assert ck.chunk_path(2, 512, 4, 32, 32, torch.bfloat16) == ck.PATH_RECURRENT
+
+
+@pytest.mark.parametrize("dims", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [70, 300])
+def test_d64_on_tensor_cores(ck, dims, T):
+    """d_k, d_v = 64 run the 128-wide kernel on zero-padded tiles (TMA fills the missing
+    channels with zeros); padded state rows and columns must stay exactly zero."""
+    dk, dv = dims
+    inp = make_inputs(2, T, 3, dk, dv, torch.bfloat16, seed=dk + 2 * dv + T, gate="signmag", s0_std=0.1)
+    o, ST = run_chunk(ck, inp)
+    assert o.shape == (2, T, 3, dv) and ST.shape == (2, 3, dk, dv)
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check(f"d{dk}x{dv} T={T}/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check(f"d{dk}x{dv} T={T}/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
 
 
 @pytest.mark.parametrize("T", [1, 2, 31, 32, 33, 63, 64, 65, 127, 128, 129, 300])
