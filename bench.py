@@ -335,6 +335,7 @@ def ours_arm(args):
 
     if not args.no_extras:
         line["kda"] = kda_measure(ck, q, k, v, a, b, o, ST, stream, world, args.steps, value)
+        line["configs"] = configs_measure(ck, dev, stream, world)
     if not args.no_e2e:
         line["e2e"] = e2e_measure(ck, inp, dev, stream, world, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -347,6 +348,44 @@ def ours_arm(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def configs_measure(ck, dev, stream, world):
+    """The workloads' other configurations: small (L2-resident and launch-bound: latency
+    only) and long (one head batch of 65536 tokens with an initial state: 16 sequences,
+    so 16 SMs work; tokens/s and the fraction of the HBM roofline)."""
+    import torch
+    from ckda_inputs import make_workload
+    out = {}
+    for name, reps in (("small", 20), ("long", 3)):
+        inp = make_workload(name)
+        B, T, H, dk, dv = inp.shape
+        q, k, v, a, b = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
+        S0 = inp.S0.to(dev)
+        o = torch.empty(B, T, H, dv, device=dev)
+        ST = torch.empty(B, H, dk, dv, device=dev)
+
+        def step():
+            ck.chunk_fwd(q, k, v, a, b, S0, o=o, S_T=ST)
+
+        step()
+        torch.cuda.synchronize()
+        assert ck.get_device_error() == 0
+        secs = time_launches(step, reps, stream)
+        value, secs = aggregate_throughput(B * T * reps, secs, world, device="cuda")
+        per = secs / reps
+        path = "chunk_tc" if ck.chunk_path(B, T, H, dk, dv, inp.q.dtype) == ck.PATH_CHUNK_TC else "recurrent"
+        ent = {"shape": f"B={B} T={T} H={H} dk={dk} dv={dv} {str(inp.q.dtype).replace('torch.', '')}",
+               "path": path, "us_per_launch": per * 1e6}
+        if name == "long":
+            bytes_tok = 2 * dk * 2 + dv * 2 + dk * 4 + 4 + dv * 4
+            alg = B * T * H * bytes_tok + 2 * B * H * dk * dv * 4
+            hbm, src = peaks()
+            ent.update({"tokens_per_s": value, "roofline": {"bound": "hbm", "achieved": alg / per / 1e9,
+                        "peak": hbm, "unit": "GB/s", "frac": alg / per / 1e9 / hbm,
+                        "alg_bytes_per_launch": alg}})
+        out[name] = ent
+    return out
 
 
 def kda_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, ckda_value):
