@@ -48,6 +48,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_chunk_fwd_workspace_bytes.restype = sz
     lib.ckda_chunk_fwd_path.argtypes = [i] * 6
     lib.ckda_chunk_fwd_path.restype = i
+    lib.ckda_chunk_fwd_segments.argtypes = [i] * 6
+    lib.ckda_chunk_fwd_segments.restype = i
     lib.ckda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 6 + [vp, sz, vp]
     lib.ckda_chunk_fwd.restype = i
     lib.ckda_recurrent_fwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 6 + [vp]
@@ -106,6 +108,11 @@ def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
 
 def chunk_path(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
     return int(load().ckda_chunk_fwd_path(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
+
+
+def chunk_segments(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Segments per sequence ckda_chunk_fwd runs side by side on the current device (1 = one pass)."""
+    return int(load().ckda_chunk_fwd_segments(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
 
 
 def _fwd_common(q, k, v, alpha, beta, S0, o, S_T):

@@ -101,6 +101,12 @@ size_t ckda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_
     return ckda::chunk_tc_workspace_bytes(B, T, H, dk, dv);
 }
 
+int ckda_chunk_fwd_segments(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {
+    if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return 1;
+    if (ckda_chunk_fwd_path(B, T, H, dk, dv, dt) != CKDA_PATH_CHUNK_TC) return 1;
+    return ckda::chunk_tc_segments(B, T, H);
+}
+
 ckda_status_t ckda_recurrent_fwd_ex(const void* q, const void* k, const void* v,
                                     const float* gate, const float* beta, const float* S0,
                                     float* o, float* S_T, int B, int T, int H, int dk, int dv,

@@ -115,6 +115,11 @@ constexpr uint32_t kTmaBytes1a = 4 * 8192;  // alpha (4 fp32 boxes)
 constexpr uint32_t kTmaBytes1b = 2 * 8192;  // k (2 bf16 boxes)
 constexpr uint32_t kTmaBytes2 = 4 * 8192;   // q + v (2 bf16 boxes each)
 
+// Launch flags (segment passes of a long sequence; see launch_chunk_tc)
+constexpr uint32_t kFlagVZero = 1u;     // v is taken as zero (not loaded; no V T^T term)
+constexpr uint32_t kFlagNoO = 2u;       // no o output
+constexpr uint32_t kFlagS0Ident = 4u;   // the state entering each segment is the identity (d_v = d_k)
+
 // Byte address (from tile base) of the 16-byte chunk `ch` (0..7) of row `row` in a
 // tile of 128-byte rows with 128-byte swizzle.
 __device__ __forceinline__ uint32_t chunk_off(int row, int ch) {
@@ -258,8 +263,9 @@ template <bool kLogGate>
 __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
-                const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta, const float* S0,
-                float* ST, int T, int H, int dk, int dv) {
+                const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta,
+                const float* S0_seg, float* ST_seg, float* ST_last, float* M_seg, int T, int H, int dk,
+                int dv_in, int seg_len, int nseg, uint32_t flags_in) {
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -286,8 +292,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, hh = warp >> 2;
     const int m = quarter * 32 + lane;            // TMEM lane = channel / feature / row
-    const int bh = blockIdx.x;
+    // CTA -> (batch, head) and segment sg of seg_len tokens (nseg segments per sequence; one
+    // segment covering all T for an unsegmented launch). Entering state: slot (bh, sg) of
+    // S0_seg (zero if NULL; identity with kFlagS0Ident). Final state: ST_last for the last
+    // segment, else slot (bh, sg) of ST_seg; NULL = not written. A slot is d_k x d_v floats.
+    // blockIdx.z = 1 runs the segment's transition product instead: identity entering state,
+    // v = 0, no o, d_v = d_k, the result written to slot (bh, sg) of M_seg.
+    const bool trans = blockIdx.z != 0;
+    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident) : flags_in;
+    const int dv = trans ? dk : dv_in;
+    if (trans) ST_seg = M_seg;
+    const int bh = blockIdx.x;                    // grid: x = (batch, head), y = segment
+    const int sg = blockIdx.y;
     const int b = bh / H, h = bh % H;
+    const int ta = sg * seg_len;
+    const int tb = min(T, ta + seg_len);
+    const size_t slot = ((size_t)bh * nseg + sg) * dk * dv;
+    const float* S0 = (flags & kFlagS0Ident) || S0_seg == nullptr ? nullptr : S0_seg + slot;
+    float* ST = (sg == nseg - 1) ? (ST_last ? ST_last + (size_t)bh * dk * dv : nullptr)
+                                 : (ST_seg ? ST_seg + slot : nullptr);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
@@ -335,17 +358,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::mbar_arrive_expect_tx(&bar_tma1b, kTmaBytes1b);
         for (int i = 0; i < 2; ++i) tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma1b, 64 * i, h, t0, b);
     };
+    const bool v_zero = (flags & kFlagVZero) != 0;
     auto issue_loads2 = [&](int t0) {
-        tc::mbar_arrive_expect_tx(&bar_tma2, kTmaBytes2);
+        tc::mbar_arrive_expect_tx(&bar_tma2, v_zero ? kTmaBytes2 / 2 : kTmaBytes2);
         for (int i = 0; i < 2; ++i) {
             tc::tma_load_4d(sm + SM_Q + i * 8192, &map_q, &bar_tma2, 64 * i, h, t0, b);
-            tc::tma_load_4d(sm + SM_V + i * 8192, &map_v, &bar_tma2, 64 * i, h, t0, b);
+            if (!v_zero) tc::tma_load_4d(sm + SM_V + i * 8192, &map_v, &bar_tma2, 64 * i, h, t0, b);
         }
     };
     auto load_beta = [&](int t0) -> float {
-        return (tid < C && t0 + tid < T) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
+        return (tid < C && t0 + tid < tb) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
     };
-    float beta_next = load_beta(0);
+    float beta_next = load_beta(ta);
 
     // C1: [O^T | Z^T] = (S0 Diag g)^T [(q e1)^T | (k e1)^T]  (3 passes), after the state copy
     auto issue_c1 = [&](uint32_t sb_) {
@@ -385,7 +409,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                        tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iv, ks != 0);
     };
     //   += (-Z^T)_hi [T_hi ; T_lo]^T + (-Z^T)_lo [T_hi ; T_lo]^T once -Z^T is in TMEM
-    auto issue_uz = [&](uint32_t sb_) {
+    auto issue_uz = [&](uint32_t sb_, bool after_v) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
         const uint32_t iz = tc::idesc_bf16(128, 128, 0, 0);   // A = -Z^T (TMEM)
 #pragma unroll
@@ -393,7 +417,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             const uint32_t aa = tm0 + (ps == 1 ? TM_ZALO : TM_ZAHI);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ts(tm0 + TM_DU, aa + ks * 8, tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iz, 1);
+                tc::mma_ts(tm0 + TM_DU, aa + ks * 8, tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iz,
+                           (after_v || ps || ks) ? 1u : 0u);
         }
         tc::mma_commit(&bar_u);
     };
@@ -413,7 +438,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     };
 
     const uint32_t sbase = tc::smem_u32(sm);
-    const int nchunks = (T + C - 1) / C;
+    const int nchunks = max(0, (tb - ta + C - 1) / C);
+    const bool want_o = (flags & kFlagNoO) == 0;
 
     if (warp >= NT / 32) {
         // ================================================================ epilogue warpgroup
@@ -449,28 +475,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
         // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
         {
-            const size_t sb = (size_t)bh * dk * dv;
+            const bool ident = (flags & kFlagS0Ident) != 0;
 #pragma unroll 1
             for (int cb = 0; cb < 8; ++cb) {
                 uint32_t x[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int c = 16 * cb + i;
-                    x[i] = __float_as_uint((S0 && c < dk && me < dv) ? S0[sb + (size_t)c * dv + me] : 0.f);
+                    const bool in = c < dk && me < dv;
+                    x[i] = __float_as_uint(ident ? ((in && c == me) ? 1.f : 0.f)
+                                                 : ((S0 && in) ? S0[(size_t)c * dv + me] : 0.f));
                 }
                 tc::tmem_st32<16>(te + TM_S + 16 * cb, x);
             }
             tc::tmem_st_wait();
         }
         if (leader && nchunks > 0) {
-            issue_loads1a(0);
-            issue_loads1b(0);
-            issue_loads2(0);
+            issue_loads1a(ta);
+            issue_loads1b(ta);
+            issue_loads2(ta);
         }
         int ck = 0;
         for (; ck < nchunks; ++ck) {
             const uint32_t par = (uint32_t)ck & 1u;
-            const int t0 = ck * C;
+            const int t0 = ta + ck * C;
             // ---------------- E1: state copy. The accumulator holds S Diag(1/kappa_prev):
             // S = acc kappa_prev, then the operand S g_ref (split into TMEM) and the new
             // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
@@ -520,7 +548,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // leader: o store, C1 (runs while the compute warps solve), the next chunk's alpha
             if (leader) {
                 tc::tc_fence_after();
-                if (ck > 0) {
+                if (ck > 0 && want_o) {
                     tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
                     tc::bulk_commit();
                 }
@@ -552,8 +580,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 efail |= !tc::mbar_wait(&bar_ht, par);
                 tc::tc_fence_after();
                 if (ck + 1 < nchunks) issue_loads1b(t0 + C);
-                issue_uv(sbase);
-                issue_uz(sbase);
+                if (!v_zero) issue_uv(sbase);
+                issue_uz(sbase, !v_zero);
             }
             // ---------------- E3: U^T -> TMEM operand of the O / state MMA
             efail |= !tc::mbar_wait(&bar_u, par);
@@ -587,8 +615,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             if (!esync_or(efail)) {
                 stage_o();
                 epi_publish();
-                if (!esync_or(false) && leader) {
-                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, (nchunks - 1) * C, b);
+                if (!esync_or(false) && leader && want_o) {
+                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, ta + (nchunks - 1) * C, b);
                     tc::bulk_commit();
                 }
             }
@@ -615,7 +643,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // ---------------- P0: gate cumulation of chunk ckn (thread = channel m, tokens 32hh .. 32hh+31),
         // the per-channel constants and the exact-path decision. True if a wait gave up.
         auto gate_logs = [&](int ckn) -> bool {
-            const int nvalid = min(C, T - ckn * C);
+            const int nvalid = min(C, tb - (ta + ckn * C));
             wfail |= !tc::mbar_wait(&bar_tma1a, ckn & 1);
             float run = 0.f;
             par = 0;
@@ -680,7 +708,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
         if (nchunks > 0 && gate_logs(0)) failed = true;
         for (int ck = 0; ck < nchunks && !failed; ++ck) {
-            const int t0 = ck * C;
+            const int t0 = ta + ck * C;
             if (tid < C) sh_beta[tid] = beta_next;
 
             // ---------------- P1: gate factors (thread = channel m, tokens 32hh .. 32hh+31)
@@ -956,7 +984,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 
         // final state: S = acc Diag(kappa_last)
         if (!failed && ST != nullptr) {
-            const size_t sb = (size_t)bh * dk * dv;
             for (int cb = 0; cb < 2; ++cb) {
                 const int c0 = 64 * hh + 32 * cb;
                 float x[32];
@@ -964,7 +991,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (c0 + i < dk && m < dv) ST[sb + (size_t)(c0 + i) * dv + m] = x[i] * sh_kref[c0 + i];
+                    if (c0 + i < dk && m < dv) ST[(size_t)(c0 + i) * dv + m] = x[i] * sh_kref[c0 + i];
             }
         }
     }
@@ -987,16 +1014,117 @@ inline bool chunk_tc_supported(int dk, int dv, int dt) {
     return dt == 1 && (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
 }
 
+// ------------------------------------------------------------------ long sequences
+// With few (batch, head) pairs the per-sequence chain of chunks is the critical path and most
+// SMs sit idle. The affine map of a segment of tokens, S_out = M S_in + N (M the product of
+// its transitions (I - beta k k^T) Diag(alpha), N the state it builds from S_in = 0), lets
+// segments run side by side:
+//   pass 1: one CTA per (sequence, segment but the last) computes N (z = 0) and M (z = 1);
+//   prefix: S_{s+1} = M_s S_s + N_s from S_0 = S0, sequentially over the segments;
+//   pass 2: every segment again from its entering state S_s, now with o and the final state.
+struct ChunkTcPlan {
+    int nseg;      // segments per sequence (1 = one CTA per sequence)
+    int seg_len;   // tokens per segment, a multiple of the chunk
+};
+
+inline int chunk_tc_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        n = 0;
+    return n > 0 ? n : 148;
+}
+
+// Picks the segment count with the least modelled time, in units of one chunk step of a CTA
+// (one CTA per SM): waves of each pass times its chunks per segment, plus a fixed cost per
+// launch and per prefix step.
+inline ChunkTcPlan chunk_tc_plan(int B, int T, int H, int sms) {
+    constexpr double kLaunchCost = 1.5, kPrefixStep = 0.5;
+    constexpr int kMaxSeg = 64;
+    const long long bh = (long long)B * H;
+    const int nch = (T + ctc::C - 1) / ctc::C;
+    auto waves = [&](long long ctas) { return (double)((ctas + sms - 1) / sms); };
+    ChunkTcPlan best{1, nch * ctc::C};
+    double best_cost = waves(bh) * nch + kLaunchCost;
+    for (int s = 2; s <= kMaxSeg && s <= nch; ++s) {
+        const int per = (nch + s - 1) / s;
+        const int ns = (nch + per - 1) / per;
+        if (ns != s) continue;   // the same split as a smaller s
+        const double cost = (waves(2 * bh * (ns - 1)) + waves(bh * ns)) * per + 3 * kLaunchCost +
+                            kPrefixStep * (ns - 1);
+        if (cost < best_cost) { best_cost = cost; best = ChunkTcPlan{ns, per * ctc::C}; }
+    }
+    return best;
+}
+
+// workspace: the entering states (B*H*nseg slots of d_k x d_v floats), then the segments'
+// transition products (B*H*nseg slots of d_k x d_k floats)
 inline size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv) {
-    (void)B; (void)T; (void)H; (void)dk; (void)dv;
-    return 0;
+    if ((long long)B * H == 0 || T <= 0) return 0;
+    const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
+    if (p.nseg == 1) return 0;
+    return (size_t)B * H * p.nseg * (size_t)dk * (size_t)(dv + dk) * sizeof(float);
+}
+
+inline int chunk_tc_segments(int B, int T, int H) {
+    if ((long long)B * H == 0 || T <= 0) return 1;
+    return chunk_tc_plan(B, T, H, chunk_tc_sm_count()).nseg;
+}
+
+// S_{s+1} = M_s S_s + N_s over the segments of one sequence (grid x), on 16 columns of the
+// state (grid y). Slot s + 1 of Sx holds N_s on entry and S_{s+1} on exit; slot 0 gets S0
+// (zero if NULL). fp32 throughout; one thread owns 8 rows of one column.
+__global__ void __launch_bounds__(256) chunk_tc_seg_prefix(float* __restrict__ Sx, const float* __restrict__ M,
+                                                           const float* __restrict__ S0, int nseg, int dk, int dv) {
+    __shared__ float sS[128][16];
+    __shared__ float sM[128][33];
+    const int bh = blockIdx.x, n0 = blockIdx.y * 16;
+    const int t = threadIdx.x, n = t & 15, rq = t >> 4;
+    const bool col_ok = n0 + n < dv;
+    float* Sb = Sx + (size_t)bh * nseg * dk * dv;
+    const float* Mb = M + (size_t)bh * nseg * dk * dk;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = rq + 16 * i;
+        const bool ok = r < dk && col_ok;
+        const float x = (ok && S0) ? S0[(size_t)bh * dk * dv + (size_t)r * dv + n0 + n] : 0.f;
+        sS[r][n] = x;
+        if (ok) Sb[(size_t)r * dv + n0 + n] = x;
+    }
+    __syncthreads();
+    for (int sg = 0; sg + 1 < nseg; ++sg) {
+        const float* Ms = Mb + (size_t)sg * dk * dk;
+        float* Sn = Sb + (size_t)(sg + 1) * dk * dv;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rq + 16 * i;
+            acc[i] = (r < dk && col_ok) ? Sn[(size_t)r * dv + n0 + n] : 0.f;
+        }
+        for (int j0 = 0; j0 < dk; j0 += 32) {
+            for (int e = t; e < dk * 32; e += 256) sM[e >> 5][e & 31] = Ms[(size_t)(e >> 5) * dk + j0 + (e & 31)];
+            __syncthreads();
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) {
+                const float a = sS[j0 + j][n];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(sM[rq + 16 * i][j], a, acc[i]);
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rq + 16 * i;
+            sS[r][n] = r < dk ? acc[i] : 0.f;
+            if (r < dk && col_ok) Sn[(size_t)r * dv + n0 + n] = acc[i];
+        }
+        __syncthreads();
+    }
 }
 
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const float* alpha, const float* beta, const float* S0, float* o, float* ST,
                                    int B, int T, int H, int dk, int dv, bool log_gate, void* workspace,
                                    cudaStream_t st) {
-    (void)workspace;
     if (!chunk_tc_supported(dk, dv, 1)) return cudaErrorNotSupported;
     CUtensorMap mk, mq, mv, ma, mo;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -1013,7 +1141,28 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         if (e != cudaSuccess) return e;
         attr_set[log_gate ? 1 : 0] = true;
     }
-    kern<<<(unsigned)(B * H), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, ST, T, H, dk, dv);
+    const unsigned nbh = (unsigned)(B * H);
+    const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
+    if (p.nseg == 1) {
+        kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, nullptr, ST, nullptr,
+                                                                     T, H, dk, dv, T, 1, 0u);
+        return cudaGetLastError();
+    }
+    if (workspace == nullptr) return cudaErrorInvalidValue;
+    float* Sx = static_cast<float*>(workspace);
+    float* Mx = Sx + (size_t)nbh * p.nseg * dk * dv;
+    // pass 1: N_s into slot s + 1 of Sx, M_s into slot s of Mx, for every segment but the last
+    kern<<<dim3(nbh, (unsigned)(p.nseg - 1), 2), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
+        mk, mq, mv, ma, mo, beta, nullptr, Sx + (size_t)dk * dv, nullptr, Mx, T, H, dk, dv, p.seg_len, p.nseg,
+        ctc::kFlagNoO);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    chunk_tc_seg_prefix<<<dim3(nbh, (unsigned)(dv / 16)), 256, 0, st>>>(Sx, Mx, S0, p.nseg, dk, dv);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // pass 2: every segment from its entering state, with o; the last one writes S_T
+    kern<<<dim3(nbh, (unsigned)p.nseg, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
+        mk, mq, mv, ma, mo, beta, Sx, nullptr, ST, nullptr, T, H, dk, dv, p.seg_len, p.nseg, 0u);
     return cudaGetLastError();
 }
 

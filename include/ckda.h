@@ -88,13 +88,27 @@ CKDA_API int ckda_abi_version(void);
 CKDA_API const char* ckda_status_string(ckda_status_t status);
 
 /*
- * Bytes of device workspace ckda_chunk_fwd needs for this problem (may be 0).
- * Invalid sizes return 0; ckda_chunk_fwd then rejects them.
+ * Bytes of device workspace ckda_chunk_fwd needs for this problem on the current
+ * device (may be 0). Nonzero when the tensor-core path splits each sequence into
+ * segments (few (b, h) pairs, long T): the segments' entering states and transition
+ * products, B*H*nseg*dk*(dv+dk) fp32. Invalid sizes return 0; ckda_chunk_fwd then
+ * rejects them.
  */
 CKDA_API size_t ckda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
 
 /* The path ckda_chunk_fwd takes for these sizes (for tests and reporting). */
 CKDA_API ckda_path_t ckda_chunk_fwd_path(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
+
+/*
+ * Segments per sequence the tensor-core path runs side by side for these sizes on
+ * the current device (1 = one pass, no workspace; for tests and reporting). A
+ * segment of tokens acts on the state as the affine map S -> M S + N (the
+ * recurrence's step composed over the segment); the path builds every segment's
+ * M and N at once, chains the entering states, then evaluates the segments again
+ * from those states. Not a step the pages describe: a scheduling choice for
+ * sequences too few to fill the GPU. Returns 1 for shapes on the recurrent path.
+ */
+CKDA_API int ckda_chunk_fwd_segments(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
 
 /*
  * Chunked forward (prefill / training forward without gradients).

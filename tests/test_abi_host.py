@@ -110,6 +110,28 @@ def test_workspace_query_and_path(lib):
     assert lib.ckda_chunk_fwd_path(8, 4096, 16, 128, 128, 0) == 0
 
 
+def test_segment_plan(lib):
+    """Host-side segment plan of the tensor-core path (148 SMs assumed without a device):
+    a batch that fills the GPU runs in one pass with no workspace; one long sequence per
+    head is split, and its workspace holds nseg entering states (dk x dv) and transition
+    products (dk x dk) per sequence, fp32."""
+    bf = 1
+    assert lib.ckda_chunk_fwd_segments(8, 4096, 16, 128, 128, bf) == 1
+    assert lib.ckda_chunk_fwd_workspace_bytes(8, 4096, 16, 128, 128, bf) == 0
+    nseg = lib.ckda_chunk_fwd_segments(1, 65536, 16, 128, 128, bf)
+    assert 1 < nseg <= 64
+    assert lib.ckda_chunk_fwd_workspace_bytes(1, 65536, 16, 128, 128, bf) == 16 * nseg * 128 * 256 * 4
+    n64 = lib.ckda_chunk_fwd_segments(1, 65536, 16, 64, 128, bf)
+    assert lib.ckda_chunk_fwd_workspace_bytes(1, 65536, 16, 64, 128, bf) == 16 * n64 * 64 * 192 * 4
+    # segments are whole chunks: never more segments than chunks
+    for T in (1, 64, 65, 128, 640, 1000):
+        assert 1 <= lib.ckda_chunk_fwd_segments(1, T, 1, 128, 128, bf) <= (T + 63) // 64
+    # the recurrent path and empty problems are never split
+    assert lib.ckda_chunk_fwd_segments(1, 65536, 16, 128, 128, 0) == 1
+    assert lib.ckda_chunk_fwd_segments(0, 65536, 16, 128, 128, bf) == 1
+    assert lib.ckda_chunk_fwd_segments(1, 65536, 16, 32, 32, bf) == 1
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     import delta_rule_attention_ckda_b200 as ck
