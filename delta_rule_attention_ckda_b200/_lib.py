@@ -58,6 +58,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_chunk_fwd_ex.restype = i
     lib.ckda_recurrent_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp]
     lib.ckda_recurrent_fwd_ex.restype = i
+    lib.ckda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp]
+    lib.ckda_chunk_fwd_noalloc.restype = i
     lib.ckda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 5 + [vp]
     lib.ckda_decode_step.restype = i
     lib.ckda_get_device_error.argtypes = [vp]
@@ -160,6 +162,25 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=Tru
                                _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate), _ptr(workspace), wbytes,
                                _stream(stream))
     _raise(st, "ckda_chunk_fwd_ex")
+    return o, S_T
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20      # CKDA_NOALLOC_SCRATCH_BYTES
+
+
+def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
+                      stream=None, gate="signed") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """ckda_chunk_fwd_noalloc: ckda_chunk_fwd_ex on the library's fixed device scratch
+    (no workspace argument; the call allocates nothing). Raises CkdaError(WORKSPACE)
+    when the problem needs more than NOALLOC_SCRATCH_BYTES of scratch. o / S_T are
+    allocated with torch only when not given."""
+    B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
+    if S_T is None and want_state:
+        S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
+    st = load().ckda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                       _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate),
+                                       _stream(stream))
+    _raise(st, "ckda_chunk_fwd_noalloc")
     return o, S_T
 
 

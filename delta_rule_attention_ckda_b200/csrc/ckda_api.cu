@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "kernels/common.cuh"
 #include "kernels/recurrent.cuh"
 #include "kernels/decode.cuh"
@@ -69,6 +71,26 @@ ckda_status_t check_fwd_args(const void* q, const void* k, const void* v, const 
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return CKDA_ERR_MISALIGNED;
     return CKDA_OK;
+}
+
+// Fixed scratch of ckda_chunk_fwd_noalloc: part of the module's device image, so the
+// runtime sets it up with the module and no call allocates it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CKDA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.
+void* noalloc_scratch() {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
 }
 
 }  // namespace
@@ -162,6 +184,24 @@ ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const void* v, con
         return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
     }
     return ckda_recurrent_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, gate_mode, stream);
+}
+
+ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* gate,
+                                     const float* beta, const float* S0, float* o, float* S_T, int B,
+                                     int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                     ckda_gate_t gate_mode, void* stream) {
+    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+    ckda_status_t s = check_fwd_args(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt);
+    if (s != CKDA_OK) return s;
+    const size_t need = ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt);
+    if (need > CKDA_NOALLOC_SCRATCH_BYTES) return CKDA_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if (need > 0) {
+        ws = noalloc_scratch();
+        if (ws == nullptr) return CKDA_ERR_CUDA;
+    }
+    return ckda_chunk_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, gate_mode, ws, need,
+                             stream);
 }
 
 ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,

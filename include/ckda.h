@@ -52,7 +52,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 2
+#define CKDA_ABI_VERSION 3
 
 typedef enum {
     CKDA_OK = 0,
@@ -152,6 +152,29 @@ CKDA_API ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const voi
                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
                                 ckda_gate_t gate_mode,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Capacity of the fixed device scratch ckda_chunk_fwd_noalloc uses: 32 MiB per device. */
+#define CKDA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * ckda_chunk_fwd_ex without a caller-supplied workspace and without any allocation.
+ * The paper has no counterpart to this call: it is a deployment variant of the
+ * segmented long-sequence path. Where that path needs scratch (see
+ * ckda_chunk_fwd_workspace_bytes), it uses a fixed array of
+ * CKDA_NOALLOC_SCRATCH_BYTES that lives in the library's device image (allocated by
+ * the CUDA runtime when the module loads on a device, never by this call); its
+ * address is looked up once per device. Arguments, layouts and results are those of
+ * ckda_chunk_fwd_ex; o, S_T and every input stay caller-owned.
+ * Errors: CKDA_ERR_WORKSPACE, with nothing launched, when the problem needs more
+ * scratch than the capacity (e.g. B*H*nseg*dk*(dv+dk)*4 > 32 MiB); otherwise as
+ * ckda_chunk_fwd_ex. The scratch is one per device: calls that need it must be
+ * ordered (e.g. issued on one stream); concurrent calls on unordered streams race.
+ */
+CKDA_API ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                const float* gate, const float* beta, const float* S0,
+                                float* o, float* S_T,
+                                int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                ckda_gate_t gate_mode, void* stream);
 
 /*
  * Token-by-token forward on CUDA cores in fp32 (the recurrent path of

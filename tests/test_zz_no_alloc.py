@@ -1,0 +1,75 @@
+"""ckda_chunk_fwd_noalloc: the segmented chunk path on the library's fixed device
+scratch instead of a caller workspace. Two consecutive calls, on different inputs so
+that the second one reuses scratch the first one filled, must give results
+bit-identical to ckda_chunk_fwd on the same inputs (same kernels, same launch plan)."""
+import ctypes
+
+import pytest
+import torch
+
+from ckda_inputs import make_inputs, make_workload
+from parity_util import to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ck():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from delta_rule_attention_ckda_b200 import build
+    build.build()
+    import delta_rule_attention_ckda_b200 as m
+    m.load()
+    return m
+
+
+def _pair(ck, inp):
+    q, k, v, a, b, s0 = to_dev(inp)
+    o_ref, S_ref = ck.chunk_fwd(q, k, v, a, b, s0)
+    o = torch.full_like(o_ref, float("nan"))
+    S = torch.full_like(S_ref, float("nan"))
+    return (q, k, v, a, b, s0), (o_ref, S_ref), (o, S)
+
+
+@pytest.mark.parametrize("shape", [(1, 1000, 2, 128, 128), (1, 1100, 2, 64, 128), (2, 300, 2, 128, 128)])
+def test_two_consecutive_calls_match_workspace_entry(ck, shape):
+    B, T, H, dk, dv = shape
+    need = ck.workspace_bytes(B, T, H, dk, dv)
+    assert need <= ck.NOALLOC_SCRATCH_BYTES
+    first = _pair(ck, make_inputs(B, T, H, dk, dv, torch.bfloat16, seed=1, gate="tanh15", s0_std=0.1))
+    second = _pair(ck, make_inputs(B, T, H, dk, dv, torch.bfloat16, seed=2, gate="signmag", s0_std=0.1))
+    for args, _, (o, S) in (first, second):
+        ck.chunk_fwd_noalloc(*args, o=o, S_T=S)
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    for _, (o_ref, S_ref), (o, S) in (first, second):
+        assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
+
+
+def test_long_workload_fits_and_matches(ck):
+    """B=1, T=65536, H=16, d=128: the segmented launch the long-context forward takes."""
+    inp = make_workload("long")
+    B, T, H, dk = inp.q.shape
+    assert ck.chunk_segments(B, T, H, dk, dk) > 1
+    assert 0 < ck.workspace_bytes(B, T, H, dk, dk) <= ck.NOALLOC_SCRATCH_BYTES
+    args, (o_ref, S_ref), (o, S) = _pair(ck, inp)
+    for _ in range(2):
+        o.fill_(float("nan"))
+        ck.chunk_fwd_noalloc(*args, o=o, S_T=S)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
+
+
+def test_oversize_problem_is_rejected_before_launch(ck):
+    """A problem whose segment buffers exceed the fixed scratch returns
+    CKDA_ERR_WORKSPACE without touching its (dummy, aligned) pointers."""
+    lib = ck.load()
+    B, T, H, d = 1, 1 << 20, 32, 128
+    assert ck.workspace_bytes(B, T, H, d, d) > ck.NOALLOC_SCRATCH_BYTES
+    p = ctypes.c_void_p(256)
+    fp = ctypes.cast(p, ctypes.POINTER(ctypes.c_float))
+    st = lib.ckda_chunk_fwd_noalloc(p, p, p, fp, fp, fp, fp, fp, B, T, H, d, d, 1, 0, None)
+    assert st == 6   # CKDA_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
