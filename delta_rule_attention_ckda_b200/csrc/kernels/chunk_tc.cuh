@@ -1,4 +1,4 @@
-// Chunked WY/UT CKDA forward on tcgen05 tensor cores (sm_100a), d_k = d_v = 128.
+// Chunked WY/UT CKDA forward on tcgen05 tensor cores (sm_100a), d_k, d_v in {64, 128}.
 //
 // Recurrence (blog post "One update, one quarter-turn", section "The mirror"):
 //   S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T,   o_t = S_t^T q_t.
@@ -33,14 +33,18 @@
 // state into the MMA operand), and the final write multiplies by the last kappa.
 // Entries above the diagonal of X Y^T may overflow; they are never read.
 //
-// B200 mapping. One CTA (256 threads) owns one (batch, head) and walks its chunks in
-// order. Everything is computed transposed so the 128 feature rows sit on the 128
-// TMEM lanes: the fp32 state lives in TMEM for the whole sequence and never
-// round-trips HBM. Every product runs on tcgen05 with bf16 operands; operands that
-// are not raw bf16 inputs are split x = hi + lo (two bf16) and each product is the
-// three passes hi*hi + hi*lo + lo*hi (relative error about 2^-17), which the fp32-state
-// tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by TMA (no
-// multicast) with 128-byte swizzle; tokens past the end read as zero and get gate 1.
+// B200 mapping. One CTA of 384 threads owns one (batch, head), or one segment of its
+// tokens, and walks the chunks in order: two compute warpgroups (gate, [P;A] epilogue,
+// solve) and one epilogue warpgroup (state copy, o tile, -Z^T and U^T into TMEM) whose
+// leader thread issues the TMA loads and stores and every MMA but [P;A]. Everything is
+// computed transposed so the 128 feature rows sit on the 128 TMEM lanes: the fp32
+// state lives in TMEM for the whole sequence and never round-trips HBM. Every product
+// runs on tcgen05 with bf16 operands; operands that are not raw bf16 inputs are split
+// x = hi + lo (hi rounded to nearest, lo the remainder truncated: |x - hi - lo| <=
+// 2^-15 |x|) and each product is the three passes hi*hi + hi*lo + lo*hi, which the
+// fp32-state tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by
+// TMA (no multicast) with 128-byte swizzle; tokens past the end read as zero and get
+// gate 1. A 64-wide d_k or d_v is the 128-wide problem with zero padding.
 //
 // Exponent safety. e1 and e2 stay inside [2^-96, 2^96] unless a chunk's gates decay by
 // more than 2^-192 in some channel; such a chunk computes A and P pair by pair on CUDA
@@ -139,8 +143,9 @@ __device__ __forceinline__ float ld_alpha_tile(const uint8_t* tile, int r, int c
 }
 
 // (a, b) -> packed bf16 hi pair and packed bf16 lo pair with hi + lo = x to within
-// 2^-17 |x|: hi is x rounded to nearest, the remainder x - hi (exact in fp32) is truncated
-// to bf16 by taking its upper half. One conversion per pair; the conversion unit is the
+// 2^-15 |x|: hi is x rounded to nearest (|x - hi| <= 2^-8 |x|), the remainder x - hi
+// (exact in fp32) is truncated to bf16 by taking its upper half (error below one unit in
+// its 8-bit significand). One conversion per pair; the conversion unit is the
 // scarce resource in the operand-splitting epilogues.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
