@@ -165,7 +165,7 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=Tru
     return o, S_T
 
 
-NOALLOC_SCRATCH_BYTES = 32 << 20      # CKDA_NOALLOC_SCRATCH_BYTES
+NOALLOC_SCRATCH_BYTES = 20 << 20      # CKDA_NOALLOC_SCRATCH_BYTES
 
 
 def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,

@@ -269,8 +269,8 @@ __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
                 const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta,
-                const float* S0_seg, float* ST_seg, float* ST_last, float* M_seg, int T, int H, int dk,
-                int dv_in, int seg_len, int nseg, uint32_t flags_in) {
+                const float* S0_head, const float* S0_seg, float* ST_seg, float* ST_last, float* M_seg,
+                int T, int H, int dk, int dv_in, int seg_len, int nseg, int sg_base, uint32_t flags_in) {
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -297,23 +297,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, hh = warp >> 2;
     const int m = quarter * 32 + lane;            // TMEM lane = channel / feature / row
-    // CTA -> (batch, head) and segment sg of seg_len tokens (nseg segments per sequence; one
-    // segment covering all T for an unsegmented launch). Entering state: slot (bh, sg) of
-    // S0_seg (zero if NULL; identity with kFlagS0Ident). Final state: ST_last for the last
-    // segment, else slot (bh, sg) of ST_seg; NULL = not written. A slot is d_k x d_v floats.
+    // CTA -> (batch, head) and segment sg = sg_base + blockIdx.y of seg_len tokens (nseg
+    // segments per sequence; one segment covering all T for an unsegmented launch).
+    // Entering state: for segment 0 the sequence's S0 in S0_head (zero if NULL), else slot
+    // (bh, sg) of S0_seg (zero if NULL). Final state: ST_last for the last segment, else slot
+    // (bh, sg) of ST_seg; NULL = not written. A slot is d_k x d_v floats. flags_in applies
+    // to segments after the first; segment 0 always writes o.
     // blockIdx.z = 1 runs the segment's transition product instead: identity entering state,
-    // v = 0, no o, d_v = d_k, the result written to slot (bh, sg) of M_seg.
+    // v = 0, no o, d_v = d_k, the result written to slot (bh, sg) of M_seg. Segment 0 needs
+    // none (its entering state is known), so those CTAs return at once.
     const bool trans = blockIdx.z != 0;
-    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident) : flags_in;
+    const int bh = blockIdx.x;                    // grid: x = (batch, head), y = segment
+    const int sg = sg_base + (int)blockIdx.y;
+    if (trans && sg == 0) return;
+    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident) : (sg == 0 ? 0u : flags_in);
     const int dv = trans ? dk : dv_in;
     if (trans) ST_seg = M_seg;
-    const int bh = blockIdx.x;                    // grid: x = (batch, head), y = segment
-    const int sg = blockIdx.y;
     const int b = bh / H, h = bh % H;
     const int ta = sg * seg_len;
     const int tb = min(T, ta + seg_len);
     const size_t slot = ((size_t)bh * nseg + sg) * dk * dv;
-    const float* S0 = (flags & kFlagS0Ident) || S0_seg == nullptr ? nullptr : S0_seg + slot;
+    const float* S0 = (flags & kFlagS0Ident) ? nullptr
+                    : sg == 0 ? (S0_head ? S0_head + (size_t)bh * dk * dv : nullptr)
+                              : (S0_seg ? S0_seg + slot : nullptr);
     float* ST = (sg == nseg - 1) ? (ST_last ? ST_last + (size_t)bh * dk * dv : nullptr)
                                  : (ST_seg ? ST_seg + slot : nullptr);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -745,12 +751,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         const float e1 = __uint_as_float(__float_as_uint(tc::ex2_approx(t)) ^ sg);
                         const float e2 = __uint_as_float(__float_as_uint(m2) ^ sg ^ sC);
                         const float kv = ld_bf16_tile(sm + SM_K, r, m);
-                        const float qv = ld_bf16_tile(sm + SM_Q, r, m);
+                        const float qv = want_o ? ld_bf16_tile(sm + SM_Q, r, m) : 0.f;
                         xk[e] = kv * e1;
                         xq[e] = qv * e1;
                         yk[e] = kv * e2;
                     }
-                    store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xq);
+                    // without o the q rows of X (read only into P and O) are left as they are
+                    if (want_o) store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xq);
                     store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xk);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) split2(yk[2 * e], yk[2 * e + 1], yh[q8][e], yl[q8][e]);
@@ -810,7 +817,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         const int s = 32 * hh + i;
                         at[s * 64 + r] = (s < r) ? br * d1[i] : 0.f;
                     }
-                } else {
+                } else if (want_o) {
                     const int r = m;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) d1[i] = (32 * hh + i <= r) ? d1[i] : 0.f;
@@ -1025,8 +1032,10 @@ inline bool chunk_tc_supported(int dk, int dv, int dt) {
 // its transitions (I - beta k k^T) Diag(alpha), N the state it builds from S_in = 0), lets
 // segments run side by side:
 //   pass 1: one CTA per (sequence, segment but the last) computes N (z = 0) and M (z = 1);
-//   prefix: S_{s+1} = M_s S_s + N_s from S_0 = S0, sequentially over the segments;
-//   pass 2: every segment again from its entering state S_s, now with o and the final state.
+//           segment 0 starts from the known S0, so it runs once, with o, and writes S_1 itself;
+//   prefix: S_{s+1} = M_s S_s + N_s from S_1, sequentially over the segments;
+//   pass 2: every segment after the first from its entering state S_s, with o; the last one
+//           writes the final state.
 struct ChunkTcPlan {
     int nseg;      // segments per sequence (1 = one CTA per sequence)
     int seg_len;   // tokens per segment, a multiple of the chunk
@@ -1054,8 +1063,8 @@ inline ChunkTcPlan chunk_tc_plan(int B, int T, int H, int sms) {
         const int per = (nch + s - 1) / s;
         const int ns = (nch + per - 1) / per;
         if (ns != s) continue;   // the same split as a smaller s
-        const double cost = (waves(2 * bh * (ns - 1)) + waves(bh * ns)) * per + 3 * kLaunchCost +
-                            kPrefixStep * (ns - 1);
+        const double cost = (waves(bh * (2 * ns - 3)) + waves(bh * (ns - 1))) * per + 3 * kLaunchCost +
+                            kPrefixStep * (ns - 2);
         if (cost < best_cost) { best_cost = cost; best = ChunkTcPlan{ns, per * ctc::C}; }
     }
     return best;
@@ -1076,10 +1085,10 @@ inline int chunk_tc_segments(int B, int T, int H) {
 }
 
 // S_{s+1} = M_s S_s + N_s over the segments of one sequence (grid x), on 16 columns of the
-// state (grid y). Slot s + 1 of Sx holds N_s on entry and S_{s+1} on exit; slot 0 gets S0
-// (zero if NULL). fp32 throughout; one thread owns 8 rows of one column.
+// state (grid y), from S_1 (slot 1 of Sx, already the true state). Slot s + 1 of Sx holds
+// N_s on entry and S_{s+1} on exit. fp32 throughout; one thread owns 8 rows of one column.
 __global__ void __launch_bounds__(256) chunk_tc_seg_prefix(float* __restrict__ Sx, const float* __restrict__ M,
-                                                           const float* __restrict__ S0, int nseg, int dk, int dv) {
+                                                           int nseg, int dk, int dv) {
     __shared__ float sS[128][16];
     __shared__ float sM[128][33];
     const int bh = blockIdx.x, n0 = blockIdx.y * 16;
@@ -1090,13 +1099,10 @@ __global__ void __launch_bounds__(256) chunk_tc_seg_prefix(float* __restrict__ S
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int r = rq + 16 * i;
-        const bool ok = r < dk && col_ok;
-        const float x = (ok && S0) ? S0[(size_t)bh * dk * dv + (size_t)r * dv + n0 + n] : 0.f;
-        sS[r][n] = x;
-        if (ok) Sb[(size_t)r * dv + n0 + n] = x;
+        sS[r][n] = (r < dk && col_ok) ? Sb[(size_t)dk * dv + (size_t)r * dv + n0 + n] : 0.f;
     }
     __syncthreads();
-    for (int sg = 0; sg + 1 < nseg; ++sg) {
+    for (int sg = 1; sg + 1 < nseg; ++sg) {
         const float* Ms = Mb + (size_t)sg * dk * dk;
         float* Sn = Sb + (size_t)(sg + 1) * dk * dv;
         float acc[8];
@@ -1149,25 +1155,29 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     const unsigned nbh = (unsigned)(B * H);
     const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
     if (p.nseg == 1) {
-        kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, nullptr, ST, nullptr,
-                                                                     T, H, dk, dv, T, 1, 0u);
+        kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mk, mq, mv, ma, mo, beta, S0, nullptr, nullptr, ST,
+                                                                     nullptr, T, H, dk, dv, T, 1, 0, 0u);
         return cudaGetLastError();
     }
     if (workspace == nullptr) return cudaErrorInvalidValue;
     float* Sx = static_cast<float*>(workspace);
     float* Mx = Sx + (size_t)nbh * p.nseg * dk * dv;
-    // pass 1: N_s into slot s + 1 of Sx, M_s into slot s of Mx, for every segment but the last
+    // pass 1, every segment but the last: segment 0 from S0 with o, its final state S_1 into
+    // slot 1 of Sx; later segments s: N_s into slot s + 1 of Sx (z = 0), M_s into slot s of
+    // Mx (z = 1)
     kern<<<dim3(nbh, (unsigned)(p.nseg - 1), 2), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
-        mk, mq, mv, ma, mo, beta, nullptr, Sx + (size_t)dk * dv, nullptr, Mx, T, H, dk, dv, p.seg_len, p.nseg,
-        ctc::kFlagNoO);
+        mk, mq, mv, ma, mo, beta, S0, nullptr, Sx + (size_t)dk * dv, nullptr, Mx, T, H, dk, dv, p.seg_len, p.nseg,
+        0, ctc::kFlagNoO);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    chunk_tc_seg_prefix<<<dim3(nbh, (unsigned)(dv / 16)), 256, 0, st>>>(Sx, Mx, S0, p.nseg, dk, dv);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // pass 2: every segment from its entering state, with o; the last one writes S_T
-    kern<<<dim3(nbh, (unsigned)p.nseg, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
-        mk, mq, mv, ma, mo, beta, Sx, nullptr, ST, nullptr, T, H, dk, dv, p.seg_len, p.nseg, 0u);
+    if (p.nseg > 2) {
+        chunk_tc_seg_prefix<<<dim3(nbh, (unsigned)(dv / 16)), 256, 0, st>>>(Sx, Mx, p.nseg, dk, dv);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // pass 2: segments 1 .. nseg - 1 from their entering states, with o; the last writes S_T
+    kern<<<dim3(nbh, (unsigned)(p.nseg - 1), 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
+        mk, mq, mv, ma, mo, beta, nullptr, Sx, nullptr, ST, nullptr, T, H, dk, dv, p.seg_len, p.nseg, 1, 0u);
     return cudaGetLastError();
 }
 

@@ -153,8 +153,9 @@ CKDA_API ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const voi
                                 ckda_gate_t gate_mode,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
-/* Capacity of the fixed device scratch ckda_chunk_fwd_noalloc uses: 32 MiB per device. */
-#define CKDA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+/* Capacity of the fixed device scratch ckda_chunk_fwd_noalloc uses: 20 MiB per device
+ * (the long-context forward, B=1, T=65536, H=16, d=128, needs exactly this on a 148-SM GPU). */
+#define CKDA_NOALLOC_SCRATCH_BYTES ((size_t)20 << 20)
 
 /*
  * ckda_chunk_fwd_ex without a caller-supplied workspace and without any allocation.
@@ -166,7 +167,7 @@ CKDA_API ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const voi
  * address is looked up once per device. Arguments, layouts and results are those of
  * ckda_chunk_fwd_ex; o, S_T and every input stay caller-owned.
  * Errors: CKDA_ERR_WORKSPACE, with nothing launched, when the problem needs more
- * scratch than the capacity (e.g. B*H*nseg*dk*(dv+dk)*4 > 32 MiB); otherwise as
+ * scratch than the capacity (B*H*nseg*dk*(dv+dk)*4 > 20 MiB); otherwise as
  * ckda_chunk_fwd_ex. The scratch is one per device: calls that need it must be
  * ordered (e.g. issued on one stream); concurrent calls on unordered streams race.
  */
