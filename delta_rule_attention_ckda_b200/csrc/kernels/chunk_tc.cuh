@@ -1086,49 +1086,85 @@ inline int chunk_tc_segments(int B, int T, int H) {
 
 // S_{s+1} = M_s S_s + N_s over the segments of one sequence (grid x), on 16 columns of the
 // state (grid y), from S_1 (slot 1 of Sx, already the true state). Slot s + 1 of Sx holds
-// N_s on entry and S_{s+1} on exit. fp32 throughout; one thread owns 8 rows of one column.
-__global__ void __launch_bounds__(256) chunk_tc_seg_prefix(float* __restrict__ Sx, const float* __restrict__ M,
-                                                           int nseg, int dk, int dv) {
-    __shared__ float sS[128][16];
-    __shared__ float sM[128][33];
+// N_s on entry and S_{s+1} on exit. fp32 throughout. The next M streams into the other
+// half of a double buffer (cp.async) while this one is applied; a thread owns a 4 x 2 tile
+// of the result, fed by 16-byte row reads of M and 8-byte reads of the 16-column block.
+constexpr int kPrefixThreads = 256;
+inline size_t seg_prefix_smem(int dk) { return 2 * (size_t)dk * dk * sizeof(float); }
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
+}
+
+__global__ void __launch_bounds__(kPrefixThreads) chunk_tc_seg_prefix(float* __restrict__ Sx, const float* __restrict__ M,
+                                                                      int nseg, int dk, int dv) {
+    extern __shared__ __align__(16) float sMbuf[];          // [2][dk * dk], row-major
+    __shared__ __align__(16) float sS[128][16];
     const int bh = blockIdx.x, n0 = blockIdx.y * 16;
-    const int t = threadIdx.x, n = t & 15, rq = t >> 4;
-    const bool col_ok = n0 + n < dv;
+    const int t = threadIdx.x;
+    const int r0 = 4 * (t >> 3), c0 = 2 * (t & 7);
+    const bool rows_ok = r0 < dk;                           // dk is a multiple of 4
     float* Sb = Sx + (size_t)bh * nseg * dk * dv;
     const float* Mb = M + (size_t)bh * nseg * dk * dk;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = rq + 16 * i;
-        sS[r][n] = (r < dk && col_ok) ? Sb[(size_t)dk * dv + (size_t)r * dv + n0 + n] : 0.f;
+    const int nvec = dk * dk / 4;                           // float4 per transition product
+    auto fetch = [&](int sg) {
+        const float4* src = reinterpret_cast<const float4*>(Mb + (size_t)sg * dk * dk);
+        float4* dst = reinterpret_cast<float4*>(sMbuf + (size_t)(sg & 1) * dk * dk);
+        for (int e = t; e < nvec; e += kPrefixThreads) cp_async16(dst + e, src + e);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    if (nseg > 2) fetch(1);
+    for (int e = t; e < 128 * 16; e += kPrefixThreads) {
+        const int r = e >> 4, n = e & 15;
+        sS[r][n] = (r < dk && n0 + n < dv) ? Sb[(size_t)dk * dv + (size_t)r * dv + n0 + n] : 0.f;
     }
-    __syncthreads();
     for (int sg = 1; sg + 1 < nseg; ++sg) {
-        const float* Ms = Mb + (size_t)sg * dk * dk;
         float* Sn = Sb + (size_t)(sg + 1) * dk * dv;
-        float acc[8];
+        float acc[4][2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = rq + 16 * i;
-            acc[i] = (r < dk && col_ok) ? Sn[(size_t)r * dv + n0 + n] : 0.f;
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                acc[a][c] = (rows_ok && n0 + c0 + c < dv) ? Sn[(size_t)(r0 + a) * dv + n0 + c0 + c] : 0.f;
+        if (sg + 2 < nseg) {
+            fetch(sg + 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-        for (int j0 = 0; j0 < dk; j0 += 32) {
-            for (int e = t; e < dk * 32; e += 256) sM[e >> 5][e & 31] = Ms[(size_t)(e >> 5) * dk + j0 + (e & 31)];
-            __syncthreads();
-#pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
-                const float a = sS[j0 + j][n];
+        __syncthreads();                                     // M_sg and S_sg visible to all
+        if (rows_ok) {
+            const float* Ms = sMbuf + (size_t)(sg & 1) * dk * dk;
+            for (int j = 0; j < dk; j += 4) {
+                float4 mr[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(sM[rq + 16 * i][j], a, acc[i]);
+                for (int a = 0; a < 4; ++a) mr[a] = *reinterpret_cast<const float4*>(Ms + (size_t)(r0 + a) * dk + j);
+                float2 sv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sv[u] = *reinterpret_cast<const float2*>(&sS[j + u][c0]);
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    acc[a][0] = fmaf(mr[a].x, sv[0].x, acc[a][0]);
+                    acc[a][1] = fmaf(mr[a].x, sv[0].y, acc[a][1]);
+                    acc[a][0] = fmaf(mr[a].y, sv[1].x, acc[a][0]);
+                    acc[a][1] = fmaf(mr[a].y, sv[1].y, acc[a][1]);
+                    acc[a][0] = fmaf(mr[a].z, sv[2].x, acc[a][0]);
+                    acc[a][1] = fmaf(mr[a].z, sv[2].y, acc[a][1]);
+                    acc[a][0] = fmaf(mr[a].w, sv[3].x, acc[a][0]);
+                    acc[a][1] = fmaf(mr[a].w, sv[3].y, acc[a][1]);
+                }
             }
-            __syncthreads();
         }
+        __syncthreads();                                     // every read of S_sg and M_sg done
+        if (rows_ok) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = rq + 16 * i;
-            sS[r][n] = r < dk ? acc[i] : 0.f;
-            if (r < dk && col_ok) Sn[(size_t)r * dv + n0 + n] = acc[i];
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    sS[r0 + a][c0 + c] = acc[a][c];
+                    if (n0 + c0 + c < dv) Sn[(size_t)(r0 + a) * dv + n0 + c0 + c] = acc[a][c];
+                }
         }
-        __syncthreads();
     }
 }
 
@@ -1171,7 +1207,15 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.nseg > 2) {
-        chunk_tc_seg_prefix<<<dim3(nbh, (unsigned)(dv / 16)), 256, 0, st>>>(Sx, Mx, p.nseg, dk, dv);
+        static bool prefix_attr = false;
+        if (!prefix_attr) {
+            e = cudaFuncSetAttribute(chunk_tc_seg_prefix, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)seg_prefix_smem(128));
+            if (e != cudaSuccess) return e;
+            prefix_attr = true;
+        }
+        chunk_tc_seg_prefix<<<dim3(nbh, (unsigned)(dv / 16)), kPrefixThreads, seg_prefix_smem(dk), st>>>(
+            Sx, Mx, p.nseg, dk, dv);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
