@@ -63,13 +63,20 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
-    """Hash of the sources of the chunk kernel; the committed DRAM-traffic figure is
-    only reported while it matches."""
+# sources that make up each profiled kernel (its code, the primitives it uses, its launch)
+KERNEL_SOURCES = {
+    "chunk_fwd_chunk_tc_layer": ["kernels/common.cuh", "kernels/chunk_tc.cuh", "kernels/tc_primitives.cuh",
+                                 "kernels/tc_host.cuh"],
+    "decode128": ["kernels/common.cuh", "kernels/decode.cuh"],
+}
+
+
+def kernel_source_hash(kernel_key):
+    """Hash of the sources of one kernel; its committed DRAM-traffic figure is only
+    reported while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "delta_rule_attention_ckda_b200", "csrc")
-    for rel in ["ckda_api.cu", "kernels/common.cuh", "kernels/chunk_tc.cuh", "kernels/tc_primitives.cuh",
-                "kernels/recurrent.cuh", "kernels/decode.cuh"]:
+    for rel in KERNEL_SOURCES[kernel_key]:
         p = os.path.join(csrc, rel)
         if os.path.exists(p):
             with open(p, "rb") as f:
@@ -84,7 +91,7 @@ def committed_traffic(kernel_key):
         with open(path) as f:
             d = json.load(f)
         ent = d.get(kernel_key)
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        if ent and ent.get("source_hash") == kernel_source_hash(kernel_key):
             return float(ent["bytes_per_launch"])
     except Exception:
         pass
