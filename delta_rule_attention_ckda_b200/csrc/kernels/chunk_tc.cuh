@@ -277,19 +277,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     __shared__ uint64_t bar_tma1a, bar_tma1b, bar_tma2, bar_ap, bar_c1, bar_u, bar_c2;   // TMA / MMA completion
     // compute -> epilogue group: per-channel constants of the chunk (hk), X / Y tiles written and
     // the alpha space free (hap), T written and A consumed (ht)
-    __shared__ uint64_t bar_hk, bar_hap, bar_ht;
+    // hk is double-buffered by chunk parity, so the compute warps may hand over the next
+    // chunk's constants before the epilogue group has waited for this chunk's
+    __shared__ uint64_t bar_hk[2], bar_hap, bar_ht;
     __shared__ uint32_t tmem_base_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
-    float* sh_fa = sh_beta + 64;            // [128] g_ref (operand copy = S g_ref)
-    float* sh_fs = sh_fa + 128;             // [128] g_ref, or Gamma_C on the exact path (accumulator)
-    float* sh_kref = sh_fs + 128;           // [128] kappa of the last chunk
-    float* sh_Lx = sh_kref + 128;           // [128] exchange: L at token 31
+    // per-channel constants, [2][128] by chunk parity: the next chunk's are written while the
+    // epilogue group may still read this chunk's
+    float* sh_fa = sh_beta + 64;            // g_ref (operand copy = S g_ref)
+    float* sh_fs = sh_fa + 256;             // g_ref, or Gamma_C on the exact path (accumulator)
+    float* sh_kref = sh_fs + 256;           // kappa of the chunk
+    float* sh_Lx = sh_kref + 256;           // [128] exchange: L at token 31
     float* sh_LC = sh_Lx + 128;             // [128] exchange: L at token 63
     uint32_t* sh_px = reinterpret_cast<uint32_t*>(sh_LC + 128);        // [128]
     uint32_t* sh_pC = sh_px + 128;                                       // [128]
     uint32_t* sh_sign = sh_pC + 128;        // [64][4] slow path: sign bits per (token, channel)
-    float* sh_kp = reinterpret_cast<float*>(sh_sign + 256);             // [128] kappa of the previous chunk
+    float* sh_kp = reinterpret_cast<float*>(sh_sign + 256);             // [2][128] kappa of the previous chunk
     float* at = reinterpret_cast<float*>(sm + SM_AT);
     float* xs = reinterpret_cast<float*>(sm + SM_XS);
     float* rs = reinterpret_cast<float*>(sm + SM_RS);
@@ -333,7 +337,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::mbar_init(&bar_c1, 1);
         tc::mbar_init(&bar_u, 1);
         tc::mbar_init(&bar_c2, 1);
-        tc::mbar_init(&bar_hk, NT);
+        tc::mbar_init(&bar_hk[0], NT);
+        tc::mbar_init(&bar_hk[1], NT);
         tc::mbar_init(&bar_hap, NT);
         tc::mbar_init(&bar_ht, NT);
         tc::fence_mbar_init();
@@ -343,7 +348,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::prefetch_tensormap(&map_a);
         tc::prefetch_tensormap(&map_o);
     }
-    if (tid < D) sh_kref[tid] = 1.f;
+    if (tid < 2 * D) sh_kref[tid] = 1.f;
     // blocks of (I + A)^{-1} above the 16 x 16 block diagonal: zero once, never written again
     for (int e = tid; e < 384; e += NT_ALL) {
         int r, g;
@@ -510,13 +515,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         for (; ck < nchunks; ++ck) {
             const uint32_t par = (uint32_t)ck & 1u;
             const int t0 = ta + ck * C;
-            // ---------------- E1: state copy. The accumulator holds S Diag(1/kappa_prev):
+            // ---------------- E1: state copy (after the previous o tile and the next alpha are on
+            // their way, so that it overlaps the solve). The accumulator holds S Diag(1/kappa_prev):
             // S = acc kappa_prev, then the operand S g_ref (split into TMEM) and the new
             // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
             // for fast-decaying channels although each factor and each result is in range.
-            efail |= !tc::mbar_wait(&bar_hk, par);             // this chunk's constants
+            efail |= !tc::mbar_wait(&bar_hk[par], (uint32_t)(ck >> 1) & 1u);   // this chunk's constants
             if (ck > 0) efail |= !tc::mbar_wait(&bar_c2, par ^ 1u);
             tc::tc_fence_after();
+            // the previous chunk's o rows, once the gate (or the exact path) is done with the
+            // alpha space; its store and the next alpha go out before the state copy
+            efail |= !tc::mbar_wait(&bar_hap, par);
+            if (ck > 0) stage_o();
+            epi_publish();
+            if (esync_or(efail)) break;
+            if (leader) {
+                tc::tc_fence_after();
+                if (ck > 0 && want_o) {
+                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
+                    tc::bulk_commit();
+                }
+                if (ck + 1 < nchunks) {
+                    tc::bulk_wait_read0();
+                    issue_loads1a(t0 + C);
+                }
+            }
             {
                 float sv[2][16];
                 tc::tmem_ld32<16>(te + TM_S, sv[0]);
@@ -529,9 +552,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     uint32_t snew[16];
 #pragma unroll
                     for (int i4 = 0; i4 < 4; ++i4) {
-                        const float4 kk = reinterpret_cast<const float4*>(sh_kp + 16 * cb)[i4];
-                        const float4 fa = reinterpret_cast<const float4*>(sh_fa + 16 * cb)[i4];
-                        const float4 fs = reinterpret_cast<const float4*>(sh_fs + 16 * cb)[i4];
+                        const float4 kk = reinterpret_cast<const float4*>(sh_kp + par * D + 16 * cb)[i4];
+                        const float4 fa = reinterpret_cast<const float4*>(sh_fa + par * D + 16 * cb)[i4];
+                        const float4 fs = reinterpret_cast<const float4*>(sh_fs + par * D + 16 * cb)[i4];
                         const float s0 = cur[4 * i4] * kk.x, s1 = cur[4 * i4 + 1] * kk.y;
                         const float s2 = cur[4 * i4 + 2] * kk.z, s3 = cur[4 * i4 + 3] * kk.w;
                         z[4 * i4] = s0 * fa.x;
@@ -550,24 +573,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
                 }
             }
-            // the previous chunk's o rows, once the gate (or the exact path) is done with the
-            // alpha space
-            efail |= !tc::mbar_wait(&bar_hap, par);
-            if (ck > 0) stage_o();
             epi_publish();
             if (esync_or(efail)) break;
-            // leader: o store, C1 (runs while the compute warps solve), the next chunk's alpha
+            // leader: C1 (runs while the compute warps solve)
             if (leader) {
                 tc::tc_fence_after();
-                if (ck > 0 && want_o) {
-                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
-                    tc::bulk_commit();
-                }
                 issue_c1(sbase);
-                if (ck + 1 < nchunks) {
-                    tc::bulk_wait_read0();
-                    issue_loads1a(t0 + C);
-                }
             }
             // ---------------- E2: -Z^T -> TMEM operand of the U MMA
             efail |= !tc::mbar_wait(&bar_c1, par);
@@ -696,16 +707,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             if (hh == 0) {
                 LC = sh_LC[m];
                 pC = sh_pC[m];
-                sh_kp[m] = sh_kref[m];
+                const int pb = ckn & 1, o = pb * D + m;
+                sh_kp[o] = sh_kref[(pb ^ 1) * D + m];
                 if (!slow) {
                     const float gref = exp2f(0.5f * LC);
-                    sh_fa[m] = gref;
-                    sh_fs[m] = gref;
-                    sh_kref[m] = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
+                    sh_fa[o] = gref;
+                    sh_fs[o] = gref;
+                    sh_kref[o] = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
                 } else {
-                    sh_fa[m] = 1.f;
-                    sh_fs[m] = (pC ? -1.f : 1.f) * exp2f(LC);
-                    sh_kref[m] = 1.f;
+                    sh_fa[o] = 1.f;
+                    sh_fs[o] = (pC ? -1.f : 1.f) * exp2f(LC);
+                    sh_kref[o] = 1.f;
                 }
             }
             if (slow) {
@@ -713,7 +725,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
             }
-            handoff(&bar_hk);                     // the epilogue group copies the state with them
+            handoff(&bar_hk[ckn & 1]);            // the epilogue group copies the state with them
             return false;
         };
 
@@ -1003,7 +1015,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (c0 + i < dk && m < dv) ST[(size_t)(c0 + i) * dv + m] = x[i] * sh_kref[c0 + i];
+                    if (c0 + i < dk && m < dv)
+                        ST[(size_t)(c0 + i) * dv + m] = x[i] * sh_kref[((nchunks - 1) & 1) * D + c0 + i];
             }
         }
     }
