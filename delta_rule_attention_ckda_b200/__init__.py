@@ -15,9 +15,9 @@ Tensors are torch CUDA tensors in [B, T, H, d] layout; q/k/v bf16 or fp32, the
 rest fp32. There is no CPU path.
 """
 from ._lib import (BF16, F32, NOALLOC_SCRATCH_BYTES, PATH_CHUNK_TC, PATH_RECURRENT, CkdaError,
-                   chunk_fwd, chunk_fwd_noalloc, chunk_path, chunk_segments, decode_step,
+                   bwd, bwd_workspace_bytes, chunk_fwd, chunk_fwd_noalloc, chunk_path, chunk_segments, decode_step,
                    get_device_error, load, recurrent_fwd, workspace_bytes, LIB_PATH)
 
-__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES", "recurrent_fwd", "decode_step",
+__all__ = ["bwd", "bwd_workspace_bytes", "chunk_fwd", "chunk_fwd_noalloc", "NOALLOC_SCRATCH_BYTES", "recurrent_fwd", "decode_step",
            "workspace_bytes", "chunk_path", "chunk_segments", "get_device_error", "load", "CkdaError", "LIB_PATH", "F32", "BF16",
            "PATH_RECURRENT", "PATH_CHUNK_TC"]

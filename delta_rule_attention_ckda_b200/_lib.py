@@ -60,6 +60,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_recurrent_fwd_ex.restype = i
     lib.ckda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp]
     lib.ckda_chunk_fwd_noalloc.restype = i
+    lib.ckda_bwd_workspace_bytes.argtypes = [i] * 6
+    lib.ckda_bwd_workspace_bytes.restype = sz
+    lib.ckda_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp] + [i] * 7 + [vp, sz, vp]
+    lib.ckda_bwd.restype = i
     lib.ckda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 5 + [vp]
     lib.ckda_decode_step.restype = i
     lib.ckda_get_device_error.argtypes = [vp]
@@ -182,6 +186,53 @@ def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_s
                                        _stream(stream))
     _raise(st, "ckda_chunk_fwd_noalloc")
     return o, S_T
+
+
+def bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    return int(load().ckda_bwd_workspace_bytes(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
+
+
+def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, grads=None,
+        workspace=None, stream=None, gate="signed"):
+    """ckda_bwd: gradients of L = <grad_o, o> + <grad_S_T, S_T> for the forward of chunk_fwd.
+    Returns a dict with dq, dk, dv, dalpha (dL/dg for gate="log"), dbeta and dS0 (None
+    unless want_dS0). Output tensors may be passed in `grads` (same keys); the workspace
+    is allocated with torch when not given."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _check(q, "q", (B, T, H, dk))
+    _check(k, "k", (B, T, H, dk), dt)
+    _check(v, "v", (B, T, H, dv), dt)
+    _check(alpha, "alpha", (B, T, H, dk), torch.float32)
+    _check(beta, "beta", (B, T, H), torch.float32)
+    _check(grad_o, "grad_o", (B, T, H, dv), torch.float32)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    if grad_S_T is not None:
+        _check(grad_S_T, "grad_S_T", (B, H, dk, dv), torch.float32)
+    g = dict(grads or {})
+    f32 = dict(device=q.device, dtype=torch.float32)
+    shapes = {"dq": (B, T, H, dk), "dk": (B, T, H, dk), "dv": (B, T, H, dv), "dalpha": (B, T, H, dk),
+              "dbeta": (B, T, H), "dS0": (B, H, dk, dv)}
+    for name, shp in shapes.items():
+        if name == "dS0" and not want_dS0:
+            g[name] = None
+            continue
+        if g.get(name) is None:
+            g[name] = torch.empty(shp, **f32)
+        _check(g[name], name, shp, torch.float32)
+    lib = load()
+    need = int(lib.ckda_bwd_workspace_bytes(B, T, H, dk, dv, _dt(q)))
+    if need and workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ckda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(grad_o),
+                      _ptr(grad_S_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]),
+                      _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q), _gate(gate),
+                      _ptr(workspace), wbytes, _stream(stream))
+    _raise(st, "ckda_bwd")
+    return g
 
 
 def recurrent_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,

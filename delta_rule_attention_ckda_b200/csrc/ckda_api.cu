@@ -13,6 +13,7 @@
 #include "kernels/recurrent.cuh"
 #include "kernels/decode.cuh"
 #include "kernels/chunk_tc.cuh"
+#include "kernels/bwd.cuh"
 
 namespace {
 
@@ -210,6 +211,63 @@ ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const 
                              size_t workspace_bytes, void* stream) {
     return ckda_chunk_fwd_ex(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt, CKDA_GATE_SIGNED,
                              workspace, workspace_bytes, stream);
+}
+
+size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {
+    (void)dt;
+    if (B <= 0 || T <= 0 || H <= 0 || !dims_ok(dk, dv)) return 0;
+    const size_t bh = (size_t)B * H, nblk = ((size_t)T + ckda::bwd::KB - 1) / ckda::bwd::KB;
+    return (bh * nblk * dk * dv + bh * ckda::bwd::SCRATCH_FLOATS_PER_CTA) * sizeof(float);
+}
+
+ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float* gate, const float* beta,
+                       const float* S0, const float* grad_o, const float* grad_S_T, float* grad_q,
+                       float* grad_k, float* grad_v, float* grad_gate, float* grad_beta, float* grad_S0,
+                       int B, int T, int H, int dk, int dv, ckda_dtype_t dt, ckda_gate_t gate_mode,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
+    if (dt != CKDA_F32 && dt != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
+    const bool any_tokens = (long long)B * T * H > 0;
+    if (any_tokens && (!q || !k || !v || !gate || !beta || !grad_o || !grad_q || !grad_k || !grad_v ||
+                       !grad_gate || !grad_beta))
+        return CKDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, gate, beta, S0, grad_o, grad_S_T, grad_q, grad_k, grad_v, grad_gate,
+                          grad_beta, grad_S0, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return CKDA_ERR_MISALIGNED;
+    const size_t need = ckda_bwd_workspace_bytes(B, T, H, dk, dv, dt);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    if ((long long)B * H == 0) return CKDA_OK;
+    if (T == 0) return copy_state(grad_S_T, grad_S0, (size_t)B * H * dk * dv, st);
+    const size_t bh = (size_t)B * H;
+    const size_t nblk = ((size_t)T + ckda::bwd::KB - 1) / ckda::bwd::KB;
+    (void)nblk;
+    float* scratch = static_cast<float*>(workspace);                  // 16-byte aligned, float4 access
+    float* ckpt = scratch + bh * ckda::bwd::SCRATCH_FLOATS_PER_CTA;
+    const bool lg = gate_mode == CKDA_GATE_LOG;
+#define CKDA_LAUNCH_BWD(TIN, LG)                                                                          \
+    do {                                                                                                  \
+        const TIN* qq = static_cast<const TIN*>(q);                                                        \
+        const TIN* kk = static_cast<const TIN*>(k);                                                        \
+        const TIN* vv = static_cast<const TIN*>(v);                                                        \
+        ckda::bwd_ckpt_kernel<TIN, LG><<<(unsigned)bh, ckda::bwd::NT, 0, st>>>(qq, kk, vv, gate, beta, S0, \
+                                                                             ckpt, T, H, dk, dv);          \
+        ckda::bwd_grad_kernel<TIN, LG><<<(unsigned)bh, ckda::bwd::NT, 0, st>>>(                            \
+            qq, kk, vv, gate, beta, grad_o, grad_S_T, ckpt, scratch, grad_q, grad_k, grad_v, grad_gate,    \
+            grad_beta, grad_S0, T, H, dk, dv);                                                             \
+    } while (0)
+    if (dt == CKDA_BF16) {
+        if (lg) CKDA_LAUNCH_BWD(__nv_bfloat16, true);
+        else CKDA_LAUNCH_BWD(__nv_bfloat16, false);
+    } else {
+        if (lg) CKDA_LAUNCH_BWD(float, true);
+        else CKDA_LAUNCH_BWD(float, false);
+    }
+#undef CKDA_LAUNCH_BWD
+    return launch_status();
 }
 
 ckda_status_t ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,

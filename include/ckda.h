@@ -52,7 +52,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 3
+#define CKDA_ABI_VERSION 4
 
 typedef enum {
     CKDA_OK = 0,
@@ -209,6 +209,40 @@ CKDA_API ckda_status_t ckda_decode_step(const void* q, const void* k, const void
                                const float* alpha, const float* beta,
                                float* S, float* o,
                                int N, int H, int dk, int dv, ckda_dtype_t dt, void* stream);
+
+/*
+ * Bytes of device workspace ckda_bwd needs (0 for empty problems): the forward state
+ * at every 8th token, B*H*ceil(T/8)*dk*dv fp32, plus a 512 KiB scratch per (b, h).
+ */
+CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
+
+/*
+ * Backward pass: the gradients of the forward map of ckda_chunk_fwd_ex for the loss
+ *     L = sum_t <grad_o_t, o_t> + <grad_S_T, S_T>
+ * (the vector-Jacobian product with cotangents grad_o and grad_S_T). The pages measure
+ * the forward and backward passes together and mention a sign-aware backward kernel
+ * (ai.info summary of the Complex KDA paper, "Main Findings"); they print no backward
+ * formulas, so this is the derivative of the recurrence itself, taken token by token
+ * in reverse on CUDA cores in fp32 from states recomputed out of checkpoints.
+ *   q, k, v, gate, beta, S0, B..dv, dt, gate_mode: as for ckda_chunk_fwd_ex (S0 may
+ *              be NULL: zero initial state; any dk, dv <= 128; fp32 or bf16 q, k, v)
+ *   grad_o     [B,T,H,dv] fp32 cotangent of o (required when B*T*H > 0)
+ *   grad_S_T   [B,H,dk,dv] fp32 cotangent of the final state, or NULL (zero)
+ *   grad_q, grad_k [B,T,H,dk] fp32 out   grad_v [B,T,H,dv] fp32 out
+ *   grad_gate  [B,T,H,dk] fp32 out: dL/dalpha (CKDA_GATE_SIGNED) or dL/dg (CKDA_GATE_LOG)
+ *   grad_beta  [B,T,H] fp32 out          grad_S0 [B,H,dk,dv] fp32 out, or NULL (not written)
+ *   workspace  device buffer of at least ckda_bwd_workspace_bytes(...) bytes, owned by
+ *              the caller.
+ * Every pointer is 16-byte aligned; outputs must not overlap inputs. Returns CKDA_OK or
+ * an error status (nothing launched on argument errors).
+ */
+CKDA_API ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float* gate,
+                                const float* beta, const float* S0, const float* grad_o,
+                                const float* grad_S_T, float* grad_q, float* grad_k, float* grad_v,
+                                float* grad_gate, float* grad_beta, float* grad_S0,
+                                int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                ckda_gate_t gate_mode, void* workspace, size_t workspace_bytes,
+                                void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears this GPU's device error word.

@@ -49,7 +49,7 @@ def test_status_strings(lib):
         s = lib.ckda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.ckda_status_string(99) == b"unknown status"
-    assert lib.ckda_abi_version() == 3
+    assert lib.ckda_abi_version() == 4
 
 
 NULL = None
@@ -130,6 +130,36 @@ def test_segment_plan(lib):
     assert lib.ckda_chunk_fwd_segments(1, 65536, 16, 128, 128, 0) == 1
     assert lib.ckda_chunk_fwd_segments(0, 65536, 16, 128, 128, bf) == 1
     assert lib.ckda_chunk_fwd_segments(1, 65536, 16, 32, 32, bf) == 1
+
+
+def test_bwd_workspace_and_argument_checks(lib):
+    """ckda_bwd's workspace: 8-token checkpoints plus a 512 KiB scratch per sequence;
+    argument errors return before anything touches the device."""
+    import ctypes
+    assert lib.ckda_bwd_workspace_bytes(2, 17, 3, 16, 8, 0) == (2 * 3 * 3 * 16 * 8 + 2 * 3 * 131072) * 4
+    assert lib.ckda_bwd_workspace_bytes(0, 17, 3, 16, 8, 0) == 0
+    assert lib.ckda_bwd_workspace_bytes(1, 0, 3, 16, 8, 0) == 0
+    assert lib.ckda_bwd_workspace_bytes(1, 4, 1, 0, 8, 0) == 0
+    p = ctypes.c_void_p(256)
+    fp = ctypes.cast(p, ctypes.POINTER(ctypes.c_float))
+    null = ctypes.POINTER(ctypes.c_float)()
+    ws = ctypes.c_void_p(4096)
+    big = 1 << 40
+    # missing grad_o
+    assert lib.ckda_bwd(p, p, p, fp, fp, null, null, null, fp, fp, fp, fp, fp, null,
+                        1, 4, 1, 16, 16, 0, 0, ws, big, None) == 1
+    # unknown gate mode, bad head size
+    assert lib.ckda_bwd(p, p, p, fp, fp, null, fp, null, fp, fp, fp, fp, fp, null,
+                        1, 4, 1, 16, 16, 0, 7, ws, big, None) == 1
+    assert lib.ckda_bwd(p, p, p, fp, fp, null, fp, null, fp, fp, fp, fp, fp, null,
+                        1, 4, 1, 129, 16, 0, 0, ws, big, None) == 1
+    # misaligned output
+    bad = ctypes.cast(ctypes.c_void_p(260), ctypes.POINTER(ctypes.c_float))
+    assert lib.ckda_bwd(p, p, p, fp, fp, null, fp, null, bad, fp, fp, fp, fp, null,
+                        1, 4, 1, 16, 16, 0, 0, ws, big, None) == 3
+    # workspace too small
+    assert lib.ckda_bwd(p, p, p, fp, fp, null, fp, null, fp, fp, fp, fp, fp, null,
+                        1, 4, 1, 16, 16, 0, 0, ws, 16, None) == 6
 
 
 def test_python_binding_refuses_cpu_tensors():
