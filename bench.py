@@ -343,6 +343,7 @@ def ours_arm(args):
     if not args.no_extras:
         line["kda"] = kda_measure(ck, q, k, v, a, b, o, ST, stream, world, args.steps, value)
         line["configs"] = configs_measure(ck, dev, stream, world)
+        line["bwd"] = bwd_measure(ck, q, k, v, a, b, stream, world)
     if not args.no_e2e:
         line["e2e"] = e2e_measure(ck, inp, dev, stream, world, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -393,6 +394,43 @@ def configs_measure(ck, dev, stream, world):
                         "alg_bytes_per_launch": alg}})
         out[name] = ent
     return out
+
+
+def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
+    """The backward pass (ckda_bwd) of the same layer step: gradients of <dO, o> for q,
+    k, v, alpha, beta and S0, from a fixed synthetic cotangent dO. Tokens/s and the
+    algorithmic HBM bytes (inputs and cotangent read once, gradients written once)."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    g = torch.Generator(device="cpu").manual_seed(11)
+    dO = torch.randn(B, T, H, dv, generator=g).to(q.device)
+    grads = {n: torch.empty(s, device=q.device) for n, s in (
+        ("dq", (B, T, H, dk)), ("dk", (B, T, H, dk)), ("dv", (B, T, H, dv)), ("dalpha", (B, T, H, dk)),
+        ("dbeta", (B, T, H)), ("dS0", (B, H, dk, dv)))}
+    ws = torch.empty(ck.bwd_workspace_bytes(B, T, H, dk, dv), device=q.device, dtype=torch.uint8)
+
+    def step():
+        ck.bwd(q, k, v, a, b, dO, None, None, grads=grads, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    barrier(world)
+    secs = time_launches(step, reps, stream)
+    assert ck.get_device_error() == 0
+    value, secs = aggregate_throughput(B * T * reps, secs, world, device="cuda")
+    per = secs / reps
+    in_bytes = 2 * dk * 2 + dv * 2 + dk * 4 + 4 + dv * 4          # q, k, v (bf16), alpha, beta, dO
+    out_bytes = 3 * dk * 4 + dv * 4 + 4                             # dq, dk, dalpha, dv, dbeta
+    alg = B * T * H * (in_bytes + out_bytes) + B * H * dk * dv * 4   # + dS0
+    hbm, _ = peaks()
+    del ws
+    return {"workload": f"layer B={B} T={T} H={H} dk={dk} dv={dv}, backward of <dO, o> (S0 = 0)",
+            "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": 2 * reps,
+            "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg,
+                         "kernels": "bwd_ckpt_kernel + bwd_grad_kernel (fp32 CUDA cores)"}}
 
 
 def kda_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, ckda_value):

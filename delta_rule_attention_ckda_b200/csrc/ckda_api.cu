@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kernels/common.cuh"
@@ -217,7 +218,11 @@ size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_
     (void)dt;
     if (B <= 0 || T <= 0 || H <= 0 || !dims_ok(dk, dv)) return 0;
     const size_t bh = (size_t)B * H, nblk = ((size_t)T + ckda::bwd::KB - 1) / ckda::bwd::KB;
-    return (bh * nblk * dk * dv + bh * ckda::bwd::SCRATCH_FLOATS_PER_CTA) * sizeof(float);
+    const size_t nsl = (size_t)ckda::bwd::slabs(dv), nrow = bh * (size_t)T;
+    return (bh * nsl * ckda::bwd::SCRATCH_FLOATS_PER_CTA     // recomputed states
+            + bh * nblk * dk * dv                             // checkpoints
+            + nsl * nrow * 3 * dk + nsl * nrow)               // per-slab partial row sums
+           * sizeof(float);
 }
 
 ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float* gate, const float* beta,
@@ -242,22 +247,29 @@ ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float*
     cudaStream_t st = as_stream(stream);
     if ((long long)B * H == 0) return CKDA_OK;
     if (T == 0) return copy_state(grad_S_T, grad_S0, (size_t)B * H * dk * dv, st);
-    const size_t bh = (size_t)B * H;
+    const size_t bh = (size_t)B * H, nrow = bh * (size_t)T;
     const size_t nblk = ((size_t)T + ckda::bwd::KB - 1) / ckda::bwd::KB;
-    (void)nblk;
+    const int nsl = ckda::bwd::slabs(dv);
     float* scratch = static_cast<float*>(workspace);                  // 16-byte aligned, float4 access
-    float* ckpt = scratch + bh * ckda::bwd::SCRATCH_FLOATS_PER_CTA;
+    float* ckpt = scratch + bh * nsl * ckda::bwd::SCRATCH_FLOATS_PER_CTA;
+    float* part = ckpt + bh * nblk * dk * dv;
+    float* partb = part + (size_t)nsl * nrow * 3 * dk;
+    const dim3 grid((unsigned)bh, (unsigned)nsl);
+    const size_t nsum = nrow * dk;
+    const unsigned sum_blocks = (unsigned)std::min<size_t>((nsum + 255) / 256, 148 * 16);
     const bool lg = gate_mode == CKDA_GATE_LOG;
 #define CKDA_LAUNCH_BWD(TIN, LG)                                                                          \
     do {                                                                                                  \
         const TIN* qq = static_cast<const TIN*>(q);                                                        \
         const TIN* kk = static_cast<const TIN*>(k);                                                        \
         const TIN* vv = static_cast<const TIN*>(v);                                                        \
-        ckda::bwd_ckpt_kernel<TIN, LG><<<(unsigned)bh, ckda::bwd::NT, 0, st>>>(qq, kk, vv, gate, beta, S0, \
-                                                                             ckpt, T, H, dk, dv);          \
-        ckda::bwd_grad_kernel<TIN, LG><<<(unsigned)bh, ckda::bwd::NT, 0, st>>>(                            \
-            qq, kk, vv, gate, beta, grad_o, grad_S_T, ckpt, scratch, grad_q, grad_k, grad_v, grad_gate,    \
-            grad_beta, grad_S0, T, H, dk, dv);                                                             \
+        ckda::bwd_ckpt_kernel<TIN, LG><<<grid, ckda::bwd::NT, 0, st>>>(qq, kk, vv, gate, beta, S0, ckpt, T, \
+                                                                     H, dk, dv);                          \
+        ckda::bwd_grad_kernel<TIN, LG><<<grid, ckda::bwd::NT, 0, st>>>(                                    \
+            qq, kk, vv, gate, beta, grad_o, grad_S_T, ckpt, scratch, part, partb, grad_v, grad_S0, B, T, H, \
+            dk, dv);                                                                                      \
+        ckda::bwd_sum_kernel<LG><<<sum_blocks, 256, 0, st>>>(part, partb, gate, grad_q, grad_k, grad_gate, \
+                                                             grad_beta, nrow, dk, nsl);                   \
     } while (0)
     if (dt == CKDA_BF16) {
         if (lg) CKDA_LAUNCH_BWD(__nv_bfloat16, true);

@@ -211,8 +211,10 @@ CKDA_API ckda_status_t ckda_decode_step(const void* q, const void* k, const void
                                int N, int H, int dk, int dv, ckda_dtype_t dt, void* stream);
 
 /*
- * Bytes of device workspace ckda_bwd needs (0 for empty problems): the forward state
- * at every 8th token, B*H*ceil(T/8)*dk*dv fp32, plus a 512 KiB scratch per (b, h).
+ * Bytes of device workspace ckda_bwd needs (0 for empty problems), all fp32: the
+ * forward state at every 8th token (B*H*ceil(T/8)*dk*dv), recomputed states (128 KiB
+ * per (b, h) and 32-column slab of the state) and per-slab partial sums of the row
+ * gradients (slabs*B*T*H*(3*dk + 1)), where slabs = ceil(dv / 32).
  */
 CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
 

@@ -133,10 +133,14 @@ def test_segment_plan(lib):
 
 
 def test_bwd_workspace_and_argument_checks(lib):
-    """ckda_bwd's workspace: 8-token checkpoints plus a 512 KiB scratch per sequence;
+    """ckda_bwd's workspace: 8-token checkpoints, recomputed states and row partials;
     argument errors return before anything touches the device."""
     import ctypes
-    assert lib.ckda_bwd_workspace_bytes(2, 17, 3, 16, 8, 0) == (2 * 3 * 3 * 16 * 8 + 2 * 3 * 131072) * 4
+    # 6 sequences, 3 checkpoint blocks, one 32-column slab: checkpoints + states + partials
+    assert lib.ckda_bwd_workspace_bytes(2, 17, 3, 16, 8, 0) == (
+        6 * 3 * 16 * 8 + 6 * 8 * 128 * 32 + 6 * 17 * (3 * 16 + 1)) * 4
+    assert lib.ckda_bwd_workspace_bytes(1, 8, 1, 128, 100, 0) == (
+        1 * 128 * 100 + 4 * 8 * 128 * 32 + 4 * 8 * (3 * 128 + 1)) * 4
     assert lib.ckda_bwd_workspace_bytes(0, 17, 3, 16, 8, 0) == 0
     assert lib.ckda_bwd_workspace_bytes(1, 0, 3, 16, 8, 0) == 0
     assert lib.ckda_bwd_workspace_bytes(1, 4, 1, 0, 8, 0) == 0
