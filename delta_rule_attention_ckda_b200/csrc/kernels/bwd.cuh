@@ -172,7 +172,7 @@ __device__ __forceinline__ void ld_scratch(float (&S)[4][4], const float4* slot)
 // Pass 1: the forward over T, keeping S_{8n - 1} (the state entering token 8n) as
 // checkpoint n (ckpt: [B*H][nblk][d_k][d_v]; checkpoint 0 = S0). Grid: (B*H, slabs).
 template <typename TIn, bool kLogGate>
-__global__ void __launch_bounds__(bwd::NT)
+__global__ void __launch_bounds__(bwd::NT, 4)
 bwd_ckpt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta, const float* S0,
                 float* __restrict__ ckpt, int T, int H, int dk, int dv) {
@@ -203,7 +203,7 @@ bwd_ckpt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
 // dv and dS0 are written directly; dq, dk, da and db as per-slab partials
 // (part: [slabs][B*T*H][3][d_k], partb: [slabs][B*T*H]).
 template <typename TIn, bool kLogGate>
-__global__ void __launch_bounds__(bwd::NT)
+__global__ void __launch_bounds__(bwd::NT, 4)
 bwd_grad_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta, const float* __restrict__ dO,
                 const float* dST, const float* __restrict__ ckpt, float* __restrict__ scratch,
