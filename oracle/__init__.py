@@ -79,11 +79,29 @@ def set_threads(n: int) -> None:
     _load().ckda_oracle_set_threads(int(n))
 
 
-def oracle_fwd(q, k, v, alpha, beta, S0=None, want_state: bool = True
+NORM_EPS = 1e-12
+
+
+def normalize_rows(x) -> np.ndarray:
+    """x / max(||x||_2, 1e-12) over the last axis, in fp64: the L2 normalisation of q and k
+    per token and head that a layer applies before the recurrence (the ai.info summary
+    of the Complex KDA paper: keys are unit vectors, ||k|| = 1, for the transition
+    (I - b k k^T) Diag(a) to be a Householder-type reflection). The floor on the norm is
+    torch.nn.functional.normalize's default; the pages give none."""
+    x = _f64(x)
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return x / np.maximum(n, NORM_EPS)
+
+
+def oracle_fwd(q, k, v, alpha, beta, S0=None, want_state: bool = True, normalize_qk: bool = False
                ) -> Tuple[np.ndarray, Optional[np.ndarray]]:
     """Run the recurrence. Shapes: q,k,alpha [B,T,H,dk]; v [B,T,H,dv]; beta [B,T,H];
-    S0 [B,H,dk,dv] or None. Returns (o [B,T,H,dv], S_T [B,H,dk,dv] or None), fp64."""
+    S0 [B,H,dk,dv] or None. With normalize_qk, q and k are first divided by their L2
+    norms per token and head (normalize_rows). Returns (o [B,T,H,dv], S_T [B,H,dk,dv]
+    or None), fp64."""
     q, k, v, alpha, beta, S0 = map(_f64, (q, k, v, alpha, beta, S0))
+    if normalize_qk:
+        q, k = normalize_rows(q), normalize_rows(k)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     assert k.shape == (B, T, H, dk) and alpha.shape == (B, T, H, dk)

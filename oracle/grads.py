@@ -36,10 +36,14 @@ def _t64(x):
     return torch.as_tensor(np.asarray(x, dtype=np.float64)).clone()
 
 
-def oracle_bwd(q, k, v, alpha, beta, dO, S0=None, dST=None) -> Dict[str, np.ndarray]:
+def oracle_bwd(q, k, v, alpha, beta, dO, S0=None, dST=None, normalize_qk: bool = False
+               ) -> Dict[str, np.ndarray]:
     """Gradients of L = <dO, o> + <dST, S_T> for the recurrence above.
     Shapes: q, k, alpha [B,T,H,dk]; v, dO [B,T,H,dv]; beta [B,T,H]; S0, dST [B,H,dk,dv]
-    (None = zero). Returns dict with keys dq, dk, dv, dalpha, dbeta, dS0 (fp64 numpy)."""
+    (None = zero). With normalize_qk the forward first divides q and k by their L2 norms
+    per token and head (floor 1e-12, as oracle.normalize_rows) and the gradients are
+    with respect to the raw q and k. Returns dict with keys dq, dk, dv, dalpha, dbeta,
+    dS0 (fp64 numpy)."""
     import torch
     q, k, v, alpha, beta, dO = (_t64(x) for x in (q, k, v, alpha, beta, dO))
     B, T, H, dk = q.shape
@@ -48,6 +52,9 @@ def oracle_bwd(q, k, v, alpha, beta, dO, S0=None, dST=None) -> Dict[str, np.ndar
     leaves = [q, k, v, alpha, beta, S0]
     for x in leaves:
         x.requires_grad_(True)
+    if normalize_qk:
+        q = q / torch.linalg.vector_norm(q, dim=-1, keepdim=True).clamp_min(1e-12)
+        k = k / torch.linalg.vector_norm(k, dim=-1, keepdim=True).clamp_min(1e-12)
     S = S0
     outs = []
     for t in range(T):

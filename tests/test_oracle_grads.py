@@ -98,3 +98,48 @@ def test_worked_quarter_turn_readout_gradient():
     for t in range(T):
         St = np.linalg.matrix_power(A, t + 1)
         np.testing.assert_allclose(g["dq"][0, t, 0], St @ dO[0, t, 0], atol=1e-12)
+
+
+def test_normalize_rows_definition():
+    """Rows end with unit norm; positive per-row scaling does not change them; a zero
+    row stays zero (the norm is floored, nothing is divided by zero)."""
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((3, 5, 2, 7))
+    x[0, 0, 0] = 0.0
+    y = oracle.normalize_rows(x)
+    n = np.linalg.norm(y, axis=-1)
+    assert np.allclose(n[x.any(axis=-1)], 1.0, atol=1e-15) and (y[0, 0, 0] == 0).all()
+    s = rng.uniform(0.1, 10.0, size=x.shape[:-1] + (1,))
+    np.testing.assert_allclose(oracle.normalize_rows(x * s), y, atol=1e-15)
+
+
+def test_normalized_forward_is_scale_invariant():
+    q, k, v, a, b, S0, dO, dST = _problem(13)
+    rng = np.random.default_rng(14)
+    sq = rng.uniform(0.2, 5.0, size=q.shape[:-1] + (1,))
+    sk = rng.uniform(0.2, 5.0, size=k.shape[:-1] + (1,))
+    o1, S1 = oracle.oracle_fwd(q, k, v, a, b, S0, normalize_qk=True)
+    o2, S2 = oracle.oracle_fwd(q * sq, k * sk, v, a, b, S0, normalize_qk=True)
+    np.testing.assert_allclose(o2, o1, atol=1e-12)
+    np.testing.assert_allclose(S2, S1, atol=1e-12)
+
+
+@pytest.mark.parametrize("which", ["q", "k"])
+def test_normalized_gradient_matches_central_differences(which):
+    q, k, v, a, b, S0, dO, dST = _problem(15)
+    q = 3.0 * q
+    k = 0.5 * k
+    g = oracle_bwd(q, k, v, a, b, dO, S0=S0, dST=dST, normalize_qk=True)
+    rng = np.random.default_rng(16)
+    x = q if which == "q" else k
+    d = rng.standard_normal(x.shape)
+    eps = 1e-6
+
+    def loss(xx):
+        qq, kk = (xx, k) if which == "q" else (q, xx)
+        o, ST = oracle.oracle_fwd(qq, kk, v, a, b, S0, normalize_qk=True)
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    fd = (loss(x + eps * d) - loss(x - eps * d)) / (2 * eps)
+    an = float(np.sum(g["d" + which] * d))
+    assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (fd, an)
