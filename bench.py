@@ -344,6 +344,7 @@ def ours_arm(args):
         line["kda"] = kda_measure(ck, q, k, v, a, b, o, ST, stream, world, args.steps, value)
         line["configs"] = configs_measure(ck, dev, stream, world)
         line["bwd"] = bwd_measure(ck, q, k, v, a, b, stream, world)
+        line["normalize_qk"] = norm_measure(ck, q, k, v, a, b, o, ST, stream, world, args.steps, value)
     if not args.no_e2e:
         line["e2e"] = e2e_measure(ck, inp, dev, stream, world, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -431,6 +432,34 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
             "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg,
                          "kernels": "bwd_ckpt_kernel + bwd_grad_kernel (fp32 CUDA cores)"}}
+
+
+def norm_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, plain_value):
+    """The layer step with q and k L2-normalised inside the kernel (CKDA_OPT_NORMALIZE_QK),
+    next to the same step fed by a separate normalisation pass (torch, bf16 in and out)."""
+    import torch
+    B, T, H, dk = q.shape
+
+    def fused():
+        ck.chunk_fwd(q, k, v, a, b, None, o=o, S_T=ST, normalize_qk=True)
+
+    def separate():
+        qn = torch.nn.functional.normalize(q.float(), dim=-1).to(q.dtype)
+        kn = torch.nn.functional.normalize(k.float(), dim=-1).to(k.dtype)
+        ck.chunk_fwd(qn, kn, v, a, b, None, o=o, S_T=ST)
+
+    out = {"workload": "layer, q and k L2-normalised per token and head"}
+    for name, fn in (("fused", fused), ("separate_torch_pass", separate)):
+        for _ in range(3):
+            fn()
+        assert ck.get_device_error() == 0
+        barrier(world)
+        secs = time_launches(fn, steps, stream)
+        value, secs = aggregate_throughput(B * T * steps, secs, world, device="cuda")
+        out[name] = {"value": value, "unit": "tokens/s", "ms_per_step": 1e3 * secs / steps}
+    out["fused_over_plain"] = out["fused"]["value"] / plain_value
+    out["gpu_launches"] = steps
+    return out
 
 
 def kda_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, ckda_value):

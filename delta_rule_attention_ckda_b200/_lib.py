@@ -143,16 +143,26 @@ def _fwd_common(q, k, v, alpha, beta, S0, o, S_T):
 GATES = {"signed": 0, "log": 1}       # ckda_gate_t: alpha in [-1,1], or g = ln(alpha) (KDA form)
 
 
+OPT_NORMALIZE_QK = 0x100              # CKDA_OPT_NORMALIZE_QK
+
+
 def _gate(gate: str) -> int:
     if gate not in GATES:
         raise ValueError(f"gate must be one of {sorted(GATES)}, got {gate!r}")
     return GATES[gate]
 
 
+def _mode(gate: str, normalize_qk: bool) -> int:
+    """The C mode argument: the gate form, OR-ed with CKDA_OPT_NORMALIZE_QK if asked."""
+    return _gate(gate) | (OPT_NORMALIZE_QK if normalize_qk else 0)
+
+
 def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
-              workspace=None, stream=None, gate="signed") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              workspace=None, stream=None, gate="signed",
+              normalize_qk=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """ckda_chunk_fwd_ex. Returns (o, S_T). `alpha` is the gate in the form `gate` names:
     "signed" (alpha in [-1,1], CKDA) or "log" (g = ln(alpha) of a non-negative gate, KDA).
+    normalize_qk: q and k are L2-normalised per token and head inside the kernels.
     Allocates o / S_T / workspace with torch when not given (the library never allocates)."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
     if S_T is None and want_state:
@@ -163,8 +173,8 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=Tru
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.ckda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o),
-                               _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate), _ptr(workspace), wbytes,
-                               _stream(stream))
+                               _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk), _ptr(workspace),
+                               wbytes, _stream(stream))
     _raise(st, "ckda_chunk_fwd_ex")
     return o, S_T
 
@@ -173,7 +183,8 @@ NOALLOC_SCRATCH_BYTES = 20 << 20      # CKDA_NOALLOC_SCRATCH_BYTES
 
 
 def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
-                      stream=None, gate="signed") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                      stream=None, gate="signed",
+                      normalize_qk=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """ckda_chunk_fwd_noalloc: ckda_chunk_fwd_ex on the library's fixed device scratch
     (no workspace argument; the call allocates nothing). Raises CkdaError(WORKSPACE)
     when the problem needs more than NOALLOC_SCRATCH_BYTES of scratch. o / S_T are
@@ -182,7 +193,7 @@ def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_s
     if S_T is None and want_state:
         S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
     st = load().ckda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
-                                       _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate),
+                                       _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk),
                                        _stream(stream))
     _raise(st, "ckda_chunk_fwd_noalloc")
     return o, S_T
@@ -193,7 +204,7 @@ def bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
 
 
 def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, grads=None,
-        workspace=None, stream=None, gate="signed"):
+        workspace=None, stream=None, gate="signed", normalize_qk=False):
     """ckda_bwd: gradients of L = <grad_o, o> + <grad_S_T, S_T> for the forward of chunk_fwd.
     Returns a dict with dq, dk, dv, dalpha (dL/dg for gate="log"), dbeta and dS0 (None
     unless want_dS0). Output tensors may be passed in `grads` (same keys); the workspace
@@ -229,20 +240,21 @@ def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, 
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.ckda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(grad_o),
                       _ptr(grad_S_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]),
-                      _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q), _gate(gate),
+                      _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q), _mode(gate, normalize_qk),
                       _ptr(workspace), wbytes, _stream(stream))
     _raise(st, "ckda_bwd")
     return g
 
 
 def recurrent_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
-                  stream=None, gate="signed") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                  stream=None, gate="signed", normalize_qk=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """ckda_recurrent_fwd_ex (fp32 SIMT token-by-token kernel). Returns (o, S_T)."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
     if S_T is None and want_state:
         S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
     st = load().ckda_recurrent_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
-                                      _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _gate(gate), _stream(stream))
+                                      _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk),
+                                      _stream(stream))
     _raise(st, "ckda_recurrent_fwd_ex")
     return o, S_T
 

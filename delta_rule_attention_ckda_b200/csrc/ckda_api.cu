@@ -39,7 +39,7 @@ ckda_status_t copy_state(const float* S0, float* S_T, size_t n, cudaStream_t st)
     return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
-template <typename TIn, bool kLogGate>
+template <typename TIn, bool kLogGate, bool kNorm>
 ckda_status_t launch_recurrent(const TIn* q, const TIn* k, const TIn* v, const float* alpha,
                                const float* beta, const float* S0, float* o, float* S_T,
                                int B, int T, int H, int dk, int dv, cudaStream_t st) {
@@ -50,7 +50,7 @@ ckda_status_t launch_recurrent(const TIn* q, const TIn* k, const TIn* v, const f
     dim3 grid((unsigned)seqs, (unsigned)((dv + cols_per_cta - 1) / cols_per_cta));
     dim3 block((unsigned)cols_per_cta);
 #define CKDA_LAUNCH_REC(DKT)                                                                  \
-    ckda::recurrent_fwd_kernel<DKT, TIn, kLogGate><<<grid, block, 0, st>>>(q, k, v, alpha, beta, S0, o, \
+    ckda::recurrent_fwd_kernel<DKT, TIn, kLogGate, kNorm><<<grid, block, 0, st>>>(q, k, v, alpha, beta, S0, o, \
                                                                   S_T, T, H, dk, dv, cols_per_cta)
     if (dk <= 16) CKDA_LAUNCH_REC(16);
     else if (dk <= 32) CKDA_LAUNCH_REC(32);
@@ -95,6 +95,16 @@ void* noalloc_scratch() {
     return addr[dev];
 }
 
+// mode = a ckda_gate_t value, optionally OR-ed with CKDA_OPT_* bits
+bool parse_mode(int mode, bool* log_gate, bool* norm_qk) {
+    const int gate = mode & 0xFF, opts = mode & ~0xFF;
+    if (gate != CKDA_GATE_SIGNED && gate != CKDA_GATE_LOG) return false;
+    if (opts & ~CKDA_OPT_NORMALIZE_QK) return false;
+    *log_gate = gate == CKDA_GATE_LOG;
+    *norm_qk = (opts & CKDA_OPT_NORMALIZE_QK) != 0;
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -134,26 +144,28 @@ int ckda_chunk_fwd_segments(int B, int T, int H, int dk, int dv, ckda_dtype_t dt
 ckda_status_t ckda_recurrent_fwd_ex(const void* q, const void* k, const void* v,
                                     const float* gate, const float* beta, const float* S0,
                                     float* o, float* S_T, int B, int T, int H, int dk, int dv,
-                                    ckda_dtype_t dt, ckda_gate_t gate_mode, void* stream) {
-    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+                                    ckda_dtype_t dt, int mode, void* stream) {
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return CKDA_ERR_INVALID_ARG;
     ckda_status_t s = check_fwd_args(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt);
     if (s != CKDA_OK) return s;
     cudaStream_t st = as_stream(stream);
     if ((long long)B * H == 0) return CKDA_OK;
     if (T == 0) return copy_state(S0, S_T, (size_t)B * H * dk * dv, st);
-    const bool lg = gate_mode == CKDA_GATE_LOG;
-    if (dt == CKDA_BF16) {
-        const auto* qb = static_cast<const __nv_bfloat16*>(q);
-        const auto* kb = static_cast<const __nv_bfloat16*>(k);
-        const auto* vb = static_cast<const __nv_bfloat16*>(v);
-        return lg ? launch_recurrent<__nv_bfloat16, true>(qb, kb, vb, gate, beta, S0, o, S_T, B, T, H, dk, dv, st)
-                  : launch_recurrent<__nv_bfloat16, false>(qb, kb, vb, gate, beta, S0, o, S_T, B, T, H, dk, dv, st);
-    }
-    const auto* qf = static_cast<const float*>(q);
-    const auto* kf = static_cast<const float*>(k);
-    const auto* vf = static_cast<const float*>(v);
-    return lg ? launch_recurrent<float, true>(qf, kf, vf, gate, beta, S0, o, S_T, B, T, H, dk, dv, st)
-              : launch_recurrent<float, false>(qf, kf, vf, gate, beta, S0, o, S_T, B, T, H, dk, dv, st);
+#define CKDA_REC(TIN)                                                                                   \
+    do {                                                                                                \
+        const auto* qq = static_cast<const TIN*>(q);                                                     \
+        const auto* kk = static_cast<const TIN*>(k);                                                     \
+        const auto* vv = static_cast<const TIN*>(v);                                                     \
+        if (lg)                                                                                         \
+            return nq ? launch_recurrent<TIN, true, true>(qq, kk, vv, gate, beta, S0, o, S_T, B, T, H, dk, dv, st) \
+                      : launch_recurrent<TIN, true, false>(qq, kk, vv, gate, beta, S0, o, S_T, B, T, H, dk, dv, st); \
+        return nq ? launch_recurrent<TIN, false, true>(qq, kk, vv, gate, beta, S0, o, S_T, B, T, H, dk, dv, st)   \
+                  : launch_recurrent<TIN, false, false>(qq, kk, vv, gate, beta, S0, o, S_T, B, T, H, dk, dv, st); \
+    } while (0)
+    if (dt == CKDA_BF16) CKDA_REC(__nv_bfloat16);
+    CKDA_REC(float);
+#undef CKDA_REC
 }
 
 ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const void* v,
@@ -166,9 +178,10 @@ ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const void* v,
 
 ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* gate,
                                 const float* beta, const float* S0, float* o, float* S_T, int B,
-                                int T, int H, int dk, int dv, ckda_dtype_t dt, ckda_gate_t gate_mode,
+                                int T, int H, int dk, int dv, ckda_dtype_t dt, int mode,
                                 void* workspace, size_t workspace_bytes, void* stream) {
-    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return CKDA_ERR_INVALID_ARG;
     ckda_status_t s = check_fwd_args(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt);
     if (s != CKDA_OK) return s;
     const size_t need = ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt);
@@ -181,18 +194,18 @@ ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const void* v, con
         cudaError_t e = ckda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
                                               static_cast<const __nv_bfloat16*>(k),
                                               static_cast<const __nv_bfloat16*>(v), gate, beta,
-                                              S0, o, S_T, B, T, H, dk, dv, gate_mode == CKDA_GATE_LOG,
-                                              workspace, st);
+                                              S0, o, S_T, B, T, H, dk, dv, lg, nq, workspace, st);
         return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
     }
-    return ckda_recurrent_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, gate_mode, stream);
+    return ckda_recurrent_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, mode, stream);
 }
 
 ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* gate,
                                      const float* beta, const float* S0, float* o, float* S_T, int B,
                                      int T, int H, int dk, int dv, ckda_dtype_t dt,
-                                     ckda_gate_t gate_mode, void* stream) {
-    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+                                     int mode, void* stream) {
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return CKDA_ERR_INVALID_ARG;
     ckda_status_t s = check_fwd_args(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt);
     if (s != CKDA_OK) return s;
     const size_t need = ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt);
@@ -202,7 +215,7 @@ ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, const void* v
         ws = noalloc_scratch();
         if (ws == nullptr) return CKDA_ERR_CUDA;
     }
-    return ckda_chunk_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, gate_mode, ws, need,
+    return ckda_chunk_fwd_ex(q, k, v, gate, beta, S0, o, S_T, B, T, H, dk, dv, dt, mode, ws, need,
                              stream);
 }
 
@@ -228,9 +241,10 @@ size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_
 ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float* gate, const float* beta,
                        const float* S0, const float* grad_o, const float* grad_S_T, float* grad_q,
                        float* grad_k, float* grad_v, float* grad_gate, float* grad_beta, float* grad_S0,
-                       int B, int T, int H, int dk, int dv, ckda_dtype_t dt, ckda_gate_t gate_mode,
+                       int B, int T, int H, int dk, int dv, ckda_dtype_t dt, int mode,
                        void* workspace, size_t workspace_bytes, void* stream) {
-    if (gate_mode != CKDA_GATE_SIGNED && gate_mode != CKDA_GATE_LOG) return CKDA_ERR_INVALID_ARG;
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return CKDA_ERR_INVALID_ARG;
     if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
     if (dt != CKDA_F32 && dt != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
     if ((long long)B * H > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
@@ -257,27 +271,32 @@ ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float*
     const dim3 grid((unsigned)bh, (unsigned)nsl);
     const size_t nsum = nrow * dk;
     const unsigned sum_blocks = (unsigned)std::min<size_t>((nsum + 255) / 256, 148 * 16);
-    const bool lg = gate_mode == CKDA_GATE_LOG;
-#define CKDA_LAUNCH_BWD(TIN, LG)                                                                          \
+#define CKDA_LAUNCH_BWD(TIN, LG, NQ)                                                                      \
     do {                                                                                                  \
         const TIN* qq = static_cast<const TIN*>(q);                                                        \
         const TIN* kk = static_cast<const TIN*>(k);                                                        \
         const TIN* vv = static_cast<const TIN*>(v);                                                        \
-        ckda::bwd_ckpt_kernel<TIN, LG><<<grid, ckda::bwd::NT, 0, st>>>(qq, kk, vv, gate, beta, S0, ckpt, T, \
-                                                                     H, dk, dv);                          \
-        ckda::bwd_grad_kernel<TIN, LG><<<grid, ckda::bwd::NT, 0, st>>>(                                    \
+        ckda::bwd_ckpt_kernel<TIN, LG, NQ><<<grid, ckda::bwd::NT, 0, st>>>(qq, kk, vv, gate, beta, S0,     \
+                                                                         ckpt, T, H, dk, dv);              \
+        ckda::bwd_grad_kernel<TIN, LG, NQ><<<grid, ckda::bwd::NT, 0, st>>>(                                \
             qq, kk, vv, gate, beta, grad_o, grad_S_T, ckpt, scratch, part, partb, grad_v, grad_S0, B, T, H, \
             dk, dv);                                                                                      \
         ckda::bwd_sum_kernel<LG><<<sum_blocks, 256, 0, st>>>(part, partb, gate, grad_q, grad_k, grad_gate, \
                                                              grad_beta, nrow, dk, nsl);                   \
+        if (NQ) {                                                                                         \
+            const unsigned nb = (unsigned)std::min<size_t>((nrow + 7) / 8, 148 * 32);                      \
+            ckda::bwd_norm_kernel<TIN><<<nb, 256, 0, st>>>(qq, grad_q, nrow, dk);                          \
+            ckda::bwd_norm_kernel<TIN><<<nb, 256, 0, st>>>(kk, grad_k, nrow, dk);                          \
+        }                                                                                                 \
     } while (0)
-    if (dt == CKDA_BF16) {
-        if (lg) CKDA_LAUNCH_BWD(__nv_bfloat16, true);
-        else CKDA_LAUNCH_BWD(__nv_bfloat16, false);
-    } else {
-        if (lg) CKDA_LAUNCH_BWD(float, true);
-        else CKDA_LAUNCH_BWD(float, false);
-    }
+#define CKDA_LAUNCH_BWD2(TIN)                                                                             \
+    do {                                                                                                  \
+        if (lg) { if (nq) CKDA_LAUNCH_BWD(TIN, true, true); else CKDA_LAUNCH_BWD(TIN, true, false); }      \
+        else { if (nq) CKDA_LAUNCH_BWD(TIN, false, true); else CKDA_LAUNCH_BWD(TIN, false, false); }       \
+    } while (0)
+    if (dt == CKDA_BF16) CKDA_LAUNCH_BWD2(__nv_bfloat16);
+    else CKDA_LAUNCH_BWD2(float);
+#undef CKDA_LAUNCH_BWD2
 #undef CKDA_LAUNCH_BWD
     return launch_status();
 }

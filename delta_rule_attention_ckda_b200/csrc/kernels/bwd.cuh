@@ -30,6 +30,8 @@
 // keeps them exactly zero.
 //
 // kLogGate: the gate input holds g = ln a; the gradient written is dg = da * a.
+// kNorm: the forward divided q and k by their L2 norms per token (floor 1e-12); the steps
+// run on the normalised values and a last kernel maps dq, dk back through the division.
 #pragma once
 #include "common.cuh"
 
@@ -49,6 +51,30 @@ struct Tok {                      // one block of tokens, fp32, zero-padded
     float v[KB][SLAB], dO[KB][SLAB];
     float b[KB];
 };
+
+// Divide the staged q and k rows by their norms (warp w: token w). Call between two
+// __syncthreads of the staging; ends with one more.
+__device__ __forceinline__ void normalize_staged(Tok& s) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int c = lane; c < D; c += 32) {
+        sq = fmaf(s.q[w][c], s.q[w][c], sq);
+        sk = fmaf(s.k[w][c], s.k[w][c], sk);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    }
+    const float iq = 1.f / fmaxf(sqrtf(sq), 1e-12f), ik = 1.f / fmaxf(sqrtf(sk), 1e-12f);
+#pragma unroll
+    for (int c = lane; c < D; c += 32) {
+        s.q[w][c] *= iq;
+        s.k[w][c] *= ik;
+    }
+    __syncthreads();
+}
 
 // Stage tokens t0 .. t0 + n - 1 of (b, h), slab columns c0 .. c0 + 31 of v and dO.
 template <typename TIn, bool kLogGate>
@@ -171,7 +197,7 @@ __device__ __forceinline__ void ld_scratch(float (&S)[4][4], const float4* slot)
 
 // Pass 1: the forward over T, keeping S_{8n - 1} (the state entering token 8n) as
 // checkpoint n (ckpt: [B*H][nblk][d_k][d_v]; checkpoint 0 = S0). Grid: (B*H, slabs).
-template <typename TIn, bool kLogGate>
+template <typename TIn, bool kLogGate, bool kNorm>
 __global__ void __launch_bounds__(bwd::NT, 4)
 bwd_ckpt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta, const float* S0,
@@ -192,6 +218,7 @@ bwd_ckpt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
         __syncthreads();                                  // previous block's tokens consumed
         stage<TIn, kLogGate>(s, q, k, v, alpha, beta, nullptr, b, h, T, H, dk, dv, t0, cnt, c0);
         __syncthreads();
+        if constexpr (kNorm) normalize_staged(s);
         for (int tt = 0; tt < cnt; ++tt) {
             fwd_step(S, s, tt, red[rb], i0, j0);
             rb ^= 1;
@@ -202,7 +229,7 @@ bwd_ckpt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
 // Pass 2: gradients, walking the checkpoint blocks in reverse. Grid: (B*H, slabs).
 // dv and dS0 are written directly; dq, dk, da and db as per-slab partials
 // (part: [slabs][B*T*H][3][d_k], partb: [slabs][B*T*H]).
-template <typename TIn, bool kLogGate>
+template <typename TIn, bool kLogGate, bool kNorm>
 __global__ void __launch_bounds__(bwd::NT, 4)
 bwd_grad_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta, const float* __restrict__ dO,
@@ -227,6 +254,7 @@ bwd_grad_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
         __syncthreads();
         stage<TIn, kLogGate>(s, q, k, v, alpha, beta, dO, b, h, T, H, dk, dv, t0, cnt, c0);
         __syncthreads();
+        if constexpr (kNorm) normalize_staged(s);
         // the block's entering states S_{t-1}, recomputed from the checkpoint
         {
             float S[4][4];
@@ -360,6 +388,39 @@ bwd_sum_kernel(const float* __restrict__ part, const float* __restrict__ partb, 
             float sb = 0.f;
             for (int sl = 0; sl < nsl; ++sl) sb += partb[(size_t)sl * nrow + row];
             dbeta[row] = sb;
+        }
+    }
+}
+
+// Pass 4 (kNorm only): the gradients with respect to the normalised rows x^ = x / n,
+// n = max(||x||, 1e-12), mapped to the raw rows: dx = (dx^ - x^ (x^ . dx^)) / n when
+// ||x|| > 1e-12, else dx^ / n. One warp per row; grad holds dx^ on entry, dx on exit.
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+bwd_norm_kernel(const TIn* __restrict__ x, float* __restrict__ grad, size_t nrow, int d) {
+    const int lane = threadIdx.x & 31;
+    for (size_t row = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrow;
+         row += ((size_t)gridDim.x * blockDim.x) >> 5) {
+        const TIn* xr = x + row * d;
+        float* gr = grad + row * d;
+        float ss = 0.f, dot = 0.f;
+        for (int c = lane; c < d; c += 32) {
+            const float xv = ld_in(xr + c);
+            ss = fmaf(xv, xv, ss);
+            dot = fmaf(xv, gr[c], dot);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        }
+        const float nrm = sqrtf(ss);
+        const float inv = 1.f / fmaxf(nrm, 1e-12f);
+        const bool floor = !(nrm > 1e-12f);
+        const float proj = dot * inv;                      // x^ . dx^
+        for (int c = lane; c < d; c += 32) {
+            const float g = gr[c];
+            gr[c] = floor ? g * inv : (g - ld_in(xr + c) * inv * proj) * inv;
         }
     }
 }

@@ -264,7 +264,9 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 //
 // kLogGate: the gate input holds g = ln a of a non-negative gate (KDA) instead of a signed
 // a; the cumulation then needs no logarithm and no sign parity.
-template <bool kLogGate>
+// kNormQK: q and k are divided by their L2 norms per token (floor 1e-12) on the way in;
+// the scale folds into the per-token factors, so the normalised values are never rounded.
+template <bool kLogGate, bool kNormQK>
 __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
@@ -294,6 +296,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     uint32_t* sh_pC = sh_px + 128;                                       // [128]
     uint32_t* sh_sign = sh_pC + 128;        // [64][4] slow path: sign bits per (token, channel)
     float* sh_kp = reinterpret_cast<float*>(sh_sign + 256);             // [2][128] kappa of the previous chunk
+    float* sh_kn = sh_kp + 256;             // [64] 1 / ||k_r|| of the chunk's tokens (kNormQK)
+    float* sh_qn = sh_kn + 64;              // [64] 1 / ||q_r||
     float* at = reinterpret_cast<float*>(sm + SM_AT);
     float* xs = reinterpret_cast<float*>(sm + SM_XS);
     float* rs = reinterpret_cast<float*>(sm + SM_RS);
@@ -744,6 +748,36 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     wfail |= !tc::mbar_wait(&bar_c1, ph_c1);
                     ph_c1 ^= 1u;
                 }
+                if constexpr (kNormQK) {
+                    // 1 / max(||x_r||, 1e-12) for k and q: thread (token r, quarter p of the
+                    // channels) sums 32 squares from four 16-byte chunks of the swizzled tile
+                    const int r = tid >> 2, p = tid & 3;
+                    const uint32_t base = (uint32_t)(p >> 1) * 8192u;
+                    float ssk = 0.f, ssq = 0.f;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const uint32_t off = base + chunk_off(r, 4 * (p & 1) + c4);
+                        const uint4 wk = *reinterpret_cast<const uint4*>(sm + SM_K + off);
+                        const uint4 wq = *reinterpret_cast<const uint4*>(sm + SM_Q + off);
+                        const uint32_t uk[4] = {wk.x, wk.y, wk.z, wk.w}, uq[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float k0 = __uint_as_float(uk[e] << 16), k1 = __uint_as_float(uk[e] & 0xFFFF0000u);
+                            const float q0 = __uint_as_float(uq[e] << 16), q1 = __uint_as_float(uq[e] & 0xFFFF0000u);
+                            ssk = fmaf(k0, k0, fmaf(k1, k1, ssk));
+                            ssq = fmaf(q0, q0, fmaf(q1, q1, ssq));
+                        }
+                    }
+                    ssk += __shfl_xor_sync(0xffffffffu, ssk, 1);
+                    ssk += __shfl_xor_sync(0xffffffffu, ssk, 2);
+                    ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
+                    ssq += __shfl_xor_sync(0xffffffffu, ssq, 2);
+                    if (p == 0) {
+                        sh_kn[r] = rsqrtf(fmaxf(ssk, 1e-24f));
+                        sh_qn[r] = rsqrtf(fmaxf(ssq, 1e-24f));
+                    }
+                    csync();
+                }
                 // per-token factors (the sign of Gamma_r is XORed into the factor's sign bit):
                 //   fast path  e1 = Gamma_r / 2^R,  e2 = 2^R / Gamma_r  (R = L_C / 2: middle of the range)
                 //   exact path e1 = Gamma_r,        e2 = Gamma_C / Gamma_r
@@ -762,8 +796,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         const float m2 = tc::ex2_approx(d2 - t);
                         const float e1 = __uint_as_float(__float_as_uint(tc::ex2_approx(t)) ^ sg);
                         const float e2 = __uint_as_float(__float_as_uint(m2) ^ sg ^ sC);
-                        const float kv = ld_bf16_tile(sm + SM_K, r, m);
-                        const float qv = want_o ? ld_bf16_tile(sm + SM_Q, r, m) : 0.f;
+                        float kv = ld_bf16_tile(sm + SM_K, r, m);
+                        float qv = want_o ? ld_bf16_tile(sm + SM_Q, r, m) : 0.f;
+                        if constexpr (kNormQK) {
+                            kv *= sh_kn[r];
+                            qv *= sh_qn[r];
+                        }
                         xk[e] = kv * e1;
                         xq[e] = qv * e1;
                         yk[e] = kv * e2;
@@ -867,9 +905,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int sc = sq + 4 * j;
-                        at[sc * 64 + r] = (sc < r) ? br * va[j] : 0.f;
+                        float av = va[j], pv = vp[j];
+                        if constexpr (kNormQK) {
+                            av *= sh_kn[r] * sh_kn[sc];
+                            pv *= sh_qn[r] * sh_kn[sc];
+                        }
+                        at[sc * 64 + r] = (sc < r) ? br * av : 0.f;
                         uint32_t hpair, lpair;
-                        split2((sc <= r) ? vp[j] : 0.f, 0.f, hpair, lpair);
+                        split2((sc <= r) ? pv : 0.f, 0.f, hpair, lpair);
                         const uint32_t offp = chunk_off(r, sc >> 3) + (uint32_t)(sc & 7) * 2u;
                         *reinterpret_cast<uint16_t*>(sm + SM_PHI + offp) = (uint16_t)(hpair & 0xffffu);
                         *reinterpret_cast<uint16_t*>(sm + SM_PLO + offp) = (uint16_t)(lpair & 0xffffu);
@@ -1183,8 +1226,8 @@ __global__ void __launch_bounds__(kPrefixThreads) chunk_tc_seg_prefix(float* __r
 
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const float* alpha, const float* beta, const float* S0, float* o, float* ST,
-                                   int B, int T, int H, int dk, int dv, bool log_gate, void* workspace,
-                                   cudaStream_t st) {
+                                   int B, int T, int H, int dk, int dv, bool log_gate, bool norm_qk,
+                                   void* workspace, cudaStream_t st) {
     if (!chunk_tc_supported(dk, dv, 1)) return cudaErrorNotSupported;
     CUtensorMap mk, mq, mv, ma, mo;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -1194,12 +1237,14 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         !tc::make_map_bthd(&mo, o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dv, 128, 64,
                            CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    static bool attr_set[2] = {false, false};
-    auto* kern = log_gate ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
-    if (!attr_set[log_gate ? 1 : 0]) {
+    static bool attr_set[4] = {false, false, false, false};
+    auto* kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
+                          : (norm_qk ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
+    const int variant = (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
+    if (!attr_set[variant]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ctc::SMEM_ALLOC);
         if (e != cudaSuccess) return e;
-        attr_set[log_gate ? 1 : 0] = true;
+        attr_set[variant] = true;
     }
     const unsigned nbh = (unsigned)(B * H);
     const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());

@@ -13,12 +13,13 @@
 // them exactly zero.
 //
 // kLogGate: the gate input holds g = ln a (a non-negative gate, a = e^g <= 1) instead of a.
+// kNorm: q and k are divided by their L2 norms per token (floor 1e-12) once staged.
 #pragma once
 #include "common.cuh"
 
 namespace ckda {
 
-template <int DK, typename TIn, bool kLogGate>
+template <int DK, typename TIn, bool kLogGate, bool kNorm>
 __global__ void __launch_bounds__(128)
 recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                      const TIn* __restrict__ v, const float* __restrict__ alpha,
@@ -29,6 +30,7 @@ recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     __shared__ float sk[TB][DK], sq[TB][DK], sa[TB][DK];
     __shared__ float sv[TB][128];
     __shared__ float sb[TB];
+    __shared__ float snk[TB], snq[TB];
 
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh % H;
@@ -59,6 +61,24 @@ recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
             sv[tt][threadIdx.x] = active ? ld_in(v + tok * dv + j) : 0.f;
         }
         __syncthreads();
+        if constexpr (kNorm) {
+            if (threadIdx.x < nt) {           // one thread per token (nt <= TB < blockDim.x)
+                float ssk = 0.f, ssq = 0.f;
+                for (int i = 0; i < DK; ++i) {
+                    ssk = fmaf(sk[threadIdx.x][i], sk[threadIdx.x][i], ssk);
+                    ssq = fmaf(sq[threadIdx.x][i], sq[threadIdx.x][i], ssq);
+                }
+                snk[threadIdx.x] = 1.f / fmaxf(sqrtf(ssk), 1e-12f);
+                snq[threadIdx.x] = 1.f / fmaxf(sqrtf(ssq), 1e-12f);
+            }
+            __syncthreads();
+            for (int idx = threadIdx.x; idx < nt * DK; idx += blockDim.x) {
+                const int tt = idx / DK, i = idx % DK;
+                sk[tt][i] *= snk[tt];
+                sq[tt][i] *= snq[tt];
+            }
+            __syncthreads();
+        }
 #pragma unroll 1
         for (int tt = 0; tt < nt; ++tt) {
             float y = 0.f;

@@ -52,7 +52,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 4
+#define CKDA_ABI_VERSION 5
 
 typedef enum {
     CKDA_OK = 0,
@@ -80,6 +80,18 @@ typedef enum {
     CKDA_GATE_SIGNED = 0,       /* alpha in [-1,1]^dk: the CKDA gate, sign and magnitude   */
     CKDA_GATE_LOG = 1           /* g = ln(alpha) <= 0 of a non-negative gate (the KDA form) */
 } ckda_gate_t;
+
+/*
+ * The `mode` argument of the *_ex calls and of ckda_bwd is a ckda_gate_t value,
+ * optionally OR-ed with option bits:
+ *   CKDA_OPT_NORMALIZE_QK: q and k are divided by their L2 norms per token and head,
+ *     x / max(||x||_2, 1e-12), before the recurrence (the layer step before the path: the
+ *     keys of the transition are unit vectors, ai.info summary of the Complex KDA paper,
+ *     "Methodology"; the floor is torch.nn.functional.normalize's default). The
+ *     normalisation is fused: the normalised values are never written to memory.
+ * Unknown bits return CKDA_ERR_INVALID_ARG.
+ */
+#define CKDA_OPT_NORMALIZE_QK 0x100
 
 /* Version of this ABI (CKDA_ABI_VERSION). */
 CKDA_API int ckda_abi_version(void);
@@ -137,20 +149,21 @@ CKDA_API ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* 
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * ckda_chunk_fwd with the gate in the form gate_mode selects. CKDA_GATE_SIGNED is
+ * ckda_chunk_fwd with the gate in the form `mode` selects. CKDA_GATE_SIGNED is
  * ckda_chunk_fwd itself. CKDA_GATE_LOG reads g = ln(alpha), fp32, in alpha's
  * [B,T,H,dk] layout, for a gate that never changes sign: the parameterisation of KDA,
  * whose gate CKDA extends from [0,1] to [-1,1] (ai.info summary of the Complex KDA paper,
  * "What This Paper Is About"). The map is the same recurrence with alpha = e^g
  * (g = -inf gives alpha = 0). It runs on the same kernels, so that CKDA's cost over KDA
  * can be measured (ai.info summary, "Main Findings": the throughput cost of the signed
- * gate). An unknown gate_mode returns CKDA_ERR_INVALID_ARG.
+ * gate). CKDA_OPT_NORMALIZE_QK may be OR-ed in (see above). An unknown mode returns
+ * CKDA_ERR_INVALID_ARG.
  */
 CKDA_API ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                                 const float* gate, const float* beta, const float* S0,
                                 float* o, float* S_T,
                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
-                                ckda_gate_t gate_mode,
+                                int mode,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* Capacity of the fixed device scratch ckda_chunk_fwd_noalloc uses: 20 MiB per device
@@ -175,7 +188,7 @@ CKDA_API ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, cons
                                 const float* gate, const float* beta, const float* S0,
                                 float* o, float* S_T,
                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
-                                ckda_gate_t gate_mode, void* stream);
+                                int mode, void* stream);
 
 /*
  * Token-by-token forward on CUDA cores in fp32 (the recurrent path of
@@ -189,12 +202,12 @@ CKDA_API ckda_status_t ckda_recurrent_fwd(const void* q, const void* k, const vo
                                  int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
                                  void* stream);
 
-/* ckda_recurrent_fwd with the gate in the form gate_mode selects (see ckda_chunk_fwd_ex). */
+/* ckda_recurrent_fwd with the gate and options `mode` selects (see ckda_chunk_fwd_ex). */
 CKDA_API ckda_status_t ckda_recurrent_fwd_ex(const void* q, const void* k, const void* v,
                                     const float* gate, const float* beta, const float* S0,
                                     float* o, float* S_T,
                                     int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
-                                    ckda_gate_t gate_mode, void* stream);
+                                    int mode, void* stream);
 
 /*
  * One recurrent decode step for N independent sequences (blog post "One update,
@@ -226,7 +239,7 @@ CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ck
  * (ai.info summary of the Complex KDA paper, "Main Findings"); they print no backward
  * formulas, so this is the derivative of the recurrence itself, taken token by token
  * in reverse on CUDA cores in fp32 from states recomputed out of checkpoints.
- *   q, k, v, gate, beta, S0, B..dv, dt, gate_mode: as for ckda_chunk_fwd_ex (S0 may
+ *   q, k, v, gate, beta, S0, B..dv, dt, mode: as for ckda_chunk_fwd_ex (S0 may
  *              be NULL: zero initial state; any dk, dv <= 128; fp32 or bf16 q, k, v)
  *   grad_o     [B,T,H,dv] fp32 cotangent of o (required when B*T*H > 0)
  *   grad_S_T   [B,H,dk,dv] fp32 cotangent of the final state, or NULL (zero)
@@ -243,7 +256,7 @@ CKDA_API ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, con
                                 const float* grad_S_T, float* grad_q, float* grad_k, float* grad_v,
                                 float* grad_gate, float* grad_beta, float* grad_S0,
                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
-                                ckda_gate_t gate_mode, void* workspace, size_t workspace_bytes,
+                                int mode, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
 /*

@@ -49,7 +49,7 @@ def test_status_strings(lib):
         s = lib.ckda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.ckda_status_string(99) == b"unknown status"
-    assert lib.ckda_abi_version() == 4
+    assert lib.ckda_abi_version() == 5
 
 
 NULL = None
@@ -164,6 +164,22 @@ def test_bwd_workspace_and_argument_checks(lib):
     # workspace too small
     assert lib.ckda_bwd(p, p, p, fp, fp, null, fp, null, fp, fp, fp, fp, fp, null,
                         1, 4, 1, 16, 16, 0, 0, ws, 16, None) == 6
+
+
+def test_mode_option_bits(lib):
+    """mode = gate form | option bits; unknown bits and gate forms are argument errors,
+    returned before anything touches the (dummy) pointers."""
+    import ctypes
+    from delta_rule_attention_ckda_b200 import _lib
+    assert _lib._mode("signed", True) == 0x100 and _lib._mode("log", False) == 1
+    p = ctypes.c_void_p(256)
+    fp = ctypes.cast(p, ctypes.POINTER(ctypes.c_float))
+    null = ctypes.POINTER(ctypes.c_float)()
+    for mode in (0x200, 0x101 | 0x400, 2, 0x1FF):
+        assert lib.ckda_chunk_fwd_ex(p, p, p, fp, fp, null, fp, null, 1, 4, 1, 16, 16, 0, mode,
+                                     None, 0, None) == 1, hex(mode)
+        assert lib.ckda_recurrent_fwd_ex(p, p, p, fp, fp, null, fp, null, 1, 4, 1, 16, 16, 0, mode,
+                                         None) == 1, hex(mode)
 
 
 def test_python_binding_refuses_cpu_tensors():
