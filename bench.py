@@ -63,7 +63,7 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# sources that make up each profiled kernel (its code, the primitives it uses, its launch)
+# device sources that make up each profiled kernel (its code and the primitives it uses)
 KERNEL_SOURCES = {
     "chunk_fwd_chunk_tc_layer": ["kernels/common.cuh", "kernels/chunk_tc.cuh", "kernels/tc_primitives.cuh",
                                  "kernels/tc_host.cuh"],

@@ -13,7 +13,7 @@
 #include "kernels/common.cuh"
 #include "kernels/recurrent.cuh"
 #include "kernels/decode.cuh"
-#include "kernels/chunk_tc.cuh"
+#include "kernels/chunk_tc_launch.cuh"
 #include "kernels/bwd.cuh"
 
 namespace {
