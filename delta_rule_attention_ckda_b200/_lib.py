@@ -66,6 +66,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_bwd.restype = i
     lib.ckda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 5 + [vp]
     lib.ckda_decode_step.restype = i
+    lib.ckda_decode_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 6 + [vp]
+    lib.ckda_decode_step_ex.restype = i
     lib.ckda_get_device_error.argtypes = [vp]
     lib.ckda_get_device_error.restype = i
     _lib = lib
@@ -259,8 +261,10 @@ def recurrent_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state
     return o, S_T
 
 
-def decode_step(q, k, v, alpha, beta, S, *, o=None, stream=None) -> torch.Tensor:
-    """ckda_decode_step: updates S [N,H,dk,dv] in place, returns o [N,H,dv]."""
+def decode_step(q, k, v, alpha, beta, S, *, o=None, stream=None, gate="signed",
+                normalize_qk=False) -> torch.Tensor:
+    """ckda_decode_step_ex: updates S [N,H,dk,dv] in place, returns o [N,H,dv]. `alpha` is
+    the gate in the form `gate` names; normalize_qk L2-normalises q and k in the step."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
@@ -273,9 +277,10 @@ def decode_step(q, k, v, alpha, beta, S, *, o=None, stream=None) -> torch.Tensor
     if o is None:
         o = torch.empty(N, H, dv, device=q.device, dtype=torch.float32)
     _check(o, "o", (N, H, dv), torch.float32)
-    st = load().ckda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
-                                 _ptr(o), N, H, dk, dv, _dt(q), _stream(stream))
-    _raise(st, "ckda_decode_step")
+    st = load().ckda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                                    _ptr(o), N, H, dk, dv, _dt(q), _mode(gate, normalize_qk),
+                                    _stream(stream))
+    _raise(st, "ckda_decode_step_ex")
     return o
 
 

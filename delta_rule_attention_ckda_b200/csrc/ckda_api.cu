@@ -301,32 +301,44 @@ ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float*
     return launch_status();
 }
 
-ckda_status_t ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
-                               const float* beta, float* S, float* o, int N, int H, int dk,
-                               int dv, ckda_dtype_t dt, void* stream) {
+ckda_status_t ckda_decode_step_ex(const void* q, const void* k, const void* v, const float* gate,
+                                  const float* beta, float* S, float* o, int N, int H, int dk, int dv,
+                                  ckda_dtype_t dt, int mode, void* stream) {
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return CKDA_ERR_INVALID_ARG;
     if (N < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
     if (dt != CKDA_F32 && dt != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
     const long long seqs = (long long)N * H;
     if (seqs == 0) return CKDA_OK;
     if (seqs > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
-    if (!q || !k || !v || !alpha || !beta || !S || !o) return CKDA_ERR_INVALID_ARG;
-    const void* ptrs[7] = {q, k, v, alpha, beta, S, o};
+    if (!q || !k || !v || !gate || !beta || !S || !o) return CKDA_ERR_INVALID_ARG;
+    const void* ptrs[7] = {q, k, v, gate, beta, S, o};
     for (const void* p : ptrs)
         if (!aligned16(p)) return CKDA_ERR_MISALIGNED;
     cudaStream_t st = as_stream(stream);
     if (dk == 128 && dv == 128) {
-        if (dt == CKDA_BF16)
-            ckda::decode128_kernel<__nv_bfloat16><<<(unsigned)seqs, 256, 0, st>>>(
-                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                static_cast<const __nv_bfloat16*>(v), alpha, beta, S, o);
-        else
-            ckda::decode128_kernel<float><<<(unsigned)seqs, 256, 0, st>>>(
-                static_cast<const float*>(q), static_cast<const float*>(k),
-                static_cast<const float*>(v), alpha, beta, S, o);
+#define CKDA_DECODE(TIN, LG, NQ)                                                                        \
+    ckda::decode128_kernel<TIN, LG, NQ><<<(unsigned)seqs, 256, 0, st>>>(                                 \
+        static_cast<const TIN*>(q), static_cast<const TIN*>(k), static_cast<const TIN*>(v), gate, beta, S, o)
+#define CKDA_DECODE2(TIN)                                                                               \
+    do {                                                                                                \
+        if (lg) { if (nq) CKDA_DECODE(TIN, true, true); else CKDA_DECODE(TIN, true, false); }            \
+        else { if (nq) CKDA_DECODE(TIN, false, true); else CKDA_DECODE(TIN, false, false); }             \
+    } while (0)
+        if (dt == CKDA_BF16) CKDA_DECODE2(__nv_bfloat16);
+        else CKDA_DECODE2(float);
+#undef CKDA_DECODE2
+#undef CKDA_DECODE
         return launch_status();
     }
     // Other sizes: a decode step is the recurrent forward with T = 1, S in place.
-    return ckda_recurrent_fwd(q, k, v, alpha, beta, S, o, S, N, 1, H, dk, dv, dt, stream);
+    return ckda_recurrent_fwd_ex(q, k, v, gate, beta, S, o, S, N, 1, H, dk, dv, dt, mode, stream);
+}
+
+ckda_status_t ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                               const float* beta, float* S, float* o, int N, int H, int dk,
+                               int dv, ckda_dtype_t dt, void* stream) {
+    return ckda_decode_step_ex(q, k, v, alpha, beta, S, o, N, H, dk, dv, dt, CKDA_GATE_SIGNED, stream);
 }
 
 ckda_status_t ckda_get_device_error(void* stream) {

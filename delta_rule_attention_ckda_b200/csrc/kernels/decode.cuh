@@ -11,12 +11,15 @@
 // CTA = 256 threads (8 warps) per (n, h). Warp w owns state rows 16w..16w+15; lane l
 // owns columns 4l..4l+3 of each, held as 16 float4 registers. Column sums over rows
 // are a per-thread partial over 16 rows plus an 8-way shared-memory reduction.
+//
+// kLogGate: the gate input holds g = ln a (a = e^g). kNorm: q and k are divided by their
+// L2 norms (floor 1e-12) once staged; both happen while the state read is in flight.
 #pragma once
 #include "common.cuh"
 
 namespace ckda {
 
-template <typename TIn>
+template <typename TIn, bool kLogGate, bool kNorm>
 __global__ void __launch_bounds__(256, 2)
 decode128_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                  const TIn* __restrict__ v, const float* __restrict__ alpha,
@@ -25,7 +28,7 @@ decode128_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     constexpr int D = 128;
     __shared__ float sk[D], sq[D], sa[D], sv[D];
     __shared__ float4 red_y[8][32], red_z[8][32];
-    __shared__ float s_kq;
+    __shared__ float s_kq, s_nk, s_nq;
 
     const int nh = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -40,10 +43,36 @@ decode128_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
         const size_t off = (size_t)nh * D + tid;
         sk[tid] = ld_in(k + off);
         sq[tid] = ld_in(q + off);
-        sa[tid] = __ldg(alpha + off);
+        const float g = __ldg(alpha + off);
+        sa[tid] = kLogGate ? expf(g) : g;
         sv[tid] = ld_in(v + off);
     }
     __syncthreads();
+    if constexpr (kNorm) {
+        if (warp == 0) {
+            float pk = 0.f, pq = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                pk = fmaf(sk[4 * lane + c], sk[4 * lane + c], pk);
+                pq = fmaf(sq[4 * lane + c], sq[4 * lane + c], pq);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                pk += __shfl_xor_sync(0xffffffffu, pk, off);
+                pq += __shfl_xor_sync(0xffffffffu, pq, off);
+            }
+            if (lane == 0) {
+                s_nk = 1.f / fmaxf(sqrtf(pk), 1e-12f);
+                s_nq = 1.f / fmaxf(sqrtf(pq), 1e-12f);
+            }
+        }
+        __syncthreads();
+        if (tid < D) {
+            sk[tid] *= s_nk;
+            sq[tid] *= s_nq;
+        }
+        __syncthreads();
+    }
 
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f), z = y;
 #pragma unroll

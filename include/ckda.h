@@ -52,7 +52,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 5
+#define CKDA_ABI_VERSION 6
 
 typedef enum {
     CKDA_OK = 0,
@@ -258,6 +258,14 @@ CKDA_API ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, con
                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
                                 int mode, void* workspace, size_t workspace_bytes,
                                 void* stream);
+
+/* ckda_decode_step with the gate form and options `mode` selects (see ckda_chunk_fwd_ex):
+ * gate holds alpha (CKDA_GATE_SIGNED) or g = ln(alpha) (CKDA_GATE_LOG), and
+ * CKDA_OPT_NORMALIZE_QK divides q and k by their L2 norms inside the step. */
+CKDA_API ckda_status_t ckda_decode_step_ex(const void* q, const void* k, const void* v,
+                               const float* gate, const float* beta,
+                               float* S, float* o,
+                               int N, int H, int dk, int dv, ckda_dtype_t dt, int mode, void* stream);
 
 /*
  * Synchronises `stream`, then reads and clears this GPU's device error word.

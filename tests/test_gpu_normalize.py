@@ -111,3 +111,32 @@ def test_bwd_normalized(ck, dtype):
     want = oracle_bwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, dO, S0=inp.S0, dST=dST, normalize_qk=True)
     for n in ("dq", "dk", "dv", "dalpha", "dbeta", "dS0"):
         check(f"norm bwd {dtype}/{n}", got[n].double().cpu().numpy(), want[n], TAU_F32)
+
+
+@pytest.mark.parametrize("dims", [(128, 128), (64, 32)])
+@pytest.mark.parametrize("gate", ["signed", "log"])
+def test_decode_normalized_and_log_gate(ck, dims, gate):
+    """Decode step with the gate form and the fused normalisation (the 128-wide kernel, and
+    the recurrent path for other sizes), three consecutive steps on one state."""
+    dk, dv = dims
+    N, H = 6, 3
+    g = torch.Generator().manual_seed(dk + dv)
+    S = (0.05 * torch.randn(N, H, dk, dv, generator=g))
+    S_ref = S.double().numpy()
+    Sd = S.cuda()
+    for t in range(3):
+        q = (torch.randn(N, H, dk, generator=g) * 3).to(torch.bfloat16)
+        k = (torch.randn(N, H, dk, generator=g) * 0.3).to(torch.bfloat16)
+        v = torch.randn(N, H, dv, generator=g).to(torch.bfloat16)
+        a = torch.tanh(1.5 + torch.randn(N, H, dk, generator=g))
+        if gate == "log":
+            a = torch.log(a.abs())
+        b = 2 * torch.sigmoid(torch.randn(N, H, generator=g))
+        o = ck.decode_step(q.cuda(), k.cuda(), v.cuda(), a.cuda(), b.cuda(), Sd, gate=gate, normalize_qk=True)
+        alpha = torch.exp(a.double()).numpy() if gate == "log" else a
+        o_ref, S_ref = oracle.oracle_fwd(q[:, None], k[:, None], v[:, None], alpha[:, None] if gate == "log"
+                                         else a[:, None], b[:, None], S_ref, normalize_qk=True)
+        check(f"norm decode {dims} {gate} step {t}/o", o.double().cpu().numpy(), o_ref[:, 0], TAU_BF16)
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    check(f"norm decode {dims} {gate}/S", Sd.double().cpu().numpy(), S_ref, TAU_BF16)
