@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -71,17 +72,24 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without comments and blank space, so that a comment edit keeps the hash."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(kernel_key):
-    """Hash of the sources of one kernel; its committed DRAM-traffic figure is only
-    reported while it matches."""
+    """Hash of the code (comments stripped) of one kernel's sources; its committed
+    DRAM-traffic figure is only reported while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "delta_rule_attention_ckda_b200", "csrc")
     for rel in KERNEL_SOURCES[kernel_key]:
         p = os.path.join(csrc, rel)
         if os.path.exists(p):
-            with open(p, "rb") as f:
+            with open(p, encoding="utf-8") as f:
                 h.update(rel.encode())
-                h.update(f.read())
+                h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

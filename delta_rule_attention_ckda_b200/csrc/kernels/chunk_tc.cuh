@@ -181,7 +181,8 @@ __device__ __forceinline__ void tmem_st_f32x32(uint32_t taddr, const float (&x)[
     tc::tmem_st32<16>(taddr + 16, b);
 }
 
-// Barrier among the 256 compute threads only (named barrier 1; the issuer warp never joins).
+// Barrier among the 256 compute threads only (named barrier 1; the epilogue warpgroup never
+// joins).
 __device__ __forceinline__ void csync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Same barrier with an OR over the threads' predicates.
@@ -224,8 +225,9 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
     return csync_or(!ok);
 }
 
-// Hand this thread's shared-memory writes and tcgen05.st to the issuer warp: complete
-// the stores, order them before the async proxy and the thread sync, then arrive.
+// Hand this thread's shared-memory writes and tcgen05.st to the epilogue warpgroup (whose
+// leader issues the MMAs that read them): complete the stores, order them before the
+// async proxy and the thread sync, then arrive.
 __device__ __forceinline__ void handoff(uint64_t* bar) {
     tc::tmem_st_wait();
     tc::fence_proxy_async_smem();
@@ -234,7 +236,7 @@ __device__ __forceinline__ void handoff(uint64_t* bar) {
 }
 
 // A copy of x the compiler cannot see through: keeps loop-invariant MMA descriptors from
-// being hoisted out of the chunk loop into (scarce) issuer registers.
+// being hoisted out of the chunk loop into (scarce) epilogue-warpgroup registers.
 __device__ __forceinline__ uint32_t opaque(uint32_t x) {
     asm volatile("mov.b32 %0, %0;" : "+r"(x));
     return x;
@@ -253,14 +255,15 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 
 // ------------------------------------------------------------------------------ kernel
 
-// Per-chunk schedule (one CTA per (batch, head)). Eight compute warps do the CUDA-core
-// work; one issuer warp issues every tcgen05 MMA group, TMA load and o store, so that the
-// compute warps never stall while an MMA group drains (an issuing thread blocks for about
-// the duration of the MMAs it issues). The compute warps hand their operands over through
+// Per-chunk schedule (one CTA per (batch, head), or per segment of one). Eight compute
+// warps do the gate, the [P;A] epilogue and the solve; four epilogue warps move the state
+// chain's operands through TMEM, and the epilogue leader issues every TMA copy and every
+// MMA group but [P;A] (an issuing thread blocks for about the duration of the MMAs it
+// issues, so issue stays off the compute warps). The groups hand operands over through
 // mbarriers; each MMA group commits to its own mbarrier. What overlaps:
-//   gate cumulation of chunk c           ||  O / state MMAs of chunk c-1
-//   o tile of chunk c-1, state copy       ||  [A ; P] MMA of chunk c
-//   [A ; P] epilogue, solve for T         ||  C1 MMA ([Z | O_inter]), k / alpha of chunk c+1
+//   factors, X and Y tiles of chunk c          ||  (epilogue: waits for them)
+//   [P;A] epilogue and solve of chunk c        ||  o tile of chunk c-1, state copy, C1, -Z^T
+//   gate cumulation of chunk c+1               ||  U MMA, U^T, O / state MMA of chunk c
 //
 // kLogGate: the gate input holds g = ln a of a non-negative gate (KDA) instead of a signed
 // a; the cumulation then needs no logarithm and no sign parity.
@@ -1008,8 +1011,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     const uint32_t zoff = chunk_off(lane, 4 + (warp & 3)) + (uint32_t)half * 8192u;
                     *reinterpret_cast<uint4*>(sm + SM_T + zoff) = make_uint4(0u, 0u, 0u, 0u);
                 }
-                // A (k-tile space) is consumed: the issuer loads the next chunk's k and alpha
-                // once the o tile has left the alpha space
+                // A (k-tile space) is consumed: the epilogue leader loads the next chunk's k
                 csync();
                 // X[32:64, 0:32]: thread -> row 32 + r2, columns 4 c4 .. 4 c4 + 3, straight into T.
                 // X[32 + r2][32 + mm] is zero for mm > r2: warps 0-3 hold rows r2 < 16.
@@ -1033,7 +1035,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 *reinterpret_cast<uint2*>(sm + SM_T + off) = make_uint2(h0, h1);
                 *reinterpret_cast<uint2*>(sm + SM_T + 8192 + off) = make_uint2(l0, l1);
             }
-            handoff(&bar_ht);                      // T tiles complete: the issuer starts V T^T
+            handoff(&bar_ht);                      // T tiles complete: the leader starts V T^T
 
             if (ck + 1 < nchunks) beta_next = load_beta(t0 + C);
 
