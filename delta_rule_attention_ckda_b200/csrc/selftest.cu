@@ -139,7 +139,37 @@ __global__ void tma_selftest_kernel(const __grid_constant__ CUtensorMap map, int
     for (int i = threadIdx.x; i < box_bytes; i += blockDim.x) out[i] = ok ? smem[i] : 0;
 }
 
+// The failure path of the bounded waits: one warp waits on phase 0 of an mbarrier that
+// no thread arrives at (or, with arrive != 0, that thread 0 completes first). The wait gives
+// up after `limit` polls, records the timeout in this library's device error word and
+// returns; the kernel then writes whether the wait succeeded and ends normally.
+__global__ void wait_timeout_selftest_kernel(uint32_t limit, int arrive, int* result) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (arrive && threadIdx.x == 0) mbar_arrive(&bar);
+    const bool ok = mbar_wait(&bar, 0, limit);
+    if (threadIdx.x == 0) result[0] = ok ? 1 : 0;
+}
+
 }  // namespace
+
+ST_API int ckda_selftest_wait(unsigned limit, int arrive, int* result_dev) {
+    wait_timeout_selftest_kernel<<<1, 32>>>(limit, arrive, result_dev);
+    return cudaGetLastError() == cudaSuccess ? 0 : 4;
+}
+
+// Synchronises the device, then reads and clears this library's device error word.
+ST_API int ckda_selftest_error_word(unsigned* word) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return 4;
+    unsigned zero = 0;
+    if (cudaMemcpyFromSymbol(word, ckda::g_error_word, sizeof(unsigned)) != cudaSuccess) return 4;
+    if (cudaMemcpyToSymbol(ckda::g_error_word, &zero, sizeof(unsigned)) != cudaSuccess) return 4;
+    return 0;
+}
 
 ST_API int ckda_selftest_gemm(const void* A, const void* B, float* D, int N, int K, int a_mode, int b_mode,
                               int neg_a, int* status_dev) {

@@ -22,7 +22,25 @@ def st():
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.ckda_selftest_gemm.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
     lib.ckda_selftest_tma.argtypes = [vp, i, i, i, i, i, i, i, i, i, i, vp, vp]
+    lib.ckda_selftest_wait.argtypes = [ctypes.c_uint, i, vp]
+    lib.ckda_selftest_error_word.argtypes = [ctypes.POINTER(ctypes.c_uint)]
     return lib
+
+
+@pytest.mark.parametrize("arrive", [0, 1])
+def test_bounded_wait_gives_up_and_reports(st, arrive):
+    """A wait on an mbarrier that nothing completes returns after its poll limit with the
+    timeout bit set in the device error word; the context stays usable afterwards (a
+    GEMM self-test still passes). With the barrier completed first, the wait succeeds
+    and nothing is reported."""
+    word = ctypes.c_uint(0)
+    assert st.ckda_selftest_error_word(ctypes.byref(word)) == 0      # clear
+    res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    assert st.ckda_selftest_wait(1024, arrive, res.data_ptr()) == 0
+    assert st.ckda_selftest_error_word(ctypes.byref(word)) == 0
+    assert int(res.item()) == arrive
+    assert (word.value & 1) == (0 if arrive else 1)
+    test_gemm_paths(st, 0, 0, 64, 64, 0)
 
 
 def swz(off):
