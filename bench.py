@@ -495,30 +495,71 @@ def kda_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, ckda_value):
 
 def e2e_measure(ck, inp, dev, stream, world, args):
     """Same metric through the public Python API with pinned host buffers; every step
-    copies its inputs host->device and reads o and S_T back."""
+    copies its inputs host->device and reads o and S_T back. Steps are pipelined over
+    three streams (inputs in, compute, results out) and two device buffer sets, so the
+    copies of neighbouring steps overlap the compute and each other, as a serving loop
+    would run them."""
     import torch
     B, T, H, dk, dv = inp.shape
     hq, hk, hv, ha, hb = (x.pin_memory() for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
     ho = torch.empty(B, T, H, dv, pin_memory=True)
     hS = torch.empty(B, H, dk, dv, pin_memory=True)
-    dq, dk_, dv_, da, db = (torch.empty_like(x, device=dev) for x in (hq, hk, hv, ha, hb))
+    sets = []
+    for _ in range(2):
+        sets.append({"in": [torch.empty_like(x, device=dev) for x in (hq, hk, hv, ha, hb)],
+                     "o": torch.empty(B, T, H, dv, device=dev), "S": torch.empty(B, H, dk, dv, device=dev)})
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of set i copied
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]     # set i computed
+    ev_out = [torch.cuda.Event() for _ in range(2)]     # results of set i read back
+    for e in ev_out:
+        e.record(stream)
 
-    def step():
-        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (da, ha), (db, hb)):
-            d.copy_(h, non_blocking=True)
-        o, S = ck.chunk_fwd(dq, dk_, dv_, da, db, None)
-        ho.copy_(o, non_blocking=True)
-        hS.copy_(S, non_blocking=True)
+    def step(i):
+        st = sets[i % 2]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[i % 2])              # the set's previous compute is done
+            for d, h in zip(st["in"], (hq, hk, hv, ha, hb)):
+                d.copy_(h, non_blocking=True)
+            ev_in[i % 2].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[i % 2])
+            s_cmp.wait_event(ev_out[i % 2])             # its previous results have left
+            q, k, v, a, b = st["in"]
+            ck.chunk_fwd(q, k, v, a, b, None, o=st["o"], S_T=st["S"], stream=s_cmp)
+            ev_cmp[i % 2].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[i % 2])
+            ho.copy_(st["o"], non_blocking=True)
+            hS.copy_(st["S"], non_blocking=True)
+            ev_out[i % 2].record(s_out)
 
-    step()
-    n = max(3, min(args.steps, 5))
+    for e in ev_cmp:
+        e.record(stream)
+    step(0)
+    step(1)
+    torch.cuda.synchronize()
+    n = max(4, min(args.steps, 8))
     barrier(world)
-    secs = time_launches(step, n, stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for x in (s_in, s_cmp, s_out):
+        x.wait_event(t0)
+    for i in range(n):
+        step(i)
+    for x in (s_in, s_cmp, s_out):
+        stream.wait_stream(x)
+    t1.record(stream)
+    t1.synchronize()
+    assert ck.get_device_error() == 0
+    secs = t0.elapsed_time(t1) / 1e3
     value, secs = aggregate_throughput(B * T * n, secs, world, device="cuda")
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, hb))
     d2h = ho.numel() * 4 + hS.numel() * 4
     return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": n}
+            "d2h_bytes_per_step": d2h, "steps": n,
+            "pipeline": "3 streams (in, compute, out), 2 device buffer sets; pinned host buffers"}
 
 
 def decode_measure(ck, dev, stream, world):
