@@ -1,9 +1,24 @@
 // Host side of the chunked tensor-core forward: the supported shapes, the segment plan for
 // long sequences, the segment-prefix kernel, the workspace and the launches.
 #pragma once
+#include <atomic>
+
 #include "chunk_tc.cuh"
 
 namespace ckda {
+
+// cudaFuncSetAttribute applies on the current device only: remember, per kernel, the
+// devices it was applied on (bit d of the mask). Setting it twice is harmless.
+inline cudaError_t ensure_smem_attr(const void* fn, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 
 // d_k, d_v in {64, 128}: a 64-wide problem runs as the 128-wide one with zero padding,
@@ -171,14 +186,13 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
         !tc::make_map_bthd(&mo, o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, B, T, H, dv, 128, 64,
                            CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    static bool attr_set[4] = {false, false, false, false};
+    static std::atomic<uint64_t> attr_done[4];
     auto* kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
                           : (norm_qk ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
     const int variant = (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
-    if (!attr_set[variant]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ctc::SMEM_ALLOC);
+    {
+        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)ctc::SMEM_ALLOC, attr_done[variant]);
         if (e != cudaSuccess) return e;
-        attr_set[variant] = true;
     }
     const unsigned nbh = (unsigned)(B * H);
     const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
@@ -199,13 +213,10 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.nseg > 2) {
-        static bool prefix_attr = false;
-        if (!prefix_attr) {
-            e = cudaFuncSetAttribute(chunk_tc_seg_prefix, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)seg_prefix_smem(128));
-            if (e != cudaSuccess) return e;
-            prefix_attr = true;
-        }
+        static std::atomic<uint64_t> prefix_done{0};
+        e = ensure_smem_attr(reinterpret_cast<const void*>(chunk_tc_seg_prefix), (int)seg_prefix_smem(128),
+                             prefix_done);
+        if (e != cudaSuccess) return e;
         chunk_tc_seg_prefix<<<dim3(nbh, (unsigned)(dv / 16)), kPrefixThreads, seg_prefix_smem(dk), st>>>(
             Sx, Mx, p.nseg, dk, dv);
         e = cudaGetLastError();
