@@ -115,9 +115,15 @@ def test_T_zero_copies_state(ck, fn):
     assert torch.count_nonzero(ST) == 0
 
 
-@pytest.mark.parametrize("fn", ["chunk", "recurrent"])
-def test_in_place_state(ck, fn):
-    inp = make_inputs(2, 150, 2, 128, 128, torch.bfloat16, seed=9, s0_std=0.05)
+@pytest.mark.parametrize("fn,shape", [("chunk", (2, 150, 2)), ("recurrent", (2, 150, 2)),
+                                      ("chunk", (1, 1000, 2))])
+def test_in_place_state(ck, fn, shape):
+    """S_T may be S0: one pass (each CTA reads its slot first and writes it last) and the
+    segmented path (S0 read by the first launch, S_T written by the last)."""
+    B, T, H = shape
+    inp = make_inputs(B, T, H, 128, 128, torch.bfloat16, seed=9, s0_std=0.05)
+    if fn == "chunk" and T == 1000:
+        assert ck.chunk_segments(B, T, H, 128, 128) > 1
     o_ref, S_ref = run_fwd(ck, fn, inp)
     q, k, v, a, b, S0 = to_dev(inp)
     f = ck.chunk_fwd if fn == "chunk" else ck.recurrent_fwd
