@@ -1,6 +1,6 @@
 /*
- * ckda.h - C ABI of the CKDA (Complex Kimi Delta Attention) forward library for
- * NVIDIA B200 (sm_100a).
+ * ckda.h - C ABI of the CKDA (Complex Kimi Delta Attention) library for NVIDIA B200
+ * (sm_100a): chunked forward, decode step and backward pass.
  *
  * The operation (Complex KDA: Understanding and Enhancing the Expressivity of Kimi
  * Delta Attention, as summarised by the blog post "One update, one quarter-turn",
@@ -19,7 +19,9 @@
  * ---------------------------------------
  * - All pointers are DEVICE pointers owned by the caller. The library allocates no
  *   device memory and keeps no per-call state; the only global state is one device
- *   error word per GPU (see ckda_get_device_error) and cached kernel attributes.
+ *   error word per GPU (see ckda_get_device_error), kernel attributes cached per GPU,
+ *   and the fixed scratch array of ckda_chunk_fwd_noalloc (part of the module's
+ *   device image).
  * - Layout is contiguous row-major, head-interleaved:
  *       q, k, alpha : [B, T, H, d_k]     v, o : [B, T, H, d_v]     beta : [B, T, H]
  *       S0, S_T, S  : [B, H, d_k, d_v]   (d_v fastest)
