@@ -359,6 +359,8 @@ def ours_arm(args):
         line["cpu_baseline"] = cpu_baseline(inp)
     if not args.no_extras and args.only == "all":
         line["decode"] = decode_measure(ck, dev, stream, world)
+    if not args.no_extras and world > 1:
+        line["cp"] = cp_measure(ck, dev, stream, world, rank)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -403,6 +405,35 @@ def configs_measure(ck, dev, stream, world):
                         "alg_bytes_per_launch": alg}})
         out[name] = ent
     return out
+
+
+def cp_measure(ck, dev, stream, world, rank, reps=3):
+    """Context parallelism (N > 1 only): the long workload (one batch of 16 heads x 65536
+    tokens with an initial state) split over the ranks in token order, each rank its
+    slice; one all-gather of the slices' affine maps per step (NCCL). Strong scaling: the
+    whole job is the one sequence batch; tokens/s over the slowest rank's time."""
+    import torch
+    from ckda_inputs import make_workload
+    from delta_rule_attention_ckda_b200 import context_parallel as cp
+    inp = make_workload("long")
+    B, T, H, dk, dv = inp.shape
+    lo, hi = (T * rank) // world, (T * (rank + 1)) // world
+    q, k, v, a, b = (x[:, lo:hi].contiguous().to(dev) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
+    S0 = inp.S0.to(dev) if rank == 0 else None
+
+    def step():
+        return cp.cp_chunk_fwd(q, k, v, a, b, S0)
+
+    step()
+    barrier(world)
+    assert ck.get_device_error() == 0
+    barrier(world)
+    secs = time_launches(step, reps, stream)
+    barrier(world)
+    value, secs = aggregate_throughput((hi - lo) * B * reps, secs, world, device="cuda")
+    return {"workload": f"long B={B} T={T} H={H} dk={dk} dv={dv} bf16, tokens split over {world} ranks",
+            "scaling": "strong", "tokens_per_s": value, "ms_per_step": 1e3 * secs / reps,
+            "exchange_bytes_per_rank": 4 * B * H * dk * (dk + dv), "collective": "all_gather (NCCL)"}
 
 
 def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):

@@ -60,6 +60,12 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_recurrent_fwd_ex.restype = i
     lib.ckda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp]
     lib.ckda_chunk_fwd_noalloc.restype = i
+    lib.ckda_chunk_fwd_maps_workspace_bytes.argtypes = [i] * 6
+    lib.ckda_chunk_fwd_maps_workspace_bytes.restype = sz
+    lib.ckda_chunk_fwd_maps.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 7 + [vp, sz, vp]
+    lib.ckda_chunk_fwd_maps.restype = i
+    lib.ckda_cp_prefix.argtypes = [fp] + [i] * 5 + [vp]
+    lib.ckda_cp_prefix.restype = i
     lib.ckda_bwd_workspace_bytes.argtypes = [i] * 6
     lib.ckda_bwd_workspace_bytes.restype = sz
     lib.ckda_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp] + [i] * 7 + [vp, sz, vp]
@@ -199,6 +205,46 @@ def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_s
                                        _stream(stream))
     _raise(st, "ckda_chunk_fwd_noalloc")
     return o, S_T
+
+
+def maps_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    return int(load().ckda_chunk_fwd_maps_workspace_bytes(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
+
+
+def chunk_fwd_maps(q, k, v, alpha, beta, *, M=None, N=None, workspace=None, stream=None, gate="signed",
+                   normalize_qk=False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """ckda_chunk_fwd_maps: the affine map S_T = M S_0 + N of every (b, h) sequence.
+    Returns (M [B,H,dk,dk], N [B,H,dk,dv]), fp32; allocated with torch when not given."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _check(q, "q", (B, T, H, dk))
+    _check(k, "k", (B, T, H, dk), dt)
+    _check(v, "v", (B, T, H, dv), dt)
+    _check(alpha, "alpha", (B, T, H, dk), torch.float32)
+    _check(beta, "beta", (B, T, H), torch.float32)
+    f32 = dict(device=q.device, dtype=torch.float32)
+    M = torch.empty(B, H, dk, dk, **f32) if M is None else M
+    N = torch.empty(B, H, dk, dv, **f32) if N is None else N
+    _check(M, "M", (B, H, dk, dk), torch.float32)
+    _check(N, "N", (B, H, dk, dv), torch.float32)
+    lib = load()
+    need = int(lib.ckda_chunk_fwd_maps_workspace_bytes(B, T, H, dk, dv, _dt(q)))
+    if need and workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ckda_chunk_fwd_maps(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(M), _ptr(N),
+                                 B, T, H, dk, dv, _dt(q), _mode(gate, normalize_qk), _ptr(workspace), wbytes,
+                                 _stream(stream))
+    _raise(st, "ckda_chunk_fwd_maps")
+    return M, N
+
+
+def cp_prefix(blocks: torch.Tensor, R: int, B: int, H: int, dk: int, dv: int, stream=None) -> torch.Tensor:
+    """ckda_cp_prefix, in place on `blocks` ([R, B*H*dk*(dk+dv)] fp32, rank r's M then N)."""
+    _check(blocks, "blocks", (R, B * H * dk * (dk + dv)), torch.float32)
+    _raise(load().ckda_cp_prefix(_ptr(blocks), R, B, H, dk, dv, _stream(stream)), "ckda_cp_prefix")
+    return blocks
 
 
 def bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:

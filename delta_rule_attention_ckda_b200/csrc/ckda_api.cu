@@ -39,19 +39,21 @@ ckda_status_t copy_state(const float* S0, float* S_T, size_t n, cudaStream_t st)
     return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
+// M_out != NULL: also the transition product into M_out (grid z = 1; see the kernel)
 template <typename TIn, bool kLogGate, bool kNorm>
 ckda_status_t launch_recurrent(const TIn* q, const TIn* k, const TIn* v, const float* alpha,
                                const float* beta, const float* S0, float* o, float* S_T,
-                               int B, int T, int H, int dk, int dv, cudaStream_t st) {
-    const int cols = dv <= 32 ? 32 : (dv <= 64 ? 64 : 128);
+                               int B, int T, int H, int dk, int dv, cudaStream_t st, float* M_out = nullptr) {
+    const int ncol = M_out ? std::max(dk, dv) : dv;
+    const int cols = ncol <= 32 ? 32 : (ncol <= 64 ? 64 : 128);
     // Few sequences: split the columns over more CTAs (one warp each).
     const long long seqs = (long long)B * H;
-    const int cols_per_cta = (seqs * ((dv + cols - 1) / cols) < 148) ? 32 : cols;
-    dim3 grid((unsigned)seqs, (unsigned)((dv + cols_per_cta - 1) / cols_per_cta));
+    const int cols_per_cta = (seqs * ((ncol + cols - 1) / cols) < 148) ? 32 : cols;
+    dim3 grid((unsigned)seqs, (unsigned)((ncol + cols_per_cta - 1) / cols_per_cta), M_out ? 2u : 1u);
     dim3 block((unsigned)cols_per_cta);
 #define CKDA_LAUNCH_REC(DKT)                                                                  \
     ckda::recurrent_fwd_kernel<DKT, TIn, kLogGate, kNorm><<<grid, block, 0, st>>>(q, k, v, alpha, beta, S0, o, \
-                                                                  S_T, T, H, dk, dv, cols_per_cta)
+                                                                  S_T, M_out, T, H, dk, dv, cols_per_cta)
     if (dk <= 16) CKDA_LAUNCH_REC(16);
     else if (dk <= 32) CKDA_LAUNCH_REC(32);
     else if (dk <= 64) CKDA_LAUNCH_REC(64);
@@ -225,6 +227,69 @@ ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const 
                              size_t workspace_bytes, void* stream) {
     return ckda_chunk_fwd_ex(q, k, v, alpha, beta, S0, o, S_T, B, T, H, dk, dv, dt, CKDA_GATE_SIGNED,
                              workspace, workspace_bytes, stream);
+}
+
+size_t ckda_chunk_fwd_maps_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {
+    if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return 0;
+    if (ckda_chunk_fwd_path(B, T, H, dk, dv, dt) != CKDA_PATH_CHUNK_TC) return 0;
+    return ckda::chunk_tc_maps_workspace_bytes(B, T, H, dk, dv);
+}
+
+ckda_status_t ckda_chunk_fwd_maps(const void* q, const void* k, const void* v, const float* gate,
+                                  const float* beta, float* M, float* N, int B, int T, int H, int dk, int dv,
+                                  ckda_dtype_t dt, int mode, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return CKDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
+    if (dt != CKDA_F32 && dt != CKDA_BF16) return CKDA_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
+    if ((long long)B * H == 0) return CKDA_OK;
+    if (!M || !N) return CKDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !gate || !beta)) return CKDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, gate, beta, M, N, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return CKDA_ERR_MISALIGNED;
+    const size_t need = ckda_chunk_fwd_maps_workspace_bytes(B, T, H, dk, dv, dt);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    if (T > 0 && ckda_chunk_fwd_path(B, T, H, dk, dv, dt) == CKDA_PATH_CHUNK_TC) {
+        cudaError_t e = ckda::launch_chunk_tc_maps(static_cast<const __nv_bfloat16*>(q),
+                                                   static_cast<const __nv_bfloat16*>(k),
+                                                   static_cast<const __nv_bfloat16*>(v), gate, beta, M, N, B, T,
+                                                   H, dk, dv, lg, nq, workspace, st);
+        return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+    }
+    // other shapes, and T = 0 (M = I, N = 0): the recurrent kernel in its map mode
+#define CKDA_MAPS(TIN)                                                                                    \
+    do {                                                                                                  \
+        const auto* qq = static_cast<const TIN*>(q);                                                       \
+        const auto* kk = static_cast<const TIN*>(k);                                                       \
+        const auto* vv = static_cast<const TIN*>(v);                                                       \
+        if (lg)                                                                                           \
+            return nq ? launch_recurrent<TIN, true, true>(qq, kk, vv, gate, beta, nullptr, nullptr, N, B, T, H, \
+                                                          dk, dv, st, M)                                  \
+                      : launch_recurrent<TIN, true, false>(qq, kk, vv, gate, beta, nullptr, nullptr, N, B, T, H, \
+                                                           dk, dv, st, M);                                \
+        return nq ? launch_recurrent<TIN, false, true>(qq, kk, vv, gate, beta, nullptr, nullptr, N, B, T, H,  \
+                                                       dk, dv, st, M)                                     \
+                  : launch_recurrent<TIN, false, false>(qq, kk, vv, gate, beta, nullptr, nullptr, N, B, T, H, \
+                                                        dk, dv, st, M);                                   \
+    } while (0)
+    if (dt == CKDA_BF16) CKDA_MAPS(__nv_bfloat16);
+    CKDA_MAPS(float);
+#undef CKDA_MAPS
+}
+
+ckda_status_t ckda_cp_prefix(float* blocks, int R, int B, int H, int dk, int dv, void* stream) {
+    if (R < 1 || B < 0 || H < 0 || !dims_ok(dk, dv)) return CKDA_ERR_INVALID_ARG;
+    if ((long long)B * H > 0x7fffffffLL) return CKDA_ERR_UNSUPPORTED;
+    if ((long long)B * H == 0 || R == 1) return CKDA_OK;
+    if (dk % 4 != 0) return CKDA_ERR_UNSUPPORTED;
+    if (blocks == nullptr) return CKDA_ERR_INVALID_ARG;
+    if (!aligned16(blocks)) return CKDA_ERR_MISALIGNED;
+    cudaError_t e = ckda::launch_cp_prefix(blocks, R, B, H, dk, dv, as_stream(stream));
+    return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
 size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {

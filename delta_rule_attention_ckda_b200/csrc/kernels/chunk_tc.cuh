@@ -123,6 +123,7 @@ constexpr uint32_t kTmaBytes2 = 4 * 8192;   // q + v (2 bf16 boxes each)
 constexpr uint32_t kFlagVZero = 1u;     // v is taken as zero (not loaded; no V T^T term)
 constexpr uint32_t kFlagNoO = 2u;       // no o output
 constexpr uint32_t kFlagS0Ident = 4u;   // the state entering each segment is the identity (d_v = d_k)
+constexpr uint32_t kFlagMapsOnly = 8u;  // every segment, the first included, builds its affine map
 
 // Byte address (from tile base) of the 16-byte chunk `ch` (0..7) of row `row` in a
 // tile of 128-byte rows with 128-byte swizzle.
@@ -317,21 +318,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // blockIdx.z = 1 runs the segment's transition product instead: identity entering state,
     // v = 0, no o, d_v = d_k, the result written to slot (bh, sg) of M_seg. Segment 0 needs
     // none (its entering state is known), so those CTAs return at once.
+    // kFlagMapsOnly in flags_in treats segment 0 like the others (the whole launch builds
+    // affine maps: z = 0 the state from zero with flags_in, z = 1 the transition product).
     const bool trans = blockIdx.z != 0;
     const int bh = blockIdx.x;                    // grid: x = (batch, head), y = segment
     const int sg = sg_base + (int)blockIdx.y;
-    if (trans && sg == 0) return;
-    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident) : (sg == 0 ? 0u : flags_in);
+    const bool direct = sg == 0 && (flags_in & kFlagMapsOnly) == 0;   // segment 0 from the known S0
+    if (trans && direct) return;
+    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident) : (direct ? 0u : flags_in);
     const int dv = trans ? dk : dv_in;
-    if (trans) ST_seg = M_seg;
     const int b = bh / H, h = bh % H;
     const int ta = sg * seg_len;
     const int tb = min(T, ta + seg_len);
     const size_t slot = ((size_t)bh * nseg + sg) * dk * dv;
     const float* S0 = (flags & kFlagS0Ident) ? nullptr
-                    : sg == 0 ? (S0_head ? S0_head + (size_t)bh * dk * dv : nullptr)
-                              : (S0_seg ? S0_seg + slot : nullptr);
-    float* ST = (sg == nseg - 1) ? (ST_last ? ST_last + (size_t)bh * dk * dv : nullptr)
+                    : direct ? (S0_head ? S0_head + (size_t)bh * dk * dv : nullptr)
+                             : (S0_seg ? S0_seg + slot : nullptr);
+    float* ST = trans ? (M_seg ? M_seg + slot : nullptr)
+              : (sg == nseg - 1) ? (ST_last ? ST_last + (size_t)bh * dk * dv : nullptr)
                                  : (ST_seg ? ST_seg + slot : nullptr);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
@@ -353,7 +357,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::prefetch_tensormap(&map_q);
         tc::prefetch_tensormap(&map_v);
         tc::prefetch_tensormap(&map_a);
-        tc::prefetch_tensormap(&map_o);
+        if ((flags & kFlagNoO) == 0) tc::prefetch_tensormap(&map_o);   // unset when no CTA writes o
     }
     if (tid < 2 * D) sh_kref[tid] = 1.f;
     // blocks of (I + A)^{-1} above the 16 x 16 block diagonal: zero once, never written again

@@ -14,6 +14,9 @@
 //
 // kLogGate: the gate input holds g = ln a (a non-negative gate, a = e^g <= 1) instead of a.
 // kNorm: q and k are divided by their L2 norms per token (floor 1e-12) once staged.
+// Affine map of the sequence (S_T = M S_0 + N): CTAs with blockIdx.z = 1 run the transition
+// product instead, from the identity (d_k x d_k) with v = 0, into M_out; o may be NULL (not
+// written) and S0 NULL, so the z = 0 CTAs then build N.
 #pragma once
 #include "common.cuh"
 
@@ -24,7 +27,7 @@ __global__ void __launch_bounds__(128)
 recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                      const TIn* __restrict__ v, const float* __restrict__ alpha,
                      const float* __restrict__ beta, const float* S0,
-                     float* __restrict__ o, float* ST,
+                     float* __restrict__ o, float* ST, float* M_out,
                      int T, int H, int dk, int dv, int cols_per_cta) {
     constexpr int TB = 16;                       // tokens staged per batch
     __shared__ float sk[TB][DK], sq[TB][DK], sa[TB][DK];
@@ -34,14 +37,18 @@ recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh % H;
+    const bool trans = blockIdx.z != 0;          // transition product: columns of the identity
+    const int ncol = trans ? dk : dv;
     const int j = blockIdx.y * cols_per_cta + threadIdx.x;
-    const bool active = (threadIdx.x < cols_per_cta) && (j < dv);
-    const size_t state_base = (size_t)bh * dk * dv;
+    const bool active = (threadIdx.x < cols_per_cta) && (j < ncol);
+    const size_t state_base = (size_t)bh * dk * ncol;
+    if (trans) o = nullptr;
 
     float s[DK];
 #pragma unroll
     for (int i = 0; i < DK; ++i)
-        s[i] = (active && S0 != nullptr && i < dk) ? S0[state_base + (size_t)i * dv + j] : 0.f;
+        s[i] = trans ? ((active && i == j) ? 1.f : 0.f)
+                     : ((active && S0 != nullptr && i < dk) ? S0[state_base + (size_t)i * dv + j] : 0.f);
 
     for (int t0 = 0; t0 < T; t0 += TB) {
         const int nt = min(TB, T - t0);
@@ -58,7 +65,7 @@ recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
         if (threadIdx.x < nt) sb[threadIdx.x] = __ldg(beta + ((size_t)b * T + t0 + threadIdx.x) * H + h);
         for (int tt = 0; tt < nt; ++tt) {
             const size_t tok = ((size_t)b * T + t0 + tt) * H + h;
-            sv[tt][threadIdx.x] = active ? ld_in(v + tok * dv + j) : 0.f;
+            sv[tt][threadIdx.x] = (active && !trans) ? ld_in(v + tok * dv + j) : 0.f;
         }
         __syncthreads();
         if constexpr (kNorm) {
@@ -94,13 +101,14 @@ recurrent_fwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                 s[i] = fmaf(sk[tt][i], u, s[i]);
                 acc = fmaf(s[i], sq[tt][i], acc);
             }
-            if (active) o[(((size_t)b * T + t0 + tt) * H + h) * dv + j] = acc;
+            if (active && o != nullptr) o[(((size_t)b * T + t0 + tt) * H + h) * dv + j] = acc;
         }
     }
-    if (active && ST != nullptr) {
+    float* out = trans ? M_out : ST;
+    if (active && out != nullptr) {
 #pragma unroll
         for (int i = 0; i < DK; ++i)
-            if (i < dk) ST[state_base + (size_t)i * dv + j] = s[i];
+            if (i < dk) out[state_base + (size_t)i * ncol + j] = s[i];
     }
 }
 

@@ -54,7 +54,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 6
+#define CKDA_ABI_VERSION 7
 
 typedef enum {
     CKDA_OK = 0,
@@ -191,6 +191,54 @@ CKDA_API ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, cons
                                 float* o, float* S_T,
                                 int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
                                 int mode, void* stream);
+
+/*
+ * Context parallelism over T (a sequence split over ranks in token order; the ai.info
+ * summary of the Complex KDA paper, "Why This Matters", names long-context models with
+ * a fixed-size recurrent state as the use). The pages describe no multi-GPU scheme:
+ * this is the plainest one the recurrence allows. A slice of tokens acts on the state
+ * entering it as an affine map, S_out = M S_in + N, with M (d_k x d_k) the product of
+ * the slice's transitions (I - beta k k^T) Diag(alpha), last token leftmost, and N
+ * (d_k x d_v) the state the slice builds from S_in = 0. Each rank after the first
+ * builds its slice's map (ckda_chunk_fwd_maps), the first runs its slice directly
+ * from S0; the ranks exchange (M, N) once (an all-gather: B*H*d_k*(d_k+d_v) floats per
+ * rank); ckda_cp_prefix chains the maps into every rank's entering state; each rank
+ * after the first then runs its slice from that state (ckda_chunk_fwd_ex) for o.
+ */
+
+/* Bytes of workspace ckda_chunk_fwd_maps needs (0 when it builds the maps in one pass):
+ * few (b, h) pairs split the slice into sub-slices built side by side, which need
+ * B*H*(nsub+1)*dk*(dk+dv) fp32. Invalid sizes return 0. */
+CKDA_API size_t ckda_chunk_fwd_maps_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
+
+/*
+ * The affine map S_T = M S_0 + N of every (b, h) sequence of T tokens, for the gate
+ * form and options in `mode` (as ckda_chunk_fwd_ex).
+ *   q, k, gate [B,T,H,dk]; v [B,T,H,dv] (dtype dt); beta [B,T,H] fp32
+ *   M  [B,H,dk,dk] fp32 out: the product of the transitions (T = 0: the identity)
+ *   N  [B,H,dk,dv] fp32 out: the final state from a zero initial state (T = 0: zero)
+ *   workspace: at least ckda_chunk_fwd_maps_workspace_bytes(...) bytes, caller-owned.
+ * Tensor-core shapes (bf16, d_k, d_v in {64, 128}) run the chunk kernel with v = 0 and
+ * an identity initial state for M; other shapes run the recurrent kernel the same way.
+ * M and N must not overlap each other or any input. Errors as ckda_chunk_fwd_ex
+ * (CKDA_ERR_INVALID_ARG for a NULL M or N).
+ */
+CKDA_API ckda_status_t ckda_chunk_fwd_maps(const void* q, const void* k, const void* v,
+                                const float* gate, const float* beta, float* M, float* N,
+                                int B, int T, int H, int dk, int dv, ckda_dtype_t dt,
+                                int mode, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The exchange step's prefix, in place on the gathered maps of R ranks in token order.
+ * `blocks` holds R consecutive blocks of B*H*dk*(dk+dv) fp32, block r = rank r's
+ * [B,H,dk,dk] M followed by its [B,H,dk,dv] N. Block 0's N is the first rank's final
+ * state (its M is not read). On return the N part of block r holds the state after
+ * rank r's tokens: rank r + 1's entering state, and for r = R - 1 the sequence's final
+ * state. fp32, S_{r} = M_r S_{r-1} + N_r in rank order. R = 1 is a no-op.
+ * Errors: CKDA_ERR_INVALID_ARG (R < 1, bad sizes, NULL blocks), CKDA_ERR_MISALIGNED,
+ * CKDA_ERR_UNSUPPORTED when dk is not a multiple of 4.
+ */
+CKDA_API ckda_status_t ckda_cp_prefix(float* blocks, int R, int B, int H, int dk, int dv, void* stream);
 
 /*
  * Token-by-token forward on CUDA cores in fp32 (the recurrent path of

@@ -49,7 +49,7 @@ def test_status_strings(lib):
         s = lib.ckda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.ckda_status_string(99) == b"unknown status"
-    assert lib.ckda_abi_version() == 6
+    assert lib.ckda_abi_version() == 7
 
 
 NULL = None
@@ -198,3 +198,47 @@ def test_gate_mode_names():
         _lib._gate("exp")
     text = open(os.path.join(ROOT, "include", "ckda.h")).read()
     assert "CKDA_GATE_SIGNED = 0" in text and "CKDA_GATE_LOG = 1" in text
+
+
+def test_maps_workspace_and_argument_checks(lib):
+    """ckda_chunk_fwd_maps: workspace only when the sequences are too few to fill the GPU
+    (then (nsub + 1) slots of [M | N] per sequence), argument errors before any launch."""
+    bf = 1
+    assert lib.ckda_chunk_fwd_maps_workspace_bytes(64, 256, 16, 128, 128, bf) == 0      # 2048 CTAs already
+    wl = lib.ckda_chunk_fwd_maps_workspace_bytes(8, 4096, 16, 128, 128, bf)             # 256 CTAs: split
+    assert wl % (128 * 128 * 256 * 4) == 0
+    assert lib.ckda_chunk_fwd_maps_workspace_bytes(1, 65536, 16, 128, 128, 0) == 0     # fp32: recurrent
+    w = lib.ckda_chunk_fwd_maps_workspace_bytes(1, 65536, 16, 128, 128, bf)
+    slot = 16 * 128 * 256 * 4
+    assert w > 0 and w % slot == 0 and 3 <= w // slot <= 65
+    assert lib.ckda_chunk_fwd_maps_workspace_bytes(1, 65536, 16, 64, 128, bf) % (16 * 64 * 192 * 4) == 0
+    assert lib.ckda_chunk_fwd_maps_workspace_bytes(-1, 64, 1, 128, 128, bf) == 0
+    p = ctypes.c_void_p(256)
+    fp = ctypes.cast(p, ctypes.POINTER(ctypes.c_float))
+    null = ctypes.POINTER(ctypes.c_float)()
+    bad = ctypes.cast(ctypes.c_void_p(260), ctypes.POINTER(ctypes.c_float))
+    args = (1, 64, 1, 16, 16, 0)
+    assert lib.ckda_chunk_fwd_maps(p, p, p, fp, fp, null, fp, *args, 0, None, 0, None) == 1     # no M
+    assert lib.ckda_chunk_fwd_maps(p, p, p, fp, fp, fp, null, *args, 0, None, 0, None) == 1     # no N
+    assert lib.ckda_chunk_fwd_maps(None, p, p, fp, fp, fp, fp, *args, 0, None, 0, None) == 1    # no q
+    assert lib.ckda_chunk_fwd_maps(p, p, p, fp, fp, bad, fp, *args, 0, None, 0, None) == 3
+    assert lib.ckda_chunk_fwd_maps(p, p, p, fp, fp, fp, fp, *args, 0x200, None, 0, None) == 1   # mode
+    assert lib.ckda_chunk_fwd_maps(p, p, p, fp, fp, fp, fp, 1, 64, 1, 0, 16, 0, 0, None, 0, None) == 1
+    assert lib.ckda_chunk_fwd_maps(p, p, p, fp, fp, fp, fp, 1, 65536, 16, 128, 128, bf, 0, None, 0,
+                                   None) == 6                                                  # workspace
+    assert lib.ckda_chunk_fwd_maps(None, None, None, null, null, null, null, 0, 64, 4, 16, 16, 0, 0, None, 0,
+                                   None) == 0                                                  # empty: nothing
+
+
+def test_cp_prefix_argument_checks(lib):
+    p = ctypes.cast(ctypes.c_void_p(256), ctypes.POINTER(ctypes.c_float))
+    null = ctypes.POINTER(ctypes.c_float)()
+    bad = ctypes.cast(ctypes.c_void_p(260), ctypes.POINTER(ctypes.c_float))
+    assert lib.ckda_cp_prefix(p, 0, 1, 1, 16, 16, None) == 1          # R < 1
+    assert lib.ckda_cp_prefix(p, 2, 1, 1, 0, 16, None) == 1           # d_k = 0
+    assert lib.ckda_cp_prefix(p, 2, 1, 1, 16, 129, None) == 1         # d_v > 128
+    assert lib.ckda_cp_prefix(null, 2, 1, 1, 16, 16, None) == 1
+    assert lib.ckda_cp_prefix(bad, 2, 1, 1, 16, 16, None) == 3
+    assert lib.ckda_cp_prefix(p, 2, 1, 1, 6, 16, None) == 2           # d_k not a multiple of 4
+    assert lib.ckda_cp_prefix(null, 1, 1, 1, 16, 16, None) == 0       # one rank: nothing to chain
+    assert lib.ckda_cp_prefix(null, 3, 0, 4, 16, 16, None) == 0       # no sequences
