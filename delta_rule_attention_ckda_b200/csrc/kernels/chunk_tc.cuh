@@ -38,13 +38,16 @@
 // solve) and one epilogue warpgroup (state copy, o tile, -Z^T and U^T into TMEM) whose
 // leader thread issues the TMA loads and stores and every MMA but [P;A]. Everything is
 // computed transposed so the 128 feature rows sit on the 128 TMEM lanes: the fp32
-// state lives in TMEM for the whole sequence and never round-trips HBM. Every product
-// runs on tcgen05 with bf16 operands; operands that are not raw bf16 inputs are split
+// state lives in TMEM for the whole sequence and never round-trips HBM. Every chunk-sized
+// product runs on tcgen05 with bf16 operands; operands that are not raw bf16 inputs are split
 // x = hi + lo (hi rounded to nearest, lo the remainder truncated: |x - hi - lo| <=
 // 2^-15 |x|) and each product is the three passes hi*hi + hi*lo + lo*hi, which the
 // fp32-state tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by
 // TMA (no multicast) with 128-byte swizzle; tokens past the end read as zero and get
-// gate 1. A 64-wide d_k or d_v is the 128-wide problem with zero padding.
+// gate 1. A 64-wide d_k or d_v is the 128-wide problem with zero padding. The solve's
+// small block products (16 and 32 wide, inside the 64 x 64 inverse) run on warp-level
+// mma.sync in three tf32 passes: latency-bound steps where a 128-row tcgen05 tile and a
+// TMEM round trip would cost more than they save.
 //
 // Exponent safety. e1 and e2 stay inside [2^-96, 2^96] unless a chunk's gates decay by
 // more than 2^-192 in some channel; such a chunk computes A and P pair by pair on CUDA
@@ -80,7 +83,7 @@ constexpr float kChunkRange = 192.f;  // -L_C bound for the fast path (factors w
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t SM_K = 0;            // k tile: 2 TMA boxes [64 tok][64 ch] bf16
-constexpr uint32_t SM_AT = 0;           //   after the gate: A column-major, at[s][r] = A_rs, fp32 [64][64]
+constexpr uint32_t SM_AT = 0;           //   after the gate: A column-major, fp32 [64][64] (at_idx)
 constexpr uint32_t SM_Q = 16384;        // q tile
 constexpr uint32_t SM_T = 16384;        //   after the gate: [T_hi ; T_lo] K-major [128 n][64 s]
 constexpr uint32_t SM_V = 32768;        // v tile (MN-major A operand of V^T T^T)
@@ -95,8 +98,9 @@ constexpr uint32_t SM_YLO = 172032;     //   K-major B operand of 192 rows for t
 constexpr uint32_t SM_PLO = 188416;
 constexpr uint32_t SM_XS = 196608;      // (I + A)^{-1}, fp32 row-major [64][XS_LD]; blocks above the
 constexpr int XS_LD = 68;               //   16 x 16 block diagonal stay zero for the whole kernel
-constexpr uint32_t SM_RS = SM_XS + 64 * XS_LD * 4;   // solve temporaries, fp32 [32][36]
-constexpr uint32_t SM_SMALL = SM_RS + 32 * 36 * 4;
+constexpr uint32_t SM_RS = SM_XS + 64 * XS_LD * 4;   // solve temporaries, fp32 [32][RS_LD]
+constexpr int RS_LD = 40;
+constexpr uint32_t SM_SMALL = SM_RS + 32 * RS_LD * 4;
 constexpr uint32_t SM_BYTES = SM_SMALL + 8192;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;       // + alignment slack
 static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
@@ -129,6 +133,38 @@ constexpr uint32_t kFlagMapsOnly = 8u;  // every segment, the first included, bu
 // tile of 128-byte rows with 128-byte swizzle.
 __device__ __forceinline__ uint32_t chunk_off(int row, int ch) {
     return (uint32_t)row * 128u + ((uint32_t)(ch ^ (row & 7)) << 4);
+}
+
+// A_rs in the column-major A tile, rows XOR-ed by 8 (s & 3) within each column: the
+// warp's fragment loads of the solve's mma (rows g, columns t) then hit 32 distinct banks.
+__device__ __forceinline__ int at_idx(int r, int s) { return s * 64 + (r ^ (8 * (s & 3))); }
+
+// One warp-level tf32 MMA, D (16 x 8) += A (16 x 8) B (8 x 8), fp32 accumulation.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D += A B to about fp32 accuracy in three tf32 passes: x = big + small with big = x with
+// its low 13 mantissa bits cleared (exactly representable) and small = x - big (exact in
+// fp32; the MMA reads its top 19 bits), D += small_A big_B + big_A small_B + big_A big_B.
+__device__ __forceinline__ void mma3_tf32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
+    uint32_t ab[4], as[4], bb[2], bs[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        ab[i] = __float_as_uint(a[i]) & 0xFFFFE000u;
+        as[i] = __float_as_uint(a[i] - __uint_as_float(ab[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        bb[i] = __float_as_uint(b[i]) & 0xFFFFE000u;
+        bs[i] = __float_as_uint(b[i] - __uint_as_float(bb[i]));
+    }
+    mma_tf32(d, as, bb);
+    mma_tf32(d, ab, bs);
+    mma_tf32(d, ab, bb);
 }
 
 // Element (r, c) of a bf16 TMA tile made of 64-channel boxes [64 tokens][128 B].
@@ -262,9 +298,12 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 // MMA group but [P;A] (an issuing thread blocks for about the duration of the MMAs it
 // issues, so issue stays off the compute warps). The groups hand operands over through
 // mbarriers; each MMA group commits to its own mbarrier. What overlaps:
-//   factors, X and Y tiles of chunk c          ||  (epilogue: waits for them)
-//   [P;A] epilogue and solve of chunk c        ||  o tile of chunk c-1, state copy, C1, -Z^T
+//   factors, X and Y tiles of chunk c          ||  state copy of chunk c (after c-1's state MMA)
+//   [P;A] epilogue and solve of chunk c        ||  o tile of chunk c-1, C1, -Z^T
 //   gate cumulation of chunk c+1               ||  U MMA, U^T, O / state MMA of chunk c
+// The two groups form two chains of about equal length per chunk (compute: factors, [P;A],
+// solve, gate; epilogue: state copy, o tile, C1, -Z^T, U, U^T, state MMA), so a phase only
+// pays off when both chains shorten.
 //
 // kLogGate: the gate input holds g = ln a of a non-negative gate (KDA) instead of a signed
 // a; the cumulation then needs no logarithm and no sign parity.
@@ -526,8 +565,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         for (; ck < nchunks; ++ck) {
             const uint32_t par = (uint32_t)ck & 1u;
             const int t0 = ta + ck * C;
-            // ---------------- E1: state copy (after the previous o tile and the next alpha are on
-            // their way, so that it overlaps the solve). The accumulator holds S Diag(1/kappa_prev):
+            // ---------------- E1: state copy, as soon as the previous state MMA is done (it overlaps
+            // the compute warps' factors), then the previous o tile once the alpha space is free,
+            // then C1. The accumulator holds S Diag(1/kappa_prev):
             // S = acc kappa_prev, then the operand S g_ref (split into TMEM) and the new
             // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
             // for fast-decaying channels although each factor and each result is in range.
@@ -536,21 +576,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             tc::tc_fence_after();
             // the previous chunk's o rows, once the gate (or the exact path) is done with the
             // alpha space; its store and the next alpha go out before the state copy
-            efail |= !tc::mbar_wait(&bar_hap, par);
-            if (ck > 0) stage_o();
-            epi_publish();
-            if (esync_or(efail)) break;
-            if (leader) {
-                tc::tc_fence_after();
-                if (ck > 0 && want_o) {
-                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
-                    tc::bulk_commit();
-                }
-                if (ck + 1 < nchunks) {
-                    tc::bulk_wait_read0();
-                    issue_loads1a(t0 + C);
-                }
-            }
             {
                 float sv[2][16];
                 tc::tmem_ld32<16>(te + TM_S, sv[0]);
@@ -584,8 +609,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
                 }
             }
+            efail |= !tc::mbar_wait(&bar_hap, par);
+            if (ck > 0) stage_o();
             epi_publish();
             if (esync_or(efail)) break;
+            if (leader) {
+                tc::tc_fence_after();
+                if (ck > 0 && want_o) {
+                    tc::tma_store_4d(&map_o, sm + SM_OT, 0, h, t0 - C, b);   // rows past T are skipped
+                    tc::bulk_commit();
+                }
+                if (ck + 1 < nchunks) {
+                    tc::bulk_wait_read0();
+                    issue_loads1a(t0 + C);
+                }
+            }
             // leader: C1 (runs while the compute warps solve)
             if (leader) {
                 tc::tc_fence_after();
@@ -872,7 +910,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int s = 32 * hh + i;
-                        at[s * 64 + r] = (s < r) ? br * d1[i] : 0.f;
+                        at[at_idx(r, s)] = (s < r) ? br * d1[i] : 0.f;
                     }
                 } else if (want_o) {
                     const int r = m;
@@ -917,7 +955,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                             av *= sh_kn[r] * sh_kn[sc];
                             pv *= sh_qn[r] * sh_kn[sc];
                         }
-                        at[sc * 64 + r] = (sc < r) ? br * av : 0.f;
+                        at[at_idx(r, sc)] = (sc < r) ? br * av : 0.f;
                         uint32_t hpair, lpair;
                         split2((sc <= r) ? pv : 0.f, 0.f, hpair, lpair);
                         const uint32_t offp = chunk_off(r, sc >> 3) + (uint32_t)(sc & 7) * 2u;
@@ -936,19 +974,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // block -X_22 A_21 X_11 (X_ii the inverses of the diagonal blocks).
             if (warp < 4 && lane < 16) {
                 // diagonal block I, column j: right-looking forward substitution; column ss of
-                // A_II is contiguous in the column-major A, so each step is 4 broadcast loads
+                // A_II is contiguous in the column-major A (4-row groups keep their order under
+                // the row XOR), so each step is 4 broadcast loads
                 const int I = warp, j = lane;
-                const float* acol = at + (16 * I) * 64 + 16 * I;
                 float acc[16];
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) acc[rr] = (rr == j) ? 1.f : 0.f;
 #pragma unroll
                 for (int ss = 0; ss < 15; ++ss) {
                     const float xv = acc[ss];             // final value of x_ss (0 above the diagonal)
+                    const int sc = 16 * I + ss;
                     float a[16];
 #pragma unroll
                     for (int g = (ss + 1) >> 2; g < 4; ++g) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(acol + ss * 64 + 4 * g);
+                        const float4 t4 = *reinterpret_cast<const float4*>(at + at_idx(16 * I + 4 * g, sc));
                         a[4 * g] = t4.x; a[4 * g + 1] = t4.y; a[4 * g + 2] = t4.z; a[4 * g + 3] = t4.w;
                     }
 #pragma unroll
@@ -958,49 +997,55 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 for (int rr = 0; rr < 16; ++rr) xs[(16 * I + rr) * XS_LD + 16 * I + j] = acc[rr];
             }
             csync();
-            // level 1 (blocks of 16 -> 32), pairs (0,1) and (2,3): R = A_10 X_00, X_10 = -X_11 R.
-            // Thread: pair pb, row r, columns 2 c2, 2 c2 + 1.
-            {
-                const int pb = tid >> 7, r = (tid >> 3) & 15, c2 = tid & 7, o = 32 * pb;
-                float2 acc = make_float2(0.f, 0.f);
+            // level 1 (blocks of 16 -> 32), pairs (0,1) and (2,3): R = A_10 X_00, X_10 = -X_11 R, on
+            // warp MMAs (m16n8k8, three tf32 passes). Warp w < 4: pair pb = w / 2, column tile
+            // nt = w % 2 (8 columns); it owns all 16 rows of its R columns, so R goes through a
+            // warp-private scratch. Fragment lanes: row g = lane / 4, column t = lane % 4.
+            const int fg = lane >> 2, ft = lane & 3;
+            if (warp < 4) {
+                const int pb = warp >> 1, nt = warp & 1, o = 32 * pb;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float a = at[(o + k) * 64 + o + 16 + r];
-                    const float2 xv = *reinterpret_cast<const float2*>(xs + (o + k) * XS_LD + o + 2 * c2);
-                    acc.x = fmaf(a, xv.x, acc.x);
-                    acc.y = fmaf(a, xv.y, acc.y);
+                for (int ks = 0; ks < 2; ++ks) {
+                    if (ks < nt) continue;                // X_00[k][c] = 0 for k < c
+                    const int s0 = o + 8 * ks + ft, s1 = s0 + 4, r0 = o + 16 + fg, r1 = r0 + 8;
+                    const float a[4] = {at[at_idx(r0, s0)], at[at_idx(r1, s0)], at[at_idx(r0, s1)], at[at_idx(r1, s1)]};
+                    const float b[2] = {xs[s0 * XS_LD + o + 8 * nt + fg], xs[s1 * XS_LD + o + 8 * nt + fg]};
+                    mma3_tf32(d, a, b);
                 }
-                *reinterpret_cast<float2*>(rs + pb * 320 + r * 20 + 2 * c2) = acc;
-                csync();
-                float2 xo = make_float2(0.f, 0.f);
+                float* sc = rs + warp * 128;              // R columns of this warp, [16][8]
+                *reinterpret_cast<float2*>(sc + fg * 8 + 2 * ft) = make_float2(d[0], d[1]);
+                *reinterpret_cast<float2*>(sc + (fg + 8) * 8 + 2 * ft) = make_float2(d[2], d[3]);
+                __syncwarp();
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int mm = 0; mm < 16; ++mm) {
-                    const float xd = xs[(o + 16 + r) * XS_LD + o + 16 + mm];   // X_11, zero above the diagonal
-                    const float2 rv = *reinterpret_cast<const float2*>(rs + pb * 320 + mm * 20 + 2 * c2);
-                    xo.x = fmaf(xd, rv.x, xo.x);
-                    xo.y = fmaf(xd, rv.y, xo.y);
+                for (int ks = 0; ks < 2; ++ks) {
+                    const int rr = o + 16 + fg, cc = o + 16 + 8 * ks + ft;   // X_11[i][k] = 0 for k > i
+                    const float a[4] = {xs[rr * XS_LD + cc], xs[(rr + 8) * XS_LD + cc], xs[rr * XS_LD + cc + 4],
+                                        xs[(rr + 8) * XS_LD + cc + 4]};
+                    const float b[2] = {sc[(8 * ks + ft) * 8 + fg], sc[(8 * ks + ft + 4) * 8 + fg]};
+                    mma3_tf32(e, a, b);
                 }
-                *reinterpret_cast<float2*>(xs + (o + 16 + r) * XS_LD + o + 2 * c2) = make_float2(-xo.x, -xo.y);
+                *reinterpret_cast<float2*>(xs + (o + 16 + fg) * XS_LD + o + 8 * nt + 2 * ft) = make_float2(-e[0], -e[1]);
+                *reinterpret_cast<float2*>(xs + (o + 24 + fg) * XS_LD + o + 8 * nt + 2 * ft) = make_float2(-e[2], -e[3]);
             }
             csync();
-            // level 2 (32 -> 64): R = A[32:64, 0:32] X[0:32, 0:32], X[32:64, 0:32] = -X[32:64, 32:64] R.
+            // level 2 (32 -> 64): R = A[32:64, 0:32] X[0:32, 0:32], X[32:64, 0:32] = -X[32:64, 32:64] R,
+            // warp (mt = w / 4, nt = w % 4): the 16 x 8 tile (rows 16 mt, columns 8 nt) of each.
             // T = X Diag(beta) is split into the MMA operand as soon as a block of X is final.
             {
-                // R: warp -> column group cg (columns 4 cg .. 4 cg + 3), lane -> row; X[k][c] = 0
-                // for k < c, so group cg runs 32 - 4 cg steps. Warps w and w + 4 share a
-                // scheduler: they take groups w and 7 - w (36 steps per scheduler).
-                const int cg = (warp < 4) ? warp : 11 - warp, r = lane;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-                for (int k = 4 * cg; k < 32; ++k) {
-                    const float a = at[k * 64 + 32 + r];
-                    const float4 xv = *reinterpret_cast<const float4*>(xs + k * XS_LD + 4 * cg);
-                    acc.x = fmaf(a, xv.x, acc.x);
-                    acc.y = fmaf(a, xv.y, acc.y);
-                    acc.z = fmaf(a, xv.z, acc.z);
-                    acc.w = fmaf(a, xv.w, acc.w);
+                const int mt = warp >> 2, nt = warp & 3;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    if (ks < nt) continue;                // X[k][c] = 0 for k < c
+                    const int s0 = 8 * ks + ft, s1 = s0 + 4, r0 = 32 + 16 * mt + fg, r1 = r0 + 8;
+                    const float a[4] = {at[at_idx(r0, s0)], at[at_idx(r1, s0)], at[at_idx(r0, s1)], at[at_idx(r1, s1)]};
+                    const float b[2] = {xs[s0 * XS_LD + 8 * nt + fg], xs[s1 * XS_LD + 8 * nt + fg]};
+                    mma3_tf32(d, a, b);
                 }
-                *reinterpret_cast<float4*>(rs + r * 36 + 4 * cg) = acc;
+                *reinterpret_cast<float2*>(rs + (16 * mt + fg) * RS_LD + 8 * nt + 2 * ft) = make_float2(d[0], d[1]);
+                *reinterpret_cast<float2*>(rs + (16 * mt + fg + 8) * RS_LD + 8 * nt + 2 * ft) = make_float2(d[2], d[3]);
                 // final blocks of T: rows 0..31 x columns 0..31 and rows 32..63 x columns 32..63
                 // (16-byte chunk ch of row tr), and the zero block rows 0..31 x columns 32..63
                 {
@@ -1017,27 +1062,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
                 // A (k-tile space) is consumed: the epilogue leader loads the next chunk's k
                 csync();
-                // X[32:64, 0:32]: thread -> row 32 + r2, columns 4 c4 .. 4 c4 + 3, straight into T.
-                // X[32 + r2][32 + mm] is zero for mm > r2: warps 0-3 hold rows r2 < 16.
-                const int r2 = tid >> 3, c4 = tid & 7;
-                const int mmax = (warp < 4) ? 16 : 32;
-                float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                for (int mm = 0; mm < mmax; ++mm) {
-                    const float xd = xs[(32 + r2) * XS_LD + 32 + mm];
-                    const float4 rv = *reinterpret_cast<const float4*>(rs + mm * 36 + 4 * c4);
-                    xo.x = fmaf(xd, rv.x, xo.x);
-                    xo.y = fmaf(xd, rv.y, xo.y);
-                    xo.z = fmaf(xd, rv.z, xo.z);
-                    xo.w = fmaf(xd, rv.w, xo.w);
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    if (ks > 2 * mt + 1) continue;        // X[32 + i][32 + k] = 0 for k > i
+                    const int rr = 32 + 16 * mt + fg, cc = 32 + 8 * ks + ft;
+                    const float a[4] = {xs[rr * XS_LD + cc], xs[(rr + 8) * XS_LD + cc], xs[rr * XS_LD + cc + 4],
+                                        xs[(rr + 8) * XS_LD + cc + 4]};
+                    const float b[2] = {rs[(8 * ks + ft) * RS_LD + 8 * nt + fg], rs[(8 * ks + ft + 4) * RS_LD + 8 * nt + fg]};
+                    mma3_tf32(e, a, b);
                 }
-                const float4 b4 = reinterpret_cast<const float4*>(sh_beta)[c4];
+                // T rows 32 + 16 mt + g (+ 8), columns 8 nt + 2 t (+ 1): -X Diag(beta), split
+                const float2 bb = *reinterpret_cast<const float2*>(sh_beta + 8 * nt + 2 * ft);
                 uint32_t h0, l0, h1, l1;
-                split2(-xo.x * b4.x, -xo.y * b4.y, h0, l0);
-                split2(-xo.z * b4.z, -xo.w * b4.w, h1, l1);
-                const uint32_t off = chunk_off(32 + r2, c4 >> 1) + (uint32_t)(c4 & 1) * 8u;
-                *reinterpret_cast<uint2*>(sm + SM_T + off) = make_uint2(h0, h1);
-                *reinterpret_cast<uint2*>(sm + SM_T + 8192 + off) = make_uint2(l0, l1);
+                split2(-e[0] * bb.x, -e[1] * bb.y, h0, l0);
+                split2(-e[2] * bb.x, -e[3] * bb.y, h1, l1);
+                const int row0 = 32 + 16 * mt + fg;
+                const uint32_t off0 = chunk_off(row0, nt) + 4u * ft, off1 = chunk_off(row0 + 8, nt) + 4u * ft;
+                *reinterpret_cast<uint32_t*>(sm + SM_T + off0) = h0;
+                *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off0) = l0;
+                *reinterpret_cast<uint32_t*>(sm + SM_T + off1) = h1;
+                *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off1) = l1;
             }
             handoff(&bar_ht);                      // T tiles complete: the leader starts V T^T
 
