@@ -529,14 +529,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // o rows of a finished chunk: TMEM -> shared tile [64 tok][128] fp32 in the alpha space
         auto stage_o = [&]() {
             float* ot = reinterpret_cast<float*>(sm + SM_OT);
+            float ov[4][16];                      // all four loads in flight, one wait
 #pragma unroll
-            for (int b16 = 0; b16 < 4; ++b16) {
-                float ov[16];
-                tc::tmem_ld32<16>(te + TM_O + 16 * b16, ov);
-                tc::tmem_ld_wait();
+            for (int b16 = 0; b16 < 4; ++b16) tc::tmem_ld32<16>(te + TM_O + 16 * b16, ov[b16]);
+            tc::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) ot[(16 * b16 + i) * D + me] = ov[i];
-            }
+            for (int b16 = 0; b16 < 4; ++b16)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ot[(16 * b16 + i) * D + me] = ov[b16][i];
         };
 
         // initial state -> accumulator (lane d_v, columns d_k); kappa_prev = 1
@@ -632,11 +632,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // ---------------- E2: -Z^T -> TMEM operand of the U MMA
             efail |= !tc::mbar_wait(&bar_c1, par);
             tc::tc_fence_after();
+            float zz[4][16];
+#pragma unroll
+            for (int b16 = 0; b16 < 4; ++b16) tc::tmem_ld32<16>(te + TM_Z + 16 * b16, zz[b16]);
+            tc::tmem_ld_wait();
 #pragma unroll
             for (int b16 = 0; b16 < 4; ++b16) {
-                float z[16];
-                tc::tmem_ld32<16>(te + TM_Z + 16 * b16, z);
-                tc::tmem_ld_wait();
+                float (&z)[16] = zz[b16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) z[i] = -z[i];
                 uint32_t hi[8], lo[8];
@@ -658,12 +660,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             efail |= !tc::mbar_wait(&bar_u, par);
             tc::tc_fence_after();
             if (leader && ck + 1 < nchunks) issue_loads2(t0 + C);      // V and T consumed
+            float uu[4][16];
+#pragma unroll
+            for (int b16 = 0; b16 < 4; ++b16) tc::tmem_ld32<16>(te + TM_DU + 16 * b16, uu[b16]);
+            tc::tmem_ld_wait();
 #pragma unroll
             for (int b16 = 0; b16 < 4; ++b16) {
-                float u[16], u2[16];
-                tc::tmem_ld32<16>(te + TM_DU + 16 * b16, u);
+                float u2[16];
                 tc::tmem_ld32<16>(te + TM_DU + 64 + 16 * b16, u2);
                 tc::tmem_ld_wait();
+                float (&u)[16] = uu[b16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) u[i] += u2[i];
                 uint32_t hi[8], lo[8];
