@@ -45,6 +45,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-extras", action="store_true")
+    p.add_argument("--cp", action="store_true",
+                   help="with N > 1: also time the long workload split over the ranks by tokens "
+                        "(context parallelism, one all-gather per step)")
     p.add_argument("--batch", type=int, default=WORKLOAD["B"],
                    help="batch size of the layer workload (smaller values for profiling captures)")
     p.add_argument("--only", default="all", choices=["all", "chunk", "decode"],
@@ -359,7 +362,7 @@ def ours_arm(args):
         line["cpu_baseline"] = cpu_baseline(inp)
     if not args.no_extras and args.only == "all":
         line["decode"] = decode_measure(ck, dev, stream, world)
-    if not args.no_extras and world > 1:
+    if args.cp and world > 1:
         line["cp"] = cp_measure(ck, dev, stream, world, rank)
     if rank == 0:
         print(json.dumps(line), flush=True)
