@@ -109,9 +109,12 @@ def cp_chunk_fwd(q, k, v, alpha, beta, S0=None, *, group=None, gate: str = "sign
     """The forward of sequences whose tokens are split over the ranks of `group`.
 
     q, k, alpha [B, T_r, H, dk], v [B, T_r, H, dv], beta [B, T_r, H]: this rank's slice
-    (same B, H, dk, dv on every rank). S0 [B, H, dk, dv] is read on rank 0 only (None =
-    zero). Returns (o [B, T_r, H, dv] of this rank's tokens, the final state [B, H, dk,
-    dv] of the whole sequences, on every rank). All ranks must call it together."""
+    (same B, H, dk, dv and dtypes on every rank; T_r may differ, and may be 0). S0 [B, H,
+    dk, dv] is read on rank 0 only (None = zero). `ops` replaces the three compute steps
+    (default: the CUDA library with `gate` and `normalize_qk`; an `ops` given carries its
+    own). Returns (o [B, T_r, H, dv] of this rank's tokens, the final state [B, H, dk, dv]
+    of the whole sequences, on every rank). All ranks must call it together; the exchange
+    needs d_k to be a multiple of 4 (ckda_cp_prefix)."""
     import torch.distributed as dist
     ops = ops or CudaOps(gate, normalize_qk)
     R = dist.get_world_size(group)
