@@ -173,3 +173,25 @@ def test_one_rank_nccl_group(ck):
         assert torch.equal(o, o2) and torch.equal(ST, ST2)
     finally:
         dist.destroy_process_group()
+
+
+def test_emulated_ranks_log_gate_and_normalisation(ck):
+    """The scheme with the KDA log gate and the fused q/k normalisation (raw, non-unit q, k)."""
+    from delta_rule_attention_ckda_b200 import context_parallel as cp
+    T, d = 600, 128
+    inp = make_inputs(1, T, 2, d, d, torch.bfloat16, seed=31, gate="log15", s0_std=0.1)
+    inp.q = (inp.q.float() * 2.5).to(torch.bfloat16)
+    inp.k = (inp.k.float() * 0.4).to(torch.bfloat16)
+    q, k, v, g, b, s0 = to_dev(inp)
+    ops = cp.CudaOps("log", normalize_qk=True)
+    edges = [0, 200, 450, T]
+    parts = [tuple(_slice(x, edges[r], edges[r + 1]) for x in (q, k, v, g, b)) for r in range(3)]
+    firsts, blocks = zip(*[cp.local_stage(r, *parts[r], s0 if r == 0 else None, ops=ops) for r in range(3)])
+    states = cp.combine(torch.stack(blocks), 1, 2, d, d, ops=ops)
+    o = torch.cat([cp.finish_stage(r, *parts[r], states, firsts[r], ops=ops) for r in range(3)], dim=1)
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    alpha = torch.exp(inp.alpha.double()).numpy()
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, alpha, inp.beta, inp.S0, normalize_qk=True)
+    check("cp log+norm/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check("cp log+norm/S", cp.final_state(states, 1, 2, d, d).double().cpu().numpy(), S_ref, TAU_BF16)
