@@ -1,6 +1,7 @@
 /*
  * ckda.h - C ABI of the CKDA (Complex Kimi Delta Attention) library for NVIDIA B200
- * (sm_100a): chunked forward, decode step and backward pass.
+ * (sm_100a): chunked forward, decode step, backward pass, and the affine maps and
+ * prefix of context parallelism over the sequence.
  *
  * The operation (Complex KDA: Understanding and Enhancing the Expressivity of Kimi
  * Delta Attention, as summarised by the blog post "One update, one quarter-turn",
