@@ -574,8 +574,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             efail |= !tc::mbar_wait(&bar_hk[par], (uint32_t)(ck >> 1) & 1u);   // this chunk's constants
             if (ck > 0) efail |= !tc::mbar_wait(&bar_c2, par ^ 1u);
             tc::tc_fence_after();
-            // the previous chunk's o rows, once the gate (or the exact path) is done with the
-            // alpha space; its store and the next alpha go out before the state copy
             {
                 float sv[2][16];
                 tc::tmem_ld32<16>(te + TM_S, sv[0]);
@@ -609,6 +607,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
                 }
             }
+            // the previous chunk's o rows, once the compute warps are done with the alpha space
+            // (hap); their store and the next alpha go out before C1
             efail |= !tc::mbar_wait(&bar_hap, par);
             if (ck > 0) stage_o();
             epi_publish();
