@@ -50,8 +50,8 @@ def parse():
                         "(context parallelism, one all-gather per step)")
     p.add_argument("--batch", type=int, default=WORKLOAD["B"],
                    help="batch size of the layer workload (smaller values for profiling captures)")
-    p.add_argument("--only", default="all", choices=["all", "chunk", "decode"],
-                   help="run only one of the two kernels (profiling captures)")
+    p.add_argument("--only", default="all", choices=["all", "chunk", "decode", "bwd"],
+                   help="run only the forward legs, the decode leg or the backward leg (profiling captures)")
     return p.parse_args()
 
 
@@ -305,6 +305,12 @@ def ours_arm(args):
         return 0
     inp = make_workload("layer", B=args.batch)
     B, T, H, dk, dv = inp.shape
+    if args.only == "bwd":
+        q, k, v, a, b = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
+        line = {"bwd": bwd_measure(ck, q, k, v, a, b, stream, world, reps=max(1, args.steps))}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
     q, k, v, a, b = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.alpha, inp.beta))
     o = torch.empty(B, T, H, dv, device=dev)
     ST = torch.empty(B, H, dk, dv, device=dev)
@@ -470,10 +476,10 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
     hbm, _ = peaks()
     del ws
     return {"workload": f"layer B={B} T={T} H={H} dk={dk} dv={dv}, backward of <dO, o> (S0 = 0)",
-            "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": 2 * reps,
+            "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": 3 * reps,
             "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg,
-                         "kernels": "bwd_ckpt_kernel + bwd_grad_kernel (fp32 CUDA cores)"}}
+                         "kernels": "bwd_ckpt_kernel + bwd_grad_kernel + bwd_sum_kernel (fp32 CUDA cores)"}}
 
 
 def norm_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, plain_value):
