@@ -195,3 +195,23 @@ def test_emulated_ranks_log_gate_and_normalisation(ck):
     o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, alpha, inp.beta, inp.S0, normalize_qk=True)
     check("cp log+norm/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
     check("cp log+norm/S", cp.final_state(states, 1, 2, d, d).double().cpu().numpy(), S_ref, TAU_BF16)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64)])
+def test_emulated_ranks_unequal_widths(ck, dk, dv):
+    """d_k != d_v on the tensor-core path: maps of d_k x d_k and d_k x d_v, the fold's two
+    chains over different column counts, a ragged last slice."""
+    from delta_rule_attention_ckda_b200 import context_parallel as cp
+    T = 1333
+    inp = make_inputs(1, T, 3, dk, dv, torch.bfloat16, seed=dk + dv, gate="tanh15", s0_std=0.1)
+    q, k, v, a, b, s0 = to_dev(inp)
+    edges = [0, 512, 1000, T]
+    parts = [tuple(_slice(x, edges[r], edges[r + 1]) for x in (q, k, v, a, b)) for r in range(3)]
+    firsts, blocks = zip(*[cp.local_stage(r, *parts[r], s0 if r == 0 else None) for r in range(3)])
+    states = cp.combine(torch.stack(blocks), 1, 3, dk, dv)
+    o = torch.cat([cp.finish_stage(r, *parts[r], states, firsts[r]) for r in range(3)], dim=1)
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check(f"cp {dk}x{dv}/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check(f"cp {dk}x{dv}/S", cp.final_state(states, 1, 3, dk, dv).double().cpu().numpy(), S_ref, TAU_BF16)
