@@ -722,16 +722,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         auto gate_logs = [&](int ckn) -> bool {
             const int nvalid = min(C, tb - (ta + ckn * C));
             wfail |= !tc::mbar_wait(&bar_tma1a, ckn & 1);
+            // this thread's 32 gate values first (every address lies inside the tile; rows past
+            // the end and channels past d_k are replaced by the neutral gate below), then the chain
+            float gv[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) gv[i] = ld_alpha_tile(sm + SM_AL, 32 * hh + i, m);
             float run = 0.f;
             par = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int r = 32 * hh + i;
                 if constexpr (kLogGate) {
-                    const float g = (r < nvalid && m < dk) ? ld_alpha_tile(sm + SM_AL, r, m) : 0.f;
+                    const float g = (r < nvalid && m < dk) ? gv[i] : 0.f;
                     run += fmaxf(g * kLog2e, kLgFloor);
                 } else {
-                    const float a = (r < nvalid && m < dk) ? ld_alpha_tile(sm + SM_AL, r, m) : 1.f;
+                    const float a = (r < nvalid && m < dk) ? gv[i] : 1.f;
                     run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
                     par |= (__float_as_uint(a + 0.f) >> 31) << i;     // -0 + 0 = +0: sign(-0) is +
                 }
@@ -836,6 +841,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 const uint32_t sC = slow ? (pC << 31) : 0u;
                 const float d2 = slow ? LC : 0.f;                       // e2 = 2^(d2 - t)
                 uint32_t yh[4][4], yl[4][4];      // Y = k e2 split, held until the tile is free
+                float kin[32], qin[32];           // this thread's k and q values first
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    kin[i] = ld_bf16_tile(sm + SM_K, 32 * hh + i, m);
+                    qin[i] = want_o ? ld_bf16_tile(sm + SM_Q, 32 * hh + i, m) : 0.f;
+                }
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
                     float xk[8], xq[8], yk[8];
@@ -847,8 +858,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         const float m2 = tc::ex2_approx(d2 - t);
                         const float e1 = __uint_as_float(__float_as_uint(tc::ex2_approx(t)) ^ sg);
                         const float e2 = __uint_as_float(__float_as_uint(m2) ^ sg ^ sC);
-                        float kv = ld_bf16_tile(sm + SM_K, r, m);
-                        float qv = want_o ? ld_bf16_tile(sm + SM_Q, r, m) : 0.f;
+                        float kv = kin[i];
+                        float qv = qin[i];
                         if constexpr (kNormQK) {
                             kv *= sh_kn[r];
                             qv *= sh_qn[r];
