@@ -301,9 +301,9 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 //   factors, X and Y tiles of chunk c          ||  state copy of chunk c (after c-1's state MMA)
 //   [P;A] epilogue and solve of chunk c        ||  o tile of chunk c-1, C1, -Z^T
 //   gate cumulation of chunk c+1               ||  U MMA, U^T, O / state MMA of chunk c
-// The two groups form two chains of about equal length per chunk (compute: factors, [P;A],
-// solve, gate; epilogue: state copy, o tile, C1, -Z^T, U, U^T, state MMA), so a phase only
-// pays off when both chains shorten.
+// The two groups form two chains of nearly equal length per chunk (compute: factors, [P;A],
+// solve, gate; epilogue: state copy, o tile, C1, -Z^T, U, U^T, state MMA), so shortening
+// one pays off only up to the length of the other.
 //
 // kLogGate: the gate input holds g = ln a of a non-negative gate (KDA) instead of a signed
 // a; the cumulation then needs no logarithm and no sign parity.
