@@ -242,3 +242,14 @@ def test_cp_prefix_argument_checks(lib):
     assert lib.ckda_cp_prefix(p, 2, 1, 1, 6, 16, None) == 2           # d_k not a multiple of 4
     assert lib.ckda_cp_prefix(null, 1, 1, 1, 16, 16, None) == 0       # one rank: nothing to chain
     assert lib.ckda_cp_prefix(null, 3, 0, 4, 16, 16, None) == 0       # no sequences
+
+
+def test_python_binding_refuses_cpu_tensors_for_maps_and_prefix():
+    """No CPU path: the map and prefix calls raise on host tensors before any library call."""
+    import torch
+    import delta_rule_attention_ckda_b200 as ck
+    x = torch.zeros(1, 4, 1, 16)
+    with pytest.raises(ValueError):
+        ck.chunk_fwd_maps(x, x, x, x, torch.zeros(1, 4, 1))
+    with pytest.raises(ValueError):
+        ck.cp_prefix(torch.zeros(2, 1 * 1 * 16 * 32), 2, 1, 1, 16, 16)
