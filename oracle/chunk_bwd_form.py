@@ -163,3 +163,55 @@ def bwd_chunked_form(q, k, v, alpha, beta, dO, S0=None, dST=None, C: int = 16) -
                 dS = g["dS0"]
             out["dS0"][bb, h] = dS
     return out
+
+
+def chunk_bwd_factored(q, k, v, a, b, S0, dO, dSC):
+    """``chunk_bwd`` in the form a tensor-core kernel would take, for gates without zeros:
+    every gate ratio as a product of per-token factors e1_r = G_r / g, e2_s = g / G_s (g a
+    per-channel reference, here |G_{C-1}|^(1/2)), so A, P and their gradients are products
+    of C x d tiles; the gate gradient collects, per token and channel, the log-derivative
+    g_r = dL/dG_r * G_r from those products and takes da_j = (sum_{r >= j} g_r) / a_j
+    (a reverse prefix sum, then a division by the gate). Returns the same dict."""
+    C, dk = q.shape
+    G = np.cumprod(a, axis=0)
+    gref = np.sqrt(np.abs(G[C - 1]))
+    e1 = G / gref
+    e2 = gref / G
+    ke1, ke2, qe1 = k * e1, k * e2, q * e1
+    Kt, Qt = G * k, G * q
+    Kh = (G[C - 1] / G) * k
+    A = b[:, None] * np.tril(ke1 @ ke2.T, k=-1)
+    P = np.tril(qe1 @ ke2.T)
+    X = np.linalg.inv(np.eye(C) + A)
+    T = X * b[None, :]
+    W = v - Kt @ S0
+    U = T @ W
+    # products, as in chunk_bwd
+    dS0 = G[C - 1][:, None] * dSC
+    dGC = np.sum(dSC * S0, axis=1)
+    dKh = U @ dSC.T
+    dU = Kh @ dSC
+    dQt = dO @ S0.T
+    dS0 += Qt.T @ dO
+    dP = np.tril(dO @ U.T)
+    dU += P.T @ dO
+    dT = dU @ W.T
+    dW = T.T @ dU
+    dKt = -dW @ S0.T
+    dS0 += -Kt.T @ dW
+    dX = dT * b[None, :]
+    db = np.sum(X * dT, axis=0)
+    dA = np.tril(-X.T @ dX @ X.T, k=-1)
+    dAb = dA * b[:, None]                                  # through the row factor b_r
+    db += np.sum(dA * np.tril(ke1 @ ke2.T, k=-1), axis=1)
+    # tile gradients: A and P are b (.) (k e1)(k e2)^T and (q e1)(k e2)^T, masked
+    d_ke1 = dAb @ ke2
+    d_qe1 = dP @ ke2
+    d_ke2 = dAb.T @ ke1 + dP.T @ qe1
+    dq = d_qe1 * e1 + dQt * G
+    dkk = d_ke1 * e1 + d_ke2 * e2 + dKt * G + dKh * (G[C - 1] / G)
+    # log-derivatives: a tile x e1 grows with G_r, x e2 shrinks with G_s
+    glog = (d_ke1 * ke1 + d_qe1 * qe1 - d_ke2 * ke2 + dKt * Kt + dQt * Qt - dKh * Kh)
+    glog[C - 1] += np.sum(dKh * Kh, axis=0) + dGC * G[C - 1]
+    da = np.cumsum(glog[::-1], axis=0)[::-1] / a
+    return dict(dq=dq, dk=dkk, dv=dW.copy(), da=da, db=db, dS0=dS0)

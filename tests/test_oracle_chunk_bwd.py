@@ -53,3 +53,26 @@ def test_zero_initial_state_and_no_state_cotangent():
     got = bwd_chunked_form(q, k, v, a, b, dO, S0=None, dST=None, C=4)
     want = oracle_bwd(q, k, v, a, b, dO, S0=None, dST=None)
     _close(got, want)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_factored_chunk_backward_equals_the_exact_one(seed):
+    """The factored form (tile products, a reverse prefix sum and a division by the gate)
+    against the exact chunk model, on one chunk with signed gates (none of them zero)."""
+    from oracle.chunk_bwd_form import chunk_bwd, chunk_bwd_factored
+    rng = np.random.default_rng(40 + seed)
+    C, dk, dv = 12, 5, 3
+    q = rng.standard_normal((C, dk))
+    k = rng.standard_normal((C, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((C, dv))
+    a = np.tanh(1.0 + rng.standard_normal((C, dk)))
+    b = 2.0 / (1.0 + np.exp(-rng.standard_normal(C)))
+    S0 = 0.3 * rng.standard_normal((dk, dv))
+    dO = rng.standard_normal((C, dv))
+    dSC = rng.standard_normal((dk, dv))
+    want = chunk_bwd(q, k, v, a, b, S0, dO, dSC)
+    got = chunk_bwd_factored(q, k, v, a, b, S0, dO, dSC)
+    for n in ("dq", "dk", "dv", "da", "db", "dS0"):
+        np.testing.assert_allclose(got[n], want[n], rtol=1e-9, atol=1e-9 * max(1.0, np.abs(want[n]).max()),
+                                   err_msg=n)
