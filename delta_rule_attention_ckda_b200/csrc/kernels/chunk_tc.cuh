@@ -42,7 +42,8 @@
 // product runs on tcgen05 with bf16 operands; operands that are not raw bf16 inputs are split
 // x = hi + lo (hi rounded to nearest, lo the remainder truncated: |x - hi - lo| <=
 // 2^-15 |x|) and each product is the three passes hi*hi + hi*lo + lo*hi, which the
-// fp32-state tolerance needs; raw V stays exact in one bf16 operand. Inputs arrive by
+// fp32-state tolerance needs; raw V stays exact in one bf16 operand. U, whose rounding a
+// chunk of cancelling updates amplifies, carries a third term (four passes in its MMA). Inputs arrive by
 // TMA (no multicast) with 128-byte swizzle; tokens past the end read as zero and get
 // gate 1. A 64-wide d_k or d_v is the 128-wide problem with zero padding. The solve's
 // small block products (16 and 32 wide, inside the 64 x 64 inverse) run on warp-level
@@ -85,7 +86,7 @@ constexpr float kChunkRange = 192.f;  // -L_C bound for the fast path (factors w
 constexpr uint32_t SM_K = 0;            // k tile: 2 TMA boxes [64 tok][64 ch] bf16
 constexpr uint32_t SM_AT = 0;           //   after the gate: A column-major, fp32 [64][64] (at_idx)
 constexpr uint32_t SM_Q = 16384;        // q tile
-constexpr uint32_t SM_T = 16384;        //   after the gate: [T_hi ; T_lo] K-major [128 n][64 s]
+constexpr uint32_t SM_T = 16384;        //   after the gate: [T_hi ; T_mid] K-major [128 n][64 s]
 constexpr uint32_t SM_V = 32768;        // v tile (MN-major A operand of V^T T^T)
 constexpr uint32_t SM_AL = 49152;       // alpha tile: 4 boxes [64 tok][32 ch] fp32
 constexpr uint32_t SM_SLOWL = 49152;    //   slow path only: L fp32 [64][128]
@@ -98,6 +99,8 @@ constexpr uint32_t SM_YLO = 172032;     //   K-major B operand of 192 rows for t
 constexpr uint32_t SM_PLO = 188416;
 constexpr uint32_t SM_XS = 196608;      // (I + A)^{-1}, fp32 row-major [64][XS_LD]; blocks above the
 constexpr int XS_LD = 68;               //   16 x 16 block diagonal stay zero for the whole kernel
+constexpr uint32_t SM_TL = SM_XS;       //   after the solve: T_lo K-major [64 n][64 s] over rows 0..29 of the
+                                        //   solve's X, which the next chunk's solve writes again
 constexpr uint32_t SM_RS = SM_XS + 64 * XS_LD * 4;   // solve temporaries, fp32 [32][RS_LD]
 constexpr int RS_LD = 40;
 constexpr uint32_t SM_SMALL = SM_RS + 32 * RS_LD * 4;
@@ -113,11 +116,13 @@ constexpr uint32_t TM_SAHI = 256;     // (S0 Diag g)^T hi / lo, packed bf16 (A o
 constexpr uint32_t TM_SALO = 320;
 constexpr uint32_t TM_ZAHI = 256;     //   after C1: -Z^T hi / lo, packed bf16 (A operand of the U MMA)
 constexpr uint32_t TM_ZALO = 288;
-constexpr uint32_t TM_UAHI = 320;     //   after the U MMA: U^T hi / lo, packed bf16 (A of C2)
+constexpr uint32_t TM_UAHI = 320;     //   after the U MMA: U^T hi / mid, packed bf16 (A of C2)
 constexpr uint32_t TM_UALO = 352;
 constexpr uint32_t TM_D1 = 384;       // [A ; P] as two partial sums: X_hi Y_hi + X_lo Y_hi | X_hi Y_lo
 constexpr uint32_t TM_DU = 384;       //   after the [A ; P] epilogue: U^T as two partial sums,
                                       //   (V^T - Z^T) T_hi^T | (V^T - Z^T) T_lo^T
+constexpr uint32_t TM_UAL3 = 384;     //   after the sums are read: U^T third term, packed bf16 (the
+                                      //   next [A ; P] waits for the O / state MMA that reads it)
 
 constexpr uint32_t kTmaBytes1a = 4 * 8192;  // alpha (4 fp32 boxes)
 constexpr uint32_t kTmaBytes1b = 2 * 8192;  // k (2 bf16 boxes)
@@ -188,6 +193,19 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     hi = *reinterpret_cast<const uint32_t*>(&h);
     const float la = a - __uint_as_float(hi << 16), lb = b - __uint_as_float(hi & 0xFFFF0000u);
+    lo = __byte_perm(__float_as_uint(la), __float_as_uint(lb), 0x7632);
+}
+
+// (a, b) -> three packed bf16 pairs with hi + mid + lo = x to within 2^-25 |x|: hi and mid
+// rounded to nearest (x - hi and x - hi - mid are exact in fp32), lo the last remainder
+// truncated. For the operand whose rounding a chunk's cancelling updates amplify most (U).
+__device__ __forceinline__ void split3(float a, float b, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    const float ra = a - __uint_as_float(hi << 16), rb = b - __uint_as_float(hi & 0xFFFF0000u);
+    const __nv_bfloat162 md = __floats2bfloat162_rn(ra, rb);
+    mid = *reinterpret_cast<const uint32_t*>(&md);
+    const float la = ra - __uint_as_float(mid << 16), lb = rb - __uint_as_float(mid & 0xFFFF0000u);
     lo = __byte_perm(__float_as_uint(la), __float_as_uint(lb), 0x7632);
 }
 
@@ -325,6 +343,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // hk is double-buffered by chunk parity, so the compute warps may hand over the next
     // chunk's constants before the epilogue group has waited for this chunk's
     __shared__ uint64_t bar_hk[2], bar_hap, bar_ht;
+    // end of the kernel: each MMA-issuing thread (epilogue leader, compute thread 0) commits to
+    // its own barrier and waits, so that no MMA it issued still writes TMEM when TMEM is freed
+    // (on the normal path everything has completed already; after a wait that gave up it has not)
+    __shared__ uint64_t bar_drain[2];
     __shared__ uint32_t tmem_base_s;
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
@@ -391,6 +413,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         tc::mbar_init(&bar_hk[1], NT);
         tc::mbar_init(&bar_hap, NT);
         tc::mbar_init(&bar_ht, NT);
+        tc::mbar_init(&bar_drain[0], 1);
+        tc::mbar_init(&bar_drain[1], 1);
         tc::fence_mbar_init();
         tc::prefetch_tensormap(&map_k);
         tc::prefetch_tensormap(&map_q);
@@ -416,16 +440,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // inputs of a chunk arrive in three groups: alpha (its space frees up once the previous
     // o tile is stored, early in the chunk before), k (its space holds A until the solve's
     // second level), then q and v (read by the U MMA)
+    // loads issued per barrier (epilogue leader only): after a wait that gave up, the leader
+    // waits for the last one of each before the CTA exits (at most one is outstanding per barrier)
+    uint32_t n1a = 0, n1b = 0, n2 = 0;
     auto issue_loads1a = [&](int t0) {
+        ++n1a;
         tc::mbar_arrive_expect_tx(&bar_tma1a, kTmaBytes1a);
         for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma1a, 32 * i, h, t0, b);
     };
     auto issue_loads1b = [&](int t0) {
+        ++n1b;
         tc::mbar_arrive_expect_tx(&bar_tma1b, kTmaBytes1b);
         for (int i = 0; i < 2; ++i) tc::tma_load_4d(sm + SM_K + i * 8192, &map_k, &bar_tma1b, 64 * i, h, t0, b);
     };
     const bool v_zero = (flags & kFlagVZero) != 0;
     auto issue_loads2 = [&](int t0) {
+        ++n2;
         tc::mbar_arrive_expect_tx(&bar_tma2, v_zero ? kTmaBytes2 / 2 : kTmaBytes2);
         for (int i = 0; i < 2; ++i) {
             tc::tma_load_4d(sm + SM_Q + i * 8192, &map_q, &bar_tma2, 64 * i, h, t0, b);
@@ -465,19 +495,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                        tc::sdesc(sb0 + SM_YHI + ks * 2048, SM_YLO - SM_YHI, 1024), i64, 1);
         tc::mma_commit(&bar_ap);
     };
-    // U^T = V^T [T_hi ; T_lo]^T, issued as soon as T is ready (N = 128: both halves at once)
+    // T has three bf16 terms (T_hi + T_mid + T_lo to about 2^-25 |T|): a chunk whose keys repeat
+    // (the quarter-turn example) amplifies T's rounding by the number of cancelling terms in
+    // the state update, so two terms (2^-17) are not enough there. U^T accumulates as two
+    // partial sums, (V^T - Z^T) T_hi^T and (V^T - Z^T) (T_mid + T_lo)^T.
+    // U^T = V^T [T_hi ; T_mid]^T (N = 128: both halves at once) + V^T T_lo^T into the second half,
+    // issued as soon as T is ready
     auto issue_uv = [&](uint32_t sb_) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
         const uint32_t iv = tc::idesc_bf16(128, 128, 1, 0);   // A = V^T (MN-major), B = T (K-major)
+        const uint32_t iv64 = tc::idesc_bf16(128, 64, 1, 0);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             tc::mma_ss(tm0 + TM_DU, tc::sdesc(sb0 + SM_V + ks * 2048, 8192, 1024),
                        tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iv, ks != 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            tc::mma_ss(tm0 + TM_DU + 64, tc::sdesc(sb0 + SM_V + ks * 2048, 8192, 1024),
+                       tc::sdesc(sb0 + SM_TL + ks * 32, 16, 1024), iv64, 1);
     };
-    //   += (-Z^T)_hi [T_hi ; T_lo]^T + (-Z^T)_lo [T_hi ; T_lo]^T once -Z^T is in TMEM
+    //   += (-Z^T)_hi [T_hi ; T_mid]^T + (-Z^T)_hi T_lo^T + (-Z^T)_lo [T_hi ; T_mid]^T once -Z^T is in
+    //   TMEM (the product of the two small terms is below the others' rounding)
     auto issue_uz = [&](uint32_t sb_, bool after_v) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
         const uint32_t iz = tc::idesc_bf16(128, 128, 0, 0);   // A = -Z^T (TMEM)
+        const uint32_t iz64 = tc::idesc_bf16(128, 64, 0, 0);
 #pragma unroll
         for (int ps = 0; ps < 2; ++ps) {
             const uint32_t aa = tm0 + (ps == 1 ? TM_ZALO : TM_ZAHI);
@@ -485,20 +527,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             for (int ks = 0; ks < 4; ++ks)
                 tc::mma_ts(tm0 + TM_DU, aa + ks * 8, tc::sdesc(sb0 + SM_T + ks * 32, 16, 1024), iz,
                            (after_v || ps || ks) ? 1u : 0u);
+            if (ps == 0) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_ts(tm0 + TM_DU + 64, aa + ks * 8, tc::sdesc(sb0 + SM_TL + ks * 32, 16, 1024), iz64, 1);
+            }
         }
         tc::mma_commit(&bar_u);
     };
-    // [acc | O^T] += U^T [(k e2) | P^T]  (3 passes, N = 192: state and output in one MMA)
+    // [acc | O^T] += U^T [(k e2) | P^T]  (N = 192: state and output in one MMA). U^T has
+    // three terms and [Y ; P] two: passes U_hi Y_hi, U_hi Y_lo, U_mid Y_hi, then U_lo Y_hi for
+    // the state only (N = 128). A chunk whose updates cancel (orthogonal steps that return the
+    // state, as in the quarter-turn example) amplifies U's rounding in the state it carries
+    // forward; a chunk's o is not carried forward and does not need the third term.
     auto issue_c2 = [&](uint32_t sb_) {
         const uint32_t sb0 = opaque(sb_), tm0 = opaque(tm);
-        const uint32_t idesc = tc::idesc_bf16(128, 192, 0, 0);
+        const uint32_t idesc = tc::idesc_bf16(128, 192, 0, 0), idesc_s = tc::idesc_bf16(128, 128, 0, 0);
 #pragma unroll
-        for (int ps = 0; ps < 3; ++ps) {
-            const uint32_t aa = tm0 + (ps == 2 ? TM_UALO : TM_UAHI);
+        for (int ps = 0; ps < 4; ++ps) {
+            const uint32_t aa = tm0 + (ps == 3 ? TM_UAL3 : ps == 2 ? TM_UALO : TM_UAHI);
             const uint32_t yb = sb0 + (ps == 1 ? SM_YLO : SM_YHI);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ts(tm0 + TM_S, aa + ks * 8, tc::sdesc(yb + ks * 32, 16, 1024), idesc, 1);
+                tc::mma_ts(tm0 + TM_S, aa + ks * 8, tc::sdesc(yb + ks * 32, 16, 1024), ps == 3 ? idesc_s : idesc, 1);
         }
         tc::mma_commit(&bar_c2);
     };
@@ -672,10 +723,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 float (&u)[16] = uu[b16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) u[i] += u2[i];
-                uint32_t hi[8], lo[8];
-                split_pack16(u, hi, lo);
+                uint32_t hi[8], mid[8], lo[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) split3(u[2 * e], u[2 * e + 1], hi[e], mid[e], lo[e]);
                 tc::tmem_st32<8>(te + TM_UAHI + 8 * b16, hi);
-                tc::tmem_st32<8>(te + TM_UALO + 8 * b16, lo);
+                tc::tmem_st32<8>(te + TM_UALO + 8 * b16, mid);
+                // columns 384 .. 415: the first half of the sums, already read above
+                tc::tmem_st32<8>(te + TM_UAL3 + 8 * b16, lo);
             }
             epi_publish();
             if (esync_or(efail)) break;
@@ -698,7 +752,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
             }
         }
-        if (leader) tc::bulk_wait0();
+        if (leader) {
+            tc::bulk_wait0();
+            tc::mma_commit(&bar_drain[0]);
+            tc::mbar_wait(&bar_drain[0], 0);
+            if (efail) {
+                // loads whose data nobody waited for: let them land before shared memory is released
+                if (n1a) tc::mbar_wait(&bar_tma1a, (n1a - 1) & 1u);
+                if (n1b) tc::mbar_wait(&bar_tma1b, (n1b - 1) & 1u);
+                if (n2) tc::mbar_wait(&bar_tma2, (n2 - 1) & 1u);
+            }
+        }
     } else {
         // ================================================================ compute warpgroups
         setmaxnreg_inc<kRegCompute>();
@@ -1064,21 +1128,35 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 *reinterpret_cast<float2*>(rs + (16 * mt + fg) * RS_LD + 8 * nt + 2 * ft) = make_float2(d[0], d[1]);
                 *reinterpret_cast<float2*>(rs + (16 * mt + fg + 8) * RS_LD + 8 * nt + 2 * ft) = make_float2(d[2], d[3]);
                 // final blocks of T: rows 0..31 x columns 0..31 and rows 32..63 x columns 32..63
-                // (16-byte chunk ch of row tr), and the zero block rows 0..31 x columns 32..63
+                // (16-byte chunk ch of row tr), and the zero block rows 0..31 x columns 32..63. The
+                // 16 x 16 blocks above the diagonal are zero without being read: the previous chunk's
+                // T_lo overwrote some of them. T_lo goes out after the barrier below, once no warp
+                // reads rows 0..31 of the solve's X.
+                uint32_t tl3[4];
+                const int half = warp >> 2, ch = (warp & 3) + 4 * half, tr = lane + 32 * half;
                 {
-                    const int half = warp >> 2, ch = (warp & 3) + 4 * half, tr = lane + 32 * half;
-                    const float4 x0 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch);
-                    const float4 x1 = *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch + 4);
+                    const bool above = (ch >> 1) > (tr >> 4);
+                    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 x0 = above ? zero4 : *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch);
+                    const float4 x1 = above ? zero4 : *reinterpret_cast<const float4*>(xs + tr * XS_LD + 8 * ch + 4);
                     const float4 b0 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[0];
                     const float4 b1 = reinterpret_cast<const float4*>(sh_beta + 8 * ch)[1];
                     const float v[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
                                         x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
-                    store_split8(sm + SM_T, sm + SM_T + 8192, tr, ch, v);
+                    uint32_t th[4], tm_[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) split3(v[2 * e2], v[2 * e2 + 1], th[e2], tm_[e2], tl3[e2]);
+                    const uint32_t off = chunk_off(tr, ch);
+                    *reinterpret_cast<uint4*>(sm + SM_T + off) = make_uint4(th[0], th[1], th[2], th[3]);
+                    *reinterpret_cast<uint4*>(sm + SM_T + 8192 + off) = make_uint4(tm_[0], tm_[1], tm_[2], tm_[3]);
                     const uint32_t zoff = chunk_off(lane, 4 + (warp & 3)) + (uint32_t)half * 8192u;
                     *reinterpret_cast<uint4*>(sm + SM_T + zoff) = make_uint4(0u, 0u, 0u, 0u);
                 }
                 // A (k-tile space) is consumed: the epilogue leader loads the next chunk's k
                 csync();
+                *reinterpret_cast<uint4*>(sm + SM_TL + chunk_off(tr, ch)) = make_uint4(tl3[0], tl3[1], tl3[2], tl3[3]);
+                if (half == 0)
+                    *reinterpret_cast<uint4*>(sm + SM_TL + chunk_off(lane, 4 + (warp & 3))) = make_uint4(0u, 0u, 0u, 0u);
                 float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
@@ -1091,15 +1169,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
                 // T rows 32 + 16 mt + g (+ 8), columns 8 nt + 2 t (+ 1): -X Diag(beta), split
                 const float2 bb = *reinterpret_cast<const float2*>(sh_beta + 8 * nt + 2 * ft);
-                uint32_t h0, l0, h1, l1;
-                split2(-e[0] * bb.x, -e[1] * bb.y, h0, l0);
-                split2(-e[2] * bb.x, -e[3] * bb.y, h1, l1);
+                uint32_t h0, m0, l0, h1, m1, l1;
+                split3(-e[0] * bb.x, -e[1] * bb.y, h0, m0, l0);
+                split3(-e[2] * bb.x, -e[3] * bb.y, h1, m1, l1);
                 const int row0 = 32 + 16 * mt + fg;
                 const uint32_t off0 = chunk_off(row0, nt) + 4u * ft, off1 = chunk_off(row0 + 8, nt) + 4u * ft;
                 *reinterpret_cast<uint32_t*>(sm + SM_T + off0) = h0;
-                *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off0) = l0;
+                *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off0) = m0;
+                *reinterpret_cast<uint32_t*>(sm + SM_TL + off0) = l0;
                 *reinterpret_cast<uint32_t*>(sm + SM_T + off1) = h1;
-                *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off1) = l1;
+                *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off1) = m1;
+                *reinterpret_cast<uint32_t*>(sm + SM_TL + off1) = l1;
             }
             handoff(&bar_ht);                      // T tiles complete: the leader starts V T^T
 
@@ -1129,6 +1209,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     if (c0 + i < dk && m < dv)
                         ST[(size_t)(c0 + i) * dv + m] = x[i] * sh_kref[((nchunks - 1) & 1) * D + c0 + i];
             }
+        }
+        if (tid == 0) {
+            tc::mma_commit(&bar_drain[1]);
+            tc::mbar_wait(&bar_drain[1], 0);
         }
     }
     tc::tc_fence_before();
