@@ -60,6 +60,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_recurrent_fwd_ex.restype = i
     lib.ckda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp] + [i] * 7 + [vp]
     lib.ckda_chunk_fwd_noalloc.restype = i
+    lib.ckda_noalloc_scratch_bytes.argtypes = []
+    lib.ckda_noalloc_scratch_bytes.restype = sz
     lib.ckda_chunk_fwd_maps_workspace_bytes.argtypes = [i] * 6
     lib.ckda_chunk_fwd_maps_workspace_bytes.restype = sz
     lib.ckda_chunk_fwd_maps.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 7 + [vp, sz, vp]
@@ -92,11 +94,15 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _check(t: torch.Tensor, name: str, shape, dtype=None):
+def _check(t: torch.Tensor, name: str, shape, dtype=None, device=None):
+    """Type, device, shape, dtype and contiguity of one tensor argument. `device`: the device
+    every tensor of the call must be on (that of its first tensor)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's tensors are on {device}")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if dtype is not None and t.dtype != dtype:
@@ -105,9 +111,24 @@ def _check(t: torch.Tensor, name: str, shape, dtype=None):
         raise ValueError(f"{name} must be contiguous")
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _device(t: torch.Tensor, name: str = "q") -> torch.device:
+    """The device of a call: that of its first tensor, which must be a CUDA tensor. The
+    library launches on the current device, so every call runs under
+    torch.cuda.device(this device)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    return t.device
+
+
+def _stream(stream, device: torch.device) -> ctypes.c_void_p:
+    """The stream to launch on: the given one, which must belong to `device`, else the
+    current stream of `device`."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the call's tensors are on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -130,21 +151,22 @@ def chunk_segments(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
 
 
 def _fwd_common(q, k, v, alpha, beta, S0, o, S_T):
+    dev = _device(q)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    _check(q, "q", (B, T, H, dk))
-    _check(k, "k", (B, T, H, dk), dt)
-    _check(v, "v", (B, T, H, dv), dt)
-    _check(alpha, "alpha", (B, T, H, dk), torch.float32)
-    _check(beta, "beta", (B, T, H), torch.float32)
+    _check(q, "q", (B, T, H, dk), None, dev)
+    _check(k, "k", (B, T, H, dk), dt, dev)
+    _check(v, "v", (B, T, H, dv), dt, dev)
+    _check(alpha, "alpha", (B, T, H, dk), torch.float32, dev)
+    _check(beta, "beta", (B, T, H), torch.float32, dev)
     if S0 is not None:
-        _check(S0, "S0", (B, H, dk, dv), torch.float32)
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
     if o is None:
-        o = torch.empty(B, T, H, dv, device=q.device, dtype=torch.float32)
-    _check(o, "o", (B, T, H, dv), torch.float32)
+        o = torch.empty(B, T, H, dv, device=dev, dtype=torch.float32)
+    _check(o, "o", (B, T, H, dv), torch.float32, dev)
     if S_T is not None:
-        _check(S_T, "S_T", (B, H, dk, dv), torch.float32)
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
     return B, T, H, dk, dv, _dt(q), o
 
 
@@ -173,21 +195,28 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=Tru
     normalize_qk: q and k are L2-normalised per token and head inside the kernels.
     Allocates o / S_T / workspace with torch when not given (the library never allocates)."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
+    dev = q.device
     if S_T is None and want_state:
-        S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
+        S_T = torch.empty(B, H, dk, dv, device=dev, dtype=torch.float32)
     lib = load()
-    need = int(lib.ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt))
-    if need and workspace is None:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.ckda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o),
-                               _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk), _ptr(workspace),
-                               wbytes, _stream(stream))
+    with torch.cuda.device(dev):
+        need = int(lib.ckda_chunk_fwd_workspace_bytes(B, T, H, dk, dv, dt))
+        if need and workspace is None:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        if workspace is not None:
+            _check(workspace, "workspace", tuple(workspace.shape), None, dev)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib.ckda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(o),
+                                   _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk), _ptr(workspace),
+                                   wbytes, _stream(stream, dev))
     _raise(st, "ckda_chunk_fwd_ex")
     return o, S_T
 
 
-NOALLOC_SCRATCH_BYTES = 20 << 20      # CKDA_NOALLOC_SCRATCH_BYTES
+def noalloc_scratch_bytes() -> int:
+    """Capacity of the fixed device scratch of chunk_fwd_noalloc (CKDA_NOALLOC_SCRATCH_BYTES,
+    read from the library)."""
+    return int(load().ckda_noalloc_scratch_bytes())
 
 
 def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state=True,
@@ -195,14 +224,16 @@ def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_s
                       normalize_qk=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """ckda_chunk_fwd_noalloc: ckda_chunk_fwd_ex on the library's fixed device scratch
     (no workspace argument; the call allocates nothing). Raises CkdaError(WORKSPACE)
-    when the problem needs more than NOALLOC_SCRATCH_BYTES of scratch. o / S_T are
+    when the problem needs more than noalloc_scratch_bytes() of scratch. o / S_T are
     allocated with torch only when not given."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
+    dev = q.device
     if S_T is None and want_state:
-        S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
-    st = load().ckda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
-                                       _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk),
-                                       _stream(stream))
+        S_T = torch.empty(B, H, dk, dv, device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        st = load().ckda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                           _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk),
+                                           _stream(stream, dev))
     _raise(st, "ckda_chunk_fwd_noalloc")
     return o, S_T
 
@@ -215,35 +246,42 @@ def chunk_fwd_maps(q, k, v, alpha, beta, *, M=None, N=None, workspace=None, stre
                    normalize_qk=False) -> Tuple[torch.Tensor, torch.Tensor]:
     """ckda_chunk_fwd_maps: the affine map S_T = M S_0 + N of every (b, h) sequence.
     Returns (M [B,H,dk,dk], N [B,H,dk,dv]), fp32; allocated with torch when not given."""
+    dev = _device(q)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    _check(q, "q", (B, T, H, dk))
-    _check(k, "k", (B, T, H, dk), dt)
-    _check(v, "v", (B, T, H, dv), dt)
-    _check(alpha, "alpha", (B, T, H, dk), torch.float32)
-    _check(beta, "beta", (B, T, H), torch.float32)
-    f32 = dict(device=q.device, dtype=torch.float32)
+    _check(q, "q", (B, T, H, dk), None, dev)
+    _check(k, "k", (B, T, H, dk), dt, dev)
+    _check(v, "v", (B, T, H, dv), dt, dev)
+    _check(alpha, "alpha", (B, T, H, dk), torch.float32, dev)
+    _check(beta, "beta", (B, T, H), torch.float32, dev)
+    f32 = dict(device=dev, dtype=torch.float32)
     M = torch.empty(B, H, dk, dk, **f32) if M is None else M
     N = torch.empty(B, H, dk, dv, **f32) if N is None else N
-    _check(M, "M", (B, H, dk, dk), torch.float32)
-    _check(N, "N", (B, H, dk, dv), torch.float32)
+    _check(M, "M", (B, H, dk, dk), torch.float32, dev)
+    _check(N, "N", (B, H, dk, dv), torch.float32, dev)
     lib = load()
-    need = int(lib.ckda_chunk_fwd_maps_workspace_bytes(B, T, H, dk, dv, _dt(q)))
-    if need and workspace is None:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.ckda_chunk_fwd_maps(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(M), _ptr(N),
-                                 B, T, H, dk, dv, _dt(q), _mode(gate, normalize_qk), _ptr(workspace), wbytes,
-                                 _stream(stream))
+    with torch.cuda.device(dev):
+        need = int(lib.ckda_chunk_fwd_maps_workspace_bytes(B, T, H, dk, dv, _dt(q)))
+        if need and workspace is None:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        if workspace is not None:
+            _check(workspace, "workspace", tuple(workspace.shape), None, dev)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib.ckda_chunk_fwd_maps(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(M), _ptr(N),
+                                     B, T, H, dk, dv, _dt(q), _mode(gate, normalize_qk), _ptr(workspace),
+                                     wbytes, _stream(stream, dev))
     _raise(st, "ckda_chunk_fwd_maps")
     return M, N
 
 
 def cp_prefix(blocks: torch.Tensor, R: int, B: int, H: int, dk: int, dv: int, stream=None) -> torch.Tensor:
     """ckda_cp_prefix, in place on `blocks` ([R, B*H*dk*(dk+dv)] fp32, rank r's M then N)."""
-    _check(blocks, "blocks", (R, B * H * dk * (dk + dv)), torch.float32)
-    _raise(load().ckda_cp_prefix(_ptr(blocks), R, B, H, dk, dv, _stream(stream)), "ckda_cp_prefix")
+    dev = _device(blocks, "blocks")
+    _check(blocks, "blocks", (R, B * H * dk * (dk + dv)), torch.float32, dev)
+    with torch.cuda.device(dev):
+        st = load().ckda_cp_prefix(_ptr(blocks), R, B, H, dk, dv, _stream(stream, dev))
+    _raise(st, "ckda_cp_prefix")
     return blocks
 
 
@@ -257,21 +295,22 @@ def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, 
     Returns a dict with dq, dk, dv, dalpha (dL/dg for gate="log"), dbeta and dS0 (None
     unless want_dS0). Output tensors may be passed in `grads` (same keys); the workspace
     is allocated with torch when not given."""
+    dev = _device(q)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    _check(q, "q", (B, T, H, dk))
-    _check(k, "k", (B, T, H, dk), dt)
-    _check(v, "v", (B, T, H, dv), dt)
-    _check(alpha, "alpha", (B, T, H, dk), torch.float32)
-    _check(beta, "beta", (B, T, H), torch.float32)
-    _check(grad_o, "grad_o", (B, T, H, dv), torch.float32)
+    _check(q, "q", (B, T, H, dk), None, dev)
+    _check(k, "k", (B, T, H, dk), dt, dev)
+    _check(v, "v", (B, T, H, dv), dt, dev)
+    _check(alpha, "alpha", (B, T, H, dk), torch.float32, dev)
+    _check(beta, "beta", (B, T, H), torch.float32, dev)
+    _check(grad_o, "grad_o", (B, T, H, dv), torch.float32, dev)
     if S0 is not None:
-        _check(S0, "S0", (B, H, dk, dv), torch.float32)
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
     if grad_S_T is not None:
-        _check(grad_S_T, "grad_S_T", (B, H, dk, dv), torch.float32)
+        _check(grad_S_T, "grad_S_T", (B, H, dk, dv), torch.float32, dev)
     g = dict(grads or {})
-    f32 = dict(device=q.device, dtype=torch.float32)
+    f32 = dict(device=dev, dtype=torch.float32)
     shapes = {"dq": (B, T, H, dk), "dk": (B, T, H, dk), "dv": (B, T, H, dv), "dalpha": (B, T, H, dk),
               "dbeta": (B, T, H), "dS0": (B, H, dk, dv)}
     for name, shp in shapes.items():
@@ -280,16 +319,19 @@ def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, 
             continue
         if g.get(name) is None:
             g[name] = torch.empty(shp, **f32)
-        _check(g[name], name, shp, torch.float32)
+        _check(g[name], name, shp, torch.float32, dev)
     lib = load()
-    need = int(lib.ckda_bwd_workspace_bytes(B, T, H, dk, dv, _dt(q)))
-    if need and workspace is None:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.ckda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(grad_o),
-                      _ptr(grad_S_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]),
-                      _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q), _mode(gate, normalize_qk),
-                      _ptr(workspace), wbytes, _stream(stream))
+    with torch.cuda.device(dev):
+        need = int(lib.ckda_bwd_workspace_bytes(B, T, H, dk, dv, _dt(q)))
+        if need and workspace is None:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        if workspace is not None:
+            _check(workspace, "workspace", tuple(workspace.shape), None, dev)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib.ckda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(grad_o),
+                          _ptr(grad_S_T), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]),
+                          _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q),
+                          _mode(gate, normalize_qk), _ptr(workspace), wbytes, _stream(stream, dev))
     _raise(st, "ckda_bwd")
     return g
 
@@ -298,11 +340,13 @@ def recurrent_fwd(q, k, v, alpha, beta, S0=None, *, o=None, S_T=None, want_state
                   stream=None, gate="signed", normalize_qk=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """ckda_recurrent_fwd_ex (fp32 SIMT token-by-token kernel). Returns (o, S_T)."""
     B, T, H, dk, dv, dt, o = _fwd_common(q, k, v, alpha, beta, S0, o, S_T)
+    dev = q.device
     if S_T is None and want_state:
-        S_T = torch.empty(B, H, dk, dv, device=q.device, dtype=torch.float32)
-    st = load().ckda_recurrent_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
-                                      _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk),
-                                      _stream(stream))
+        S_T = torch.empty(B, H, dk, dv, device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        st = load().ckda_recurrent_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                          _ptr(o), _ptr(S_T), B, T, H, dk, dv, dt, _mode(gate, normalize_qk),
+                                          _stream(stream, dev))
     _raise(st, "ckda_recurrent_fwd_ex")
     return o, S_T
 
@@ -311,25 +355,32 @@ def decode_step(q, k, v, alpha, beta, S, *, o=None, stream=None, gate="signed",
                 normalize_qk=False) -> torch.Tensor:
     """ckda_decode_step_ex: updates S [N,H,dk,dv] in place, returns o [N,H,dv]. `alpha` is
     the gate in the form `gate` names; normalize_qk L2-normalises q and k in the step."""
+    dev = _device(q)
     N, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    _check(q, "q", (N, H, dk))
-    _check(k, "k", (N, H, dk), dt)
-    _check(v, "v", (N, H, dv), dt)
-    _check(alpha, "alpha", (N, H, dk), torch.float32)
-    _check(beta, "beta", (N, H), torch.float32)
-    _check(S, "S", (N, H, dk, dv), torch.float32)
+    _check(q, "q", (N, H, dk), None, dev)
+    _check(k, "k", (N, H, dk), dt, dev)
+    _check(v, "v", (N, H, dv), dt, dev)
+    _check(alpha, "alpha", (N, H, dk), torch.float32, dev)
+    _check(beta, "beta", (N, H), torch.float32, dev)
+    _check(S, "S", (N, H, dk, dv), torch.float32, dev)
     if o is None:
-        o = torch.empty(N, H, dv, device=q.device, dtype=torch.float32)
-    _check(o, "o", (N, H, dv), torch.float32)
-    st = load().ckda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
-                                    _ptr(o), N, H, dk, dv, _dt(q), _mode(gate, normalize_qk),
-                                    _stream(stream))
+        o = torch.empty(N, H, dv, device=dev, dtype=torch.float32)
+    _check(o, "o", (N, H, dv), torch.float32, dev)
+    with torch.cuda.device(dev):
+        st = load().ckda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                                        _ptr(o), N, H, dk, dv, _dt(q), _mode(gate, normalize_qk),
+                                        _stream(stream, dev))
     _raise(st, "ckda_decode_step_ex")
     return o
 
 
-def get_device_error(stream=None) -> int:
-    """ckda_get_device_error: synchronises the stream; returns the status code."""
-    return int(load().ckda_get_device_error(_stream(stream)))
+def get_device_error(stream=None, device=None) -> int:
+    """ckda_get_device_error on `device` (default: the stream's, else the current device):
+    synchronises the stream; returns the status code."""
+    if device is None:
+        device = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    device = torch.device(device)
+    with torch.cuda.device(device):
+        return int(load().ckda_get_device_error(_stream(stream, device)))

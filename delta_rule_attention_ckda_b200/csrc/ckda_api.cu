@@ -221,6 +221,8 @@ ckda_status_t ckda_chunk_fwd_noalloc(const void* q, const void* k, const void* v
                              stream);
 }
 
+size_t ckda_noalloc_scratch_bytes(void) { return CKDA_NOALLOC_SCRATCH_BYTES; }
+
 ckda_status_t ckda_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
                              const float* beta, const float* S0, float* o, float* S_T, int B,
                              int T, int H, int dk, int dv, ckda_dtype_t dt, void* workspace,

@@ -55,7 +55,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 7
+#define CKDA_ABI_VERSION 8
 
 typedef enum {
     CKDA_OK = 0,
@@ -169,9 +169,15 @@ CKDA_API ckda_status_t ckda_chunk_fwd_ex(const void* q, const void* k, const voi
                                 int mode,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
-/* Capacity of the fixed device scratch ckda_chunk_fwd_noalloc uses: 20 MiB per device
- * (the long-context forward, B=1, T=65536, H=16, d=128, needs exactly this on a 148-SM GPU). */
+/* Capacity of the fixed device scratch ckda_chunk_fwd_noalloc uses: 20 MiB per device.
+ * It is sized for a 148-SM GPU (B200), where the long-context forward (B=1, T=65536, H=16,
+ * d=128) needs exactly this; the segment plan depends on the SM count, so on a GPU with
+ * more SMs the same problem may need more and is then rejected. */
 #define CKDA_NOALLOC_SCRATCH_BYTES ((size_t)20 << 20)
+
+/* CKDA_NOALLOC_SCRATCH_BYTES as compiled into this library (for bindings that cannot read
+ * the macro). */
+CKDA_API size_t ckda_noalloc_scratch_bytes(void);
 
 /*
  * ckda_chunk_fwd_ex without a caller-supplied workspace and without any allocation.

@@ -49,7 +49,7 @@ def test_status_strings(lib):
         s = lib.ckda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.ckda_status_string(99) == b"unknown status"
-    assert lib.ckda_abi_version() == 7
+    assert lib.ckda_abi_version() == 8
 
 
 NULL = None
@@ -253,3 +253,54 @@ def test_python_binding_refuses_cpu_tensors_for_maps_and_prefix():
         ck.chunk_fwd_maps(x, x, x, x, torch.zeros(1, 4, 1))
     with pytest.raises(ValueError):
         ck.cp_prefix(torch.zeros(2, 1 * 1 * 16 * 32), 2, 1, 1, 16, 16)
+
+
+def test_noalloc_capacity_getter(lib):
+    """The fixed scratch capacity is read from the library, not restated in Python."""
+    import delta_rule_attention_ckda_b200 as ck
+    text = open(HEADER).read()
+    assert "#define CKDA_NOALLOC_SCRATCH_BYTES ((size_t)20 << 20)" in text
+    assert lib.ckda_noalloc_scratch_bytes() == 20 << 20
+    assert ck.noalloc_scratch_bytes() == 20 << 20
+
+
+class _FakeCuda(__import__("torch").Tensor):
+    """A host tensor that reports a CUDA device: lets the binding's device checks run on a
+    machine without a GPU (the checks raise before any library call or device access)."""
+    _dev = None
+
+    @property
+    def device(self):
+        return self._dev
+
+
+def _on(t, dev):
+    import torch
+    f = t.as_subclass(_FakeCuda)
+    f._dev = torch.device(dev)
+    return f
+
+
+@pytest.mark.parametrize("entry", ["chunk_fwd", "recurrent_fwd", "chunk_fwd_noalloc", "chunk_fwd_maps",
+                                   "bwd", "decode_step"])
+def test_python_binding_refuses_mixed_devices(entry):
+    """Every tensor of a call must sit on the first tensor's device: the library launches on
+    the current device with that device's stream, so a tensor on another GPU is an error,
+    raised on the host before any launch."""
+    import torch
+    import delta_rule_attention_ckda_b200 as ck
+    if entry == "decode_step":
+        q, k, v, a = (_on(torch.zeros(2, 1, 16), "cuda:0") for _ in range(4))
+        b = _on(torch.zeros(2, 1), "cuda:0")
+        S = _on(torch.zeros(2, 1, 16, 16), "cuda:1")
+        with pytest.raises(ValueError, match="cuda:1"):
+            ck.decode_step(q, k, v, a, b, S)
+        return
+    q, v, a = (_on(torch.zeros(1, 4, 1, 16), "cuda:0") for _ in range(3))
+    k = _on(torch.zeros(1, 4, 1, 16), "cuda:1")
+    b = _on(torch.zeros(1, 4, 1), "cuda:0")
+    args = (q, k, v, a, b)
+    if entry == "bwd":
+        args = args + (_on(torch.zeros(1, 4, 1, 16), "cuda:0"),)
+    with pytest.raises(ValueError, match="cuda:1"):
+        getattr(ck, entry)(*args)
