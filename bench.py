@@ -33,7 +33,13 @@ METRIC = "CKDA fwd tokens/s at H=16,d=128,T=4096; % of tensor-core/HBM roofline"
 WORKLOAD = dict(B=8, T=4096, H=16, dk=128, dv=128)
 BYTES_PER_TOKEN_HEAD = 2 * 128 * 2 + 128 * 2 + 128 * 4 + 4 + 128 * 4   # q,k,v bf16; alpha, beta, o fp32
 FLOPS_PER_TOKEN_HEAD = 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128         # minimal count, chunk 64
+FLOPS_DENSE_TILE_PER_TOKEN_HEAD = 2 * 64 * (3 * 128 + 2 * 128) + 6 * 128 * 128   # 64 x 64 tiles in full
+# Multiply-adds the chunk kernel issues per 64-token chunk (tcgen05, M = 128, K = 16 each):
+#   [P;A]  8 x N=128 + 8 x N=64;  C1  24 x N=128;  U  12 x N=128 + 8 x N=64;
+#   O / state  12 x N=192 + 4 x N=128
+ISSUED_MMA_MACS_PER_CHUNK = 128 * 16 * (8 * 128 + 8 * 64 + 24 * 128 + 12 * 128 + 8 * 64 + 12 * 192 + 4 * 128)
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -67,6 +73,17 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure of MEASURED_PEAKS.json (the layer step is a short
+    kernel timed on its own), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 # device sources that make up each profiled kernel (its code and the primitives it uses)
 KERNEL_SOURCES = {
     "chunk_fwd_chunk_tc_layer": ["kernels/common.cuh", "kernels/chunk_tc.cuh", "kernels/tc_primitives.cuh",
@@ -96,17 +113,24 @@ def kernel_source_hash(kernel_key):
     return h.hexdigest()[:16]
 
 
-def committed_traffic(kernel_key):
+def committed_profile(kernel_key):
+    """The committed ncu figures of a kernel (profiles/dram_traffic.json), or None once the
+    kernel's code no longer hashes to the value recorded with them."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         ent = d.get(kernel_key)
         if ent and ent.get("source_hash") == kernel_source_hash(kernel_key):
-            return float(ent["bytes_per_launch"])
+            return ent
     except Exception:
         pass
     return None
+
+
+def committed_traffic(kernel_key):
+    ent = committed_profile(kernel_key)
+    return None if ent is None else float(ent["bytes_per_launch"])
 
 
 class ClockSampler:
@@ -223,6 +247,18 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(inp, target_s=12.0):
     import oracle
     oracle.build()
@@ -235,10 +271,20 @@ def cpu_baseline(inp, target_s=12.0):
     n_seq = min(B * H, rounds * min(cores, B * H))
     dt = oracle_sample(inp, n_seq)
     tokens = n_seq * T / H            # token-heads / H = tokens with all heads
+    # one thread, two sequences, scaled by count to the whole layer workload
+    oracle.set_threads(1)
+    n1 = 2
+    d1 = oracle_sample(inp, n1)
+    oracle.set_threads(cores)
     return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"{n_seq} of {B * H} (batch, head) sequences x T={T} of the layer workload, "
                       f"fp64 sequential loop, OpenMP over sequences, {dt:.2f} s wall",
-            "seconds": dt}
+            "seconds": dt,
+            "one_thread": {"sequences": n1, "seconds": d1, "layer_seconds_est": d1 / n1 * B * H,
+                           "value": n1 * T / H / d1, "unit": "tokens/s",
+                           "how": f"{n1} sequences x T={T} on one thread, scaled by count to the "
+                                  f"{B * H} sequences of the layer workload"}}
 
 
 # ----------------------------------------------------------------------------- arms
@@ -341,11 +387,22 @@ def ours_arm(args):
     hbm, src = peaks()
     achieved = alg_bytes / per_launch / 1e9
     kernel_key = f"chunk_fwd_{path}_layer"
+    prof = committed_profile(kernel_key)
+    tpeak, tsrc = tensor_peak()
+    nchunks = B * H * ((T + 63) // 64)
+    issued = 2.0 * ISSUED_MMA_MACS_PER_CHUNK * nchunks / per_launch / 1e12
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "traffic": committed_traffic(kernel_key),
+            "frac": achieved / hbm, "traffic": None if prof is None else float(prof["bytes_per_launch"]),
             "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6.65 TB/s",
             "kernel": kernel_key, "alg_bytes_per_launch": alg_bytes,
-            "tflops_minimal": B * T * H * FLOPS_PER_TOKEN_HEAD / per_launch / 1e12}
+            "tflops_minimal": B * T * H * FLOPS_PER_TOKEN_HEAD / per_launch / 1e12,
+            "tflops_dense_tile": B * T * H * FLOPS_DENSE_TILE_PER_TOKEN_HEAD / per_launch / 1e12,
+            "tflops_issued_mma": issued,
+            "issued_mma_frac_of_bf16_peak": issued / tpeak,
+            "bf16_peak_tflops": tpeak, "bf16_peak_source": f"{tsrc} (MEASURED_PEAKS.json bf16_tflops, burst)",
+            "tensor_pipe_pct": None if prof is None else prof.get("tensor_pipe_pct"),
+            "tensor_pipe_pct_source": "committed ncu capture (max over SMs / mean over 148 SMs), "
+                                      "null once the kernel's code changed since"}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_launch,
@@ -629,12 +686,16 @@ def decode_measure(ck, dev, stream, world):
     bytes_call = N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4)
     hbm, src = peaks()
     gbs = bytes_call / per / 1e9
+    traffic = committed_traffic("decode128")
+    roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "alg_bytes_per_launch": bytes_call, "kernel": "decode128", "traffic": traffic}
+    if traffic is not None:
+        # part of the 268 MB state stays in the 126 MB L2 between back-to-back calls, so the
+        # DRAM bytes of a call are below its algorithmic bytes: the fraction on DRAM bytes
+        roof["dram_gbs"] = traffic / per / 1e9
+        roof["dram_frac"] = traffic / per / 1e9 / hbm
     return {"workload": "decode N=256 H=16 d=128 fp32 state, 1024 calls", "us_per_call": per * 1e6,
-            "tokens_per_s": tok_s, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm,
-                                                         "unit": "GB/s", "frac": gbs / hbm,
-                                                         "alg_bytes_per_launch": bytes_call,
-                                                         "kernel": "decode128", "traffic": committed_traffic("decode128")},
-            "gpu_launches": calls}
+            "tokens_per_s": tok_s, "roofline": roof, "gpu_launches": calls}
 
 
 def main():

@@ -333,7 +333,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
                 const __grid_constant__ CUtensorMap map_o, const float* __restrict__ beta,
                 const float* S0_head, const float* S0_seg, float* ST_seg, float* ST_last, float* M_seg,
-                int T, int H, int dk, int dv_in, int seg_len, int nseg, int sg_base, uint32_t flags_in) {
+                int T, int H, int dk, int dv_in, int seg_len, int nseg, int sg_base, uint32_t flags_in,
+                float* S_ck) {
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -399,6 +400,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
               : (sg == nseg - 1) ? (ST_last ? ST_last + (size_t)bh * dk * dv : nullptr)
                                  : (ST_seg ? ST_seg + slot : nullptr);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    // S_ck != NULL: the state entering every chunk is also written, [B*H][ceil(T/64)][d_k][d_v]
+    // fp32 (the checkpoints of the backward pass), by the CTAs that carry the true state:
+    // segment 0 from S0, and every segment of the pass that starts from the entering states
+    const bool store_states = S_ck != nullptr && !trans && (direct || sg_base > 0);
+    float* const Sck_seq = store_states ? S_ck + (size_t)bh * ((T + C - 1) / C) * dk * dv : nullptr;
 
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
     if (tid == 0) {
@@ -656,6 +662,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     tc::tmem_st32<8>(te + TM_SAHI + 8 * cb, hi);
                     tc::tmem_st32<8>(te + TM_SALO + 8 * cb, lo);
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
+                    if (store_states && me < dv) {
+                        // S[c][v] = acc[c][v] kappa_prev[c]; lanes are consecutive v: 128-byte rows
+                        float* dst = Sck_seq + ((size_t)(ta / C + ck) * dk + 16 * cb) * dv + me;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (16 * cb + i < dk) dst[(size_t)i * dv] = cur[i] * sh_kp[par * D + 16 * cb + i];
+                    }
                 }
             }
             // the previous chunk's o rows, once the compute warps are done with the alpha space

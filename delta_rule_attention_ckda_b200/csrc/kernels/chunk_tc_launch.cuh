@@ -241,7 +241,7 @@ inline bool make_chunk_tc_maps(ChunkTcMaps& m, const __nv_bfloat16* q, const __n
 
 using ChunkTcKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, const float*,
                                const float*, const float*, float*, float*, float*, int, int, int, int, int, int, int,
-                               uint32_t);
+                               uint32_t, float*);
 
 // the kernel instance for the gate form and the q/k normalisation, with its shared-memory
 // attribute set on the current device
@@ -253,10 +253,11 @@ inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKerne
     return ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)ctc::SMEM_ALLOC, attr_done[variant]);
 }
 
+// S_ck != NULL: also the state entering every chunk, [B*H][ceil(T/64)][dk][dv] fp32.
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const float* alpha, const float* beta, const float* S0, float* o, float* ST,
                                    int B, int T, int H, int dk, int dv, bool log_gate, bool norm_qk,
-                                   void* workspace, cudaStream_t st) {
+                                   void* workspace, cudaStream_t st, float* S_ck = nullptr) {
     if (!chunk_tc_supported(dk, dv, 1)) return cudaErrorNotSupported;
     ChunkTcMaps mp;
     if (o == nullptr || !make_chunk_tc_maps(mp, q, k, v, alpha, o, B, T, H, dk, dv)) return cudaErrorInvalidValue;
@@ -269,7 +270,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
     if (p.nseg == 1) {
         kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
-                                                                     nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, 0u);
+                                                                     nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, 0u, S_ck);
         return cudaGetLastError();
     }
     if (workspace == nullptr) return cudaErrorInvalidValue;
@@ -280,7 +281,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     // Mx (z = 1)
     kern<<<dim3(nbh, (unsigned)(p.nseg - 1), 2), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
         mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr, Sx + (size_t)dk * dv, nullptr, Mx, T, H, dk, dv, p.seg_len,
-        p.nseg, 0, ctc::kFlagNoO);
+        p.nseg, 0, ctc::kFlagNoO, S_ck);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.nseg > 2) {
@@ -294,7 +295,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     // pass 2: segments 1 .. nseg - 1 from their entering states, with o; the last writes S_T
     kern<<<dim3(nbh, (unsigned)(p.nseg - 1), 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
         mp.k, mp.q, mp.v, mp.a, mp.o, beta, nullptr, Sx, nullptr, ST, nullptr, T, H, dk, dv, p.seg_len, p.nseg, 1,
-        0u);
+        0u, S_ck);
     return cudaGetLastError();
 }
 
@@ -351,7 +352,7 @@ inline cudaError_t launch_chunk_tc_maps(const __nv_bfloat16* q, const __nv_bfloa
         // one segment: N is its final state (ST_last), M its transition product (slot bh)
         kern<<<dim3(nbh, 1, 2), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, nullptr,
                                                                      nullptr, nullptr, Nout, Mout, T, H, dk, dv, T, 1,
-                                                                     0, fl);
+                                                                     0, fl, nullptr);
         return cudaGetLastError();
     }
     if (workspace == nullptr) return cudaErrorInvalidValue;
@@ -361,7 +362,8 @@ inline cudaError_t launch_chunk_tc_maps(const __nv_bfloat16* q, const __nv_bfloa
     float* Nw = static_cast<float*>(workspace);
     float* Mw = Nw + (size_t)nbh * ns1 * dk * dv;
     kern<<<dim3(nbh, (unsigned)p.nseg, 2), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
-        mp.k, mp.q, mp.v, mp.a, mp.o, beta, nullptr, nullptr, Nw, nullptr, Mw, T, H, dk, dv, p.seg_len, ns1, 0, fl);
+        mp.k, mp.q, mp.v, mp.a, mp.o, beta, nullptr, nullptr, Nw, nullptr, Mw, T, H, dk, dv, p.seg_len, ns1, 0, fl,
+        nullptr);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long sdv = (long long)dk * dv, sdk = (long long)dk * dk;
