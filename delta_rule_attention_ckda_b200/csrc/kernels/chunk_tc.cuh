@@ -327,7 +327,9 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 // a; the cumulation then needs no logarithm and no sign parity.
 // kNormQK: q and k are divided by their L2 norms per token (floor 1e-12) on the way in;
 // the scale folds into the per-token factors, so the normalised values are never rounded.
-template <bool kLogGate, bool kNormQK>
+// kStoreStates: S_ck receives the state entering every chunk (the backward's checkpoints);
+// a separate instance, so that the forward carries none of its code.
+template <bool kLogGate, bool kNormQK, bool kStoreStates = false>
 __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
@@ -403,7 +405,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // S_ck != NULL: the state entering every chunk is also written, [B*H][ceil(T/64)][d_k][d_v]
     // fp32 (the checkpoints of the backward pass), by the CTAs that carry the true state:
     // segment 0 from S0, and every segment of the pass that starts from the entering states
-    const bool store_states = S_ck != nullptr && !trans && (direct || sg_base > 0);
+    const bool store_states = kStoreStates && S_ck != nullptr && !trans && (direct || sg_base > 0);
     float* const Sck_seq = store_states ? S_ck + (size_t)bh * ((T + C - 1) / C) * dk * dv : nullptr;
 
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
@@ -662,7 +664,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     tc::tmem_st32<8>(te + TM_SAHI + 8 * cb, hi);
                     tc::tmem_st32<8>(te + TM_SALO + 8 * cb, lo);
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
-                    if (store_states && me < dv) {
+                    if (kStoreStates && store_states && me < dv) {
                         // S[c][v] = acc[c][v] kappa_prev[c]; lanes are consecutive v: 128-byte rows
                         float* dst = Sck_seq + ((size_t)(ta / C + ck) * dk + 16 * cb) * dv + me;
 #pragma unroll

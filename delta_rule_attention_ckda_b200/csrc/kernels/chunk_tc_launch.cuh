@@ -243,13 +243,18 @@ using ChunkTcKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMa
                                const float*, const float*, float*, float*, float*, int, int, int, int, int, int, int,
                                uint32_t, float*);
 
-// the kernel instance for the gate form and the q/k normalisation, with its shared-memory
+// the kernel instance for the gate form and the q/k normalisation (and, for the backward's
+// checkpoints, the one that stores every chunk's entering state), with its shared-memory
 // attribute set on the current device
-inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKernel& kern) {
-    static std::atomic<uint64_t> attr_done[4];
-    kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
-                    : (norm_qk ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
-    const int variant = (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
+inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKernel& kern, bool store_states = false) {
+    static std::atomic<uint64_t> attr_done[8];
+    if (store_states)
+        kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true, true> : chunk_tc_kernel<true, false, true>)
+                        : (norm_qk ? chunk_tc_kernel<false, true, true> : chunk_tc_kernel<false, false, true>);
+    else
+        kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
+                        : (norm_qk ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
+    const int variant = (store_states ? 4 : 0) + (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
     return ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)ctc::SMEM_ALLOC, attr_done[variant]);
 }
 
@@ -263,7 +268,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     if (o == nullptr || !make_chunk_tc_maps(mp, q, k, v, alpha, o, B, T, H, dk, dv)) return cudaErrorInvalidValue;
     ChunkTcKernel kern = nullptr;
     {
-        cudaError_t e = chunk_tc_kernel_for(log_gate, norm_qk, kern);
+        cudaError_t e = chunk_tc_kernel_for(log_gate, norm_qk, kern, S_ck != nullptr);
         if (e != cudaSuccess) return e;
     }
     const unsigned nbh = (unsigned)(B * H);
