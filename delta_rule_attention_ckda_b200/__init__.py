@@ -16,14 +16,14 @@ Entry points (thin ctypes wrappers over libckda.so, see include/ckda.h):
 Tensors are torch CUDA tensors in [B, T, H, d] layout; q/k/v bf16 or fp32, the
 rest fp32. There is no CPU path.
 """
-from ._lib import (BF16, F32, PATH_CHUNK_TC, PATH_RECURRENT, CkdaError,
-                   bwd, bwd_workspace_bytes, chunk_fwd, chunk_fwd_maps, chunk_fwd_noalloc, chunk_path, chunk_segments,
+from ._lib import (BF16, BWD_CHUNK_TC, BWD_RECURRENT, F32, PATH_CHUNK_TC, PATH_RECURRENT, CkdaError,
+                   bwd, bwd_path, bwd_workspace_bytes, chunk_fwd, chunk_fwd_maps, chunk_fwd_noalloc, chunk_path, chunk_segments,
                    cp_prefix, decode_step, get_device_error, load, maps_workspace_bytes, noalloc_scratch_bytes,
                    recurrent_fwd,
                    workspace_bytes, LIB_PATH)
 from . import context_parallel
 
-__all__ = ["bwd", "bwd_workspace_bytes", "chunk_fwd", "chunk_fwd_maps", "maps_workspace_bytes", "cp_prefix",
+__all__ = ["bwd", "bwd_path", "BWD_CHUNK_TC", "BWD_RECURRENT", "bwd_workspace_bytes", "chunk_fwd", "chunk_fwd_maps", "maps_workspace_bytes", "cp_prefix",
            "context_parallel", "chunk_fwd_noalloc", "noalloc_scratch_bytes", "recurrent_fwd", "decode_step",
            "workspace_bytes", "chunk_path", "chunk_segments", "get_device_error", "load", "CkdaError", "LIB_PATH", "F32", "BF16",
            "PATH_RECURRENT", "PATH_CHUNK_TC"]

@@ -70,6 +70,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ckda_cp_prefix.restype = i
     lib.ckda_bwd_workspace_bytes.argtypes = [i] * 6
     lib.ckda_bwd_workspace_bytes.restype = sz
+    lib.ckda_bwd_workspace_bytes_ex.argtypes = [i] * 7
+    lib.ckda_bwd_workspace_bytes_ex.restype = sz
+    lib.ckda_bwd_path.argtypes = [i] * 7
+    lib.ckda_bwd_path.restype = i
     lib.ckda_bwd.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp, fp] + [i] * 7 + [vp, sz, vp]
     lib.ckda_bwd.restype = i
     lib.ckda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp] + [i] * 5 + [vp]
@@ -285,8 +289,17 @@ def cp_prefix(blocks: torch.Tensor, R: int, B: int, H: int, dk: int, dv: int, st
     return blocks
 
 
-def bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
-    return int(load().ckda_bwd_workspace_bytes(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype))))
+BWD_RECURRENT, BWD_CHUNK_TC = 0, 1
+
+
+def bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, gate="signed", normalize_qk=False) -> int:
+    return int(load().ckda_bwd_workspace_bytes_ex(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype)),
+                                                  _mode(gate, normalize_qk)))
+
+
+def bwd_path(B, T, H, dk, dv, dtype=torch.bfloat16, gate="signed", normalize_qk=False) -> int:
+    """ckda_bwd_path: BWD_CHUNK_TC (tensor cores) or BWD_RECURRENT (CUDA cores, fp32)."""
+    return int(load().ckda_bwd_path(B, T, H, dk, dv, _dt(torch.empty(0, dtype=dtype)), _mode(gate, normalize_qk)))
 
 
 def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, grads=None,
@@ -322,7 +335,7 @@ def bwd(q, k, v, alpha, beta, grad_o, S0=None, grad_S_T=None, *, want_dS0=True, 
         _check(g[name], name, shp, torch.float32, dev)
     lib = load()
     with torch.cuda.device(dev):
-        need = int(lib.ckda_bwd_workspace_bytes(B, T, H, dk, dv, _dt(q)))
+        need = int(lib.ckda_bwd_workspace_bytes_ex(B, T, H, dk, dv, _dt(q), _mode(gate, normalize_qk)))
         if need and workspace is None:
             workspace = torch.empty(need, device=dev, dtype=torch.uint8)
         if workspace is not None:

@@ -15,6 +15,7 @@
 #include "kernels/decode.cuh"
 #include "kernels/chunk_tc_launch.cuh"
 #include "kernels/bwd.cuh"
+#include "kernels/bwd_tc_launch.cuh"
 
 namespace {
 
@@ -95,6 +96,11 @@ void* noalloc_scratch() {
         addr[dev] = p;
     }
     return addr[dev];
+}
+
+size_t ckda_bwd_workspace_bytes_recurrent_impl(int B, int T, int H, int dk, int dv);
+inline size_t ckda_bwd_workspace_bytes_recurrent(int B, int T, int H, int dk, int dv) {
+    return ckda_bwd_workspace_bytes_recurrent_impl(B, T, H, dk, dv);
 }
 
 // mode = a ckda_gate_t value, optionally OR-ed with CKDA_OPT_* bits
@@ -294,8 +300,29 @@ ckda_status_t ckda_cp_prefix(float* blocks, int R, int B, int H, int dk, int dv,
     return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
+ckda_bwd_path_t ckda_bwd_path(int B, int T, int H, int dk, int dv, ckda_dtype_t dt, int mode) {
+    (void)B; (void)T; (void)H;
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq) || !dims_ok(dk, dv)) return CKDA_BWD_RECURRENT;
+    return ckda::bwd_tc_supported(dk, dv, dt, nq) ? CKDA_BWD_CHUNK_TC : CKDA_BWD_RECURRENT;
+}
+
+size_t ckda_bwd_workspace_bytes_ex(int B, int T, int H, int dk, int dv, ckda_dtype_t dt, int mode) {
+    if (B <= 0 || T <= 0 || H <= 0 || !dims_ok(dk, dv)) return 0;
+    bool lg = false, nq = false;
+    if (!parse_mode(mode, &lg, &nq)) return 0;
+    if (ckda_bwd_path(B, T, H, dk, dv, dt, mode) == CKDA_BWD_CHUNK_TC) return ckda::bwd_tc_layout(B, T, H, dk, dv).total;
+    return ckda_bwd_workspace_bytes_recurrent(B, T, H, dk, dv);
+}
+
 size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt) {
-    (void)dt;
+    return ckda_bwd_workspace_bytes_ex(B, T, H, dk, dv, dt, CKDA_GATE_SIGNED);
+}
+
+}  // extern "C"
+
+namespace {
+size_t ckda_bwd_workspace_bytes_recurrent_impl(int B, int T, int H, int dk, int dv) {
     if (B <= 0 || T <= 0 || H <= 0 || !dims_ok(dk, dv)) return 0;
     const size_t bh = (size_t)B * H, nblk = ((size_t)T + ckda::bwd::KB - 1) / ckda::bwd::KB;
     const size_t nsl = (size_t)ckda::bwd::slabs(dv), nrow = bh * (size_t)T;
@@ -304,6 +331,9 @@ size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_
             + nsl * nrow * 3 * dk + nsl * nrow)               // per-slab partial row sums
            * sizeof(float);
 }
+}  // namespace
+
+extern "C" {
 
 ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float* gate, const float* beta,
                        const float* S0, const float* grad_o, const float* grad_S_T, float* grad_q,
@@ -323,11 +353,18 @@ ckda_status_t ckda_bwd(const void* q, const void* k, const void* v, const float*
                           grad_beta, grad_S0, workspace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return CKDA_ERR_MISALIGNED;
-    const size_t need = ckda_bwd_workspace_bytes(B, T, H, dk, dv, dt);
+    const size_t need = ckda_bwd_workspace_bytes_ex(B, T, H, dk, dv, dt, mode);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CKDA_ERR_WORKSPACE;
     cudaStream_t st = as_stream(stream);
     if ((long long)B * H == 0) return CKDA_OK;
     if (T == 0) return copy_state(grad_S_T, grad_S0, (size_t)B * H * dk * dv, st);
+    if (ckda_bwd_path(B, T, H, dk, dv, dt, mode) == CKDA_BWD_CHUNK_TC) {
+        cudaError_t e = ckda::launch_bwd_tc(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                            static_cast<const __nv_bfloat16*>(v), gate, beta, S0, grad_o, grad_S_T,
+                                            grad_q, grad_k, grad_v, grad_gate, grad_beta, grad_S0, B, T, H, dk, dv, lg,
+                                            workspace, st);
+        return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+    }
     const size_t bh = (size_t)B * H, nrow = bh * (size_t)T;
     const size_t nblk = ((size_t)T + ckda::bwd::KB - 1) / ckda::bwd::KB;
     const int nsl = ckda::bwd::slabs(dv);

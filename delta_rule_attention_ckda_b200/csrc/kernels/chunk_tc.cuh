@@ -389,7 +389,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const int sg = sg_base + (int)blockIdx.y;
     const bool direct = sg == 0 && (flags_in & kFlagMapsOnly) == 0;   // segment 0 from the known S0
     if (trans && direct) return;
-    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident) : (direct ? 0u : flags_in);
+    // the checkpoint instance may run the direct segment without o (the backward needs states only)
+    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident)
+                                 : (direct ? (kStoreStates ? (flags_in & kFlagNoO) : 0u) : flags_in);
     const int dv = trans ? dk : dv_in;
     const int b = bh / H, h = bh % H;
     const int ta = sg * seg_len;

@@ -258,14 +258,18 @@ inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKerne
     return ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)ctc::SMEM_ALLOC, attr_done[variant]);
 }
 
-// S_ck != NULL: also the state entering every chunk, [B*H][ceil(T/64)][dk][dv] fp32.
+// S_ck != NULL: also the state entering every chunk, [B*H][ceil(T/64)][dk][dv] fp32; with it,
+// no_o runs every segment without o (o may then be NULL).
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const float* alpha, const float* beta, const float* S0, float* o, float* ST,
                                    int B, int T, int H, int dk, int dv, bool log_gate, bool norm_qk,
-                                   void* workspace, cudaStream_t st, float* S_ck = nullptr) {
+                                   void* workspace, cudaStream_t st, float* S_ck = nullptr, bool no_o = false) {
     if (!chunk_tc_supported(dk, dv, 1)) return cudaErrorNotSupported;
+    if (no_o && S_ck == nullptr) return cudaErrorInvalidValue;
+    const uint32_t extra = no_o ? ctc::kFlagNoO : 0u;
     ChunkTcMaps mp;
-    if (o == nullptr || !make_chunk_tc_maps(mp, q, k, v, alpha, o, B, T, H, dk, dv)) return cudaErrorInvalidValue;
+    if ((o == nullptr && !no_o) || !make_chunk_tc_maps(mp, q, k, v, alpha, no_o ? nullptr : o, B, T, H, dk, dv))
+        return cudaErrorInvalidValue;
     ChunkTcKernel kern = nullptr;
     {
         cudaError_t e = chunk_tc_kernel_for(log_gate, norm_qk, kern, S_ck != nullptr);
@@ -275,7 +279,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
     if (p.nseg == 1) {
         kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
-                                                                     nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, 0u, S_ck);
+                                                                     nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, extra, S_ck);
         return cudaGetLastError();
     }
     if (workspace == nullptr) return cudaErrorInvalidValue;
@@ -300,7 +304,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     // pass 2: segments 1 .. nseg - 1 from their entering states, with o; the last writes S_T
     kern<<<dim3(nbh, (unsigned)(p.nseg - 1), 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(
         mp.k, mp.q, mp.v, mp.a, mp.o, beta, nullptr, Sx, nullptr, ST, nullptr, T, H, dk, dv, p.seg_len, p.nseg, 1,
-        0u, S_ck);
+        extra, S_ck);
     return cudaGetLastError();
 }
 

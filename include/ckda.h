@@ -55,7 +55,7 @@ extern "C" {
 #endif
 
 #define CKDA_MAX_D 128
-#define CKDA_ABI_VERSION 8
+#define CKDA_ABI_VERSION 9
 
 typedef enum {
     CKDA_OK = 0,
@@ -280,12 +280,30 @@ CKDA_API ckda_status_t ckda_decode_step(const void* q, const void* k, const void
                                float* S, float* o,
                                int N, int H, int dk, int dv, ckda_dtype_t dt, void* stream);
 
+/* Which kernels ckda_bwd runs for a problem. */
+typedef enum {
+    CKDA_BWD_RECURRENT = 0,     /* token by token on CUDA cores, fp32 (any d <= 128, fp32 or bf16)  */
+    CKDA_BWD_CHUNK_TC = 1       /* chunked on tcgen05 tensor cores (bf16, d_k and d_v in {64, 128},
+                                   no CKDA_OPT_NORMALIZE_QK)                                          */
+} ckda_bwd_path_t;
+
+/* The kernels ckda_bwd runs for these sizes, dtype and mode (for tests and reporting). */
+CKDA_API ckda_bwd_path_t ckda_bwd_path(int B, int T, int H, int dk, int dv, ckda_dtype_t dt, int mode);
+
 /*
- * Bytes of device workspace ckda_bwd needs (0 for empty problems), all fp32: the
- * forward state at every 8th token (B*H*ceil(T/8)*dk*dv), recomputed states (128 KiB
- * per (b, h) and 32-column slab of the state) and per-slab partial sums of the row
- * gradients (slabs*B*T*H*(3*dk + 1)), where slabs = ceil(dv / 32).
+ * Bytes of device workspace ckda_bwd needs for the mode it is called with (0 for empty
+ * problems or an invalid mode), all fp32.
+ * CKDA_BWD_CHUNK_TC: the state entering every 64-token chunk and the cotangent of the state
+ *   leaving it (2 * B*H*ceil(T/64)*dk*dv), the chunks' dWx = (I + A)^{-T} dU
+ *   (B*H*ceil(T/64)*64*dv), plus the forward's segment workspace when few sequences split
+ *   (ckda_chunk_fwd_workspace_bytes), each part 256-byte aligned.
+ * CKDA_BWD_RECURRENT: the forward state at every 8th token (B*H*ceil(T/8)*dk*dv), recomputed
+ *   states (128 KiB per (b, h) and 32-column slab of the state) and per-slab partial sums of
+ *   the row gradients (slabs*B*T*H*(3*dk + 1)), where slabs = ceil(dv / 32).
  */
+CKDA_API size_t ckda_bwd_workspace_bytes_ex(int B, int T, int H, int dk, int dv, ckda_dtype_t dt, int mode);
+
+/* ckda_bwd_workspace_bytes_ex for mode CKDA_GATE_SIGNED. */
 CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ckda_dtype_t dt);
 
 /*
@@ -294,8 +312,13 @@ CKDA_API size_t ckda_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, ck
  * (the vector-Jacobian product with cotangents grad_o and grad_S_T). The pages measure
  * the forward and backward passes together and mention a sign-aware backward kernel
  * (ai.info summary of the Complex KDA paper, "Main Findings"); they print no backward
- * formulas, so this is the derivative of the recurrence itself, taken token by token
- * in reverse on CUDA cores in fp32 from states recomputed out of checkpoints.
+ * formulas, so this is the derivative of the recurrence itself. Two implementations
+ * (ckda_bwd_path): for bf16 q/k/v with d_k, d_v in {64, 128} and no q/k normalisation, the
+ * chunked form on tensor cores (a forward pass that keeps every chunk's entering state, the
+ * state cotangent chunk by chunk in reverse, then every chunk's gradients side by side; the
+ * products split into bf16 terms as in the forward, so its error is of the bf16 forward's
+ * order, not of fp32); otherwise token by token in reverse on CUDA cores in fp32 from states
+ * recomputed out of checkpoints.
  *   q, k, v, gate, beta, S0, B..dv, dt, mode: as for ckda_chunk_fwd_ex (S0 may
  *              be NULL: zero initial state; any dk, dv <= 128; fp32 or bf16 q, k, v)
  *   grad_o     [B,T,H,dv] fp32 cotangent of o (required when B*T*H > 0)

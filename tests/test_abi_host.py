@@ -49,7 +49,7 @@ def test_status_strings(lib):
         s = lib.ckda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.ckda_status_string(99) == b"unknown status"
-    assert lib.ckda_abi_version() == 8
+    assert lib.ckda_abi_version() == 9
 
 
 NULL = None

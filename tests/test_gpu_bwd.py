@@ -1,11 +1,13 @@
 """Parity of the backward pass (ckda_bwd) against the fp64 gradient oracle.
 
 Every gradient (q, k, v, gate, beta, S0) is compared element by element with the
-oracle's on the same inputs: max-abs error <= tau * RMS(oracle gradient), tau = 1e-4
-(the path computes in fp32 whatever the input dtype; bf16 inputs are converted
-exactly, so the same bound applies). Cases cover ragged checkpoint blocks, odd and
-unequal head sizes, a zero or given initial state and final-state cotangent, the log
-gate, fast-decaying and zero gates, and sampled sequences of the full-size layer.
+oracle's on the same inputs: max-abs error <= tau * RMS(oracle gradient). tau = 1e-4 on
+the CUDA-core path (fp32 arithmetic whatever the input dtype; bf16 inputs are converted
+exactly), 3e-3 on the tensor-core path that bf16 shapes with d in {64, 128} take (its
+products split operands into bf16 terms, as the forward's do, so it is held to the
+bf16 forward's bound). Cases cover ragged chunks and checkpoint blocks, odd and unequal
+head sizes, a zero or given initial state and final-state cotangent, the log gate,
+fast-decaying and zero gates, and sampled sequences of the full-size layer.
 """
 import numpy as np
 import pytest
@@ -17,6 +19,7 @@ from parity_util import check, to_dev
 
 pytestmark = pytest.mark.gpu
 TAU = 1e-4
+TAU_TC = 3e-3
 NAMES = [("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dalpha", "dalpha"), ("dbeta", "dbeta"), ("dS0", "dS0")]
 
 
@@ -48,6 +51,12 @@ def _run(ck, inp, dO, dST, gate="signed", alpha=None):
     return {n: (None if x is None else x.double().cpu().numpy()) for n, x in g.items()}
 
 
+def _tau(ck, inp, gate="signed"):
+    B, T, H, dk, dv = inp.shape
+    tc_path = ck.bwd_path(B, T, H, dk, dv, inp.q.dtype, gate=gate) == ck.BWD_CHUNK_TC
+    return TAU_TC if tc_path else TAU
+
+
 def _compare(tag, got, want, tau=TAU):
     for gn, on in NAMES:
         check(f"{tag}/{gn}", got[gn], want[on], tau)
@@ -62,7 +71,7 @@ def test_bwd_matches_oracle(ck, shape, dtype):
     dO, dST = _cotangents(B, T, H, dk, dv, seed=T)
     got = _run(ck, inp, dO, dST)
     want = oracle_bwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, dO, S0=inp.S0, dST=dST)
-    _compare(f"bwd {shape} {dtype}", got, want)
+    _compare(f"bwd {shape} {dtype}", got, want, _tau(ck, inp))
 
 
 def test_bwd_zero_state_no_final_cotangent(ck):
@@ -70,7 +79,7 @@ def test_bwd_zero_state_no_final_cotangent(ck):
     dO, _ = _cotangents(2, 70, 2, 32, 48, seed=4, with_dst=False)
     got = _run(ck, inp, dO, None)
     want = oracle_bwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, dO, S0=None, dST=None)
-    _compare("bwd S0=0", got, want)
+    _compare("bwd S0=0", got, want, _tau(ck, inp))
 
 
 def test_bwd_log_gate(ck):
@@ -83,7 +92,7 @@ def test_bwd_log_gate(ck):
     a = torch.exp(g.double())
     want = oracle_bwd(inp.q, inp.k, inp.v, a, inp.beta, dO, S0=inp.S0, dST=dST)
     want["dalpha"] = want["dalpha"] * a.numpy()
-    _compare("bwd loggate", got, want)
+    _compare("bwd loggate", got, want, _tau(ck, inp, gate="log"))
 
 
 def test_bwd_extreme_gates(ck):
@@ -98,7 +107,7 @@ def test_bwd_extreme_gates(ck):
     want = oracle_bwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, dO, S0=inp.S0, dST=dST)
     for v in got.values():
         assert v is None or np.isfinite(v).all()
-    _compare("bwd extreme", got, want)
+    _compare("bwd extreme", got, want, _tau(ck, inp))
 
 
 def test_bwd_layer_workload_sampled(ck):
@@ -113,4 +122,4 @@ def test_bwd_layer_workload_sampled(ck):
         want = oracle_bwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.alpha), sl(inp.beta), sl(dO))
         sub = {n: got[n][bb:bb + 1, :, hh:hh + 1] for n in ("dq", "dk", "dv", "dalpha", "dbeta")}
         sub["dS0"] = got["dS0"][bb:bb + 1, hh:hh + 1]
-        _compare(f"bwd layer ({bb},{hh})", sub, want)
+        _compare(f"bwd layer ({bb},{hh})", sub, want, _tau(ck, inp))
