@@ -505,7 +505,9 @@ def cp_measure(ck, dev, stream, world, rank, reps=3):
 def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
     """The backward pass (ckda_bwd) of the same layer step: gradients of <dO, o> for q,
     k, v, alpha, beta and S0, from a fixed synthetic cotangent dO. Tokens/s and the
-    algorithmic HBM bytes (inputs and cotangent read once, gradients written once)."""
+    algorithmic HBM bytes (inputs and cotangent read once, gradients written once). Then
+    forward + backward for the signed gate and for KDA's form of it (g = ln|alpha| through
+    the log-gate mode), the pair the pages compare."""
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -515,6 +517,7 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
         ("dq", (B, T, H, dk)), ("dk", (B, T, H, dk)), ("dv", (B, T, H, dv)), ("dalpha", (B, T, H, dk)),
         ("dbeta", (B, T, H)), ("dS0", (B, H, dk, dv)))}
     ws = torch.empty(ck.bwd_workspace_bytes(B, T, H, dk, dv), device=q.device, dtype=torch.uint8)
+    tc = ck.bwd_path(B, T, H, dk, dv, q.dtype) == ck.BWD_CHUNK_TC
 
     def step():
         ck.bwd(q, k, v, a, b, dO, None, None, grads=grads, workspace=ws)
@@ -531,12 +534,38 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
     out_bytes = 3 * dk * 4 + dv * 4 + 4                             # dq, dk, dalpha, dv, dbeta
     alg = B * T * H * (in_bytes + out_bytes) + B * H * dk * dv * 4   # + dS0
     hbm, _ = peaks()
+    kernels = ("chunk_tc_kernel (forward, chunk checkpoints) + chunk_bwd_chain_kernel + chunk_bwd_grad_kernel "
+               "(tcgen05)" if tc else "bwd_ckpt_kernel + bwd_grad_kernel + bwd_sum_kernel (fp32 CUDA cores)")
+    out = {"workload": f"layer B={B} T={T} H={H} dk={dk} dv={dv}, backward of <dO, o> (S0 = 0)",
+           "path": "chunk_tc" if tc else "recurrent",
+           "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": 3 * reps,
+           "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
+                        "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg, "kernels": kernels}}
+
+    # forward + backward, signed gate against KDA's non-negative log gate
+    o = torch.empty(B, T, H, dv, device=q.device)
+    ST = torch.empty(B, H, dk, dv, device=q.device)
+    glog = torch.log(a.abs())
+    fb = {}
+    for name, gate, gin in (("ckda", "signed", a), ("kda", "log", glog)):
+        def fwd_bwd(gate=gate, gin=gin):
+            ck.chunk_fwd(q, k, v, gin, b, None, o=o, S_T=ST, gate=gate)
+            ck.bwd(q, k, v, gin, b, dO, None, None, grads=grads, workspace=ws, gate=gate)
+
+        fwd_bwd()
+        torch.cuda.synchronize()
+        assert ck.get_device_error() == 0
+        barrier(world)
+        s = time_launches(fwd_bwd, reps, stream)
+        assert ck.get_device_error() == 0
+        _, s = aggregate_throughput(B * T * reps, s, world, device="cuda")
+        fb[name] = 1e3 * s / reps
+    out["fwd_bwd"] = {"workload": "layer: forward (o, S_T) then backward, per step",
+                      "ckda_ms": fb["ckda"], "kda_ms": fb["kda"],
+                      "kda_gate": "g = ln|alpha| (non-negative gate) through the log-gate mode",
+                      "ckda_over_kda_throughput": fb["kda"] / fb["ckda"], "gpu_launches": 4 * reps}
     del ws
-    return {"workload": f"layer B={B} T={T} H={H} dk={dk} dv={dv}, backward of <dO, o> (S0 = 0)",
-            "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": 3 * reps,
-            "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
-                         "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg,
-                         "kernels": "bwd_ckpt_kernel + bwd_grad_kernel + bwd_sum_kernel (fp32 CUDA cores)"}}
+    return out
 
 
 def norm_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, plain_value):
