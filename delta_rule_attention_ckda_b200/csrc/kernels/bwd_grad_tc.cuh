@@ -9,10 +9,9 @@
 //   d(q e1) = dP (k e2),  d(k e1) = Diag(b) dA (k e2),  d(k e2) = dP^T (q e1) + (Diag(b) dA)^T (k e1)
 //   dQt = dO S0^T,  dKt = -Diag(b) dWx S0^T,  dKh = U dS_C^T
 //   dq = d(q e1) e1 + dQt G,   dk = d(k e1) e1 + d(k e2) e2 + dKt G + dKh (Gamma_C / G)
-//   log-derivative of the gate products, per token and channel:
-//   gl = d(k e1) k e1 + d(q e1) q e1 - d(k e2) k e2 + dKt k G + dQt q G - dKh k Gamma_C / G,
-//   the last token also gets sum_r dKh k Gamma_C / G + <dS_C, S0>_row Gamma_C, and
-//   d alpha_j = (sum_{r >= j} gl_r) / alpha_j  (for the log gate, dg_j = sum_{r >= j} gl_r)
+//   the gate: d alpha_j alpha_j is the sum of the terms whose gate product contains alpha_j,
+//   the pairs s < j <= r of the P / A ratios, sum_{r >= j} of the dKt, dQt terms, sum_{s < j} of
+//   the dKh terms and <dS_C, S0> Gamma_C (for the log gate that sum is dg_j itself)
 //   d beta = rowsum(W (.) dWx) + rowsum(dA (.) L),   L = tril((k e1)(k e2)^T, -1)
 // (the pages print no backward: this is the derivative of the forward as written).
 //
@@ -23,10 +22,11 @@
 //   G8   [dP ; dA]^T-less: D[r'][s]   = [dO ; dWx] U^T         (K = d_v, two halves)
 //   G11  D[c][r'] = S0 [dO ; dWx]^T    (dQt^T | (dWx S0^T)^T)
 //   G12  D[c][s]  = dS_C U^T           (dKh^T)
-//   G9   D[c][r'] = (k e2)^T [dP ; b dA]^T   (d(q e1)^T | d(k e1)^T)
-//   G10  D[c][s]  = [q e1 ; k e1]^T [dP ; b dA]   (d(k e2)^T)
-// so the last pass has every term of a (channel, token) pair on one thread, which also runs
-// the reverse prefix sum of the gate gradient over its tokens.
+//   Facc, Q1, Q2  D[c][r'] = (k e2)^T [dP ; b dA]^T over the tokens of earlier 16-token blocks
+//   CP, G10       D[c][s]  = [q e1 ; k e1]^T [dP ; b dA] over the rows of later blocks, or all rows
+// so the last pass has every term of a (channel, token) pair on one thread: d(q e1), d(k e1)
+// are Facc plus the token's own block (CUDA cores), and the gate's pair sums across each cut
+// are the block products plus the pairs inside a block (CUDA cores, 120 per block and channel).
 #pragma once
 #include "chunk_tc.cuh"
 
@@ -60,7 +60,7 @@ constexpr int XS_LD = ctc::XS_LD;
 constexpr uint32_t SM_RS = SM_XS + 64 * XS_LD * 4;
 constexpr int RS_LD = ctc::RS_LD;
 constexpr uint32_t SM_SMALL = 202752;
-constexpr uint32_t SM_BYTES = SM_SMALL + 8192;
+constexpr uint32_t SM_BYTES = SM_SMALL + 10240;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;
 // Phase B (over phase A's consumed tiles):
 constexpr uint32_t SM_UHI = 0;          // U K-major [64 s][64 v] per d_v half (2 blocks), hi / lo
@@ -75,9 +75,15 @@ constexpr uint32_t SM_QE1 = 49152;      // q e1 [64 r][128 c] (exact path: L of 
 constexpr uint32_t SM_KE1 = 81920;      // k e1 (exact path: k)
 constexpr uint32_t SM_KE2 = 114688;     // k e2 (exact path: q)
 constexpr uint32_t SM_CUM = 147456;     // pair sums per cut position j and channel, [64 j][128 c]
+// The factored last pass (the MMA operand X is consumed): the gate gradient's per-(token, channel)
+// sums within a block, fp32 [64 r][128 c]
+constexpr uint32_t SM_TV = 81920;
 static_assert(SM_RS + 32 * RS_LD * 4 <= SM_SMALL, "solve scratch overlaps the small arrays");
 static_assert(SM_DPLO + 16384 <= SM_SMALL, "dP tile overlaps the small arrays");
 static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
+// small arrays in floats: beta 64, g / kappa / L exchange / L_C / parities 6 x 128, signs 256,
+// d beta 64, three [2][128] exchanges, Q_1 128, the gate phase's running sum [2][128]
+static_assert((64 + 6 * 128 + 256 + 64 + 3 * 256 + 128 + 256) * 4 <= SM_BYTES - SM_SMALL, "small arrays overflow");
 
 // TMEM columns (512). Phase A:
 constexpr uint32_t TM_SA = 0;           // (S0 Diag g)^T hi / lo, packed bf16 [d_v lanes][d_k]
@@ -94,8 +100,12 @@ constexpr uint32_t TM_DSLO = 96;
 constexpr uint32_t TM_G8 = 128;         // [dP ; dA] accumulator [r' lanes][64 s]
 constexpr uint32_t TM_G11 = 192;        // [c lanes][128 r']
 constexpr uint32_t TM_G12 = 320;        // [c lanes][64 s]
-constexpr uint32_t TM_G9 = 0;           //   after G11 / G12: [c lanes][128 r']
-constexpr uint32_t TM_G10 = 128;        //   after the G8 epilogue: [c lanes][64 s]
+// after the G8 epilogue (columns of the phase-B operands and of G8 are free):
+constexpr uint32_t TM_FACC = 0;         // pairs from earlier blocks, per tile row rho >= 32 (96 columns)
+constexpr uint32_t TM_CP = 96;          // pairs from later blocks, per token of blocks 0..2 (48)
+constexpr uint32_t TM_Q2 = 144;         // block 3's rows against blocks 0, 1 (32)
+constexpr uint32_t TM_G10 = 384;        // d(k e2) [c lanes][64 s]
+constexpr uint32_t TM_Q1 = 448;         // rows of blocks 2, 3 against block 0 (64)
 
 }  // namespace cbg
 
@@ -103,7 +113,8 @@ template <bool kLogGate>
 __global__ void __launch_bounds__(cbg::NTG, 1)
 chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
-                      const float* __restrict__ gate, const float* __restrict__ beta,
+                      const float* __restrict__ gate, const __nv_bfloat16* __restrict__ kraw,
+                      const __nv_bfloat16* __restrict__ qraw, const float* __restrict__ beta,
                       const float* __restrict__ dO, const float* __restrict__ Sck, const float* __restrict__ dSC,
                       const float* __restrict__ dWx, float* grad_q, float* grad_k, float* grad_gate,
                       float* grad_beta, int T, int H, int dk, int dv) {
@@ -131,6 +142,9 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     float* sh_db = reinterpret_cast<float*>(sh_sign + 256);       // [64] d beta accumulator
     float* sh_red = sh_db + 64;             // [2][128] cross-half exchange per channel
     float* sh_dgc = sh_red + 256;           // [2][128] <dS_C, S0> per channel, per d_v quarter pair
+    float* sh_red2 = sh_dgc + 256;          // [2][128] second cross-half exchange
+    float* sh_q1 = sh_red2 + 256;           // [128] the block sum Q_1 per channel
+    float* sh_run16 = sh_q1 + 128;          // [2][128] the gate phase's running log2 sum after 16 tokens
     float* at = reinterpret_cast<float*>(sm + SM_AT);
     float* xs = reinterpret_cast<float*>(sm + SM_XS);
     float* rs = reinterpret_cast<float*>(sm + SM_RS);
@@ -190,6 +204,9 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         tc::tc_fence_after();
     };
     auto sync_or = [&](bool p) -> bool { return __syncthreads_or(p) != 0; };
+    // [dP ; dA] fp32 table [128 r'][64 s]: 16-byte chunks XOR-swizzled by the row, so that a warp's
+    // rows store without bank conflicts and a row's chunks still read as float4
+    auto dpa_idx = [](int row, int col) -> int { return row * C + ((((col >> 2) ^ (row & 15)) << 2) | (col & 3)); };
 
     // ================================================================ phase A: the forward's quantities
     // gate cumulation: thread = channel m, tokens 32 hh .. 32 hh + 31 (as in the forward)
@@ -235,6 +252,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             bad = (-LC > kChunkRange);
         }
         slow = sync_or(bad);
+        sh_run16[hh * 128 + m] = L[15];
         LC = sh_LC[m];
         pC = sh_pC[m];
         if (hh == 0) {
@@ -262,23 +280,55 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         }
     }
     // factors: e1 = sgn 2^(L - R), e2 = sgn 2^(R - L) with R = L_C / 2 (exact path: e1 = Gamma,
-    // e2 = Gamma_C / Gamma); this thread's k and q values stay in registers for the last pass
+    // e2 = Gamma_C / Gamma); the last pass recomputes L and reads k, q again per 16-token block
     const float cref = slow ? 0.f : 0.5f * LC;
     const uint32_t sCbit = slow ? (pC << 31) : 0u;
     const float d2ref = slow ? LC : 0.f;
-    float kin[32], qin[32];
+    // k and q of this thread's tokens as one packed bf16 pair each (q high, k low): exact, and half
+    // the registers of two float arrays
+    uint32_t kq[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        kin[i] = ctc::ld_bf16_tile(sm + SM_K, 32 * hh + i, m);
-        qin[i] = ctc::ld_bf16_tile(sm + SM_Q, 32 * hh + i, m);
+        const float kf = ctc::ld_bf16_tile(sm + SM_K, 32 * hh + i, m);
+        const float qf = ctc::ld_bf16_tile(sm + SM_Q, 32 * hh + i, m);
+        kq[i] = (__float_as_uint(qf) & 0xffff0000u) | (__float_as_uint(kf) >> 16);
     }
-    auto factor_e1 = [&](int i) -> float {
+    auto kin = [&](int i) -> float { return __uint_as_float(kq[i] << 16); };
+    auto qin = [&](int i) -> float { return __uint_as_float(kq[i] & 0xffff0000u); };
+    auto fe1 = [&](float Lv, int i) -> float {
         const uint32_t sg = (par << (31 - i)) & 0x80000000u;
-        return __uint_as_float(__float_as_uint(tc::ex2_approx(L[i] - cref)) ^ sg);
+        return __uint_as_float(__float_as_uint(tc::ex2_approx(Lv - cref)) ^ sg);
     };
-    auto factor_e2 = [&](int i) -> float {
+    auto fe2 = [&](float Lv, int i) -> float {
         const uint32_t sg = (par << (31 - i)) & 0x80000000u;
-        return __uint_as_float(__float_as_uint(tc::ex2_approx(d2ref - (L[i] - cref))) ^ sg ^ sCbit);
+        return __uint_as_float(__float_as_uint(tc::ex2_approx(d2ref - (Lv - cref))) ^ sg ^ sCbit);
+    };
+    auto factor_e1 = [&](int i) -> float { return fe1(L[i], i); };
+    auto factor_e2 = [&](int i) -> float { return fe2(L[i], i); };
+    // one 16-token block of this thread's tokens (32 hh + 16 jb ..): the cumulative log2 gate by the
+    // gate phase's operations in the same order (so bit-identical), and k, q from global memory
+    // (read by this CTA's first loads, so normally still in L2), packed q high / k low
+    auto load_block = [&](int jb, float (&Lb)[16], uint32_t (&kqb)[16]) {
+        float run = jb ? sh_run16[hh * 128 + m] : 0.f;
+        const float lofs = hh ? sh_Lx[m] : 0.f;
+        const uint16_t* kr = reinterpret_cast<const uint16_t*>(kraw);
+        const uint16_t* qr = reinterpret_cast<const uint16_t*>(qraw);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int r = 32 * hh + 16 * jb + u;
+            const bool valid = r < nvalid && m < dk;
+            const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + m;
+            if constexpr (kLogGate) {
+                const float gg = valid ? __ldg(gate + o) : 0.f;
+                run += fmaxf(gg * kLog2e, kLgFloor);
+            } else {
+                const float a = valid ? __ldg(gate + o) : 1.f;
+                run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+            }
+            Lb[u] = run + lofs;
+            const uint32_t kb = valid ? (uint32_t)__ldg(kr + o) : 0u, qb = valid ? (uint32_t)__ldg(qr + o) : 0u;
+            kqb[u] = (qb << 16) | kb;
+        }
     };
 #pragma unroll
     for (int q8 = 0; q8 < 4; ++q8) {
@@ -287,9 +337,9 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         for (int e = 0; e < 8; ++e) {
             const int i = 8 * q8 + e;
             const float e1 = factor_e1(i), e2 = factor_e2(i);
-            xk[e] = kin[i] * e1;
-            xq[e] = qin[i] * e1;
-            yk[e] = kin[i] * e2;
+            xk[e] = kin(i) * e1;
+            xq[e] = qin(i) * e1;
+            yk[e] = kin(i) * e2;
         }
         store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xq);
         store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xk);
@@ -359,6 +409,14 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         }
     }
     if (sync_or(fail)) goto done;
+
+    // this thread's column of the entering state (lane v, channels 64 hh ..), in flight during the solve
+    float s0c[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const int c = 64 * hh + i;
+        s0c[i] = (c < dk && m < dv) ? __ldg(S0 + (size_t)c * dv + m) : 0.f;
+    }
 
     // solve: X = (I + A)^{-1} (the forward's blocked solve), T = X Diag(b) in three bf16 terms
     if (warp < 4 && lane < 16) {
@@ -474,15 +532,12 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     }
     // S0 Diag(g) -> TMEM operand [d_v lanes][d_k]: thread (lane v, half hh) takes columns 64 hh ..
     {
-#pragma unroll 1
+#pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             const int c0 = 64 * hh + 16 * cb;
             float z[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int c = c0 + i;
-                z[i] = (c < dk && m < dv) ? S0[(size_t)c * dv + m] * sh_g[c] : 0.f;
-            }
+            for (int i = 0; i < 16; ++i) z[i] = s0c[16 * cb + i] * sh_g[c0 + i];
             uint32_t hi[8], lo[8];
             split_pack16(z, hi, lo);
             tc::tmem_st32<8>(tl + TM_SA + c0 / 2, hi);
@@ -522,6 +577,13 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     tc::tmem_st_wait();
     tc::tc_fence_before();
     __syncthreads();
+    // dWx of this thread's column (lane v, tokens 32 hh ..), in flight during the U product
+    float wdx[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int s = 32 * hh + i;
+        wdx[i] = (m < dv && s < nvalid) ? __ldg(dWxc + (size_t)s * dv + m) : 0.f;
+    }
     // U^T = (V - Z)^T [T_hi ; T_mid]^T + (V - Z)^T T_lo^T: the forward's U product
     if (tid == 0) {
         tc::tc_fence_after();
@@ -554,6 +616,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         tc::tmem_ld32<32>(tl + TM_DU + 64 + 32 * hh, u2);
         tc::tmem_ld_wait();
         const int v = m, vh = v >> 6, vc = v & 63;
+        float w[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int s = 32 * hh + i;
@@ -564,15 +627,23 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             const uint32_t off = (uint32_t)vh * 8192u + chunk_off(s, vc >> 3) + (uint32_t)(vc & 7) * 2u;
             *reinterpret_cast<__nv_bfloat16*>(sm + SM_UHI + off) = hb;
             *reinterpret_cast<__nv_bfloat16*>(sm + SM_ULO + off) = lb;
-            // W = V - Z at (s, v); dWx at (s, v)
+            // W = V - Z at (s, v) times dWx at (s, v)
             const float vv = ctc::ld_bf16_tile(sm + SM_V, s, v);
-            const float w = (v < dv && s < nvalid) ? (vv - zreg[i]) * dWxc[(size_t)s * dv + v] : 0.f;
-            // sum over the warp's 32 d_v lanes, then the four lane quarters via shared atomics
-            float red = w;
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) red += __shfl_xor_sync(0xffffffffu, red, o2);
-            if (lane == 0) atomicAdd(&sh_db[s], red);
+            w[i] = (v < dv && s < nvalid) ? (vv - zreg[i]) * wdx[i] : 0.f;
         }
+        // sum over the warp's 32 d_v lanes for all 32 tokens at once (halving exchange: lane l ends
+        // with token 32 hh + l), then over the four lane quarters by shared atomics
+#pragma unroll
+        for (int off2 = 16; off2 >= 1; off2 >>= 1) {
+            const bool up = (lane & off2) != 0;
+#pragma unroll
+            for (int k = 0; k < off2; ++k) {
+                const float send = up ? w[k] : w[k + off2];
+                const float keep = up ? w[k + off2] : w[k];
+                w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off2);
+            }
+        }
+        atomicAdd(&sh_db[32 * hh + lane], w[0]);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -581,44 +652,44 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     // ================================================================ phase B: the gradient products
     {
         float dgc = 0.f;                     // <dS_C, S0> over this thread's d_v columns (channel m)
+        // one d_v half's operands, loaded into registers a half ahead (the next half's loads are in
+        // flight during this half's products):
+        //   [dO ; dWx] rows (thread: row r' = tid / 2, 32 v) -> K-major smem [128 r'][64 v]
+        //   S0 and dS_C rows (thread: lane c, v = 64 vh + 32 hh ..) -> TMEM [d_k lanes][32 packed columns]
+        float x[32], s0v[32], dsv[32];
+        const int rp_b = tid >> 1, vq_b = tid & 1;
+        auto load_b = [&](int vh) {
+            const int r = rp_b & 63;
+            const bool is_do = rp_b < 64;
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const int v = 64 * vh + 32 * vq_b + 4 * j4;
+                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r < nvalid && v < dv) {
+                    f = is_do ? __ldg(reinterpret_cast<const float4*>(dO + (((size_t)b * T + t0 + r) * H + h) * dv + v))
+                              : __ldg(reinterpret_cast<const float4*>(dWxc + (size_t)r * dv + v));
+                }
+                x[4 * j4] = f.x; x[4 * j4 + 1] = f.y; x[4 * j4 + 2] = f.z; x[4 * j4 + 3] = f.w;
+            }
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const int v = 64 * vh + 32 * hh + 4 * j4;
+                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = a4;
+                if (m < dk && v < dv) {
+                    a4 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)m * dv + v));
+                    d4 = __ldg(reinterpret_cast<const float4*>(dS + (size_t)m * dv + v));
+                }
+                s0v[4 * j4] = a4.x; s0v[4 * j4 + 1] = a4.y; s0v[4 * j4 + 2] = a4.z; s0v[4 * j4 + 3] = a4.w;
+                dsv[4 * j4] = d4.x; dsv[4 * j4 + 1] = d4.y; dsv[4 * j4 + 2] = d4.z; dsv[4 * j4 + 3] = d4.w;
+            }
+        };
+        load_b(0);
 #pragma unroll 1
         for (int vh = 0; vh < 2; ++vh) {
             if (vh == 1 && dv <= 64) break;
-            // [dO ; dWx] of this d_v half -> K-major [128 r'][64 v] (thread: row r' = tid / 2, 32 v)
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_STHI, sm + SM_STLO, rp_b, 4 * vq_b + q8, x + 8 * q8);
             {
-                const int rp = tid >> 1, vq = tid & 1;
-                const int r = rp & 63;
-                const bool is_do = rp < 64;
-                float x[32];
-#pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const int v = 64 * vh + 32 * vq + 4 * j4;
-                    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (r < nvalid && v < dv) {
-                        f = is_do ? *reinterpret_cast<const float4*>(dO + (((size_t)b * T + t0 + r) * H + h) * dv + v)
-                                  : *reinterpret_cast<const float4*>(dWxc + (size_t)r * dv + v);
-                    }
-                    x[4 * j4] = f.x; x[4 * j4 + 1] = f.y; x[4 * j4 + 2] = f.z; x[4 * j4 + 3] = f.w;
-                }
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_STHI, sm + SM_STLO, rp, 4 * vq + q8, x + 8 * q8);
-            }
-            // S0 and dS_C rows of this d_v half -> TMEM operands [d_k lanes][32 packed columns]:
-            // thread (lane c, hh) takes v = 64 vh + 32 hh ..
-            {
-                const int c = m;
-                float s0v[32], dsv[32];
-#pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const int v = 64 * vh + 32 * hh + 4 * j4;
-                    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = a4;
-                    if (c < dk && v < dv) {
-                        a4 = *reinterpret_cast<const float4*>(S0 + (size_t)c * dv + v);
-                        d4 = *reinterpret_cast<const float4*>(dS + (size_t)c * dv + v);
-                    }
-                    s0v[4 * j4] = a4.x; s0v[4 * j4 + 1] = a4.y; s0v[4 * j4 + 2] = a4.z; s0v[4 * j4 + 3] = a4.w;
-                    dsv[4 * j4] = d4.x; dsv[4 * j4 + 1] = d4.y; dsv[4 * j4 + 2] = d4.z; dsv[4 * j4 + 3] = d4.w;
-                }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) dgc = fmaf(s0v[j], dsv[j], dgc);
                 uint32_t hi[16], lo[16];
@@ -656,29 +727,31 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
                 }
                 tc::mma_commit(&bar_mma);
             }
+            if (vh == 0 && dv > 64) load_b(1);
             mma_wait();
             if (sync_or(fail)) goto done;
         }
         // <dS_C, S0>_c: the two token-half threads of channel c hold disjoint d_v columns
         sh_dgc[hh * 128 + m] = dgc;
     }
-    // G8 epilogue: [dP ; b dA] tile rows (thread: lane r', tokens 32 hh ..), d beta's rowsum(dA (.) L)
+    // G8 epilogue: [dP ; dA] into the fp32 table and [dP ; b dA] into the bf16 MMA tile (thread:
+    // lane r', tokens 32 hh ..), d beta's rowsum(dA (.) L). The bf16 tile's rows are interleaved by
+    // token block (row 32 blk + 16 half + u for token 16 blk + u of half dP / dA), so that the rows of
+    // every run of blocks are one contiguous MMA operand.
     {
         float g8[32];
         tc::tmem_ld32<32>(tl + TM_G8 + 32 * hh, g8);
         tc::tmem_ld_wait();
-        const int rp = m;
+        const int half = m >> 6, r = m & 63;
         float vals[32];
         float* dpa = reinterpret_cast<float*>(sm + SM_DPA);
-        if (rp < C) {
-            const int r = rp;
+        if (half == 0) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                vals[i] = (32 * hh + i <= r) ? g8[i] : 0.f;
-                dpa[rp * C + 32 * hh + i] = vals[i];
+                g8[i] = (32 * hh + i <= r) ? g8[i] : 0.f;
+                vals[i] = g8[i];
             }
         } else {
-            const int r = rp - C;
             const float br = sh_beta[r];
             float l[32];
             if (!slow) {
@@ -692,18 +765,22 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             float red = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const int s = 32 * hh + i;
-                const float da = (s < r) ? -g8[i] : 0.f;
-                dpa[rp * C + s] = da;
+                const int s2 = 32 * hh + i;
+                g8[i] = (s2 < r) ? -g8[i] : 0.f;
                 // entries of X Y^T above the diagonal may overflow: never read them
-                if (!slow && s < r) red = fmaf(da, l[i], red);
+                if (!slow && s2 < r) red = fmaf(g8[i], l[i], red);
                 // the exact path keeps dA itself (its pairwise pass applies b and forms rowsum(dA L))
-                vals[i] = slow ? da : br * da;
+                vals[i] = slow ? g8[i] : br * g8[i];
             }
             if (!slow) atomicAdd(&sh_db[r], red);
         }
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_DPHI, sm + SM_DPLO, rp, 4 * hh + q8, vals + 8 * q8);
+        for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(dpa + dpa_idx(m, 32 * hh + 4 * q4)) =
+                make_float4(g8[4 * q4], g8[4 * q4 + 1], g8[4 * q4 + 2], g8[4 * q4 + 3]);
+        const int rho = 32 * (r >> 4) + 16 * half + (r & 15);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + q8, vals + 8 * q8);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -719,11 +796,17 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         float* kall = reinterpret_cast<float*>(sm + SM_KE1);      // [64][128] fp32 (X, Y unused here)
         float* qall = reinterpret_cast<float*>(sm + SM_KE2);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hh + i;
-            Lsl[r * D + m] = L[i];
-            kall[r * D + m] = kin[i];
-            qall[r * D + m] = qin[i];
+        for (int jb = 0; jb < 2; ++jb) {
+            float Lb[16];
+            uint32_t kqb[16];
+            load_block(jb, Lb, kqb);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int r = 32 * hh + 16 * jb + u;
+                Lsl[r * D + m] = Lb[u];
+                kall[r * D + m] = __uint_as_float(kqb[u] << 16);
+                qall[r * D + m] = __uint_as_float(kqb[u] & 0xffff0000u);
+            }
         }
         __syncthreads();
         const int c = m;
@@ -733,7 +816,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             return ((sr ^ ss) ? -1.f : 1.f) * tc::ex2_approx(Lsl[r * D + c] - Lsl[s2 * D + c]);
         };
         const float* dpa = reinterpret_cast<const float*>(sm + SM_DPA);
-        auto tile = [&](int row, int col) -> float { return dpa[row * C + col]; };   // [dP ; dA]
+        auto tile = [&](int row, int col) -> float { return dpa[dpa_idx(row, col)]; };   // [dP ; dA]
 #pragma unroll 1
         for (int i = 0; i < 32; ++i) {
             const int r = 32 * hh + i;
@@ -747,7 +830,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             gq[i] = aq;
             gk1[i] = sh_beta[r] * ak;
             // rowsum(dA (.) L)_r, L_rs = sum_c k_rc k_sc R_rsc: this channel's share k_rc ak
-            float red = kin[i] * ak;
+            float red = kall[r * D + c] * ak;
 #pragma unroll
             for (int o2 = 16; o2 > 0; o2 >>= 1) red += __shfl_xor_sync(0xffffffffu, red, o2);
             if (lane == 0) atomicAdd(&sh_db[r], red);
@@ -766,23 +849,43 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         }
         __syncthreads();
     }
-    // G9: (k e2)^T [dP ; b dA]^T (N = 128, K = tokens);  G10: [q e1 ; k e1]^T [dP ; b dA] (N = 64, K = 128)
+    // Gate-gradient partial products and d(k e2), fast path, one commit. With the tokens in four
+    // blocks of 16, every pair (r, s) with s < j <= r whose tokens lie in different blocks enters
+    // one of these products, each of which holds only pairs that cross the cuts it serves
+    // (rho = the tile's interleaved row of token r, half dP or b dA):
+    //   Facc [c][rho - 32] = sum over tokens s of blocks before r's of (k e2)_{s c} [dP ; b dA]_{rho s}
+    //   Q1   [c][rho - 64] = the same over block 0 only, rows of blocks 2, 3
+    //   Q2   [c][rho - 96] = the same over blocks 0, 1, rows of block 3
+    //   CP   [c][s]        = sum over rows of blocks after s's of [q e1 ; k e1]_{rho c} [dP ; b dA]_{rho s}
+    //   G10  [c][s]        = the same over every row: d(k e2)
+    // Pairs inside one block are summed on CUDA cores in the last pass.
     if (!slow && tid == 0) {
         tc::tc_fence_after();
-        const uint32_t i9 = tc::idesc_bf16(128, 128, 0, 0), i10 = tc::idesc_bf16(128, 64, 0, 1);
+        const uint32_t i10 = tc::idesc_bf16(128, 64, 0, 1), i64 = tc::idesc_bf16(128, 64, 0, 0),
+                       i32 = tc::idesc_bf16(128, 32, 0, 0);
         for (int ps = 0; ps < 3; ++ps) {
             const uint32_t yb = sb + (ps == 2 ? SM_YLO : SM_YHI);
-            const uint32_t db9 = sb + (ps == 1 ? SM_DPLO : SM_DPHI);
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(tm + TM_G9, tc::sdesc(yb + ks * 32, 16, 1024), tc::sdesc(db9 + ks * 32, 16, 1024), i9,
-                           (ps | ks) != 0);
-        }
-        for (int ps = 0; ps < 3; ++ps) {
             const uint32_t xb = sb + (ps == 2 ? SM_XLO : SM_XHI);
-            const uint32_t db10 = sb + (ps == 1 ? SM_DPLO : SM_DPHI);
-            for (int ks = 0; ks < 8; ++ks)
-                tc::mma_ss(tm + TM_G10, tc::sdesc(xb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                           tc::sdesc(db10 + ks * 2048, 8192, 1024), i10, (ps | ks) != 0);
+            const uint32_t db = sb + (ps == 1 ? SM_DPLO : SM_DPHI);
+            // K = tokens of block S, rows rho >= 32 (S + 1); S = 0 covers every column
+            for (int S = 0; S < 3; ++S)
+                tc::mma_ss(tm + TM_FACC + 32 * S, tc::sdesc(yb + S * 32, 16, 1024),
+                           tc::sdesc(db + 4096 * (S + 1) + S * 32, 16, 1024),
+                           tc::idesc_bf16(128, 96 - 32 * S, 0, 0), (S | ps) != 0);
+            tc::mma_ss(tm + TM_Q1, tc::sdesc(yb, 16, 1024), tc::sdesc(db + 8192, 16, 1024), i64, ps != 0);
+            for (int S = 0; S < 2; ++S)
+                tc::mma_ss(tm + TM_Q2, tc::sdesc(yb + S * 32, 16, 1024), tc::sdesc(db + 12288 + S * 32, 16, 1024),
+                           i32, (S | ps) != 0);
+            // K = rows of block R (half dP, then b dA), N = tokens of blocks before R; R = 3 covers every column
+            for (int R = 3; R >= 1; --R)
+                for (int hf = 0; hf < 2; ++hf)
+                    tc::mma_ss(tm + TM_CP, tc::sdesc(xb + hf * 16384 + R * 32, 16, 1024),
+                               tc::sdesc(db + 4096 * R + 2048 * hf, 8192, 1024), tc::idesc_bf16(128, 16 * R, 0, 1),
+                               (R != 3 || hf != 0 || ps != 0) ? 1u : 0u);
+            for (int R = 0; R < 4; ++R)
+                for (int hf = 0; hf < 2; ++hf)
+                    tc::mma_ss(tm + TM_G10, tc::sdesc(xb + hf * 16384 + R * 32, 16, 1024),
+                               tc::sdesc(db + 4096 * R + 2048 * hf, 8192, 1024), i10, (R | hf | ps) != 0);
         }
         tc::mma_commit(&bar_mma);
     }
@@ -791,141 +894,300 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
 
     // ================================================================ last pass: thread = channel c,
     // tokens 32 hh .. 32 hh + 31
-    {
+    if (!slow) {
         const int c = m;
         const float g = sh_g[c], kap = sh_kap[c];
-        float dqe[32], dke[32], dke2[32], dqt[32], dkt[32], dkh[32];
-        if (!slow) {
-            tc::tmem_ld32<32>(tl + TM_G9 + 32 * hh, dqe);
-            tc::tmem_ld32<32>(tl + TM_G9 + 64 + 32 * hh, dke);
-            tc::tmem_ld_wait();
-            tc::tmem_ld32<32>(tl + TM_G10 + 32 * hh, dke2);
-            tc::tmem_ld_wait();
-        }
-        tc::tmem_ld32<32>(tl + TM_G11 + 32 * hh, dqt);
-        tc::tmem_ld_wait();
-        tc::tmem_ld32<32>(tl + TM_G11 + 64 + 32 * hh, dkt);
-        tc::tmem_ld32<32>(tl + TM_G12 + 32 * hh, dkh);
-        tc::tmem_ld_wait();
-        float sfx[32], pre[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hh + i;
-            const float e1 = factor_e1(i), e2 = factor_e2(i);
-            // Gamma_r and Gamma_C / Gamma_r (the exact path's factors are these already)
-            const float G = e1 * g, Gr = slow ? e2 : e2 * kap;
-            const float br = sh_beta[r];
-            const float kv = kin[i], qv = qin[i];
-            const float dKt = -br * dkt[i];
-            // d(q e1) e1, d(k e1) e1, d(k e2) e2: from the tile products, or pair by pair
-            const float tq = slow ? gq[i] : dqe[i] * e1;
-            const float tk1 = slow ? gk1[i] : dke[i] * e1;
-            const float tk2 = slow ? gk2[i] : dke2[i] * e2;
-            const float dq = tq + dqt[i] * G;
-            const float dkv = tk1 + tk2 + dKt * G + dkh[i] * Gr;
-            // the gate products through Gamma_r (Kt, Qt) and through Gamma_C / Gamma_r (Kh)
-            sfx[i] = (dKt * kv + dqt[i] * qv) * G;
-            pre[i] = dkh[i] * kv * Gr;
-            if (r < nvalid && c < dk) {
-                const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
-                grad_q[o] = dq;
-                grad_k[o] = dkv;
-            }
-        }
-        // d alpha_j alpha_j = sum of the terms whose gate product contains alpha_j:
-        //   pairs (r, s) with s < j <= r of the P / A ratios  +  sum_{r >= j} Kt, Qt terms
-        //   + sum_{s < j} Kh terms  +  <dS_C, S0>_c Gamma_C.
-        // Each sum holds only such terms (no cancelling pair enters), so dividing by alpha_j
-        // stays accurate for small and zero gates.
-        // Pair sums: row prefix RP(r, j) = sum_{s < j} w_rs, added to cut j for every j <= r,
-        //   w_rs = (q_r dP_rs + b_r k_r dA_rs) k_s Gamma_r / Gamma_s  (channel c)
-        // rows split between the two threads of a channel with equal work
-        float* tq1 = reinterpret_cast<float*>(sm + SM_QE1);
-        float* tk1t = reinterpret_cast<float*>(sm + SM_KE1);
-        float* tk2t = reinterpret_cast<float*>(sm + SM_KE2);
-        float* cum = reinterpret_cast<float*>(sm + SM_CUM);
         const float* dpa = reinterpret_cast<const float*>(sm + SM_DPA);
-        if (!slow) {
+        float* t_v = reinterpret_cast<float*>(sm + SM_TV);
+        float sfx_b[2] = {0.f, 0.f}, pre_b[2] = {0.f, 0.f};   // this thread's blocks' gate-term totals
+        float q1 = 0.f, q2 = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = 32 * hh + i;
-                const float e1 = factor_e1(i), e2 = factor_e2(i);
-                tq1[r * D + c] = qin[i] * e1;
-                tk1t[r * D + c] = kin[i] * e1;
-                tk2t[r * D + c] = kin[i] * e2;
+        for (int jb = 0; jb < 2; ++jb) {
+            const int J = 2 * hh + jb;
+            float Lb[16];
+            uint32_t kqb[16];
+            load_block(jb, Lb, kqb);
+            float y[16], xq[16], xk[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float e1 = fe1(Lb[u], 16 * jb + u), e2 = fe2(Lb[u], 16 * jb + u);
+                const float kv = __uint_as_float(kqb[u] << 16), qv = __uint_as_float(kqb[u] & 0xffff0000u);
+                y[u] = kv * e2;
+                xq[u] = qv * e1;
+                xk[u] = kv * e1;
             }
-        }
+            // pairs inside the block: gq_r = sum_{s <= r} dP_rs y_s, gk_r = sum_{s < r} dA_rs y_s (this
+            // block's share of d(q e1), d(k e1) / b) and, for every cut j of the block, the pairs
+            // s < j <= r: cum_j += (q e1)_r gq_r^(j - 1) + b_r (k e1)_r gk_r^(j - 1)
+            float gqd[16], gkd[16], cum[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) cum[(32 * hh + i) * D + c] = 0.f;
-        __syncthreads();
-        {
-#pragma unroll 1
-            for (int rr = 0; rr < 32; ++rr) {
-                const int r = (hh == 0) ? (rr < 16 ? rr : 32 + rr) : 16 + rr;
-                if (r >= nvalid) continue;
-                const float br = sh_beta[r];
-                float aq, ak;
-                if (!slow) {
-                    aq = tq1[r * D + c];
-                    ak = br * tk1t[r * D + c];
-                } else {
-                    aq = tk2t[r * D + c];            // q (exact-path table)
-                    ak = br * tk1t[r * D + c];       // b k
-                }
-                float rp = 0.f;
-#pragma unroll 4
-                for (int s2 = 0; s2 < r; ++s2) {
-                    const float w0 = aq * dpa[r * C + s2] + ak * dpa[(C + r) * C + s2];
-                    float w;
-                    if (!slow) {
-                        w = w0 * tk2t[s2 * D + c];
-                    } else {
-                        const float* Lsl = tq1;
-                        const uint32_t sr = (sh_sign[r * 4 + (c >> 5)] >> (c & 31)) & 1u;
-                        const uint32_t ss = (sh_sign[s2 * 4 + (c >> 5)] >> (c & 31)) & 1u;
-                        w = w0 * tk1t[s2 * D + c] * ((sr ^ ss) ? -1.f : 1.f) *
-                            tc::ex2_approx(Lsl[r * D + c] - Lsl[s2 * D + c]);
+            for (int u = 0; u < 16; ++u) cum[u] = 0.f;
+#pragma unroll
+            for (int ru = 0; ru < 16; ++ru) {
+                const int r = 16 * J + ru;
+                const float* rowp = dpa + r * C;
+                const float* rowa = dpa + (C + r) * C;
+                const float aq = xq[ru], ak = sh_beta[r] * xk[ru];
+                float gq = 0.f, gk = 0.f;
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    if (4 * v4 > ru) break;
+                    const int sw = ((4 * J + v4) ^ ru) << 2;      // row & 15 == ru for both halves
+                    const float4 p4 = *reinterpret_cast<const float4*>(rowp + sw);
+                    const float4 a4 = *reinterpret_cast<const float4*>(rowa + sw);
+                    const float pv[4] = {p4.x, p4.y, p4.z, p4.w}, av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int su = 4 * v4 + e;
+                        if (su < ru) {
+                            gq = fmaf(pv[e], y[su], gq);
+                            gk = fmaf(av[e], y[su], gk);
+                            cum[su + 1] = fmaf(aq, gq, fmaf(ak, gk, cum[su + 1]));
+                        } else if (su == ru) {
+                            gq = fmaf(pv[e], y[su], gq);
+                        }
                     }
-                    rp += w;
-                    atomicAdd(&cum[(s2 + 1) * D + c], rp);
+                }
+                gqd[ru] = gq;
+                gkd[ru] = gk;
+            }
+            // tokens of earlier blocks: Facc completes d(q e1), d(k e1) and gives the pairs from
+            // earlier blocks, RP_r = (q e1)_r Facc_r(dP) + (k e1)_r Facc_r(b dA)
+            float rp[16], dqa[16], dka[16];
+            {
+                float fq[16], fk[16];
+                if (J > 0) {
+                    tc::tmem_ld32<16>(tl + TM_FACC + (uint32_t)(32 * (J - 1)), fq);
+                    tc::tmem_ld32<16>(tl + TM_FACC + (uint32_t)(32 * (J - 1) + 16), fk);
+                    tc::tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) fq[u] = fk[u] = 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int r = 16 * J + u;
+                    const float e1 = fe1(Lb[u], 16 * jb + u);
+                    dqa[u] = (fq[u] + gqd[u]) * e1;
+                    dka[u] = fmaf(sh_beta[r], gkd[u], fk[u]) * e1;
+                    rp[u] = fmaf(xq[u], fq[u], xk[u] * fk[u]);
                 }
             }
-        }
-        __syncthreads();
-        // suffix sums of the Gamma_r terms and prefix sums of the Kh terms over the chunk
-        float sfx_tot = 0.f, pre_tot = 0.f;
+            // d(k e2) and the pairs from later blocks that end in this block's tokens
+            float cpv[16];
+            {
+                float g10[16], cp[16];
+                tc::tmem_ld32<16>(tl + TM_G10 + 16 * J, g10);
+                if (J < 3) tc::tmem_ld32<16>(tl + TM_CP + (uint32_t)(16 * J), cp);
+                tc::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) { sfx_tot += sfx[i]; pre_tot += pre[i]; }
-        sh_red[hh * 128 + c] = sfx_tot;
-        __syncthreads();
-        const float sfx_after = (hh == 0) ? sh_red[128 + c] : 0.f;      // second half's Gamma_r terms
-        __syncthreads();
-        sh_red[hh * 128 + c] = pre_tot;
-        __syncthreads();
-        const float pre_before = (hh == 1) ? sh_red[c] : 0.f;           // first half's Kh terms
-        const float gC = g * kap;                                       // Gamma_C
-        const float cst = (sh_dgc[c] + sh_dgc[128 + c]) * gC;
-        float suf = sfx_after, prf = pre_before;
-        float tot[32];
+                for (int u = 0; u < 16; ++u) {
+                    dka[u] = fmaf(g10[u], fe2(Lb[u], 16 * jb + u), dka[u]);
+                    cpv[u] = (J < 3) ? y[u] * cp[u] : 0.f;
+                }
+            }
+            // the pairs from later blocks ending in this block's tokens, and the block's own rows
+            {
+                float run = 0.f;
 #pragma unroll
-        for (int i = 31; i >= 0; --i) {
-            suf += sfx[i];
-            tot[i] = suf;
-        }
+                for (int u = 0; u < 16; ++u) {
+                    cum[u] += run;
+                    run += cpv[u];
+                }
+                run = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            tot[i] += prf + cst;
-            prf += pre[i];
+                for (int u = 15; u >= 0; --u) {
+                    run += rp[u];
+                    cum[u] += run;
+                }
+            }
+            // block sums Q_1 (rows of blocks 2, 3 against block 0) and Q_2 (rows of block 3 against
+            // blocks 0, 1): the pairs that cross the whole of block 1 or block 2
+            if (hh == 1) {
+                float t1[16], t2[16];
+                tc::tmem_ld32<16>(tl + TM_Q1 + (uint32_t)(32 * (J - 2)), t1);
+                tc::tmem_ld32<16>(tl + TM_Q1 + (uint32_t)(32 * (J - 2) + 16), t2);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) q1 = fmaf(xq[u], t1[u], fmaf(xk[u], t2[u], q1));
+                if (J == 3) {
+                    tc::tmem_ld32<16>(tl + TM_Q2, t1);
+                    tc::tmem_ld32<16>(tl + TM_Q2 + 16, t2);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) q2 = fmaf(xq[u], t1[u], fmaf(xk[u], t2[u], q2));
+                }
+            }
+            // the S0 and dS_C products: the rest of dq, dk and the gate's terms through Gamma_r (Kt, Qt:
+            // summed over r >= j) and through Gamma_C / Gamma_s (Kh: summed over s < j), here within
+            // the block; the other blocks' totals are added at the end
+            {
+                float dqt[16], dkt[16], dkh[16];
+                tc::tmem_ld32<16>(tl + TM_G11 + 16 * J, dqt);
+                tc::tmem_ld32<16>(tl + TM_G11 + 64 + 16 * J, dkt);
+                tc::tmem_ld32<16>(tl + TM_G12 + 16 * J, dkh);
+                tc::tmem_ld_wait();
+                float sf[16], pr[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int r = 16 * J + u;
+                    const float G = fe1(Lb[u], 16 * jb + u) * g, Gr = fe2(Lb[u], 16 * jb + u) * kap;
+                    const float kv = __uint_as_float(kqb[u] << 16), qv = __uint_as_float(kqb[u] & 0xffff0000u);
+                    const float dKt = -sh_beta[r] * dkt[u];
+                    const float dq = fmaf(dqt[u], G, dqa[u]);
+                    const float dkv = fmaf(dKt, G, fmaf(dkh[u], Gr, dka[u]));
+                    sf[u] = (dKt * kv + dqt[u] * qv) * G;
+                    pr[u] = dkh[u] * kv * Gr;
+                    if (r < nvalid && c < dk) {
+                        const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
+                        grad_q[o] = dq;
+                        grad_k[o] = dkv;
+                    }
+                }
+                float run = 0.f;
+#pragma unroll
+                for (int u = 15; u >= 0; --u) {
+                    run += sf[u];
+                    cum[u] += run;
+                }
+                sfx_b[jb] = run;
+                run = 0.f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    cum[u] += run;
+                    run += pr[u];
+                }
+                pre_b[jb] = run;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) t_v[(16 * J + u) * D + c] = cum[u];
+            }
         }
+        // d alpha_j alpha_j = the terms whose gate product contains alpha_j: the pair sums above,
+        // sum_{r >= j} of the Kt, Qt terms, sum_{s < j} of the Kh terms and <dS_C, S0>_c Gamma_C.
+        // Each holds only such terms (no cancelling pair enters), so dividing by alpha_j stays
+        // accurate for small and zero gates.
+        sh_red[hh * 128 + c] = sfx_b[0] + sfx_b[1];
+        sh_red2[hh * 128 + c] = pre_b[0] + pre_b[1];
+        if (hh == 1) sh_q1[c] = q1;
+        __syncthreads();
+        const float cst = (sh_dgc[c] + sh_dgc[128 + c]) * (g * kap);   // <dS_C, S0>_c Gamma_C
+        // per block: the other blocks' Kt, Qt totals after it, Kh totals before it, the block sum Q
+        const float other_sfx = (hh == 0) ? sh_red[128 + c] : 0.f;
+        const float other_pre = (hh == 1) ? sh_red2[c] : 0.f;
+        const float add0 = cst + other_sfx + other_pre + sfx_b[1] + ((hh == 1) ? q2 : 0.f);
+        const float add1 = cst + other_sfx + other_pre + pre_b[0] + ((hh == 0) ? sh_q1[c] : 0.f);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int r = 32 * hh + i;
             if (r < nvalid && c < dk) {
                 const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
-                const float cumj = tot[i] + cum[r * D + c];
+                const float cumj = t_v[r * D + c] + ((i < 16) ? add0 : add1);
                 float dg;
                 if constexpr (kLogGate) {
                     dg = cumj;                                  // d/dg = alpha d/dalpha
+                } else {
+                    // 1 / alpha as sign * 2^(-log2|alpha|), with the forward's floor on log2|alpha|
+                    const float a = __ldg(gate + o);
+                    const float la = fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+                    dg = ((__float_as_uint(a + 0.f) >> 31) ? -cumj : cumj) * tc::ex2_approx(-la);
+                }
+                grad_gate[o] = dg;
+            }
+        }
+        if (tid < C && tid < nvalid) grad_beta[((size_t)b * T + t0 + tid) * H + h] = sh_db[tid];
+    } else {
+        // exact path (a chunk's gate range too wide for the factored tiles): the pairwise sums
+        // above for d(q e1) e1, d(k e1) e1, d(k e2) e2, and the crossing pair sums per cut on CUDA
+        // cores; the gate's other terms as on the factored path, per 16-token block
+        const int c = m;
+        const float g = sh_g[c], kap = sh_kap[c];
+        const float* Lsl = reinterpret_cast<const float*>(sm + SM_QE1);
+        const float* kall = reinterpret_cast<const float*>(sm + SM_KE1);
+        const float* qall = reinterpret_cast<const float*>(sm + SM_KE2);
+        float* cum = reinterpret_cast<float*>(sm + SM_CUM);
+        const float* dpa = reinterpret_cast<const float*>(sm + SM_DPA);
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) cum[(32 * hh + i) * D + c] = 0.f;
+        __syncthreads();
+        // pair sums: row prefix RP(r, j) = sum_{s < j} w_rs, added to cut j for every j <= r,
+        //   w_rs = (q_r dP_rs + b_r k_r dA_rs) k_s Gamma_r / Gamma_s  (channel c)
+        // rows split between the two threads of a channel with equal work
+#pragma unroll 1
+        for (int rr = 0; rr < 32; ++rr) {
+            const int r = (hh == 0) ? (rr < 16 ? rr : 32 + rr) : 16 + rr;
+            if (r >= nvalid) continue;
+            const float aq = qall[r * D + c];
+            const float ak = sh_beta[r] * kall[r * D + c];
+            const uint32_t sr = (sh_sign[r * 4 + (c >> 5)] >> (c & 31)) & 1u;
+            float rp = 0.f;
+#pragma unroll 4
+            for (int s2 = 0; s2 < r; ++s2) {
+                const uint32_t ss = (sh_sign[s2 * 4 + (c >> 5)] >> (c & 31)) & 1u;
+                const float w0 = aq * dpa[dpa_idx(r, s2)] + ak * dpa[dpa_idx(C + r, s2)];
+                rp += w0 * kall[s2 * D + c] * ((sr ^ ss) ? -1.f : 1.f) *
+                      tc::ex2_approx(Lsl[r * D + c] - Lsl[s2 * D + c]);
+                atomicAdd(&cum[(s2 + 1) * D + c], rp);
+            }
+        }
+        __syncthreads();
+        float sfx_b[2] = {0.f, 0.f}, pre_b[2] = {0.f, 0.f};
+#pragma unroll
+        for (int jb = 0; jb < 2; ++jb) {
+            const int J = 2 * hh + jb;
+            float dqt[16], dkt[16], dkh[16];
+            tc::tmem_ld32<16>(tl + TM_G11 + 16 * J, dqt);
+            tc::tmem_ld32<16>(tl + TM_G11 + 64 + 16 * J, dkt);
+            tc::tmem_ld32<16>(tl + TM_G12 + 16 * J, dkh);
+            tc::tmem_ld_wait();
+            float sf[16], pr[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = 16 * jb + u, r = 16 * J + u;
+                // Gamma_r and Gamma_C / Gamma_r (the exact path's factors are these already)
+                const float Lr = Lsl[r * D + c];
+                const float G = fe1(Lr, i) * g, Gr = fe2(Lr, i);
+                const float kv = kall[r * D + c], qv = qall[r * D + c];
+                const float dKt = -sh_beta[r] * dkt[u];
+                const float dq = gq[i] + dqt[u] * G;
+                const float dkv = gk1[i] + gk2[i] + dKt * G + dkh[u] * Gr;
+                sf[u] = (dKt * kv + dqt[u] * qv) * G;
+                pr[u] = dkh[u] * kv * Gr;
+                if (r < nvalid && c < dk) {
+                    const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
+                    grad_q[o] = dq;
+                    grad_k[o] = dkv;
+                }
+            }
+            float run = 0.f;
+#pragma unroll
+            for (int u = 15; u >= 0; --u) {
+                run += sf[u];
+                cum[(16 * J + u) * D + c] += run;
+            }
+            sfx_b[jb] = run;
+            run = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                cum[(16 * J + u) * D + c] += run;
+                run += pr[u];
+            }
+            pre_b[jb] = run;
+        }
+        sh_red[hh * 128 + c] = sfx_b[0] + sfx_b[1];
+        sh_red2[hh * 128 + c] = pre_b[0] + pre_b[1];
+        __syncthreads();
+        const float cst = (sh_dgc[c] + sh_dgc[128 + c]) * (g * kap);   // Gamma_C on this path is kap
+        const float other = ((hh == 0) ? sh_red[128 + c] : 0.f) + ((hh == 1) ? sh_red2[c] : 0.f);
+        const float add0 = cst + other + sfx_b[1], add1 = cst + other + pre_b[0];
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+            const int r = 32 * hh + i;
+            if (r < nvalid && c < dk) {
+                const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
+                const float cumj = cum[r * D + c] + ((i < 16) ? add0 : add1);
+                float dg;
+                if constexpr (kLogGate) {
+                    dg = cumj;
                 } else {
                     const float a = __ldg(gate + o);
                     const float la = fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);

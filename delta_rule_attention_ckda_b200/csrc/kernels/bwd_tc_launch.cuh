@@ -70,7 +70,7 @@ inline cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // 3. every chunk's gradients, all chunks side by side
-    grad<<<nbh * nch, cbg::NTG, cbg::SMEM_ALLOC, st>>>(mk, mq, mv, ma, gate, beta, dO, Sck, dSC, dWx, grad_q, grad_k,
+    grad<<<nbh * nch, cbg::NTG, cbg::SMEM_ALLOC, st>>>(mk, mq, mv, ma, gate, k, q, beta, dO, Sck, dSC, dWx, grad_q, grad_k,
                                                       grad_gate, grad_beta, T, H, dk, dv);
     return cudaGetLastError();
 }

@@ -23,11 +23,15 @@ __device__ __forceinline__ uint32_t sw_off(int row, int col, int rows) {
     return swz128(logical);
 }
 
-// D[M][N] = A[M][K] * B[K][N] (optionally -A), one CTA of 128 threads, M = 128.
+// D[M][ns] = A[M][kb : kb + kn] * B[kb : kb + kn][n0 : n0 + ns] (optionally -A), one CTA of 128
+// threads, M = 128: the whole [K][N] B operand is staged, and the MMAs take a sub-tile of it
+// through the descriptors' start addresses (rows of a K-major B, columns inside the swizzle
+// atom of an MN-major B, and whole 16-wide K steps).
 // a_mode: 0 smem K-major, 1 smem MN-major, 2 tmem. b_mode: 0 smem K-major, 1 smem MN-major.
 __global__ void __launch_bounds__(128) gemm_selftest_kernel(const __nv_bfloat16* A, const __nv_bfloat16* B,
                                                             float* D, int N, int K, int a_mode, int b_mode,
-                                                            int neg_a, int* status) {
+                                                            int neg_a, int n0, int ns, int kb, int kn,
+                                                            int* status) {
     constexpr int M = 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -78,20 +82,21 @@ __global__ void __launch_bounds__(128) gemm_selftest_kernel(const __nv_bfloat16*
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-        const uint32_t idesc = idesc_bf16(M, N, a_mode == 1, b_mode == 1, neg_a);
+        const uint32_t idesc = idesc_bf16(M, ns, a_mode == 1, b_mode == 1, neg_a);
         const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
-        for (int ks = 0; ks < K / 16; ++ks) {
+        for (int ks = kb / 16; ks < (kb + kn) / 16; ++ks) {
             const int k0 = ks * 16;
             uint64_t bdesc;
-            if (b_mode == 0) bdesc = sdesc(b_base + (k0 / 64) * N * 128 + (k0 % 64) * 2, 16, 1024);
-            else bdesc = sdesc(b_base + k0 * 128, K * 128, 1024);
+            if (b_mode == 0) bdesc = sdesc(b_base + (k0 / 64) * N * 128 + n0 * 128 + (k0 % 64) * 2, 16, 1024);
+            else bdesc = sdesc(b_base + k0 * 128 + n0 * 2, K * 128, 1024);
+            const bool acc = ks > kb / 16;
             if (a_mode == 2) {
-                mma_ts(tbase + d_col, tbase + a_col + ks * 8, bdesc, idesc, ks > 0);
+                mma_ts(tbase + d_col, tbase + a_col + ks * 8, bdesc, idesc, acc);
             } else {
                 uint64_t adesc;
                 if (a_mode == 0) adesc = sdesc(a_base + (k0 / 64) * M * 128 + (k0 % 64) * 2, 16, 1024);
                 else adesc = sdesc(a_base + k0 * 128, K * 128, 1024);
-                mma_ss(tbase + d_col, adesc, bdesc, idesc, ks > 0);
+                mma_ss(tbase + d_col, adesc, bdesc, idesc, acc);
             }
         }
         mma_commit(&bar);
@@ -99,12 +104,12 @@ __global__ void __launch_bounds__(128) gemm_selftest_kernel(const __nv_bfloat16*
     const bool ok = mbar_wait(&bar, 0);
     tc_fence_after();
     if (ok) {
-        for (int c0 = 0; c0 < N; c0 += 16) {
+        for (int c0 = 0; c0 < ns; c0 += 16) {
             float r[16];
             tmem_ld32<16>(tmem_addr(tbase, (uint32_t)(warp * 32), d_col + c0), r);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) D[tid * N + c0 + j] = r[j];
+            for (int j = 0; j < 16; ++j) D[tid * ns + c0 + j] = r[j];
         }
     } else if (tid == 0) {
         *status = 1;
@@ -182,8 +187,27 @@ ST_API int ckda_selftest_gemm(const void* A, const void* B, float* D, int N, int
     const int smem = 128 * Kp * 2 + Kp * N * 2 + 1024;
     cudaFuncSetAttribute(gemm_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     gemm_selftest_kernel<<<1, 128, smem>>>(static_cast<const __nv_bfloat16*>(A),
-                                           static_cast<const __nv_bfloat16*>(B), D, N, K, a_mode, b_mode, neg_a,
-                                           status_dev);
+                                           static_cast<const __nv_bfloat16*>(B), D, N, K, a_mode, b_mode, neg_a, 0,
+                                           N, 0, K, status_dev);
+    return cudaGetLastError() == cudaSuccess ? 0 : 4;
+}
+
+// The same product on a sub-tile: D [128][ns] = A[:, kb : kb + kn] B[kb : kb + kn, n0 : n0 + ns], A in
+// K-major shared memory, B staged whole ([K][N]). K-major B: n0 a multiple of 8 (whole 8-row groups);
+// MN-major B (N = 64): n0 a multiple of 8 with n0 + ns <= 64 (inside one swizzle atom row).
+ST_API int ckda_selftest_gemm_sub(const void* A, const void* B, float* D, int N, int K, int b_mode, int n0, int ns,
+                                  int kb, int kn, int* status_dev) {
+    if (N < 16 || N > 256 || N % 16 || K < 16 || K > 128 || K % 16 || b_mode < 0 || b_mode > 1) return 1;
+    if (b_mode == 1 && N != 64) return 1;
+    if (b_mode == 0 && K % 64 && K > 64) return 1;
+    if (ns < 16 || ns % 16 || n0 < 0 || n0 % 8 || n0 + ns > N) return 1;
+    if (kb < 0 || kb % 16 || kn < 16 || kn % 16 || kb + kn > K) return 1;
+    const int Kp = K < 64 ? 64 : K;
+    const int smem = 128 * Kp * 2 + Kp * N * 2 + 1024;
+    cudaFuncSetAttribute(gemm_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    gemm_selftest_kernel<<<1, 128, smem>>>(static_cast<const __nv_bfloat16*>(A),
+                                           static_cast<const __nv_bfloat16*>(B), D, N, K, 0, b_mode, 0, n0, ns, kb,
+                                           kn, status_dev);
     return cudaGetLastError() == cudaSuccess ? 0 : 4;
 }
 

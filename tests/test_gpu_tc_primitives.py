@@ -21,6 +21,7 @@ def st():
     lib = ctypes.CDLL(build.SELFTEST_LIB)
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.ckda_selftest_gemm.argtypes = [vp, vp, vp, i, i, i, i, i, vp]
+    lib.ckda_selftest_gemm_sub.argtypes = [vp, vp, vp] + [i] * 7 + [vp]
     lib.ckda_selftest_tma.argtypes = [vp, i, i, i, i, i, i, i, i, i, i, vp, vp]
     lib.ckda_selftest_wait.argtypes = [ctypes.c_uint, i, vp]
     lib.ckda_selftest_error_word.argtypes = [ctypes.POINTER(ctypes.c_uint)]
@@ -66,6 +67,30 @@ def test_gemm_paths(st, a_mode, b_mode, N, K, neg):
     ref = A.double() @ B.double()
     if neg:
         ref = -ref
+    err = (D.double().cpu() - ref).abs().max().item()
+    assert err <= 1e-5 * ref.abs().max().item(), f"max err {err}"
+
+
+@pytest.mark.parametrize("b_mode,N,K,n0,ns,kb,kn", [
+    (0, 128, 64, 16, 48, 0, 16), (0, 128, 64, 80, 48, 0, 16), (0, 128, 64, 32, 32, 0, 32),
+    (0, 128, 64, 112, 16, 0, 48), (1, 64, 128, 0, 16, 16, 48), (1, 64, 128, 16, 16, 32, 32),
+    (1, 64, 128, 32, 16, 48, 16), (1, 64, 128, 0, 64, 64, 64), (1, 64, 64, 48, 16, 16, 16)])
+def test_gemm_sub_tiles(st, b_mode, N, K, n0, ns, kb, kn):
+    """Sub-tiles of a staged operand through the descriptors alone: rows of a K-major B,
+    16-wide column ranges inside the swizzle atom of an MN-major B, and a range of K steps
+    (the gate gradient's partial products over earlier or later token blocks)."""
+    g = torch.Generator().manual_seed(N + 7 * K + n0 + 3 * kb + b_mode)
+    A = torch.randn(128, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(K, N, generator=g).to(torch.bfloat16)
+    dA, dB = A.cuda(), B.cuda()
+    D = torch.full((128, ns), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = st.ckda_selftest_gemm_sub(dA.data_ptr(), dB.data_ptr(), D.data_ptr(), N, K, b_mode, n0, ns, kb, kn,
+                                   status.data_ptr())
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = A[:, kb:kb + kn].double() @ B[kb:kb + kn, n0:n0 + ns].double()
     err = (D.double().cpu() - ref).abs().max().item()
     assert err <= 1e-5 * ref.abs().max().item(), f"max err {err}"
 
