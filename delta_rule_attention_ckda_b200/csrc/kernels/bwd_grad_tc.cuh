@@ -69,15 +69,14 @@ constexpr uint32_t SM_STHI = 49152;     // [dO ; dWx] K-major [128 r'][64 v] of 
 constexpr uint32_t SM_STLO = 65536;
 constexpr uint32_t SM_DPHI = 32768;     // [dP ; b dA] [128 r'][64 s] (K-major B of G9, MN-major B of G10)
 constexpr uint32_t SM_DPLO = SM_XS;
+constexpr uint32_t SM_PS0 = 32768;      // phase B: S0 columns of one d_v quarter, fp32 [d_k][32] (TMA, swizzled)
+constexpr uint32_t SM_PDS = SM_XS;      //          dS_C columns of the same quarter
 // The last pass (after G9 / G10): fp32 tables for the gate gradient's pair sums
 constexpr uint32_t SM_DPA = 0;          // [dP ; dA] fp32 [128 r'][64 s] (written by the G8 epilogue)
 constexpr uint32_t SM_QE1 = 49152;      // q e1 [64 r][128 c] (exact path: L of the tokens)
 constexpr uint32_t SM_KE1 = 81920;      // k e1 (exact path: k)
 constexpr uint32_t SM_KE2 = 114688;     // k e2 (exact path: q)
 constexpr uint32_t SM_CUM = 147456;     // pair sums per cut position j and channel, [64 j][128 c]
-// The factored last pass (the MMA operand X is consumed): the gate gradient's per-(token, channel)
-// sums within a block, fp32 [64 r][128 c]
-constexpr uint32_t SM_TV = 81920;
 static_assert(SM_RS + 32 * RS_LD * 4 <= SM_SMALL, "solve scratch overlaps the small arrays");
 static_assert(SM_DPLO + 16384 <= SM_SMALL, "dP tile overlaps the small arrays");
 static_assert(SMEM_ALLOC <= 232448, "shared memory map exceeds 227 KB");
@@ -113,6 +112,7 @@ template <bool kLogGate>
 __global__ void __launch_bounds__(cbg::NTG, 1)
 chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
+                      const __grid_constant__ CUtensorMap map_s0, const __grid_constant__ CUtensorMap map_dsc,
                       const float* __restrict__ gate, const __nv_bfloat16* __restrict__ kraw,
                       const __nv_bfloat16* __restrict__ qraw, const float* __restrict__ beta,
                       const float* __restrict__ dO, const float* __restrict__ Sck, const float* __restrict__ dSC,
@@ -196,6 +196,8 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     const uint32_t tl = tm + lane_base;
     uint32_t mph = 0;                       // phase of bar_mma
     bool fail = false;
+    // TMA phases of bar_tma issued (thread 0) and waited for (each thread): phase 0 is the first loads
+    uint32_t tma_next = 1, tma_done = 1;
     // every thread waits for an MMA group that thread 0 committed; a wait that gives up is
     // OR-reduced at the CTA barrier that follows, where the CTA stops together
     auto mma_wait = [&]() {
@@ -356,9 +358,11 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     if (!slow) {
         if (tid == 0) {
             const uint32_t i128 = tc::idesc_bf16(128, 128, 1, 1), i64 = tc::idesc_bf16(128, 64, 1, 1);
+            #pragma unroll 1
             for (int ks = 0; ks < 8; ++ks)
                 tc::mma_ss(tm + TM_D1, tc::sdesc(sb + SM_XHI + ks * 2048, 16384, 1024),
                            tc::sdesc(sb + SM_YHI + ks * 2048, SM_YLO - SM_YHI, 1024), i128, ks != 0);
+            #pragma unroll 1
             for (int ks = 0; ks < 8; ++ks)
                 tc::mma_ss(tm + TM_D1, tc::sdesc(sb + SM_XLO + ks * 2048, 16384, 1024),
                            tc::sdesc(sb + SM_YHI + ks * 2048, SM_YLO - SM_YHI, 1024), i64, 1);
@@ -552,9 +556,11 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     if (tid == 0) {
         tc::tc_fence_after();
         const uint32_t id = tc::idesc_bf16(128, 64, 0, 1);
+        #pragma unroll 1
         for (int ps = 0; ps < 3; ++ps) {
             const uint32_t aa = tm + TM_SA + (ps == 2 ? 64 : 0);
             const uint32_t xb = sb + (ps == 1 ? SM_XLO : SM_XHI) + 16384;
+            #pragma unroll 1
             for (int ks = 0; ks < 8; ++ks)
                 tc::mma_ts(tm + TM_Z, aa + ks * 8, tc::sdesc(xb + ks * 2048, 8192, 1024), id, (ps | ks) != 0);
         }
@@ -589,17 +595,22 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         tc::tc_fence_after();
         const uint32_t iv = tc::idesc_bf16(128, 128, 1, 0), iv64 = tc::idesc_bf16(128, 64, 1, 0);
         const uint32_t iz = tc::idesc_bf16(128, 128, 0, 0), iz64 = tc::idesc_bf16(128, 64, 0, 0);
+        #pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
             tc::mma_ss(tm + TM_DU, tc::sdesc(sb + SM_V + ks * 2048, 8192, 1024), tc::sdesc(sb + SM_T + ks * 32, 16, 1024),
                        iv, ks != 0);
+        #pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
             tc::mma_ss(tm + TM_DU + 64, tc::sdesc(sb + SM_V + ks * 2048, 8192, 1024),
                        tc::sdesc(sb + SM_TL + ks * 32, 16, 1024), iv64, 1);
+        #pragma unroll 1
         for (int ps = 0; ps < 2; ++ps) {
             const uint32_t aa = tm + (ps == 1 ? TM_ZALO : TM_ZAHI);
+            #pragma unroll 1
             for (int ks = 0; ks < 4; ++ks)
                 tc::mma_ts(tm + TM_DU, aa + ks * 8, tc::sdesc(sb + SM_T + ks * 32, 16, 1024), iz, 1);
             if (ps == 0)
+                #pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_ts(tm + TM_DU + 64, aa + ks * 8, tc::sdesc(sb + SM_TL + ks * 32, 16, 1024), iz64, 1);
         }
@@ -652,13 +663,23 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     // ================================================================ phase B: the gradient products
     {
         float dgc = 0.f;                     // <dS_C, S0> over this thread's d_v columns (channel m)
-        // one d_v half's operands, loaded into registers a half ahead (the next half's loads are in
-        // flight during this half's products):
-        //   [dO ; dWx] rows (thread: row r' = tid / 2, 32 v) -> K-major smem [128 r'][64 v]
-        //   S0 and dS_C rows (thread: lane c, v = 64 vh + 32 hh ..) -> TMEM [d_k lanes][32 packed columns]
-        float x[32], s0v[32], dsv[32];
+        // Per d_v half: [dO ; dWx] rows (thread: row r' = tid / 2, 32 v) -> K-major smem [128 r'][64 v],
+        // loaded into registers a half ahead. Per d_v quarter: the S0 and dS_C columns by TMA (the
+        // next quarter's copies run during this quarter's products) -> TMEM operands [d_k lanes][16
+        // packed columns] (thread: lane c, v = 32 vq + 16 hh ..)
+        const int nq = dv > 64 ? 4 : 2;
+        const uint32_t qbytes = 2u * (uint32_t)dk * 128u;
+        const int srow = (int)(slot * (size_t)dk);
+        auto issue_q = [&](int vq) {         // thread 0
+            tc::mbar_arrive_expect_tx(&bar_tma, qbytes);
+            tc::tma_load_4d(sm + SM_PS0, &map_s0, &bar_tma, 32 * vq, 0, srow, 0);
+            tc::tma_load_4d(sm + SM_PDS, &map_dsc, &bar_tma, 32 * vq, 0, srow, 0);
+            ++tma_next;
+        };
+        if (tid == 0) issue_q(0);
+        float x[32];
         const int rp_b = tid >> 1, vq_b = tid & 1;
-        auto load_b = [&](int vh) {
+        auto load_x = [&](int vh) {
             const int r = rp_b & 63;
             const bool is_do = rp_b < 64;
 #pragma unroll
@@ -671,68 +692,89 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
                 }
                 x[4 * j4] = f.x; x[4 * j4 + 1] = f.y; x[4 * j4 + 2] = f.z; x[4 * j4 + 3] = f.w;
             }
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-                const int v = 64 * vh + 32 * hh + 4 * j4;
-                float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = a4;
-                if (m < dk && v < dv) {
-                    a4 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)m * dv + v));
-                    d4 = __ldg(reinterpret_cast<const float4*>(dS + (size_t)m * dv + v));
-                }
-                s0v[4 * j4] = a4.x; s0v[4 * j4 + 1] = a4.y; s0v[4 * j4 + 2] = a4.z; s0v[4 * j4 + 3] = a4.w;
-                dsv[4 * j4] = d4.x; dsv[4 * j4 + 1] = d4.y; dsv[4 * j4 + 2] = d4.z; dsv[4 * j4 + 3] = d4.w;
-            }
         };
-        load_b(0);
+        load_x(0);
 #pragma unroll 1
         for (int vh = 0; vh < 2; ++vh) {
             if (vh == 1 && dv <= 64) break;
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_STHI, sm + SM_STLO, rp_b, 4 * vq_b + q8, x + 8 * q8);
-            {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) dgc = fmaf(s0v[j], dsv[j], dgc);
-                uint32_t hi[16], lo[16];
-                ctc::split_pack32(s0v, hi, lo);
-                tc::tmem_st32<16>(tl + TM_S0HI + 16 * hh, hi);
-                tc::tmem_st32<16>(tl + TM_S0LO + 16 * hh, lo);
-                ctc::split_pack32(dsv, hi, lo);
-                tc::tmem_st32<16>(tl + TM_DSHI + 16 * hh, hi);
-                tc::tmem_st32<16>(tl + TM_DSLO + 16 * hh, lo);
-            }
-            tc::tmem_st_wait();
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
-                tc::tc_fence_after();
-                const uint32_t i8 = tc::idesc_bf16(128, 64, 0, 0), i11 = tc::idesc_bf16(128, 128, 0, 0),
-                               i12 = tc::idesc_bf16(128, 64, 0, 0);
-                for (int ps = 0; ps < 3; ++ps) {
-                    const uint32_t stb = sb + (ps == 2 ? SM_STLO : SM_STHI);
-                    const uint32_t ub = sb + (ps == 1 ? SM_ULO : SM_UHI) + (uint32_t)vh * 8192u;
-                    const uint32_t s0a = tm + (ps == 2 ? TM_S0LO : TM_S0HI);
-                    const uint32_t dsa = tm + (ps == 2 ? TM_DSLO : TM_DSHI);
-                    const uint32_t stb11 = sb + (ps == 1 ? SM_STLO : SM_STHI);
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint32_t acc = (vh | ps | ks) != 0;
-                        // G8: [dO ; dWx] U^T
-                        tc::mma_ss(tm + TM_G8, tc::sdesc(stb + ks * 32, 16, 1024), tc::sdesc(ub + ks * 32, 16, 1024), i8,
-                                   acc);
-                        // G11: S0 [dO ; dWx]^T
-                        tc::mma_ts(tm + TM_G11, s0a + ks * 8, tc::sdesc(stb11 + ks * 32, 16, 1024), i11, acc);
-                        // G12: dS_C U^T
-                        tc::mma_ts(tm + TM_G12, dsa + ks * 8, tc::sdesc(ub + ks * 32, 16, 1024), i12, acc);
-                    }
+            if (vh == 0 && dv > 64) load_x(1);
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                const int vq = 2 * vh + qq;
+                {
+                    const bool ok = tc::mbar_wait(&bar_tma, (uint32_t)(1 + vq) & 1u);
+                    fail |= !ok;
+                    if (ok) ++tma_done;
                 }
-                tc::mma_commit(&bar_mma);
+                {
+                    float s0v[16], dsv[16];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t off = (uint32_t)m * 128u + ((uint32_t)((4 * hh + t) ^ (m & 7)) << 4);
+                        float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = a4;
+                        if (m < dk) {
+                            a4 = *reinterpret_cast<const float4*>(sm + SM_PS0 + off);
+                            d4 = *reinterpret_cast<const float4*>(sm + SM_PDS + off);
+                        }
+                        s0v[4 * t] = a4.x; s0v[4 * t + 1] = a4.y; s0v[4 * t + 2] = a4.z; s0v[4 * t + 3] = a4.w;
+                        dsv[4 * t] = d4.x; dsv[4 * t + 1] = d4.y; dsv[4 * t + 2] = d4.z; dsv[4 * t + 3] = d4.w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) dgc = fmaf(s0v[j], dsv[j], dgc);
+                    uint32_t hi[8], lo[8];
+                    split_pack16(s0v, hi, lo);
+                    tc::tmem_st32<8>(tl + TM_S0HI + 16 * qq + 8 * hh, hi);
+                    tc::tmem_st32<8>(tl + TM_S0LO + 16 * qq + 8 * hh, lo);
+                    split_pack16(dsv, hi, lo);
+                    tc::tmem_st32<8>(tl + TM_DSHI + 16 * qq + 8 * hh, hi);
+                    tc::tmem_st32<8>(tl + TM_DSLO + 16 * qq + 8 * hh, lo);
+                }
+                tc::tmem_st_wait();
+                tc::fence_proxy_async_smem();
+                tc::tc_fence_before();
+                __syncthreads();
+                if (tid == 0) {
+                    tc::tc_fence_after();
+                    // every thread has read this quarter's copies: the next quarter's run during the products
+                    if (vq + 1 < nq) issue_q(vq + 1);
+                    const uint32_t i8 = tc::idesc_bf16(128, 64, 0, 0), i11 = tc::idesc_bf16(128, 128, 0, 0),
+                                   i12 = tc::idesc_bf16(128, 64, 0, 0);
+#pragma unroll 1
+                    for (int ps = 0; ps < 3; ++ps) {
+                        const uint32_t stb = sb + (ps == 2 ? SM_STLO : SM_STHI);
+                        const uint32_t ub = sb + (ps == 1 ? SM_ULO : SM_UHI) + (uint32_t)vh * 8192u;
+                        const uint32_t s0a = tm + (ps == 2 ? TM_S0LO : TM_S0HI);
+                        const uint32_t dsa = tm + (ps == 2 ? TM_DSLO : TM_DSHI);
+                        const uint32_t stb11 = sb + (ps == 1 ? SM_STLO : SM_STHI);
+#pragma unroll 1
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const int kk = 2 * qq + ks;   // K step of 16 within this d_v half
+                            const uint32_t acc = (vh | ps | kk) != 0;
+                            // G8: [dO ; dWx] U^T
+                            tc::mma_ss(tm + TM_G8, tc::sdesc(stb + kk * 32, 16, 1024), tc::sdesc(ub + kk * 32, 16, 1024),
+                                       i8, acc);
+                            // G11: S0 [dO ; dWx]^T
+                            tc::mma_ts(tm + TM_G11, s0a + kk * 8, tc::sdesc(stb11 + kk * 32, 16, 1024), i11, acc);
+                            // G12: dS_C U^T
+                            tc::mma_ts(tm + TM_G12, dsa + kk * 8, tc::sdesc(ub + kk * 32, 16, 1024), i12, acc);
+                        }
+                    }
+                    if (qq == 1) tc::mma_commit(&bar_mma);
+                }
             }
-            if (vh == 0 && dv > 64) load_b(1);
             mma_wait();
             if (sync_or(fail)) goto done;
         }
         // <dS_C, S0>_c: the two token-half threads of channel c hold disjoint d_v columns
         sh_dgc[hh * 128 + m] = dgc;
+    }
+    // the gate tile again (phase B's staging there is consumed), for the last pass's gate logs
+    if (!slow && tid == 0) {
+        tc::mbar_arrive_expect_tx(&bar_tma, 4 * 8192);
+        for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma, 32 * i, h, t0, b);
+        ++tma_next;
     }
     // G8 epilogue: [dP ; dA] into the fp32 table and [dP ; b dA] into the bf16 MMA tile (thread:
     // lane r', tokens 32 hh ..), d beta's rowsum(dA (.) L). The bf16 tile's rows are interleaved by
@@ -863,34 +905,40 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         tc::tc_fence_after();
         const uint32_t i10 = tc::idesc_bf16(128, 64, 0, 1), i64 = tc::idesc_bf16(128, 64, 0, 0),
                        i32 = tc::idesc_bf16(128, 32, 0, 0);
+        #pragma unroll 1
         for (int ps = 0; ps < 3; ++ps) {
             const uint32_t yb = sb + (ps == 2 ? SM_YLO : SM_YHI);
             const uint32_t xb = sb + (ps == 2 ? SM_XLO : SM_XHI);
             const uint32_t db = sb + (ps == 1 ? SM_DPLO : SM_DPHI);
             // K = tokens of block S, rows rho >= 32 (S + 1); S = 0 covers every column
+            #pragma unroll 1
             for (int S = 0; S < 3; ++S)
                 tc::mma_ss(tm + TM_FACC + 32 * S, tc::sdesc(yb + S * 32, 16, 1024),
                            tc::sdesc(db + 4096 * (S + 1) + S * 32, 16, 1024),
                            tc::idesc_bf16(128, 96 - 32 * S, 0, 0), (S | ps) != 0);
             tc::mma_ss(tm + TM_Q1, tc::sdesc(yb, 16, 1024), tc::sdesc(db + 8192, 16, 1024), i64, ps != 0);
+            #pragma unroll 1
             for (int S = 0; S < 2; ++S)
                 tc::mma_ss(tm + TM_Q2, tc::sdesc(yb + S * 32, 16, 1024), tc::sdesc(db + 12288 + S * 32, 16, 1024),
                            i32, (S | ps) != 0);
             // K = rows of block R (half dP, then b dA), N = tokens of blocks before R; R = 3 covers every column
+            #pragma unroll 1
             for (int R = 3; R >= 1; --R)
+                #pragma unroll 1
                 for (int hf = 0; hf < 2; ++hf)
                     tc::mma_ss(tm + TM_CP, tc::sdesc(xb + hf * 16384 + R * 32, 16, 1024),
                                tc::sdesc(db + 4096 * R + 2048 * hf, 8192, 1024), tc::idesc_bf16(128, 16 * R, 0, 1),
                                (R != 3 || hf != 0 || ps != 0) ? 1u : 0u);
+            #pragma unroll 1
             for (int R = 0; R < 4; ++R)
+                #pragma unroll 1
                 for (int hf = 0; hf < 2; ++hf)
                     tc::mma_ss(tm + TM_G10, tc::sdesc(xb + hf * 16384 + R * 32, 16, 1024),
                                tc::sdesc(db + 4096 * R + 2048 * hf, 8192, 1024), i10, (R | hf | ps) != 0);
         }
         tc::mma_commit(&bar_mma);
     }
-    if (!slow) mma_wait();
-    if (sync_or(fail)) goto done;
+    if (slow && sync_or(fail)) goto done;
 
     // ================================================================ last pass: thread = channel c,
     // tokens 32 hh .. 32 hh + 31
@@ -898,24 +946,62 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         const int c = m;
         const float g = sh_g[c], kap = sh_kap[c];
         const float* dpa = reinterpret_cast<const float*>(sm + SM_DPA);
-        float* t_v = reinterpret_cast<float*>(sm + SM_TV);
-        float sfx_b[2] = {0.f, 0.f}, pre_b[2] = {0.f, 0.f};   // this thread's blocks' gate-term totals
+        // within-block gate sums per (token, channel), fp32: tokens 0..31 in the D hi tile's
+        // space, 32..63 in the D lo tile's (both consumed by the products above)
+        float* t_v = reinterpret_cast<float*>(sm + (hh ? SM_DPLO : SM_DPHI));
+        // this thread's blocks' gate-term totals
+        float sfx0 = 0.f, sfx1 = 0.f, pre0 = 0.f, pre1 = 0.f;
         float q1 = 0.f, q2 = 0.f;
+        {
+            // the gate tile reloaded after phase B (the TMA phase after the d_v quarters)
+            const bool ok = tc::mbar_wait(&bar_tma, (uint32_t)(dv > 64 ? 5 : 3) & 1u);
+            fail |= !ok;
+            if (ok) ++tma_done;
+        }
+        // 16 consecutive values x = hi + lo of row `row` of a factored tile pair (tokens 16 J ..)
+        auto rd16 = [&](uint32_t hi_off, uint32_t lo_off, int row, int J, float (&x)[16]) {
 #pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const uint32_t off = chunk_off(row, 2 * J + k2);
+                const uint4 h4 = *reinterpret_cast<const uint4*>(sm + hi_off + off);
+                const uint4 l4 = *reinterpret_cast<const uint4*>(sm + lo_off + off);
+                const uint32_t hv[4] = {h4.x, h4.y, h4.z, h4.w}, lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x[8 * k2 + 2 * e] = __uint_as_float(hv[e] << 16) + __uint_as_float(lv[e] << 16);
+                    x[8 * k2 + 2 * e + 1] = __uint_as_float(hv[e] & 0xffff0000u) + __uint_as_float(lv[e] & 0xffff0000u);
+                }
+            }
+        };
+        // one copy of the block's code for both blocks (every instruction here runs once per chunk,
+        // so its fetch, not its issue, is what a second unrolled copy costs)
+#pragma unroll 1
         for (int jb = 0; jb < 2; ++jb) {
             const int J = 2 * hh + jb;
+            // the block's gate logs from the reloaded tile, by the gate phase's operations in the same
+            // order (bit-identical), and q e1, k e1, k e2 from the factored tiles (to 2^-16)
             float Lb[16];
-            uint32_t kqb[16];
-            load_block(jb, Lb, kqb);
-            float y[16], xq[16], xk[16];
+            {
+                float run = jb ? sh_run16[hh * 128 + c] : 0.f;
+                const float lofs = hh ? sh_Lx[c] : 0.f;
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const float e1 = fe1(Lb[u], 16 * jb + u), e2 = fe2(Lb[u], 16 * jb + u);
-                const float kv = __uint_as_float(kqb[u] << 16), qv = __uint_as_float(kqb[u] & 0xffff0000u);
-                y[u] = kv * e2;
-                xq[u] = qv * e1;
-                xk[u] = kv * e1;
+                for (int u = 0; u < 16; ++u) {
+                    const int r = 16 * J + u;
+                    const float av = ctc::ld_alpha_tile(sm + SM_AL, r, c);
+                    if constexpr (kLogGate) {
+                        const float gg = (r < nvalid && c < dk) ? av : 0.f;
+                        run += fmaxf(gg * kLog2e, kLgFloor);
+                    } else {
+                        const float a = (r < nvalid && c < dk) ? av : 1.f;
+                        run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+                    }
+                    Lb[u] = run + lofs;
+                }
             }
+            float y[16], xq[16], xk[16];
+            rd16(SM_XHI, SM_XLO, c, J, xq);
+            rd16(SM_XHI + 16384, SM_XLO + 16384, c, J, xk);
+            rd16(SM_YHI, SM_YLO, c, J, y);
             // pairs inside the block: gq_r = sum_{s <= r} dP_rs y_s, gk_r = sum_{s < r} dA_rs y_s (this
             // block's share of d(q e1), d(k e1) / b) and, for every cut j of the block, the pairs
             // s < j <= r: cum_j += (q e1)_r gq_r^(j - 1) + b_r (k e1)_r gk_r^(j - 1)
@@ -950,6 +1036,11 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
                 }
                 gqd[ru] = gq;
                 gkd[ru] = gk;
+            }
+            // block 0's gate logs, tile reads and in-block pairs ran during the products above
+            if (jb == 0) {
+                mma_wait();
+                if (sync_or(fail)) goto done;
             }
             // tokens of earlier blocks: Facc completes d(q e1), d(k e1) and gives the pairs from
             // earlier blocks, RP_r = (q e1)_r Facc_r(dP) + (k e1)_r Facc_r(b dA)
@@ -1032,12 +1123,12 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
                 for (int u = 0; u < 16; ++u) {
                     const int r = 16 * J + u;
                     const float G = fe1(Lb[u], 16 * jb + u) * g, Gr = fe2(Lb[u], 16 * jb + u) * kap;
-                    const float kv = __uint_as_float(kqb[u] << 16), qv = __uint_as_float(kqb[u] & 0xffff0000u);
                     const float dKt = -sh_beta[r] * dkt[u];
                     const float dq = fmaf(dqt[u], G, dqa[u]);
                     const float dkv = fmaf(dKt, G, fmaf(dkh[u], Gr, dka[u]));
-                    sf[u] = (dKt * kv + dqt[u] * qv) * G;
-                    pr[u] = dkh[u] * kv * Gr;
+                    // k Gamma_r = (k e1) g, q Gamma_r = (q e1) g, k Gamma_C / Gamma_r = (k e2) kappa
+                    sf[u] = (dKt * xk[u] + dqt[u] * xq[u]) * g;
+                    pr[u] = dkh[u] * y[u] * kap;
                     if (r < nvalid && c < dk) {
                         const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
                         grad_q[o] = dq;
@@ -1050,44 +1141,44 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
                     run += sf[u];
                     cum[u] += run;
                 }
-                sfx_b[jb] = run;
+                if (jb == 0) sfx0 = run; else sfx1 = run;
                 run = 0.f;
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     cum[u] += run;
                     run += pr[u];
                 }
-                pre_b[jb] = run;
+                if (jb == 0) pre0 = run; else pre1 = run;
 #pragma unroll
-                for (int u = 0; u < 16; ++u) t_v[(16 * J + u) * D + c] = cum[u];
+                for (int u = 0; u < 16; ++u) t_v[(16 * jb + u) * D + c] = cum[u];
             }
         }
         // d alpha_j alpha_j = the terms whose gate product contains alpha_j: the pair sums above,
         // sum_{r >= j} of the Kt, Qt terms, sum_{s < j} of the Kh terms and <dS_C, S0>_c Gamma_C.
         // Each holds only such terms (no cancelling pair enters), so dividing by alpha_j stays
         // accurate for small and zero gates.
-        sh_red[hh * 128 + c] = sfx_b[0] + sfx_b[1];
-        sh_red2[hh * 128 + c] = pre_b[0] + pre_b[1];
+        sh_red[hh * 128 + c] = sfx0 + sfx1;
+        sh_red2[hh * 128 + c] = pre0 + pre1;
         if (hh == 1) sh_q1[c] = q1;
         __syncthreads();
         const float cst = (sh_dgc[c] + sh_dgc[128 + c]) * (g * kap);   // <dS_C, S0>_c Gamma_C
         // per block: the other blocks' Kt, Qt totals after it, Kh totals before it, the block sum Q
         const float other_sfx = (hh == 0) ? sh_red[128 + c] : 0.f;
         const float other_pre = (hh == 1) ? sh_red2[c] : 0.f;
-        const float add0 = cst + other_sfx + other_pre + sfx_b[1] + ((hh == 1) ? q2 : 0.f);
-        const float add1 = cst + other_sfx + other_pre + pre_b[0] + ((hh == 0) ? sh_q1[c] : 0.f);
-#pragma unroll
+        const float add0 = cst + other_sfx + other_pre + sfx1 + ((hh == 1) ? q2 : 0.f);
+        const float add1 = cst + other_sfx + other_pre + pre0 + ((hh == 0) ? sh_q1[c] : 0.f);
+#pragma unroll 2
         for (int i = 0; i < 32; ++i) {
             const int r = 32 * hh + i;
             if (r < nvalid && c < dk) {
                 const size_t o = (((size_t)b * T + t0 + r) * H + h) * dk + c;
-                const float cumj = t_v[r * D + c] + ((i < 16) ? add0 : add1);
+                const float cumj = t_v[i * D + c] + ((i < 16) ? add0 : add1);
                 float dg;
                 if constexpr (kLogGate) {
                     dg = cumj;                                  // d/dg = alpha d/dalpha
                 } else {
                     // 1 / alpha as sign * 2^(-log2|alpha|), with the forward's floor on log2|alpha|
-                    const float a = __ldg(gate + o);
+                    const float a = ctc::ld_alpha_tile(sm + SM_AL, r, c);
                     const float la = fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
                     dg = ((__float_as_uint(a + 0.f) >> 31) ? -cumj : cumj) * tc::ex2_approx(-la);
                 }
@@ -1203,9 +1294,11 @@ done:
     tc::tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-        // no MMA of this CTA may still write TMEM when it is freed
+        // no MMA of this CTA may still write TMEM when it is freed, and no TMA copy its shared
+        // memory when it exits
         tc::mma_commit(&bar_mma);
         tc::mbar_wait(&bar_mma, mph);
+        for (uint32_t p = tma_done; p < tma_next; ++p) tc::mbar_wait(&bar_tma, p & 1u);
     }
     __syncthreads();
     if (warp == 0) {

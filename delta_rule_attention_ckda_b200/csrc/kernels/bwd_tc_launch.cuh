@@ -57,6 +57,13 @@ inline cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
         !tc::make_map_bthd(&ma, gate, f32, 4, B, T, H, dk, 32, 64) ||
         !tc::make_map_bthd(&mdo, dO, f32, 4, B, T, H, dv, 32, 64))
         return cudaErrorInvalidValue;
+    // the checkpoints and state cotangents as rows [B*H*chunks*d_k][d_v]: one d_v quarter of a chunk's
+    // d_k rows per copy
+    CUtensorMap ms0, mdsc;
+    const int ckrows = B * H * ((T + ctc::C - 1) / ctc::C) * dk;
+    if (!tc::make_map_bthd(&ms0, Sck, f32, 4, 1, ckrows, 1, dv, 32, dk) ||
+        !tc::make_map_bthd(&mdsc, dSC, f32, 4, 1, ckrows, 1, dv, 32, dk))
+        return cudaErrorInvalidValue;
     static std::atomic<uint64_t> chain_attr[2], grad_attr[2];
     auto chain = log_gate ? chunk_bwd_chain_kernel<true> : chunk_bwd_chain_kernel<false>;
     auto grad = log_gate ? chunk_bwd_grad_kernel<true> : chunk_bwd_grad_kernel<false>;
@@ -70,7 +77,7 @@ inline cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // 3. every chunk's gradients, all chunks side by side
-    grad<<<nbh * nch, cbg::NTG, cbg::SMEM_ALLOC, st>>>(mk, mq, mv, ma, gate, k, q, beta, dO, Sck, dSC, dWx, grad_q, grad_k,
+    grad<<<nbh * nch, cbg::NTG, cbg::SMEM_ALLOC, st>>>(mk, mq, mv, ma, ms0, mdsc, gate, k, q, beta, dO, Sck, dSC, dWx, grad_q, grad_k,
                                                       grad_gate, grad_beta, T, H, dk, dv);
     return cudaGetLastError();
 }
