@@ -133,6 +133,10 @@ constexpr uint32_t kFlagVZero = 1u;     // v is taken as zero (not loaded; no V 
 constexpr uint32_t kFlagNoO = 2u;       // no o output
 constexpr uint32_t kFlagS0Ident = 4u;   // the state entering each segment is the identity (d_v = d_k)
 constexpr uint32_t kFlagMapsOnly = 8u;  // every segment, the first included, builds its affine map
+constexpr uint32_t kFlagRedo = 16u;     // direct launch after the fast instance: only the sequences it
+                                        // marked run (aux = o)
+// the fast instance's mark in o[b][T-1][h][0] of a sequence it left (a NaN no arithmetic produces)
+constexpr uint32_t kRedoMark = 0x7FC0DE5Au;
 
 // Byte address (from tile base) of the 16-byte chunk `ch` (0..7) of row `row` in a
 // tile of 128-byte rows with 128-byte swizzle.
@@ -329,7 +333,12 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 // the scale folds into the per-token factors, so the normalised values are never rounded.
 // kStoreStates: S_ck receives the state entering every chunk (the backward's checkpoints);
 // a separate instance, so that the forward carries none of its code.
-template <bool kLogGate, bool kNormQK, bool kStoreStates = false>
+// kFast: one sequence per CTA from S0 (the direct launch) without the exact path's code. A
+// chunk whose gate range needs the exact path stops the CTA, which marks the sequence in its
+// o (S_ck then points at o); a second launch of the general instance with kFlagRedo runs the
+// marked sequences again from the start. The exact path's code, never run on ordinary gates,
+// otherwise shares the instruction cache with the chunk loop, which it then no longer fits.
+template <bool kLogGate, bool kNormQK, bool kStoreStates = false, bool kFast = false>
 __global__ void __launch_bounds__(ctc::NT_ALL, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
@@ -351,6 +360,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // (on the normal path everything has completed already; after a wait that gave up it has not)
     __shared__ uint64_t bar_drain[2];
     __shared__ uint32_t tmem_base_s;
+    __shared__ uint32_t sh_bail;            // kFast: a chunk needs the exact path; the CTA stops
 
     float* sh_beta = reinterpret_cast<float*>(sm + SM_SMALL);          // [64]
     // per-channel constants, [2][128] by chunk parity: the next chunk's are written while the
@@ -384,13 +394,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // none (its entering state is known), so those CTAs return at once.
     // kFlagMapsOnly in flags_in treats segment 0 like the others (the whole launch builds
     // affine maps: z = 0 the state from zero with flags_in, z = 1 the transition product).
-    const bool trans = blockIdx.z != 0;
+    if (!kFast && (flags_in & kFlagRedo) != 0) {
+        // the fast instance's second pass: only the sequences it marked run, from the start
+        const int b0 = (int)blockIdx.x / H, h0 = (int)blockIdx.x % H;
+        const volatile float* mk = S_ck + (((size_t)b0 * T + (T - 1)) * H + h0) * dv_in;
+        if (__float_as_uint(*mk) != kRedoMark) return;
+    }
+    const bool trans = !kFast && blockIdx.z != 0;
     const int bh = blockIdx.x;                    // grid: x = (batch, head), y = segment
     const int sg = sg_base + (int)blockIdx.y;
     const bool direct = sg == 0 && (flags_in & kFlagMapsOnly) == 0;   // segment 0 from the known S0
     if (trans && direct) return;
     // the checkpoint instance may run the direct segment without o (the backward needs states only)
-    const uint32_t flags = trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident)
+    const uint32_t flags = kFast ? 0u
+                         : trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident)
                                  : (direct ? (kStoreStates ? (flags_in & kFlagNoO) : 0u) : flags_in);
     const int dv = trans ? dk : dv_in;
     const int b = bh / H, h = bh % H;
@@ -433,6 +450,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         if ((flags & kFlagNoO) == 0) tc::prefetch_tensormap(&map_o);   // unset when no CTA writes o
     }
     if (tid < 2 * D) sh_kref[tid] = 1.f;
+    if (tid == 0) sh_bail = 0u;
     // blocks of (I + A)^{-1} above the 16 x 16 block diagonal: zero once, never written again
     for (int e = tid; e < 384; e += NT_ALL) {
         int r, g;
@@ -623,6 +641,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             issue_loads2(ta);
         }
         int ck = 0;
+        bool ebail = false;
         for (; ck < nchunks; ++ck) {
             const uint32_t par = (uint32_t)ck & 1u;
             const int t0 = ta + ck * C;
@@ -633,6 +652,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
             // for fast-decaying channels although each factor and each result is in range.
             efail |= !tc::mbar_wait(&bar_hk[par], (uint32_t)(ck >> 1) & 1u);   // this chunk's constants
+            if constexpr (kFast) {
+                // the compute warps stopped at this chunk (it needs the exact path): every epilogue
+                // thread waited for the same hand-off, so all leave here together
+                if (*reinterpret_cast<volatile uint32_t*>(&sh_bail) != 0u) {
+                    ebail = true;
+                    break;
+                }
+            }
             if (ck > 0) efail |= !tc::mbar_wait(&bar_c2, par ^ 1u);
             tc::tc_fence_after();
             {
@@ -773,11 +800,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             tc::bulk_wait0();
             tc::mma_commit(&bar_drain[0]);
             tc::mbar_wait(&bar_drain[0], 0);
-            if (efail) {
+            if (efail || ebail) {
                 // loads whose data nobody waited for: let them land before shared memory is released
                 if (n1a) tc::mbar_wait(&bar_tma1a, (n1a - 1) & 1u);
                 if (n1b) tc::mbar_wait(&bar_tma1b, (n1b - 1) & 1u);
                 if (n2) tc::mbar_wait(&bar_tma2, (n2 - 1) & 1u);
+            }
+            if constexpr (kFast) {
+                // mark the sequence for the general instance's second pass (S_ck points at o; the
+                // last token's row is in a chunk this CTA did not reach, so nothing else writes it)
+                if (ebail) S_ck[(((size_t)b * T + (T - 1)) * H + h) * dv_in] = __uint_as_float(kRedoMark);
             }
         }
     } else {
@@ -845,12 +877,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 bad = (-LC > kChunkRange);
             }
             slow = csync_or(bad);
+            if constexpr (kFast) {
+                if (slow) {
+                    // the general instance redoes this sequence: hand the (unused) constants over
+                    // so that the epilogue group sees the stop where it waits for them
+                    if (tid == 0) sh_bail = 1u;
+                    handoff(&bar_hk[ckn & 1]);
+                    return true;
+                }
+            }
             if (hh == 0) {
                 LC = sh_LC[m];
                 pC = sh_pC[m];
                 const int pb = ckn & 1, o = pb * D + m;
                 sh_kp[o] = sh_kref[(pb ^ 1) * D + m];
-                if (!slow) {
+                if (kFast || !slow) {
                     const float gref = exp2f(0.5f * LC);
                     sh_fa[o] = gref;
                     sh_fs[o] = gref;
@@ -861,7 +902,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     sh_kref[o] = 1.f;
                 }
             }
-            if (slow) {
+            if (!kFast && slow) {
                 float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) Ls[(32 * hh + i) * D + m] = L[i] + Lofs;
@@ -918,9 +959,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 // per-token factors (the sign of Gamma_r is XORed into the factor's sign bit):
                 //   fast path  e1 = Gamma_r / 2^R,  e2 = 2^R / Gamma_r  (R = L_C / 2: middle of the range)
                 //   exact path e1 = Gamma_r,        e2 = Gamma_C / Gamma_r
-                const float c1 = slow ? -Lofs : 0.5f * LC - Lofs;     // t = L_r - R, or L_r
-                const uint32_t sC = slow ? (pC << 31) : 0u;
-                const float d2 = slow ? LC : 0.f;                       // e2 = 2^(d2 - t)
+                const float c1 = (!kFast && slow) ? -Lofs : 0.5f * LC - Lofs;     // t = L_r - R, or L_r
+                const uint32_t sC = (!kFast && slow) ? (pC << 31) : 0u;
+                const float d2 = (!kFast && slow) ? LC : 0.f;                       // e2 = 2^(d2 - t)
                 uint32_t yh[4][4], yl[4][4];      // Y = k e2 split, held until the tile is free
                 float kin[32], qin[32];           // this thread's k and q values first
 #pragma unroll
@@ -967,7 +1008,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     *reinterpret_cast<uint4*>(sm + SM_YHI + off) = make_uint4(yh[q8][0], yh[q8][1], yh[q8][2], yh[q8][3]);
                     *reinterpret_cast<uint4*>(sm + SM_YLO + off) = make_uint4(yl[q8][0], yl[q8][1], yl[q8][2], yl[q8][3]);
                 }
-                if (slow) {
+                if (!kFast && slow) {
                     // sign bits of Gamma per (token, channel): word [r][m/32], bit m%32
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -978,7 +1019,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             }
             // X, Y tiles written and the alpha space free (exact path: after its pairwise
             // evaluation): the epilogue group stages the previous o tile and issues C1
-            if (!slow) handoff(&bar_hap);
+            if (kFast || !slow) handoff(&bar_hap);
             else {
                 tc::fence_proxy_async_smem();
                 tc::tc_fence_before();
@@ -986,7 +1027,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             if (csync_or(wfail)) { failed = true; break; }
 
             // ---------------- P2: [A ; P] = X Y  (3 passes) or the exact pairwise path
-            if (!slow) {
+            if (kFast || !slow) {
                 // one compute thread issues the [P ; A] MMA; every compute warp waits for it
                 if (tid == 0) {
                     tc::tc_fence_after();

@@ -246,15 +246,19 @@ using ChunkTcKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMa
 // the kernel instance for the gate form and the q/k normalisation (and, for the backward's
 // checkpoints, the one that stores every chunk's entering state), with its shared-memory
 // attribute set on the current device
-inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKernel& kern, bool store_states = false) {
-    static std::atomic<uint64_t> attr_done[8];
+inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKernel& kern, bool store_states = false,
+                                       bool fast = false) {
+    static std::atomic<uint64_t> attr_done[12];
     if (store_states)
         kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true, true> : chunk_tc_kernel<true, false, true>)
                         : (norm_qk ? chunk_tc_kernel<false, true, true> : chunk_tc_kernel<false, false, true>);
+    else if (fast)
+        kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true, false, true> : chunk_tc_kernel<true, false, false, true>)
+                        : (norm_qk ? chunk_tc_kernel<false, true, false, true> : chunk_tc_kernel<false, false, false, true>);
     else
         kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
                         : (norm_qk ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
-    const int variant = (store_states ? 4 : 0) + (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
+    const int variant = (store_states ? 4 : fast ? 8 : 0) + (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
     return ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)ctc::SMEM_ALLOC, attr_done[variant]);
 }
 
@@ -278,6 +282,22 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     const unsigned nbh = (unsigned)(B * H);
     const ChunkTcPlan p = chunk_tc_plan(B, T, H, chunk_tc_sm_count());
     if (p.nseg == 1) {
+        if (S_ck == nullptr && T > 0) {
+            // the plain forward: the instance without the exact path's code, then the general one
+            // over the sequences it marked (a chunk's gate range past the factored tiles); the
+            // second launch's other CTAs read one value and leave
+            ChunkTcKernel fast = nullptr;
+            cudaError_t e = chunk_tc_kernel_for(log_gate, norm_qk, fast, false, true);
+            if (e != cudaSuccess) return e;
+            fast<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
+                                                                         nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, 0u, o);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
+                                                                         nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0,
+                                                                         ctc::kFlagRedo, o);
+            return cudaGetLastError();
+        }
         kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
                                                                      nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, extra, S_ck);
         return cudaGetLastError();
