@@ -87,6 +87,42 @@ def test_extreme_decay_takes_exact_path(ck):
     check("extreme/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
 
 
+def test_exact_path_chunks_on_the_direct_launch(ck):
+    """One CTA per sequence (the direct launch, 128 sequences): sequences with a chunk past the
+    factored tiles' range (in the first, a middle and the last, partial chunk) are left by the
+    instance without the exact path and redone from the start by the general one; every
+    sequence, redone or not, matches the oracle."""
+    B, T, H = 8, 190, 16
+    assert ck.chunk_segments(B, T, H, 128, 128) == 1
+    inp = make_inputs(B, T, H, 128, 128, torch.bfloat16, seed=21, gate="tanh15", s0_std=0.3)
+    inp.alpha[0, 70:75, 0, :40] = 1e-20         # chunk 1
+    inp.alpha[3, 3:9, 5, 60:70] = -1e-22        # chunk 0: the CTA stops before its first chunk
+    inp.alpha[7, 150:156, 15, :] = 1e-25        # chunk 2, the partial last chunk
+    inp.alpha[5, 100, 2, :] = 0.0               # zero gates alone stay on the factored path
+    o, ST = run_chunk(ck, inp)
+    assert ck.get_device_error() == 0
+    assert torch.isfinite(o).all() and torch.isfinite(ST).all()
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, inp.alpha, inp.beta, inp.S0)
+    check("direct-exact/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check("direct-exact/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
+def test_exact_path_chunks_on_the_direct_launch_log_gate(ck):
+    """The same with the gate given as g = ln a (KDA form): a run of g = -50 (2^-72 per token)
+    in one sequence's middle chunk."""
+    B, T, H = 8, 256, 16
+    inp = make_inputs(B, T, H, 128, 128, torch.bfloat16, seed=22, gate="log15", s0_std=0.2)
+    g = inp.alpha.clone()
+    g[2, 120:126, 9, :32] = -50.0
+    q, k, v, _, b, s0 = to_dev(inp)
+    o, ST = ck.chunk_fwd(q, k, v, g.cuda(), b, s0, gate="log")
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    o_ref, S_ref = oracle.oracle_fwd(inp.q, inp.k, inp.v, torch.exp(g.double()), inp.beta, inp.S0)
+    check("direct-exact-log/o", o.double().cpu().numpy(), o_ref, TAU_BF16)
+    check("direct-exact-log/S", ST.double().cpu().numpy(), S_ref, TAU_BF16)
+
+
 @pytest.mark.parametrize("mag", [0.5, 0.2, 0.15, 0.1])
 def test_fast_decaying_channels(ck, mag):
     """Channels whose gates shrink the state by up to 2^-210 per chunk: 0.5, 0.2 and 0.15
