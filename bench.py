@@ -323,6 +323,18 @@ def reference_arm(args):
     return 0
 
 
+def fwd_launches(ck, B, T, H, dk, dv, dtype=None):
+    """Kernel launches of one chunk_fwd call: the tensor-core direct launch is two (the
+    instance without the exact path, then the general one over the sequences it left), the
+    segmented one three (segment maps, the fold, the segments from their entering states),
+    the recurrent path one."""
+    import torch
+    dtype = dtype or torch.bfloat16
+    if ck.chunk_path(B, T, H, dk, dv, dtype) != ck.PATH_CHUNK_TC:
+        return 1
+    return 2 if ck.chunk_segments(B, T, H, dk, dv, dtype) == 1 else 3
+
+
 def time_launches(fn, steps, stream):
     import torch
     ev0 = torch.cuda.Event(enable_timing=True)
@@ -412,7 +424,7 @@ def ours_arm(args):
                        "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
                        "path": path, "l2": "inputs larger than L2 (~950 MB per step vs 126 MB), no flush",
                        "state": "S0 = 0 (not read), S_T written"},
-            "roofline": roof, "gpu_launches": args.steps, "clocks": clocks}
+            "roofline": roof, "gpu_launches": args.steps * fwd_launches(ck, B, T, H, dk, dv), "clocks": clocks}
 
     if not args.no_extras:
         line["kda"] = kda_measure(ck, q, k, v, a, b, o, ST, stream, world, args.steps, value)
@@ -538,7 +550,7 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
                "(tcgen05)" if tc else "bwd_ckpt_kernel + bwd_grad_kernel + bwd_sum_kernel (fp32 CUDA cores)")
     out = {"workload": f"layer B={B} T={T} H={H} dk={dk} dv={dv}, backward of <dO, o> (S0 = 0)",
            "path": "chunk_tc" if tc else "recurrent",
-           "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": 3 * reps,
+           "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": (4 if tc else 3) * reps,
            "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
                         "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg, "kernels": kernels}}
 
@@ -563,7 +575,8 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
     out["fwd_bwd"] = {"workload": "layer: forward (o, S_T) then backward, per step",
                       "ckda_ms": fb["ckda"], "kda_ms": fb["kda"],
                       "kda_gate": "g = ln|alpha| (non-negative gate) through the log-gate mode",
-                      "ckda_over_kda_throughput": fb["kda"] / fb["ckda"], "gpu_launches": 4 * reps}
+                      "ckda_over_kda_throughput": fb["kda"] / fb["ckda"],
+                      "gpu_launches": (fwd_launches(ck, B, T, H, dk, dv) + (4 if tc else 3)) * reps}
     del ws
     return out
 
@@ -592,7 +605,7 @@ def norm_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, plain_value):
         value, secs = aggregate_throughput(B * T * steps, secs, world, device="cuda")
         out[name] = {"value": value, "unit": "tokens/s", "ms_per_step": 1e3 * secs / steps}
     out["fused_over_plain"] = out["fused"]["value"] / plain_value
-    out["gpu_launches"] = steps
+    out["gpu_launches"] = steps * fwd_launches(ck, B, T, H, dk, v.shape[-1])
     return out
 
 
@@ -616,7 +629,7 @@ def kda_measure(ck, q, k, v, a, b, o, ST, stream, world, steps, ckda_value):
     value, secs = aggregate_throughput(B * T * steps, secs, world, device="cuda")
     return {"workload": "layer, gate given as g = ln|alpha| (non-negative gate, KDA form)",
             "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * secs / steps,
-            "ckda_over_kda": ckda_value / value, "gpu_launches": steps}
+            "ckda_over_kda": ckda_value / value, "gpu_launches": steps * fwd_launches(ck, B, T, H, dk, dk)}
 
 
 def e2e_measure(ck, inp, dev, stream, world, args):

@@ -395,9 +395,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // kFlagMapsOnly in flags_in treats segment 0 like the others (the whole launch builds
     // affine maps: z = 0 the state from zero with flags_in, z = 1 the transition product).
     if (!kFast && (flags_in & kFlagRedo) != 0) {
-        // the fast instance's second pass: only the sequences it marked run, from the start
+        // the fast instance's second pass: only the sequences it marked run, from the start (the
+        // mark is in o, or with checkpoints in the last chunk's checkpoint)
         const int b0 = (int)blockIdx.x / H, h0 = (int)blockIdx.x % H;
-        const volatile float* mk = S_ck + (((size_t)b0 * T + (T - 1)) * H + h0) * dv_in;
+        const int nch = (T + C - 1) / C;
+        const volatile float* mk = kStoreStates ? S_ck + ((size_t)blockIdx.x * nch + (nch - 1)) * dk * dv_in
+                                                : S_ck + (((size_t)b0 * T + (T - 1)) * H + h0) * dv_in;
         if (__float_as_uint(*mk) != kRedoMark) return;
     }
     const bool trans = !kFast && blockIdx.z != 0;
@@ -406,7 +409,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const bool direct = sg == 0 && (flags_in & kFlagMapsOnly) == 0;   // segment 0 from the known S0
     if (trans && direct) return;
     // the checkpoint instance may run the direct segment without o (the backward needs states only)
-    const uint32_t flags = kFast ? 0u
+    const uint32_t flags = kFast ? (kStoreStates ? (flags_in & kFlagNoO) : 0u)
                          : trans ? (flags_in | kFlagVZero | kFlagNoO | kFlagS0Ident)
                                  : (direct ? (kStoreStates ? (flags_in & kFlagNoO) : 0u) : flags_in);
     const int dv = trans ? dk : dv_in;
@@ -687,19 +690,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         snew[4 * i4 + 1] = __float_as_uint(s1 * fs.y);
                         snew[4 * i4 + 2] = __float_as_uint(s2 * fs.z);
                         snew[4 * i4 + 3] = __float_as_uint(s3 * fs.w);
+                        if constexpr (kStoreStates) {
+                            // the checkpoint S[c][v] = acc[c][v] kappa_prev[c]; lanes are consecutive v
+                            // (128-byte rows); d_k is 64 or 128, so the 4 rows are in or out together
+                            if (store_states && me < dv && 16 * cb + 4 * i4 < dk) {
+                                float* dst = Sck_seq + ((size_t)(ta / C + ck) * dk + 16 * cb + 4 * i4) * dv + me;
+                                dst[0] = s0;
+                                dst[(size_t)dv] = s1;
+                                dst[2 * (size_t)dv] = s2;
+                                dst[3 * (size_t)dv] = s3;
+                            }
+                        }
                     }
                     uint32_t hi[8], lo[8];
                     split_pack16(z, hi, lo);
                     tc::tmem_st32<8>(te + TM_SAHI + 8 * cb, hi);
                     tc::tmem_st32<8>(te + TM_SALO + 8 * cb, lo);
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
-                    if (kStoreStates && store_states && me < dv) {
-                        // S[c][v] = acc[c][v] kappa_prev[c]; lanes are consecutive v: 128-byte rows
-                        float* dst = Sck_seq + ((size_t)(ta / C + ck) * dk + 16 * cb) * dv + me;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (16 * cb + i < dk) dst[(size_t)i * dv] = cur[i] * sh_kp[par * D + 16 * cb + i];
-                    }
                 }
             }
             // the previous chunk's o rows, once the compute warps are done with the alpha space
@@ -807,9 +814,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 if (n2) tc::mbar_wait(&bar_tma2, (n2 - 1) & 1u);
             }
             if constexpr (kFast) {
-                // mark the sequence for the general instance's second pass (S_ck points at o; the
-                // last token's row is in a chunk this CTA did not reach, so nothing else writes it)
-                if (ebail) S_ck[(((size_t)b * T + (T - 1)) * H + h) * dv_in] = __uint_as_float(kRedoMark);
+                // mark the sequence for the general instance's second pass: in o (S_ck points at it;
+                // the last token's row is in a chunk this CTA did not reach) or, with checkpoints, in
+                // the last chunk's checkpoint (written only when that chunk starts)
+                if (ebail) {
+                    if constexpr (kStoreStates)
+                        Sck_seq[(size_t)(nchunks - 1) * dk * dv] = __uint_as_float(kRedoMark);
+                    else
+                        S_ck[(((size_t)b * T + (T - 1)) * H + h) * dv_in] = __uint_as_float(kRedoMark);
+                }
             }
         }
     } else {

@@ -248,8 +248,11 @@ using ChunkTcKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMa
 // attribute set on the current device
 inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKernel& kern, bool store_states = false,
                                        bool fast = false) {
-    static std::atomic<uint64_t> attr_done[12];
-    if (store_states)
+    static std::atomic<uint64_t> attr_done[16];
+    if (store_states && fast)
+        kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true, true, true> : chunk_tc_kernel<true, false, true, true>)
+                        : (norm_qk ? chunk_tc_kernel<false, true, true, true> : chunk_tc_kernel<false, false, true, true>);
+    else if (store_states)
         kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true, true> : chunk_tc_kernel<true, false, true>)
                         : (norm_qk ? chunk_tc_kernel<false, true, true> : chunk_tc_kernel<false, false, true>);
     else if (fast)
@@ -258,7 +261,7 @@ inline cudaError_t chunk_tc_kernel_for(bool log_gate, bool norm_qk, ChunkTcKerne
     else
         kern = log_gate ? (norm_qk ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
                         : (norm_qk ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
-    const int variant = (store_states ? 4 : fast ? 8 : 0) + (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
+    const int variant = (store_states ? 4 : 0) + (fast ? 8 : 0) + (log_gate ? 2 : 0) + (norm_qk ? 1 : 0);
     return ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)ctc::SMEM_ALLOC, attr_done[variant]);
 }
 
@@ -296,6 +299,21 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
             kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
                                                                          nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0,
                                                                          ctc::kFlagRedo, o);
+            return cudaGetLastError();
+        }
+        if (T > 0) {
+            // with checkpoints: the same pair of launches, the mark in the last chunk's checkpoint
+            ChunkTcKernel fast = nullptr;
+            cudaError_t e = chunk_tc_kernel_for(log_gate, norm_qk, fast, true, true);
+            if (e != cudaSuccess) return e;
+            fast<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
+                                                                         nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0, extra,
+                                                                         S_ck);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,
+                                                                         nullptr, ST, nullptr, T, H, dk, dv, T, 1, 0,
+                                                                         extra | ctc::kFlagRedo, S_ck);
             return cudaGetLastError();
         }
         kern<<<dim3(nbh, 1, 1), ctc::NT_ALL, ctc::SMEM_ALLOC, st>>>(mp.k, mp.q, mp.v, mp.a, mp.o, beta, S0, nullptr,

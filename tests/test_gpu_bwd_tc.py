@@ -91,3 +91,32 @@ def test_quarter_turn_repeated(ck):
     from test_gpu_chunk_tc import quarter_turn_inputs
     inp = quarter_turn_inputs(1, 512, 2, seed=11)
     run_case(ck, "bwd-tc quarter-turn", inp, seed=12)
+
+
+def test_direct_launch_with_exact_path_chunks(ck):
+    """One CTA per sequence for the checkpoint forward (128 sequences): the sequences whose gates
+    leave the factored range in some chunk (first, middle, partial last) are left by the
+    checkpoint instance without the exact path and redone by the general one; the gradients of
+    those and of ordinary sequences match the oracle (sampled sequences, each sliced out)."""
+    B, T, H = 8, 190, 16
+    assert ck.chunk_segments(B, T, H, 128, 128) == 1
+    inp = make_inputs(B, T, H, 128, 128, torch.bfloat16, seed=31, gate="tanh15", s0_std=0.3)
+    inp.alpha[0, 70:75, 0, :40] = 1e-20         # chunk 1
+    inp.alpha[3, 3:9, 5, 60:70] = -1e-22        # chunk 0
+    inp.alpha[7, 150:156, 15, :] = 1e-25        # the partial last chunk
+    g = torch.Generator().manual_seed(32)
+    dO = torch.randn(B, T, H, 128, generator=g)
+    dST = torch.randn(B, H, 128, 128, generator=g)
+    q, k, v, a, b, s0 = to_dev(inp)
+    got = ck.bwd(q, k, v, a, b, dO.cuda(), s0, dST.cuda())
+    torch.cuda.synchronize()
+    assert ck.get_device_error() == 0
+    for (bb, hh) in [(0, 0), (3, 5), (7, 15), (2, 9)]:
+        sl = lambda x: x[bb:bb + 1, :, hh:hh + 1]
+        want = oracle_bwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.alpha), sl(inp.beta), sl(dO),
+                          S0=inp.S0[bb:bb + 1, hh:hh + 1], dST=dST[bb:bb + 1, hh:hh + 1])
+        for n in NAMES:
+            x = got[n][bb:bb + 1, hh:hh + 1] if n == "dS0" else got[n][bb:bb + 1, :, hh:hh + 1]
+            x = x.double().cpu().numpy()
+            assert np.isfinite(x).all(), (bb, hh, n)
+            check(f"bwd-tc direct-exact ({bb},{hh})/{n}", x, want[n], TAU_TC)
