@@ -546,11 +546,12 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
     out_bytes = 3 * dk * 4 + dv * 4 + 4                             # dq, dk, dalpha, dv, dbeta
     alg = B * T * H * (in_bytes + out_bytes) + B * H * dk * dv * 4   # + dS0
     hbm, _ = peaks()
-    kernels = ("chunk_tc_kernel (forward, chunk checkpoints) + chunk_bwd_chain_kernel + chunk_bwd_grad_kernel "
-               "(tcgen05)" if tc else "bwd_ckpt_kernel + bwd_grad_kernel + bwd_sum_kernel (fp32 CUDA cores)")
+    kernels = ("chunk_tc_kernel (forward with chunk checkpoints, then its redo pass) + chunk_bwd_chain_kernel + "
+               "chunk_bwd_grad_kernel + chunk_bwd_grad_exact_kernel (tcgen05)" if tc
+               else "bwd_ckpt_kernel + bwd_grad_kernel + bwd_sum_kernel (fp32 CUDA cores)")
     out = {"workload": f"layer B={B} T={T} H={H} dk={dk} dv={dv}, backward of <dO, o> (S0 = 0)",
            "path": "chunk_tc" if tc else "recurrent",
-           "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": (4 if tc else 3) * reps,
+           "value": value, "unit": "tokens/s", "ms_per_step": 1e3 * per, "gpu_launches": (5 if tc else 3) * reps,
            "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm, "unit": "GB/s",
                         "frac": alg / per / 1e9 / hbm, "alg_bytes_per_launch": alg, "kernels": kernels}}
 
@@ -576,7 +577,7 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
                       "ckda_ms": fb["ckda"], "kda_ms": fb["kda"],
                       "kda_gate": "g = ln|alpha| (non-negative gate) through the log-gate mode",
                       "ckda_over_kda_throughput": fb["kda"] / fb["ckda"],
-                      "gpu_launches": (fwd_launches(ck, B, T, H, dk, dv) + (4 if tc else 3)) * reps}
+                      "gpu_launches": (fwd_launches(ck, B, T, H, dk, dv) + (5 if tc else 3)) * reps}
     del ws
     return out
 

@@ -108,16 +108,19 @@ constexpr uint32_t TM_Q1 = 448;         // rows of blocks 2, 3 against block 0 (
 
 }  // namespace cbg
 
-template <bool kLogGate>
-__global__ void __launch_bounds__(cbg::NTG, 1)
-chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
-                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
-                      const __grid_constant__ CUtensorMap map_s0, const __grid_constant__ CUtensorMap map_dsc,
-                      const float* __restrict__ gate, const __nv_bfloat16* __restrict__ kraw,
-                      const __nv_bfloat16* __restrict__ qraw, const float* __restrict__ beta,
-                      const float* __restrict__ dO, const float* __restrict__ Sck, const float* __restrict__ dSC,
-                      const float* __restrict__ dWx, float* grad_q, float* grad_k, float* grad_gate,
-                      float* grad_beta, int T, int H, int dk, int dv) {
+// One chunk's gradients (cid = (batch, head) * chunks + chunk). kExact = false: the factored
+// path; a chunk whose gate range needs the exact path is only flagged in slow_flags (1, else 0)
+// and left to the kExact instance, which runs flagged chunks only. Keeping the exact path's
+// code out of the factored instance keeps it out of that kernel's instruction stream.
+template <bool kLogGate, bool kExact>
+__device__ __forceinline__ void
+grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap& map_v, const CUtensorMap& map_a,
+           const CUtensorMap& map_s0, const CUtensorMap& map_dsc, const float* __restrict__ gate,
+           const __nv_bfloat16* __restrict__ kraw, const __nv_bfloat16* __restrict__ qraw,
+           const float* __restrict__ beta, const float* __restrict__ dO, const float* __restrict__ Sck,
+           const float* __restrict__ dSC, const float* __restrict__ dWx, float* grad_q, float* grad_k,
+           float* grad_gate, float* grad_beta, int T, int H, int dk, int dv, int cid, uint8_t* slow_flags,
+           bool relinquish) {
     using namespace cbg;
     using ctc::chunk_off;
     using ctc::at_idx;
@@ -153,8 +156,8 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     const int quarter = warp & 3, hh = warp >> 2;
     const int m = quarter * 32 + lane;      // TMEM lane: channel, feature or row
     const int nchunks = (T + C - 1) / C;
-    const int ck = blockIdx.x % nchunks;
-    const int bh = blockIdx.x / nchunks;
+    const int ck = cid % nchunks;
+    const int bh = cid / nchunks;
     const int b = bh / H, h = bh % H;
     const int t0 = ck * C;
     const int nvalid = min(C, T - t0);
@@ -217,7 +220,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     uint32_t par = 0;
     float LC = 0.f, Lofs = 0.f;
     uint32_t pC = 0;
-    bool slow;
+    bool slow_rt;                           // the chunk's gate range needs the exact path
     {
         float gv[32];
 #pragma unroll
@@ -253,12 +256,15 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             sh_pC[m] = pC;
             bad = (-LC > kChunkRange);
         }
-        slow = sync_or(bad);
+        slow_rt = sync_or(bad);
+        if constexpr (!kExact) {
+            if (tid == 0) slow_flags[cid] = slow_rt ? 1 : 0;
+        }
         sh_run16[hh * 128 + m] = L[15];
         LC = sh_LC[m];
         pC = sh_pC[m];
         if (hh == 0) {
-            if (!slow) {
+            if (!kExact) {
                 sh_g[m] = exp2f(0.5f * LC);
                 sh_kap[m] = (pC ? -1.f : 1.f) * exp2f(LC - 0.5f * LC);
             } else {
@@ -269,7 +275,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         // L relative to the chunk start: add the first half's total on the second half
 #pragma unroll
         for (int i = 0; i < 32; ++i) L[i] += Lofs;
-        if (slow) {
+        if (kExact) {
             float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
             __syncthreads();                 // every alpha value read before L overwrites the tile
 #pragma unroll
@@ -283,9 +289,9 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     }
     // factors: e1 = sgn 2^(L - R), e2 = sgn 2^(R - L) with R = L_C / 2 (exact path: e1 = Gamma,
     // e2 = Gamma_C / Gamma); the last pass recomputes L and reads k, q again per 16-token block
-    const float cref = slow ? 0.f : 0.5f * LC;
-    const uint32_t sCbit = slow ? (pC << 31) : 0u;
-    const float d2ref = slow ? LC : 0.f;
+    const float cref = kExact ? 0.f : 0.5f * LC;
+    const uint32_t sCbit = kExact ? (pC << 31) : 0u;
+    const float d2ref = kExact ? LC : 0.f;
     // k and q of this thread's tokens as one packed bf16 pair each (q high, k low): exact, and half
     // the registers of two float arrays
     uint32_t kq[32];
@@ -355,7 +361,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     const uint32_t sb = tc::smem_u32(sm);
     // [P ; A] = X Y^T (3 passes) into TM_D1 (the exact path computes A pairwise instead; its L is
     // then read from the at[] tile, which keeps Diag(b) L)
-    if (!slow) {
+    if (!kExact) {
         if (tid == 0) {
             const uint32_t i128 = tc::idesc_bf16(128, 128, 1, 1), i64 = tc::idesc_bf16(128, 64, 1, 1);
             #pragma unroll 1
@@ -412,7 +418,8 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
             at[at_idx(r, sc)] = (sc < r) ? br * va[j] : 0.f;
         }
     }
-    if (sync_or(fail)) goto done;
+    // the factored instance leaves a chunk that needs the exact path (flagged above)
+    if (sync_or(fail || (!kExact && slow_rt))) goto done;
 
     // this thread's column of the entering state (lane v, channels 64 hh ..), in flight during the solve
     float s0c[64];
@@ -771,7 +778,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         sh_dgc[hh * 128 + m] = dgc;
     }
     // the gate tile again (phase B's staging there is consumed), for the last pass's gate logs
-    if (!slow && tid == 0) {
+    if (!kExact && tid == 0) {
         tc::mbar_arrive_expect_tx(&bar_tma, 4 * 8192);
         for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma, 32 * i, h, t0, b);
         ++tma_next;
@@ -796,7 +803,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         } else {
             const float br = sh_beta[r];
             float l[32];
-            if (!slow) {
+            if (!kExact) {
                 float l2[32];
                 tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, l);
                 tc::tmem_ld32<32>(tl + TM_D1 + 64 + 32 * hh, l2);
@@ -810,11 +817,11 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
                 const int s2 = 32 * hh + i;
                 g8[i] = (s2 < r) ? -g8[i] : 0.f;
                 // entries of X Y^T above the diagonal may overflow: never read them
-                if (!slow && s2 < r) red = fmaf(g8[i], l[i], red);
+                if (!kExact && s2 < r) red = fmaf(g8[i], l[i], red);
                 // the exact path keeps dA itself (its pairwise pass applies b and forms rowsum(dA L))
-                vals[i] = slow ? g8[i] : br * g8[i];
+                vals[i] = kExact ? g8[i] : br * g8[i];
             }
-            if (!slow) atomicAdd(&sh_db[r], red);
+            if (!kExact) atomicAdd(&sh_db[r], red);
         }
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
@@ -833,7 +840,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     //   gk2_s = sum_{r>=s} (dP_rs q_r + b_r dA_rs k_r) R_rs,   R_rs = Gamma_r / Gamma_s (channel c),
     // which stand for d(q e1) e1, d(k e1) e1 and d(k e2) e2, and rowsum(dA (.) L) for d beta
     float gq[32], gk1[32], gk2[32];
-    if (slow) {
+    if (kExact) {
         float* Lsl = reinterpret_cast<float*>(sm + SM_QE1);       // [64 r][128 c] fp32 (G8 done)
         float* kall = reinterpret_cast<float*>(sm + SM_KE1);      // [64][128] fp32 (X, Y unused here)
         float* qall = reinterpret_cast<float*>(sm + SM_KE2);
@@ -901,7 +908,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
     //   CP   [c][s]        = sum over rows of blocks after s's of [q e1 ; k e1]_{rho c} [dP ; b dA]_{rho s}
     //   G10  [c][s]        = the same over every row: d(k e2)
     // Pairs inside one block are summed on CUDA cores in the last pass.
-    if (!slow && tid == 0) {
+    if (!kExact && tid == 0) {
         tc::tc_fence_after();
         const uint32_t i10 = tc::idesc_bf16(128, 64, 0, 1), i64 = tc::idesc_bf16(128, 64, 0, 0),
                        i32 = tc::idesc_bf16(128, 32, 0, 0);
@@ -938,11 +945,11 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_co
         }
         tc::mma_commit(&bar_mma);
     }
-    if (slow && sync_or(fail)) goto done;
+    if (kExact && sync_or(fail)) goto done;
 
     // ================================================================ last pass: thread = channel c,
     // tokens 32 hh .. 32 hh + 31
-    if (!slow) {
+    if (!kExact) {
         const int c = m;
         const float g = sh_g[c], kap = sh_kap[c];
         const float* dpa = reinterpret_cast<const float*>(sm + SM_DPA);
@@ -1301,11 +1308,63 @@ done:
         for (uint32_t p = tma_done; p < tma_next; ++p) tc::mbar_wait(&bar_tma, p & 1u);
     }
     __syncthreads();
+    if (tid == 0) {
+        tc::mbar_inval(&bar_tma);
+        tc::mbar_inval(&bar_mma);
+    }
     if (warp == 0) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tm, 512);
-        tc::tmem_relinquish();
+        if (relinquish) tc::tmem_relinquish();
     }
+    __syncthreads();
+}
+
+template <bool kLogGate>
+__global__ void __launch_bounds__(cbg::NTG, 1)
+chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
+                      const __grid_constant__ CUtensorMap map_s0, const __grid_constant__ CUtensorMap map_dsc,
+                      const float* __restrict__ gate, const __nv_bfloat16* __restrict__ kraw,
+                      const __nv_bfloat16* __restrict__ qraw, const float* __restrict__ beta,
+                      const float* __restrict__ dO, const float* __restrict__ Sck, const float* __restrict__ dSC,
+                      const float* __restrict__ dWx, float* grad_q, float* grad_k, float* grad_gate,
+                      float* grad_beta, int T, int H, int dk, int dv, uint8_t* slow_flags) {
+    grad_chunk<kLogGate, false>(map_k, map_q, map_v, map_a, map_s0, map_dsc, gate, kraw, qraw, beta, dO, Sck, dSC, dWx,
+                                grad_q, grad_k, grad_gate, grad_beta, T, H, dk, dv, (int)blockIdx.x, slow_flags, true);
+}
+
+// The chunks the factored kernel flagged: each CTA takes 32 consecutive flags per step (one warp
+// reads them, a ballot lists the set ones), strided over the grid, and runs those chunks in turn.
+template <bool kLogGate>
+__global__ void __launch_bounds__(cbg::NTG, 1)
+chunk_bwd_grad_exact_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                            const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
+                            const __grid_constant__ CUtensorMap map_s0, const __grid_constant__ CUtensorMap map_dsc,
+                            const float* __restrict__ gate, const __nv_bfloat16* __restrict__ kraw,
+                            const __nv_bfloat16* __restrict__ qraw, const float* __restrict__ beta,
+                            const float* __restrict__ dO, const float* __restrict__ Sck,
+                            const float* __restrict__ dSC, const float* __restrict__ dWx, float* grad_q,
+                            float* grad_k, float* grad_gate, float* grad_beta, int T, int H, int dk, int dv,
+                            const uint8_t* __restrict__ slow_flags, int total) {
+    __shared__ uint32_t s_mask;
+    for (int base = 32 * (int)blockIdx.x; base < total; base += 32 * (int)gridDim.x) {
+        if (threadIdx.x < 32) {
+            const int c = base + (int)threadIdx.x;
+            const uint32_t mask = __ballot_sync(0xffffffffu, c < total && slow_flags[c] != 0);
+            if (threadIdx.x == 0) s_mask = mask;
+        }
+        __syncthreads();
+        uint32_t mask = s_mask;
+        __syncthreads();
+        while (mask != 0u) {
+            const int j = __ffs(mask) - 1;
+            mask &= mask - 1u;
+            grad_chunk<kLogGate, true>(map_k, map_q, map_v, map_a, map_s0, map_dsc, gate, kraw, qraw, beta, dO, Sck, dSC,
+                                       dWx, grad_q, grad_k, grad_gate, grad_beta, T, H, dk, dv, base + j, nullptr, false);
+        }
+    }
+    if (threadIdx.x < 32) tc::tmem_relinquish();
 }
 
 }  // namespace ckda

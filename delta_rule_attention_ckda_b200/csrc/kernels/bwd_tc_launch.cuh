@@ -1,5 +1,6 @@
-// Host side of the backward pass on tensor cores: supported shapes, workspace and the three
-// launches (forward with chunk checkpoints, the reverse chain, the per-chunk gradients).
+// Host side of the backward pass on tensor cores: supported shapes, workspace and the launches
+// (forward with chunk checkpoints, the reverse chain, the per-chunk gradients and their
+// exact-path chunks).
 #pragma once
 #include "chunk_tc_launch.cuh"
 #include "bwd_chain_tc.cuh"
@@ -14,10 +15,11 @@ inline bool bwd_tc_supported(int dk, int dv, int dt, bool norm_qk) {
 }
 
 // workspace, fp32: the state entering every chunk and the cotangent of the state leaving
-// it ([B*H][chunks][d_k][d_v] each), dWx ([B*H][chunks][64][d_v]), then whatever the
+// it ([B*H][chunks][d_k][d_v] each), dWx ([B*H][chunks][64][d_v]), a byte per chunk (the
+// chunks the gradients kernel leaves to its exact-path instance), then whatever the
 // forward's segmented launch needs
 struct BwdTcLayout {
-    size_t ck_off, dsc_off, dwx_off, fwd_off, total;
+    size_t ck_off, dsc_off, dwx_off, flag_off, fwd_off, total;
 };
 
 inline BwdTcLayout bwd_tc_layout(int B, int T, int H, int dk, int dv) {
@@ -27,7 +29,8 @@ inline BwdTcLayout bwd_tc_layout(int B, int T, int H, int dk, int dv) {
     l.ck_off = 0;
     l.dsc_off = align(l.ck_off + bh * n * dk * dv * sizeof(float));
     l.dwx_off = align(l.dsc_off + bh * n * dk * dv * sizeof(float));
-    l.fwd_off = align(l.dwx_off + bh * n * ctc::C * dv * sizeof(float));
+    l.flag_off = align(l.dwx_off + bh * n * ctc::C * dv * sizeof(float));
+    l.fwd_off = align(l.flag_off + bh * n);
     l.total = l.fwd_off + chunk_tc_workspace_bytes(B, T, H, dk, dv);
     return l;
 }
@@ -44,6 +47,7 @@ inline cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
     float* Sck = reinterpret_cast<float*>(ws + l.ck_off);
     float* dSC = reinterpret_cast<float*>(ws + l.dsc_off);
     float* dWx = reinterpret_cast<float*>(ws + l.dwx_off);
+    uint8_t* flags = ws + l.flag_off;
     void* fwd_ws = (l.total > l.fwd_off) ? ws + l.fwd_off : nullptr;
     // 1. the forward from S0, keeping every chunk's entering state (no o)
     cudaError_t e = launch_chunk_tc(q, k, v, gate, beta, S0, nullptr, nullptr, B, T, H, dk, dv, log_gate, false,
@@ -64,12 +68,15 @@ inline cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
     if (!tc::make_map_bthd(&ms0, Sck, f32, 4, 1, ckrows, 1, dv, 32, dk) ||
         !tc::make_map_bthd(&mdsc, dSC, f32, 4, 1, ckrows, 1, dv, 32, dk))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> chain_attr[2], grad_attr[2];
+    static std::atomic<uint64_t> chain_attr[2], grad_attr[2], exact_attr[2];
     auto chain = log_gate ? chunk_bwd_chain_kernel<true> : chunk_bwd_chain_kernel<false>;
     auto grad = log_gate ? chunk_bwd_grad_kernel<true> : chunk_bwd_grad_kernel<false>;
+    auto exact = log_gate ? chunk_bwd_grad_exact_kernel<true> : chunk_bwd_grad_exact_kernel<false>;
     e = ensure_smem_attr(reinterpret_cast<const void*>(chain), (int)cbw::SMEM_ALLOC, chain_attr[log_gate ? 1 : 0]);
     if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(grad), (int)cbg::SMEM_ALLOC, grad_attr[log_gate ? 1 : 0]);
+    if (e != cudaSuccess) return e;
+    e = ensure_smem_attr(reinterpret_cast<const void*>(exact), (int)cbg::SMEM_ALLOC, exact_attr[log_gate ? 1 : 0]);
     if (e != cudaSuccess) return e;
     const unsigned nbh = (unsigned)(B * H), nch = (unsigned)((T + ctc::C - 1) / ctc::C);
     chain<<<nbh, ctc::NT_ALL, cbw::SMEM_ALLOC, st>>>(mk, mq, ma, mdo, beta, dST, dSC, dWx, grad_v, grad_S0, T, H, dk,
@@ -78,7 +85,16 @@ inline cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
     if (e != cudaSuccess) return e;
     // 3. every chunk's gradients, all chunks side by side
     grad<<<nbh * nch, cbg::NTG, cbg::SMEM_ALLOC, st>>>(mk, mq, mv, ma, ms0, mdsc, gate, k, q, beta, dO, Sck, dSC, dWx, grad_q, grad_k,
-                                                      grad_gate, grad_beta, T, H, dk, dv);
+                                                      grad_gate, grad_beta, T, H, dk, dv, flags);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // 4. the chunks whose gate range needs the exact path (none on ordinary gates: one flag read
+    //    per chunk, 32 per CTA step)
+    const int total = (int)(nbh * nch);
+    const int ngrid = std::max(1, std::min(chunk_tc_sm_count(), (total + 31) / 32));
+    exact<<<(unsigned)ngrid, cbg::NTG, cbg::SMEM_ALLOC, st>>>(mk, mq, mv, ma, ms0, mdsc, gate, k, q, beta, dO, Sck, dSC, dWx,
+                                                             grad_q, grad_k, grad_gate, grad_beta, T, H, dk, dv, flags,
+                                                             total);
     return cudaGetLastError();
 }
 
