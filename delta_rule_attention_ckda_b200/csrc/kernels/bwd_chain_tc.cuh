@@ -339,14 +339,15 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
             if (it > 0) efail |= !tc::mbar_wait(&bar_m4, par ^ 1u);
             tc::tc_fence_after();
             {
-                float sv[2][16];
-                tc::tmem_ld32<16>(te + TM_S, sv[0]);
-                float* dst = dSC_seq + (size_t)c * chunk_state;
-#pragma unroll
+                // one 16-column block per step, its TMEM load waited for in the step: this kernel's
+                // chunk loop does not fit the instruction cache, so its code size, not its load
+                // latency, sets this epilogue's time
+                float* dst = dSC_seq + (size_t)c * chunk_state + me;
+#pragma unroll 1
                 for (int cb = 0; cb < 8; ++cb) {
-                    float (&cur)[16] = sv[cb & 1];
+                    float cur[16];
+                    tc::tmem_ld32<16>(te + TM_S + 16 * cb, cur);
                     tc::tmem_ld_wait();
-                    if (cb + 1 < 8) tc::tmem_ld32<16>(te + TM_S + 16 * (cb + 1), sv[(cb + 1) & 1]);
                     float z[16];
                     uint32_t snew[16];
 #pragma unroll
@@ -374,11 +375,12 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
                     tc::tmem_st32<8>(te + TM_SAHI + 8 * cb, hi);
                     tc::tmem_st32<8>(te + TM_SALO + 8 * cb, lo);
                     tc::tmem_st32<16>(te + TM_S + 16 * cb, snew);
-                    if (me < dv) {
-                        // dS_C[c][v]: lanes are consecutive v, so each store is a 128-byte row piece
+                    // dS_C[c][v]: lanes are consecutive v, so each store is a 128-byte row piece; d_k
+                    // is 64 or 128, so the block's 16 rows are in or out together
+                    if (me < dv && 16 * cb < dk) {
+                        float* d0 = dst + (size_t)(16 * cb) * dv;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (16 * cb + i < dk) dst[(size_t)(16 * cb + i) * dv + me] = cur[i];
+                        for (int i = 0; i < 16; ++i) d0[(size_t)i * dv] = cur[i];
                     }
                 }
             }
@@ -427,23 +429,25 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
             {
                 const int t0 = c * C;
                 const int nvalid = min(C, T - t0);
-                float ww[4][16];
-#pragma unroll
-                for (int b16 = 0; b16 < 4; ++b16) tc::tmem_ld32<16>(te + TM_DW + 16 * b16, ww[b16]);
-                tc::tmem_ld_wait();
                 float* wdst = dWx_seq + (size_t)c * C * dv + me;
-#pragma unroll
+                float* vdst = grad_v + (((size_t)b * T + t0) * H + h) * dv + me;
+                const size_t vstride = (size_t)H * dv;
+                // one 16-token block per step (code size over load batching, as in E1)
+#pragma unroll 1
                 for (int b16 = 0; b16 < 4; ++b16) {
+                    float ww[16];
+                    tc::tmem_ld32<16>(te + TM_DW + 16 * b16, ww);
+                    tc::tmem_ld_wait();
                     float w[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int s = 16 * b16 + i;
                         const float bs = sh_beta[par * 64 + s];
                         if (me < dv) {
-                            wdst[(size_t)s * dv] = ww[b16][i];
-                            if (s < nvalid) grad_v[(((size_t)b * T + t0 + s) * H + h) * dv + me] = bs * ww[b16][i];
+                            wdst[(size_t)s * dv] = ww[i];
+                            if (s < nvalid) vdst[(size_t)s * vstride] = bs * ww[i];
                         }
-                        w[i] = bs * ww[b16][i];
+                        w[i] = bs * ww[i];
                     }
                     uint32_t hi[8], mi[8], lo[8];
 #pragma unroll
@@ -621,7 +625,7 @@ chunk_bwd_chain_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_c
                     store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
                 }
                 if (slow) {
-#pragma unroll
+#pragma unroll 1
                     for (int i = 0; i < 32; ++i) {
                         const unsigned bits = __ballot_sync(0xffffffffu, (par >> i) & 1u);
                         if (lane == 0) sh_sign[(32 * hh + i) * 4 + quarter] = bits;
