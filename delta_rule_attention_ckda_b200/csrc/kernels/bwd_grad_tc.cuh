@@ -164,8 +164,8 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const size_t slot = ((size_t)bh * nchunks + ck);
     const float* S0 = Sck + slot * dk * dv;
-    const float* dS = dSC + slot * dk * dv;
     const float* dWxc = dWx + slot * C * dv;
+    const float* wxp = dWxc + (size_t)(32 * hh) * dv + m;   // this thread's dWx column, tokens 32 hh ..
 
     if (warp == 0) tc::tmem_alloc(&tmem_base_s, 512);
     if (tid == 0) {
@@ -179,6 +179,9 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
             tc::tma_load_4d(sm + SM_V + i * 8192, &map_v, &bar_tma, 64 * i, h, t0, b);
         }
         for (int i = 0; i < 4; ++i) tc::tma_load_4d(sm + SM_AL + i * 8192, &map_a, &bar_tma, 32 * i, h, t0, b);
+        // the entering state and dWx rows, read by plain loads later in phase A: into L2 now
+        tc::prefetch_l2_bulk(S0, (uint32_t)(dk * dv) * 4u);
+        tc::prefetch_l2_bulk(dWxc, (uint32_t)(C * dv) * 4u);
     }
     if (tid < C) {
         sh_beta[tid] = (tid < nvalid) ? __ldg(beta + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
@@ -216,28 +219,53 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     // ================================================================ phase A: the forward's quantities
     // gate cumulation: thread = channel m, tokens 32 hh .. 32 hh + 31 (as in the forward)
     fail |= !tc::mbar_wait(&bar_tma, 0);
-    float L[32];
+    float L[32];                            // the exact instance's cumulative log2 gates
     uint32_t par = 0;
     float LC = 0.f, Lofs = 0.f;
     uint32_t pC = 0;
     bool slow_rt;                           // the chunk's gate range needs the exact path
+    // element (token r, channel c) of the alpha tile (the layout ctc::ld_alpha_tile reads)
+    auto al_elem = [&](int r, int c) -> float* {
+        return reinterpret_cast<float*>(sm + SM_AL + (uint32_t)(c >> 5) * 8192u +
+                                        tc::swz128((uint32_t)r * 128u + (uint32_t)(c & 31) * 4u));
+    };
+    // one token's step of the cumulation; returns the gate's sign bit
+    auto gate_step = [&](float av, int r, float& run) -> uint32_t {
+        if constexpr (kLogGate) {
+            const float g = (r < nvalid && m < dk) ? av : 0.f;
+            run += fmaxf(g * kLog2e, kLgFloor);
+            return 0u;
+        } else {
+            const float a = (r < nvalid && m < dk) ? av : 1.f;
+            run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
+            return __float_as_uint(a + 0.f) >> 31;
+        }
+    };
     {
-        float gv[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) gv[i] = ctc::ld_alpha_tile(sm + SM_AL, 32 * hh + i, m);
         float run = 0.f;
+        if constexpr (kExact) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hh + i;
-            if constexpr (kLogGate) {
-                const float g = (r < nvalid && m < dk) ? gv[i] : 0.f;
-                run += fmaxf(g * kLog2e, kLgFloor);
-            } else {
-                const float a = (r < nvalid && m < dk) ? gv[i] : 1.f;
-                run += fmaxf(tc::lg2_approx(fabsf(a)), kLgFloor);
-                par |= (__float_as_uint(a + 0.f) >> 31) << i;
+            for (int i = 0; i < 32; ++i) {
+                par |= gate_step(*al_elem(32 * hh + i, m), 32 * hh + i, run) << i;
+                L[i] = run;
             }
-            L[i] = run;
+            sh_run16[hh * 128 + m] = L[15];
+        } else {
+            // 16 tokens per step; each thread's running log2 sum replaces its own alpha values in
+            // the tile (the last pass loads the gate tile again)
+#pragma unroll 1
+            for (int jb = 0; jb < 2; ++jb) {
+                uint32_t p16 = 0;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int r = 32 * hh + 16 * jb + u;
+                    float* e = al_elem(r, m);
+                    p16 |= gate_step(*e, r, run) << u;
+                    *e = run;
+                }
+                par |= p16 << (16 * jb);
+                if (jb == 0) sh_run16[hh * 128 + m] = run;
+            }
         }
         par ^= par << 1;
         par ^= par << 2;
@@ -250,7 +278,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         if (hh == 1) {
             Lofs = sh_Lx[m];
             if (sh_px[m]) par = ~par;
-            LC = L[31] + Lofs;
+            LC = run + Lofs;
             pC = par >> 31;
             sh_LC[m] = LC;
             sh_pC[m] = pC;
@@ -260,7 +288,6 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         if constexpr (!kExact) {
             if (tid == 0) slow_flags[cid] = slow_rt ? 1 : 0;
         }
-        sh_run16[hh * 128 + m] = L[15];
         LC = sh_LC[m];
         pC = sh_pC[m];
         if (hh == 0) {
@@ -272,10 +299,10 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
                 sh_kap[m] = (pC ? -1.f : 1.f) * exp2f(LC);
             }
         }
-        // L relative to the chunk start: add the first half's total on the second half
+        if constexpr (kExact) {
+            // L relative to the chunk start: add the first half's total on the second half
 #pragma unroll
-        for (int i = 0; i < 32; ++i) L[i] += Lofs;
-        if (kExact) {
+            for (int i = 0; i < 32; ++i) L[i] += Lofs;
             float* Ls = reinterpret_cast<float*>(sm + SM_SLOWL);
             __syncthreads();                 // every alpha value read before L overwrites the tile
 #pragma unroll
@@ -292,17 +319,6 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     const float cref = kExact ? 0.f : 0.5f * LC;
     const uint32_t sCbit = kExact ? (pC << 31) : 0u;
     const float d2ref = kExact ? LC : 0.f;
-    // k and q of this thread's tokens as one packed bf16 pair each (q high, k low): exact, and half
-    // the registers of two float arrays
-    uint32_t kq[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float kf = ctc::ld_bf16_tile(sm + SM_K, 32 * hh + i, m);
-        const float qf = ctc::ld_bf16_tile(sm + SM_Q, 32 * hh + i, m);
-        kq[i] = (__float_as_uint(qf) & 0xffff0000u) | (__float_as_uint(kf) >> 16);
-    }
-    auto kin = [&](int i) -> float { return __uint_as_float(kq[i] << 16); };
-    auto qin = [&](int i) -> float { return __uint_as_float(kq[i] & 0xffff0000u); };
     auto fe1 = [&](float Lv, int i) -> float {
         const uint32_t sg = (par << (31 - i)) & 0x80000000u;
         return __uint_as_float(__float_as_uint(tc::ex2_approx(Lv - cref)) ^ sg);
@@ -311,8 +327,6 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         const uint32_t sg = (par << (31 - i)) & 0x80000000u;
         return __uint_as_float(__float_as_uint(tc::ex2_approx(d2ref - (Lv - cref))) ^ sg ^ sCbit);
     };
-    auto factor_e1 = [&](int i) -> float { return fe1(L[i], i); };
-    auto factor_e2 = [&](int i) -> float { return fe2(L[i], i); };
     // one 16-token block of this thread's tokens (32 hh + 16 jb ..): the cumulative log2 gate by the
     // gate phase's operations in the same order (so bit-identical), and k, q from global memory
     // (read by this CTA's first loads, so normally still in L2), packed q high / k low
@@ -338,20 +352,29 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
             kqb[u] = (qb << 16) | kb;
         }
     };
+    // X = [q e1 ; k e1], Y = k e2 for this thread's tokens, 8 at a time (the factored instance: 16
+    // tokens per step, L from the tile, where it is relative to this half's start)
+#pragma unroll (kExact ? 2 : 1)
+    for (int jb = 0; jb < 2; ++jb) {
 #pragma unroll
-    for (int q8 = 0; q8 < 4; ++q8) {
-        float xk[8], xq[8], yk[8];
+        for (int q8 = 0; q8 < 2; ++q8) {
+            float xk[8], xq[8], yk[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = 8 * q8 + e;
-            const float e1 = factor_e1(i), e2 = factor_e2(i);
-            xk[e] = kin(i) * e1;
-            xq[e] = qin(i) * e1;
-            yk[e] = kin(i) * e2;
+            for (int e = 0; e < 8; ++e) {
+                const int i = 16 * jb + 8 * q8 + e, r = 32 * hh + i;
+                float Lv;
+                if constexpr (kExact) Lv = L[i];
+                else Lv = *al_elem(r, m) + Lofs;
+                const float kf = ctc::ld_bf16_tile(sm + SM_K, r, m), qf = ctc::ld_bf16_tile(sm + SM_Q, r, m);
+                const float e1 = fe1(Lv, i), e2 = fe2(Lv, i);
+                xk[e] = kf * e1;
+                xq[e] = qf * e1;
+                yk[e] = kf * e2;
+            }
+            store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + 2 * jb + q8, xq);
+            store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + 2 * jb + q8, xk);
+            store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + 2 * jb + q8, yk);
         }
-        store_split8(sm + SM_XHI, sm + SM_XLO, m, 4 * hh + q8, xq);
-        store_split8(sm + SM_XHI + 16384, sm + SM_XLO + 16384, m, 4 * hh + q8, xk);
-        store_split8(sm + SM_YHI, sm + SM_YLO, m, 4 * hh + q8, yk);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -375,17 +398,20 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
             tc::mma_commit(&bar_mma);
         }
         mma_wait();
-        float d1[32], d2[32];
-        tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, d1);
-        tc::tmem_ld32<32>(tl + TM_D1 + 64 + 32 * hh, d2);
-        tc::tmem_ld_wait();
-        if (m >= C) {
-            const int r = m - C;
-            const float br = sh_beta[r];
+#pragma unroll 1
+        for (int jh = 0; jh < 2; ++jh) {
+            float d1[16], d2[16];
+            tc::tmem_ld32<16>(tl + TM_D1 + 32 * hh + 16 * jh, d1);
+            tc::tmem_ld32<16>(tl + TM_D1 + 64 + 32 * hh + 16 * jh, d2);
+            tc::tmem_ld_wait();
+            if (m >= C) {
+                const int r = m - C;
+                const float br = sh_beta[r];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int s = 32 * hh + i;
-                at[at_idx(r, s)] = (s < r) ? br * (d1[i] + d2[i]) : 0.f;
+                for (int i = 0; i < 16; ++i) {
+                    const int s = 32 * hh + 16 * jh + i;
+                    at[at_idx(r, s)] = (s < r) ? br * (d1[i] + d2[i]) : 0.f;
+                }
             }
         }
     } else {
@@ -421,13 +447,6 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     // the factored instance leaves a chunk that needs the exact path (flagged above)
     if (sync_or(fail || (!kExact && slow_rt))) goto done;
 
-    // this thread's column of the entering state (lane v, channels 64 hh ..), in flight during the solve
-    float s0c[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-        const int c = 64 * hh + i;
-        s0c[i] = (c < dk && m < dv) ? __ldg(S0 + (size_t)c * dv + m) : 0.f;
-    }
 
     // solve: X = (I + A)^{-1} (the forward's blocked solve), T = X Diag(b) in three bf16 terms
     if (warp < 4 && lane < 16) {
@@ -541,14 +560,20 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off1) = m1;
         *reinterpret_cast<uint32_t*>(sm + SM_TL + off1) = l1;
     }
-    // S0 Diag(g) -> TMEM operand [d_v lanes][d_k]: thread (lane v, half hh) takes columns 64 hh ..
+    // S0 Diag(g) -> TMEM operand [d_v lanes][d_k]: thread (lane v, half hh) takes columns 64 hh ..,
+    // 16 per step from the entering state's column v (in L2 since the kernel's start; d_k is 64 or
+    // 128, so a half's channels are all in or all out)
     {
-#pragma unroll
+        const bool s0ok = 64 * hh < dk && m < dv;
+#pragma unroll 1
         for (int cb = 0; cb < 4; ++cb) {
             const int c0 = 64 * hh + 16 * cb;
+            const float* p = S0 + (size_t)c0 * dv + m;
             float z[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = s0c[16 * cb + i] * sh_g[c0 + i];
+            for (int i = 0; i < 16; ++i) z[i] = s0ok ? __ldg(p + (size_t)i * dv) : 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z[i] *= sh_g[c0 + i];
             uint32_t hi[8], lo[8];
             split_pack16(z, hi, lo);
             tc::tmem_st32<8>(tl + TM_SA + c0 / 2, hi);
@@ -574,29 +599,31 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         tc::mma_commit(&bar_mma);
     }
     mma_wait();
-    // -Z^T -> TMEM operand (thread: lane v, tokens 32 hh ..)
-    float zreg[32];
+    // -Z^T -> TMEM operand (thread: lane v, tokens 32 hh .., 16 per step); Z^T stays in TM_Z for the
+    // U epilogue
     {
-        tc::tmem_ld32<32>(tl + TM_Z + 32 * hh, zreg);
-        tc::tmem_ld_wait();
-        float nz[32];
+#pragma unroll 1
+        for (int jh = 0; jh < 2; ++jh) {
+            float nz[16];
+            tc::tmem_ld32<16>(tl + TM_Z + 32 * hh + 16 * jh, nz);
+            tc::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) nz[i] = -zreg[i];
-        uint32_t hi[16], lo[16];
-        ctc::split_pack32(nz, hi, lo);
-        tc::tmem_st32<16>(tl + TM_ZAHI + 16 * hh, hi);
-        tc::tmem_st32<16>(tl + TM_ZALO + 16 * hh, lo);
+            for (int i = 0; i < 16; ++i) nz[i] = -nz[i];
+            uint32_t hi[8], lo[8];
+            split_pack16(nz, hi, lo);
+            tc::tmem_st32<8>(tl + TM_ZAHI + 16 * hh + 8 * jh, hi);
+            tc::tmem_st32<8>(tl + TM_ZALO + 16 * hh + 8 * jh, lo);
+        }
     }
     tc::tmem_st_wait();
     tc::tc_fence_before();
     __syncthreads();
-    // dWx of this thread's column (lane v, tokens 32 hh ..), in flight during the U product
-    float wdx[32];
+    // dWx of this thread's column (lane v, tokens 32 hh ..): the first 16 in flight during the U
+    // product. The workspace holds all 64 rows of every chunk, so the rows past the sequence's end
+    // are read too and masked where they are used.
+    float wdx[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int s = 32 * hh + i;
-        wdx[i] = (m < dv && s < nvalid) ? __ldg(dWxc + (size_t)s * dv + m) : 0.f;
-    }
+    for (int i = 0; i < 16; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)i * dv) : 0.f;
     // U^T = (V - Z)^T [T_hi ; T_mid]^T + (V - Z)^T T_lo^T: the forward's U product
     if (tid == 0) {
         tc::tc_fence_after();
@@ -627,41 +654,51 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     if (sync_or(fail)) goto done;
 
     // U -> K-major tiles [64 s][64 v] per d_v half (hi / lo), and d beta's rowsum(W (.) dWx):
-    // thread (lane v, tokens 32 hh ..)
+    // thread (lane v, tokens 32 hh .., 16 per step)
     {
-        float u1[32], u2[32];
-        tc::tmem_ld32<32>(tl + TM_DU + 32 * hh, u1);
-        tc::tmem_ld32<32>(tl + TM_DU + 64 + 32 * hh, u2);
-        tc::tmem_ld_wait();
         const int v = m, vh = v >> 6, vc = v & 63;
-        float w[32];
+#pragma unroll 1
+        for (int jh = 0; jh < 2; ++jh) {
+            float u1[16], u2[16], zr[16];
+            tc::tmem_ld32<16>(tl + TM_DU + 32 * hh + 16 * jh, u1);
+            tc::tmem_ld32<16>(tl + TM_DU + 64 + 32 * hh + 16 * jh, u2);
+            tc::tmem_ld32<16>(tl + TM_Z + 32 * hh + 16 * jh, zr);
+            tc::tmem_ld_wait();
+            float w[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int s = 32 * hh + i;
-            const float u = u1[i] + u2[i];
-            __nv_bfloat16 hb, lb;
-            const float uh = __bfloat162float(hb = __float2bfloat16_rn(u));
-            lb = __float2bfloat16_rn(u - uh);
-            const uint32_t off = (uint32_t)vh * 8192u + chunk_off(s, vc >> 3) + (uint32_t)(vc & 7) * 2u;
-            *reinterpret_cast<__nv_bfloat16*>(sm + SM_UHI + off) = hb;
-            *reinterpret_cast<__nv_bfloat16*>(sm + SM_ULO + off) = lb;
-            // W = V - Z at (s, v) times dWx at (s, v)
-            const float vv = ctc::ld_bf16_tile(sm + SM_V, s, v);
-            w[i] = (v < dv && s < nvalid) ? (vv - zreg[i]) * wdx[i] : 0.f;
-        }
-        // sum over the warp's 32 d_v lanes for all 32 tokens at once (halving exchange: lane l ends
-        // with token 32 hh + l), then over the four lane quarters by shared atomics
-#pragma unroll
-        for (int off2 = 16; off2 >= 1; off2 >>= 1) {
-            const bool up = (lane & off2) != 0;
-#pragma unroll
-            for (int k = 0; k < off2; ++k) {
-                const float send = up ? w[k] : w[k + off2];
-                const float keep = up ? w[k + off2] : w[k];
-                w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off2);
+            for (int i = 0; i < 16; ++i) {
+                const int s = 32 * hh + 16 * jh + i;
+                const float u = u1[i] + u2[i];
+                __nv_bfloat16 hb, lb;
+                const float uh = __bfloat162float(hb = __float2bfloat16_rn(u));
+                lb = __float2bfloat16_rn(u - uh);
+                const uint32_t off = (uint32_t)vh * 8192u + chunk_off(s, vc >> 3) + (uint32_t)(vc & 7) * 2u;
+                *reinterpret_cast<__nv_bfloat16*>(sm + SM_UHI + off) = hb;
+                *reinterpret_cast<__nv_bfloat16*>(sm + SM_ULO + off) = lb;
+                // W = V - Z at (s, v) times dWx at (s, v)
+                const float vv = ctc::ld_bf16_tile(sm + SM_V, s, v);
+                w[i] = (v < dv && s < nvalid) ? (vv - zr[i]) * wdx[i] : 0.f;
             }
+            if (jh == 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)(16 + i) * dv) : 0.f;
+            }
+            // sum over the warp's 32 d_v lanes for the 16 tokens at once (halving exchange within
+            // each 16-lane half: lane l ends with token l & 15, then the two halves add), then over
+            // the four lane quarters by shared atomics
+#pragma unroll
+            for (int off2 = 8; off2 >= 1; off2 >>= 1) {
+                const bool up = (lane & off2) != 0;
+#pragma unroll
+                for (int k = 0; k < off2; ++k) {
+                    const float send = up ? w[k] : w[k + off2];
+                    const float keep = up ? w[k + off2] : w[k];
+                    w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off2);
+                }
+            }
+            w[0] += __shfl_xor_sync(0xffffffffu, w[0], 16);
+            if (lane < 16) atomicAdd(&sh_db[32 * hh + 16 * jh + lane], w[0]);
         }
-        atomicAdd(&sh_db[32 * hh + lane], w[0]);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -788,48 +825,53 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     // token block (row 32 blk + 16 half + u for token 16 blk + u of half dP / dA), so that the rows of
     // every run of blocks are one contiguous MMA operand.
     {
-        float g8[32];
-        tc::tmem_ld32<32>(tl + TM_G8 + 32 * hh, g8);
-        tc::tmem_ld_wait();
-        const int half = m >> 6, r = m & 63;
-        float vals[32];
+        const int half = m >> 6, r = m & 63;   // warp-uniform half
         float* dpa = reinterpret_cast<float*>(sm + SM_DPA);
-        if (half == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                g8[i] = (32 * hh + i <= r) ? g8[i] : 0.f;
-                vals[i] = g8[i];
-            }
-        } else {
-            const float br = sh_beta[r];
-            float l[32];
-            if (!kExact) {
-                float l2[32];
-                tc::tmem_ld32<32>(tl + TM_D1 + 32 * hh, l);
-                tc::tmem_ld32<32>(tl + TM_D1 + 64 + 32 * hh, l2);
+        const float br = sh_beta[r];
+        const int rho = 32 * (r >> 4) + 16 * half + (r & 15);
+        float red = 0.f;
+        // 16 tokens per step
+#pragma unroll 1
+        for (int jh = 0; jh < 2; ++jh) {
+            const int s0 = 32 * hh + 16 * jh;
+            float g8[16], l[16], vals[16];
+            tc::tmem_ld32<16>(tl + TM_G8 + s0, g8);
+            if (!kExact && half == 1) {
+                float l2[16];
+                tc::tmem_ld32<16>(tl + TM_D1 + s0, l);
+                tc::tmem_ld32<16>(tl + TM_D1 + 64 + s0, l2);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) l[i] += l2[i];
+                for (int i = 0; i < 16; ++i) l[i] += l2[i];
+            } else {
+                tc::tmem_ld_wait();
             }
-            float red = 0.f;
+            if (half == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int s2 = 32 * hh + i;
-                g8[i] = (s2 < r) ? -g8[i] : 0.f;
-                // entries of X Y^T above the diagonal may overflow: never read them
-                if (!kExact && s2 < r) red = fmaf(g8[i], l[i], red);
-                // the exact path keeps dA itself (its pairwise pass applies b and forms rowsum(dA L))
-                vals[i] = kExact ? g8[i] : br * g8[i];
+                for (int i = 0; i < 16; ++i) {
+                    g8[i] = (s0 + i <= r) ? g8[i] : 0.f;
+                    vals[i] = g8[i];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int s2 = s0 + i;
+                    g8[i] = (s2 < r) ? -g8[i] : 0.f;
+                    // entries of X Y^T above the diagonal may overflow: never read them
+                    if (!kExact && s2 < r) red = fmaf(g8[i], l[i], red);
+                    // the exact path keeps dA itself (its pairwise pass applies b and forms rowsum(dA L))
+                    vals[i] = kExact ? g8[i] : br * g8[i];
+                }
             }
-            if (!kExact) atomicAdd(&sh_db[r], red);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<float4*>(dpa + dpa_idx(m, s0 + 4 * q4)) =
+                    make_float4(g8[4 * q4], g8[4 * q4 + 1], g8[4 * q4 + 2], g8[4 * q4 + 3]);
+#pragma unroll
+            for (int q8 = 0; q8 < 2; ++q8)
+                store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + 2 * jh + q8, vals + 8 * q8);
         }
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-            *reinterpret_cast<float4*>(dpa + dpa_idx(m, 32 * hh + 4 * q4)) =
-                make_float4(g8[4 * q4], g8[4 * q4 + 1], g8[4 * q4 + 2], g8[4 * q4 + 3]);
-        const int rho = 32 * (r >> 4) + 16 * half + (r & 15);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + q8, vals + 8 * q8);
+        if (!kExact && half == 1) atomicAdd(&sh_db[r], red);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
