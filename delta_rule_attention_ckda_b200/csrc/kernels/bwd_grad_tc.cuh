@@ -108,6 +108,40 @@ constexpr uint32_t TM_Q1 = 448;         // rows of blocks 2, 3 against block 0 (
 
 }  // namespace cbg
 
+// One out-of-line copy of the 8-value split and store into 16-byte chunk `off` of a hi and a lo
+// tile (shared-memory addresses): called from several phases, it keeps their instruction stream
+// short.
+__device__ __noinline__ void split8_store(uint32_t hi_s, uint32_t lo_s, uint32_t off, float x0, float x1, float x2,
+                                          float x3, float x4, float x5, float x6, float x7) {
+    uint32_t ph[4], pl[4];
+    ctc::split2(x0, x1, ph[0], pl[0]);
+    ctc::split2(x2, x3, ph[1], pl[1]);
+    ctc::split2(x4, x5, ph[2], pl[2]);
+    ctc::split2(x6, x7, ph[3], pl[3]);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hi_s + off), "r"(ph[0]), "r"(ph[1]), "r"(ph[2]),
+                 "r"(ph[3]) : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lo_s + off), "r"(pl[0]), "r"(pl[1]), "r"(pl[2]),
+                 "r"(pl[3]) : "memory");
+}
+
+// One out-of-line copy of the 16-value split into packed bf16 hi / lo pairs and their TMEM stores
+// (8 columns each at t_hi and t_lo; every lane of the warp calls it).
+__device__ __noinline__ void split16_tmem(uint32_t t_hi, uint32_t t_lo, float x0, float x1, float x2, float x3,
+                                          float x4, float x5, float x6, float x7, float x8, float x9, float x10,
+                                          float x11, float x12, float x13, float x14, float x15) {
+    uint32_t hi[8], lo[8];
+    ctc::split2(x0, x1, hi[0], lo[0]);
+    ctc::split2(x2, x3, hi[1], lo[1]);
+    ctc::split2(x4, x5, hi[2], lo[2]);
+    ctc::split2(x6, x7, hi[3], lo[3]);
+    ctc::split2(x8, x9, hi[4], lo[4]);
+    ctc::split2(x10, x11, hi[5], lo[5]);
+    ctc::split2(x12, x13, hi[6], lo[6]);
+    ctc::split2(x14, x15, hi[7], lo[7]);
+    tc::tmem_st32<8>(t_hi, hi);
+    tc::tmem_st32<8>(t_lo, lo);
+}
+
 // One chunk's gradients (cid = (batch, head) * chunks + chunk). kExact = false: the factored
 // path; a chunk whose gate range needs the exact path is only flagged in slow_flags (1, else 0)
 // and left to the kExact instance, which runs flagged chunks only. Keeping the exact path's
@@ -126,7 +160,16 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     using ctc::at_idx;
     using ctc::split2;
     using ctc::split3;
-    using ctc::store_split8;
+    // split 16 values into TMEM hi / lo operand columns through the out-of-line copy
+    auto split_tmem16 = [&](uint32_t t_hi, uint32_t t_lo, const float (&x)[16]) {
+        split16_tmem(t_hi, t_lo, x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], x[8], x[9], x[10], x[11], x[12], x[13],
+                     x[14], x[15]);
+    };
+    // ctc::store_split8 through the out-of-line copy
+    auto store_split8 = [&](uint8_t* hi, uint8_t* lo, int row, int ch, const float* x) {
+        split8_store(tc::smem_u32(hi), tc::smem_u32(lo), ctc::chunk_off(row, ch), x[0], x[1], x[2], x[3], x[4], x[5],
+                     x[6], x[7]);
+    };
     using ctc::split_pack16;
     using ctc::mma3_tf32;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -399,17 +442,17 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         }
         mma_wait();
 #pragma unroll 1
-        for (int jh = 0; jh < 2; ++jh) {
-            float d1[16], d2[16];
-            tc::tmem_ld32<16>(tl + TM_D1 + 32 * hh + 16 * jh, d1);
-            tc::tmem_ld32<16>(tl + TM_D1 + 64 + 32 * hh + 16 * jh, d2);
+        for (int j8 = 0; j8 < 4; ++j8) {
+            float d1[8], d2[8];
+            tc::tmem_ld32<8>(tl + TM_D1 + 32 * hh + 8 * j8, d1);
+            tc::tmem_ld32<8>(tl + TM_D1 + 64 + 32 * hh + 8 * j8, d2);
             tc::tmem_ld_wait();
             if (m >= C) {
                 const int r = m - C;
                 const float br = sh_beta[r];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int s = 32 * hh + 16 * jh + i;
+                for (int i = 0; i < 8; ++i) {
+                    const int s = 32 * hh + 8 * j8 + i;
                     at[at_idx(r, s)] = (s < r) ? br * (d1[i] + d2[i]) : 0.f;
                 }
             }
@@ -476,7 +519,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         if (warp < 4) {
             const int pb = warp >> 1, nt = warp & 1, o = 32 * pb;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
             for (int ks = 0; ks < 2; ++ks) {
                 if (ks < nt) continue;
                 const int s0 = o + 8 * ks + ft, s1 = s0 + 4, r0 = o + 16 + fg, r1 = r0 + 8;
@@ -489,7 +532,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
             *reinterpret_cast<float2*>(sc + (fg + 8) * 8 + 2 * ft) = make_float2(d[2], d[3]);
             __syncwarp();
             float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
             for (int ks = 0; ks < 2; ++ks) {
                 const int rr = o + 16 + fg, cc = o + 16 + 8 * ks + ft;
                 const float a[4] = {xs[rr * XS_LD + cc], xs[(rr + 8) * XS_LD + cc], xs[rr * XS_LD + cc + 4],
@@ -503,7 +546,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         __syncthreads();
         const int mt = warp >> 2, nt = warp & 3;
         float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks) {
             if (ks < nt) continue;
             const int s0 = 8 * ks + ft, s1 = s0 + 4, r0 = 32 + 16 * mt + fg, r1 = r0 + 8;
@@ -538,7 +581,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         if (half == 0)
             *reinterpret_cast<uint4*>(sm + SM_TL + chunk_off(lane, 4 + (warp & 3))) = make_uint4(0u, 0u, 0u, 0u);
         float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks) {
             if (ks > 2 * mt + 1) continue;
             const int rr = 32 + 16 * mt + fg, cc = 32 + 8 * ks + ft;
@@ -574,10 +617,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
             for (int i = 0; i < 16; ++i) z[i] = s0ok ? __ldg(p + (size_t)i * dv) : 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) z[i] *= sh_g[c0 + i];
-            uint32_t hi[8], lo[8];
-            split_pack16(z, hi, lo);
-            tc::tmem_st32<8>(tl + TM_SA + c0 / 2, hi);
-            tc::tmem_st32<8>(tl + TM_SA + 64 + c0 / 2, lo);
+            split_tmem16(tl + TM_SA + c0 / 2, tl + TM_SA + 64 + c0 / 2, z);
         }
     }
     tc::tmem_st_wait();
@@ -609,21 +649,18 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
             tc::tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) nz[i] = -nz[i];
-            uint32_t hi[8], lo[8];
-            split_pack16(nz, hi, lo);
-            tc::tmem_st32<8>(tl + TM_ZAHI + 16 * hh + 8 * jh, hi);
-            tc::tmem_st32<8>(tl + TM_ZALO + 16 * hh + 8 * jh, lo);
+            split_tmem16(tl + TM_ZAHI + 16 * hh + 8 * jh, tl + TM_ZALO + 16 * hh + 8 * jh, nz);
         }
     }
     tc::tmem_st_wait();
     tc::tc_fence_before();
     __syncthreads();
-    // dWx of this thread's column (lane v, tokens 32 hh ..): the first 16 in flight during the U
+    // dWx of this thread's column (lane v, tokens 32 hh ..): the first 8 in flight during the U
     // product. The workspace holds all 64 rows of every chunk, so the rows past the sequence's end
     // are read too and masked where they are used.
-    float wdx[16];
+    float wdx[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)i * dv) : 0.f;
+    for (int i = 0; i < 8; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)i * dv) : 0.f;
     // U^T = (V - Z)^T [T_hi ; T_mid]^T + (V - Z)^T T_lo^T: the forward's U product
     if (tid == 0) {
         tc::tc_fence_after();
@@ -654,40 +691,45 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     if (sync_or(fail)) goto done;
 
     // U -> K-major tiles [64 s][64 v] per d_v half (hi / lo), and d beta's rowsum(W (.) dWx):
-    // thread (lane v, tokens 32 hh .., 16 per step)
+    // thread (lane v, tokens 32 hh .., 8 per step)
     {
         const int v = m, vh = v >> 6, vc = v & 63;
+        const uint32_t vcol = (uint32_t)vc * 2u;
 #pragma unroll 1
-        for (int jh = 0; jh < 2; ++jh) {
-            float u1[16], u2[16], zr[16];
-            tc::tmem_ld32<16>(tl + TM_DU + 32 * hh + 16 * jh, u1);
-            tc::tmem_ld32<16>(tl + TM_DU + 64 + 32 * hh + 16 * jh, u2);
-            tc::tmem_ld32<16>(tl + TM_Z + 32 * hh + 16 * jh, zr);
+        for (int j8 = 0; j8 < 4; ++j8) {
+            float u1[8], u2[8], zr[8];
+            tc::tmem_ld32<8>(tl + TM_DU + 32 * hh + 8 * j8, u1);
+            tc::tmem_ld32<8>(tl + TM_DU + 64 + 32 * hh + 8 * j8, u2);
+            tc::tmem_ld32<8>(tl + TM_Z + 32 * hh + 8 * j8, zr);
             tc::tmem_ld_wait();
-            float w[16];
+            float w[8];
+            // (s, v) in the U tiles and in the v tile: both are [64 s][64 v] bf16 per d_v half with
+            // the 128-byte swizzle, so one offset serves the three; s = 32 hh + 8 j8 + i has
+            // s & 7 = i
+            const uint32_t rowb = (uint32_t)vh * 8192u + (uint32_t)(32 * hh + 8 * j8) * 128u;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int s = 32 * hh + 16 * jh + i;
+            for (int i = 0; i < 8; ++i) {
+                const int s = 32 * hh + 8 * j8 + i;
                 const float u = u1[i] + u2[i];
                 __nv_bfloat16 hb, lb;
                 const float uh = __bfloat162float(hb = __float2bfloat16_rn(u));
                 lb = __float2bfloat16_rn(u - uh);
-                const uint32_t off = (uint32_t)vh * 8192u + chunk_off(s, vc >> 3) + (uint32_t)(vc & 7) * 2u;
+                const uint32_t off = rowb + (uint32_t)i * 128u + (vcol ^ ((uint32_t)i << 4));
                 *reinterpret_cast<__nv_bfloat16*>(sm + SM_UHI + off) = hb;
                 *reinterpret_cast<__nv_bfloat16*>(sm + SM_ULO + off) = lb;
                 // W = V - Z at (s, v) times dWx at (s, v)
-                const float vv = ctc::ld_bf16_tile(sm + SM_V, s, v);
+                const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + SM_V + off));
                 w[i] = (v < dv && s < nvalid) ? (vv - zr[i]) * wdx[i] : 0.f;
             }
-            if (jh == 0) {
+            if (j8 < 3) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)(16 + i) * dv) : 0.f;
+                for (int i = 0; i < 8; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)(8 * j8 + 8 + i) * dv) : 0.f;
             }
-            // sum over the warp's 32 d_v lanes for the 16 tokens at once (halving exchange within
-            // each 16-lane half: lane l ends with token l & 15, then the two halves add), then over
+            // sum over the warp's 32 d_v lanes for the 8 tokens at once (halving exchange within
+            // each 8-lane group: lane l ends with token l & 7, then the four groups add), then over
             // the four lane quarters by shared atomics
 #pragma unroll
-            for (int off2 = 8; off2 >= 1; off2 >>= 1) {
+            for (int off2 = 4; off2 >= 1; off2 >>= 1) {
                 const bool up = (lane & off2) != 0;
 #pragma unroll
                 for (int k = 0; k < off2; ++k) {
@@ -696,8 +738,9 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
                     w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off2);
                 }
             }
+            w[0] += __shfl_xor_sync(0xffffffffu, w[0], 8);
             w[0] += __shfl_xor_sync(0xffffffffu, w[0], 16);
-            if (lane < 16) atomicAdd(&sh_db[32 * hh + 16 * jh + lane], w[0]);
+            if (lane < 8) atomicAdd(&sh_db[32 * hh + 8 * j8 + lane], w[0]);
         }
     }
     tc::fence_proxy_async_smem();
@@ -723,17 +766,18 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         if (tid == 0) issue_q(0);
         float x[32];
         const int rp_b = tid >> 1, vq_b = tid & 1;
+        // this thread's row: dO of token r' (r' < 64) or dWx of token r' - 64; its 32 columns of a d_v
+        // half lie all inside d_v or all outside (d_v is 64 or 128)
+        const float* xrow = (rp_b < 64) ? dO + (((size_t)b * T + t0 + rp_b) * H + h) * dv
+                                        : dWxc + (size_t)(rp_b - 64) * dv;
+        const bool xrow_ok = (rp_b & 63) < nvalid;
         auto load_x = [&](int vh) {
-            const int r = rp_b & 63;
-            const bool is_do = rp_b < 64;
+            const int v0 = 64 * vh + 32 * vq_b;
+            const bool ok = xrow_ok && v0 < dv;
+            const float4* src = reinterpret_cast<const float4*>(xrow + v0);
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4) {
-                const int v = 64 * vh + 32 * vq_b + 4 * j4;
-                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r < nvalid && v < dv) {
-                    f = is_do ? __ldg(reinterpret_cast<const float4*>(dO + (((size_t)b * T + t0 + r) * H + h) * dv + v))
-                              : __ldg(reinterpret_cast<const float4*>(dWxc + (size_t)r * dv + v));
-                }
+                const float4 f = ok ? __ldg(src + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
                 x[4 * j4] = f.x; x[4 * j4 + 1] = f.y; x[4 * j4 + 2] = f.z; x[4 * j4 + 3] = f.w;
             }
         };
@@ -767,13 +811,8 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
                     }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) dgc = fmaf(s0v[j], dsv[j], dgc);
-                    uint32_t hi[8], lo[8];
-                    split_pack16(s0v, hi, lo);
-                    tc::tmem_st32<8>(tl + TM_S0HI + 16 * qq + 8 * hh, hi);
-                    tc::tmem_st32<8>(tl + TM_S0LO + 16 * qq + 8 * hh, lo);
-                    split_pack16(dsv, hi, lo);
-                    tc::tmem_st32<8>(tl + TM_DSHI + 16 * qq + 8 * hh, hi);
-                    tc::tmem_st32<8>(tl + TM_DSLO + 16 * qq + 8 * hh, lo);
+                    split_tmem16(tl + TM_S0HI + 16 * qq + 8 * hh, tl + TM_S0LO + 16 * qq + 8 * hh, s0v);
+                    split_tmem16(tl + TM_DSHI + 16 * qq + 8 * hh, tl + TM_DSLO + 16 * qq + 8 * hh, dsv);
                 }
                 tc::tmem_st_wait();
                 tc::fence_proxy_async_smem();
@@ -830,31 +869,31 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         const float br = sh_beta[r];
         const int rho = 32 * (r >> 4) + 16 * half + (r & 15);
         float red = 0.f;
-        // 16 tokens per step
+        // 8 tokens per step
 #pragma unroll 1
-        for (int jh = 0; jh < 2; ++jh) {
-            const int s0 = 32 * hh + 16 * jh;
-            float g8[16], l[16], vals[16];
-            tc::tmem_ld32<16>(tl + TM_G8 + s0, g8);
+        for (int j8 = 0; j8 < 4; ++j8) {
+            const int s0 = 32 * hh + 8 * j8;
+            float g8[8], l[8], vals[8];
+            tc::tmem_ld32<8>(tl + TM_G8 + s0, g8);
             if (!kExact && half == 1) {
-                float l2[16];
-                tc::tmem_ld32<16>(tl + TM_D1 + s0, l);
-                tc::tmem_ld32<16>(tl + TM_D1 + 64 + s0, l2);
+                float l2[8];
+                tc::tmem_ld32<8>(tl + TM_D1 + s0, l);
+                tc::tmem_ld32<8>(tl + TM_D1 + 64 + s0, l2);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) l[i] += l2[i];
+                for (int i = 0; i < 8; ++i) l[i] += l2[i];
             } else {
                 tc::tmem_ld_wait();
             }
             if (half == 0) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     g8[i] = (s0 + i <= r) ? g8[i] : 0.f;
                     vals[i] = g8[i];
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     const int s2 = s0 + i;
                     g8[i] = (s2 < r) ? -g8[i] : 0.f;
                     // entries of X Y^T above the diagonal may overflow: never read them
@@ -864,12 +903,10 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
                 }
             }
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
+            for (int q4 = 0; q4 < 2; ++q4)
                 *reinterpret_cast<float4*>(dpa + dpa_idx(m, s0 + 4 * q4)) =
                     make_float4(g8[4 * q4], g8[4 * q4 + 1], g8[4 * q4 + 2], g8[4 * q4 + 3]);
-#pragma unroll
-            for (int q8 = 0; q8 < 2; ++q8)
-                store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + 2 * jh + q8, vals + 8 * q8);
+            store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + j8, vals);
         }
         if (!kExact && half == 1) atomicAdd(&sh_db[r], red);
     }
@@ -1216,7 +1253,7 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         const float other_pre = (hh == 1) ? sh_red2[c] : 0.f;
         const float add0 = cst + other_sfx + other_pre + sfx1 + ((hh == 1) ? q2 : 0.f);
         const float add1 = cst + other_sfx + other_pre + pre0 + ((hh == 0) ? sh_q1[c] : 0.f);
-#pragma unroll 2
+#pragma unroll 1
         for (int i = 0; i < 32; ++i) {
             const int r = 32 * hh + i;
             if (r < nvalid && c < dk) {

@@ -72,7 +72,10 @@ __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// The poll loop stays rolled: try_wait already suspends the thread for a while, and an unrolled
+// copy at every wait site would only lengthen the kernel's instruction stream.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = kSpinLimit) {
+#pragma unroll 1
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, phase)) return true;
     report_error(kErrTimeout);
@@ -147,6 +150,14 @@ __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint
 // 32 lanes x 32-bit, N consecutive columns: thread t of the warp gets lane (lane0 + t).
 template <int N>
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld32<8>(uint32_t taddr, float (&r)[8]) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
 
 template <>
 __device__ __forceinline__ void tmem_ld32<16>(uint32_t taddr, float (&r)[16]) {
