@@ -279,8 +279,9 @@ __device__ __forceinline__ void split_pack16(const float (&x)[16], uint32_t (&hi
 }
 
 // Every compute thread waits on the barrier; true if any of them timed out.
+template <bool kRolled = true>
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity) {
-    const bool ok = tc::mbar_wait(bar, parity);
+    const bool ok = tc::mbar_wait<kRolled>(bar, parity);
     return csync_or(!ok);
 }
 
@@ -346,6 +347,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 const float* S0_head, const float* S0_seg, float* ST_seg, float* ST_last, float* M_seg,
                 int T, int H, int dk, int dv_in, int seg_len, int nseg, int sg_base, uint32_t flags_in,
                 float* S_ck) {
+    // the mbarrier poll loops: left to the compiler's unrolling in the direct launch's plain
+    // instance (measured faster there), rolled in the others (shorter code)
+    constexpr bool kRollWaits = !(kFast && !kStoreStates);
     using namespace ctc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -654,7 +658,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // S = acc kappa_prev, then the operand S g_ref (split into TMEM) and the new
             // accumulator S fs. Two separate products: kappa_prev g_ref alone can underflow fp32
             // for fast-decaying channels although each factor and each result is in range.
-            efail |= !tc::mbar_wait(&bar_hk[par], (uint32_t)(ck >> 1) & 1u);   // this chunk's constants
+            efail |= !tc::mbar_wait<kRollWaits>(&bar_hk[par], (uint32_t)(ck >> 1) & 1u);   // this chunk's constants
             if constexpr (kFast) {
                 // the compute warps stopped at this chunk (it needs the exact path): every epilogue
                 // thread waited for the same hand-off, so all leave here together
@@ -663,7 +667,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     break;
                 }
             }
-            if (ck > 0) efail |= !tc::mbar_wait(&bar_c2, par ^ 1u);
+            if (ck > 0) efail |= !tc::mbar_wait<kRollWaits>(&bar_c2, par ^ 1u);
             tc::tc_fence_after();
             {
                 float sv[2][16];
@@ -711,7 +715,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             }
             // the previous chunk's o rows, once the compute warps are done with the alpha space
             // (hap); their store and the next alpha go out before C1
-            efail |= !tc::mbar_wait(&bar_hap, par);
+            efail |= !tc::mbar_wait<kRollWaits>(&bar_hap, par);
             if (ck > 0) stage_o();
             epi_publish();
             if (esync_or(efail)) break;
@@ -732,7 +736,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 issue_c1(sbase);
             }
             // ---------------- E2: -Z^T -> TMEM operand of the U MMA
-            efail |= !tc::mbar_wait(&bar_c1, par);
+            efail |= !tc::mbar_wait<kRollWaits>(&bar_c1, par);
             tc::tc_fence_after();
             float zz[4][16];
 #pragma unroll
@@ -752,14 +756,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             if (esync_or(efail)) break;
             // leader: once T is written (and A consumed): the next chunk's k, then U
             if (leader) {
-                efail |= !tc::mbar_wait(&bar_ht, par);
+                efail |= !tc::mbar_wait<kRollWaits>(&bar_ht, par);
                 tc::tc_fence_after();
                 if (ck + 1 < nchunks) issue_loads1b(t0 + C);
                 if (!v_zero) issue_uv(sbase);
                 issue_uz(sbase, !v_zero);
             }
             // ---------------- E3: U^T -> TMEM operand of the O / state MMA
-            efail |= !tc::mbar_wait(&bar_u, par);
+            efail |= !tc::mbar_wait<kRollWaits>(&bar_u, par);
             tc::tc_fence_after();
             if (leader && ck + 1 < nchunks) issue_loads2(t0 + C);      // V and T consumed
             float uu[4][16];
@@ -791,7 +795,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
         // last chunk's o rows, once its O MMA is done and the previous o tile has been stored
         if (ck == nchunks && nchunks > 0) {
-            efail |= !tc::mbar_wait(&bar_c2, (uint32_t)(nchunks - 1) & 1u);
+            efail |= !tc::mbar_wait<kRollWaits>(&bar_c2, (uint32_t)(nchunks - 1) & 1u);
             tc::tc_fence_after();
             if (leader) tc::bulk_wait_read0();
             if (!esync_or(efail)) {
@@ -806,12 +810,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         if (leader) {
             tc::bulk_wait0();
             tc::mma_commit(&bar_drain[0]);
-            tc::mbar_wait(&bar_drain[0], 0);
+            tc::mbar_wait<kRollWaits>(&bar_drain[0], 0);
             if (efail || ebail) {
                 // loads whose data nobody waited for: let them land before shared memory is released
-                if (n1a) tc::mbar_wait(&bar_tma1a, (n1a - 1) & 1u);
-                if (n1b) tc::mbar_wait(&bar_tma1b, (n1b - 1) & 1u);
-                if (n2) tc::mbar_wait(&bar_tma2, (n2 - 1) & 1u);
+                if (n1a) tc::mbar_wait<kRollWaits>(&bar_tma1a, (n1a - 1) & 1u);
+                if (n1b) tc::mbar_wait<kRollWaits>(&bar_tma1b, (n1b - 1) & 1u);
+                if (n2) tc::mbar_wait<kRollWaits>(&bar_tma2, (n2 - 1) & 1u);
             }
             if constexpr (kFast) {
                 // mark the sequence for the general instance's second pass: in o (S_ck points at it;
@@ -847,7 +851,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // the per-channel constants and the exact-path decision. True if a wait gave up.
         auto gate_logs = [&](int ckn) -> bool {
             const int nvalid = min(C, tb - (ta + ckn * C));
-            wfail |= !tc::mbar_wait(&bar_tma1a, ckn & 1);
+            wfail |= !tc::mbar_wait<kRollWaits>(&bar_tma1a, ckn & 1);
             // this thread's 32 gate values first (every address lies inside the tile; rows past
             // the end and channels past d_k are replaced by the neutral gate below), then the chain
             float gv[32];
@@ -932,11 +936,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             // ---------------- P1: gate factors (thread = channel m, tokens 32hh .. 32hh+31)
             {
                 // k, q and v of this chunk
-                wfail |= !tc::mbar_wait(&bar_tma1b, ck & 1);
-                wfail |= !tc::mbar_wait(&bar_tma2, ck & 1);
+                wfail |= !tc::mbar_wait<kRollWaits>(&bar_tma1b, ck & 1);
+                wfail |= !tc::mbar_wait<kRollWaits>(&bar_tma2, ck & 1);
                 // the previous chunk's C1 reads X: wait for it before overwriting
                 if (ck > 0) {
-                    wfail |= !tc::mbar_wait(&bar_c1, ph_c1);
+                    wfail |= !tc::mbar_wait<kRollWaits>(&bar_c1, ph_c1);
                     ph_c1 ^= 1u;
                 }
                 if constexpr (kNormQK) {
@@ -1011,7 +1015,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
                 // the previous chunk's O / state MMA reads Y and P: wait for it before writing Y
                 if (ck > 0) {
-                    wfail |= !tc::mbar_wait(&bar_c2, ph_c2);
+                    wfail |= !tc::mbar_wait<kRollWaits>(&bar_c2, ph_c2);
                     ph_c2 ^= 1u;
                     tc::tc_fence_after();
                 }
@@ -1046,7 +1050,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     tc::tc_fence_after();
                     issue_ap(sbase);
                 }
-                wfail |= !tc::mbar_wait(&bar_ap, ph_ap);
+                wfail |= !tc::mbar_wait<kRollWaits>(&bar_ap, ph_ap);
                 ph_ap ^= 1u;
                 tc::tc_fence_after();
                 // ---------------- P3: A (fp32, column-major) and P (hi/lo) out of TMEM
@@ -1264,7 +1268,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         if (!failed && csync_or(wfail)) failed = true;
         // last chunk's state MMA
         if (!failed && nchunks > 0) {
-            if (wait_all(&bar_c2, ph_c2)) failed = true;
+            if (wait_all<kRollWaits>(&bar_c2, ph_c2)) failed = true;
             else tc::tc_fence_after();
         }
 
@@ -1283,7 +1287,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
         if (tid == 0) {
             tc::mma_commit(&bar_drain[1]);
-            tc::mbar_wait(&bar_drain[1], 0);
+            tc::mbar_wait<kRollWaits>(&bar_drain[1], 0);
         }
     }
     tc::tc_fence_before();

@@ -72,12 +72,21 @@ __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// The poll loop stays rolled: try_wait already suspends the thread for a while, and an unrolled
-// copy at every wait site would only lengthen the kernel's instruction stream.
+// Bounded wait. kRolled (the default) keeps the poll loop rolled: try_wait already suspends the
+// thread for a while, and the copy the compiler otherwise unrolls at every wait site lengthens
+// the kernel's instruction stream (by 30 to 70 KB in the backward kernels). kRolled = false
+// leaves the unrolling to the compiler, which the forward's direct-launch instance measures
+// about 1% faster with.
+template <bool kRolled = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = kSpinLimit) {
+    if constexpr (kRolled) {
 #pragma unroll 1
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, phase)) return true;
+        for (uint32_t i = 0; i < limit; ++i)
+            if (mbar_try_wait(bar, phase)) return true;
+    } else {
+        for (uint32_t i = 0; i < limit; ++i)
+            if (mbar_try_wait(bar, phase)) return true;
+    }
     report_error(kErrTimeout);
     return false;
 }
