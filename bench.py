@@ -559,7 +559,7 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
     o = torch.empty(B, T, H, dv, device=q.device)
     ST = torch.empty(B, H, dk, dv, device=q.device)
     glog = torch.log(a.abs())
-    fb = {}
+    steps = {}
     for name, gate, gin in (("ckda", "signed", a), ("kda", "log", glog)):
         def fwd_bwd(gate=gate, gin=gin):
             ck.chunk_fwd(q, k, v, gin, b, None, o=o, S_T=ST, gate=gate)
@@ -568,16 +568,25 @@ def bwd_measure(ck, q, k, v, a, b, stream, world, reps=3):
         fwd_bwd()
         torch.cuda.synchronize()
         assert ck.get_device_error() == 0
-        barrier(world)
-        s = time_launches(fwd_bwd, reps, stream)
-        assert ck.get_device_error() == 0
-        _, s = aggregate_throughput(B * T * reps, s, world, device="cuda")
-        fb[name] = 1e3 * s / reps
+        steps[name] = fwd_bwd
+    # trials alternating the two gates; each arm's median (one trial is a few ms, so a single one
+    # is at the mercy of a transient)
+    trials = 5
+    fb = {name: [] for name in steps}
+    barrier(world)
+    for _ in range(trials):
+        for name, fn in steps.items():
+            s = time_launches(fn, reps, stream)
+            assert ck.get_device_error() == 0
+            _, s = aggregate_throughput(B * T * reps, s, world, device="cuda")
+            fb[name].append(1e3 * s / reps)
+    med = {name: sorted(t)[len(t) // 2] for name, t in fb.items()}
     out["fwd_bwd"] = {"workload": "layer: forward (o, S_T) then backward, per step",
-                      "ckda_ms": fb["ckda"], "kda_ms": fb["kda"],
+                      "ckda_ms": med["ckda"], "kda_ms": med["kda"],
+                      "timing": f"median of {trials} trials of {reps} steps per gate, the gates alternating",
                       "kda_gate": "g = ln|alpha| (non-negative gate) through the log-gate mode",
-                      "ckda_over_kda_throughput": fb["kda"] / fb["ckda"],
-                      "gpu_launches": (fwd_launches(ck, B, T, H, dk, dv) + (5 if tc else 3)) * reps}
+                      "ckda_over_kda_throughput": med["kda"] / med["ckda"],
+                      "gpu_launches": (fwd_launches(ck, B, T, H, dk, dv) + (5 if tc else 3)) * reps * trials}
     del ws
     return out
 

@@ -442,17 +442,17 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         }
         mma_wait();
 #pragma unroll 1
-        for (int j8 = 0; j8 < 4; ++j8) {
-            float d1[8], d2[8];
-            tc::tmem_ld32<8>(tl + TM_D1 + 32 * hh + 8 * j8, d1);
-            tc::tmem_ld32<8>(tl + TM_D1 + 64 + 32 * hh + 8 * j8, d2);
+        for (int jh = 0; jh < 2; ++jh) {
+            float d1[16], d2[16];
+            tc::tmem_ld32<16>(tl + TM_D1 + 32 * hh + 16 * jh, d1);
+            tc::tmem_ld32<16>(tl + TM_D1 + 64 + 32 * hh + 16 * jh, d2);
             tc::tmem_ld_wait();
             if (m >= C) {
                 const int r = m - C;
                 const float br = sh_beta[r];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int s = 32 * hh + 8 * j8 + i;
+                for (int i = 0; i < 16; ++i) {
+                    const int s = 32 * hh + 16 * jh + i;
                     at[at_idx(r, s)] = (s < r) ? br * (d1[i] + d2[i]) : 0.f;
                 }
             }
@@ -655,12 +655,6 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     tc::tmem_st_wait();
     tc::tc_fence_before();
     __syncthreads();
-    // dWx of this thread's column (lane v, tokens 32 hh ..): the first 8 in flight during the U
-    // product. The workspace holds all 64 rows of every chunk, so the rows past the sequence's end
-    // are read too and masked where they are used.
-    float wdx[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)i * dv) : 0.f;
     // U^T = (V - Z)^T [T_hi ; T_mid]^T + (V - Z)^T T_lo^T: the forward's U product
     if (tid == 0) {
         tc::tc_fence_after();
@@ -691,45 +685,44 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     if (sync_or(fail)) goto done;
 
     // U -> K-major tiles [64 s][64 v] per d_v half (hi / lo), and d beta's rowsum(W (.) dWx):
-    // thread (lane v, tokens 32 hh .., 8 per step)
+    // thread (lane v, tokens 32 hh .., 16 per step)
+    // dWx comes from this thread's column (in L2 since the kernel's start); the workspace holds all
+    // 64 rows of every chunk, so the rows past the sequence's end are read too and masked here.
     {
         const int v = m, vh = v >> 6, vc = v & 63;
         const uint32_t vcol = (uint32_t)vc * 2u;
 #pragma unroll 1
-        for (int j8 = 0; j8 < 4; ++j8) {
-            float u1[8], u2[8], zr[8];
-            tc::tmem_ld32<8>(tl + TM_DU + 32 * hh + 8 * j8, u1);
-            tc::tmem_ld32<8>(tl + TM_DU + 64 + 32 * hh + 8 * j8, u2);
-            tc::tmem_ld32<8>(tl + TM_Z + 32 * hh + 8 * j8, zr);
+        for (int jh = 0; jh < 2; ++jh) {
+            float u1[16], u2[16], zr[16];
+            tc::tmem_ld32<16>(tl + TM_DU + 32 * hh + 16 * jh, u1);
+            tc::tmem_ld32<16>(tl + TM_DU + 64 + 32 * hh + 16 * jh, u2);
+            tc::tmem_ld32<16>(tl + TM_Z + 32 * hh + 16 * jh, zr);
             tc::tmem_ld_wait();
-            float w[8];
+            float w[16];
             // (s, v) in the U tiles and in the v tile: both are [64 s][64 v] bf16 per d_v half with
-            // the 128-byte swizzle, so one offset serves the three; s = 32 hh + 8 j8 + i has
-            // s & 7 = i
-            const uint32_t rowb = (uint32_t)vh * 8192u + (uint32_t)(32 * hh + 8 * j8) * 128u;
+            // the 128-byte swizzle, so one offset serves the three; s = 32 hh + 16 jh + i has
+            // s & 7 = i & 7
+            const uint32_t rowb = (uint32_t)vh * 8192u + (uint32_t)(32 * hh + 16 * jh) * 128u;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int s = 32 * hh + 8 * j8 + i;
+            for (int i = 0; i < 16; ++i) {
+                const int s = 32 * hh + 16 * jh + i;
                 const float u = u1[i] + u2[i];
                 __nv_bfloat16 hb, lb;
                 const float uh = __bfloat162float(hb = __float2bfloat16_rn(u));
                 lb = __float2bfloat16_rn(u - uh);
-                const uint32_t off = rowb + (uint32_t)i * 128u + (vcol ^ ((uint32_t)i << 4));
+                const uint32_t off = rowb + (uint32_t)i * 128u + (vcol ^ ((uint32_t)(i & 7) << 4));
                 *reinterpret_cast<__nv_bfloat16*>(sm + SM_UHI + off) = hb;
                 *reinterpret_cast<__nv_bfloat16*>(sm + SM_ULO + off) = lb;
                 // W = V - Z at (s, v) times dWx at (s, v)
                 const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + SM_V + off));
-                w[i] = (v < dv && s < nvalid) ? (vv - zr[i]) * wdx[i] : 0.f;
+                const float wd = (m < dv) ? __ldg(wxp + (size_t)(16 * jh + i) * dv) : 0.f;
+                w[i] = (v < dv && s < nvalid) ? (vv - zr[i]) * wd : 0.f;
             }
-            if (j8 < 3) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) wdx[i] = (m < dv) ? __ldg(wxp + (size_t)(8 * j8 + 8 + i) * dv) : 0.f;
-            }
-            // sum over the warp's 32 d_v lanes for the 8 tokens at once (halving exchange within
-            // each 8-lane group: lane l ends with token l & 7, then the four groups add), then over
+            // sum over the warp's 32 d_v lanes for the 16 tokens at once (halving exchange within
+            // each 16-lane half: lane l ends with token l & 15, then the two halves add), then over
             // the four lane quarters by shared atomics
 #pragma unroll
-            for (int off2 = 4; off2 >= 1; off2 >>= 1) {
+            for (int off2 = 8; off2 >= 1; off2 >>= 1) {
                 const bool up = (lane & off2) != 0;
 #pragma unroll
                 for (int k = 0; k < off2; ++k) {
@@ -738,9 +731,8 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
                     w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off2);
                 }
             }
-            w[0] += __shfl_xor_sync(0xffffffffu, w[0], 8);
             w[0] += __shfl_xor_sync(0xffffffffu, w[0], 16);
-            if (lane < 8) atomicAdd(&sh_db[32 * hh + 8 * j8 + lane], w[0]);
+            if (lane < 16) atomicAdd(&sh_db[32 * hh + 16 * jh + lane], w[0]);
         }
     }
     tc::fence_proxy_async_smem();
@@ -869,31 +861,31 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         const float br = sh_beta[r];
         const int rho = 32 * (r >> 4) + 16 * half + (r & 15);
         float red = 0.f;
-        // 8 tokens per step
+        // 16 tokens per step
 #pragma unroll 1
-        for (int j8 = 0; j8 < 4; ++j8) {
-            const int s0 = 32 * hh + 8 * j8;
-            float g8[8], l[8], vals[8];
-            tc::tmem_ld32<8>(tl + TM_G8 + s0, g8);
+        for (int jh = 0; jh < 2; ++jh) {
+            const int s0 = 32 * hh + 16 * jh;
+            float g8[16], l[16], vals[16];
+            tc::tmem_ld32<16>(tl + TM_G8 + s0, g8);
             if (!kExact && half == 1) {
-                float l2[8];
-                tc::tmem_ld32<8>(tl + TM_D1 + s0, l);
-                tc::tmem_ld32<8>(tl + TM_D1 + 64 + s0, l2);
+                float l2[16];
+                tc::tmem_ld32<16>(tl + TM_D1 + s0, l);
+                tc::tmem_ld32<16>(tl + TM_D1 + 64 + s0, l2);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) l[i] += l2[i];
+                for (int i = 0; i < 16; ++i) l[i] += l2[i];
             } else {
                 tc::tmem_ld_wait();
             }
             if (half == 0) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     g8[i] = (s0 + i <= r) ? g8[i] : 0.f;
                     vals[i] = g8[i];
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     const int s2 = s0 + i;
                     g8[i] = (s2 < r) ? -g8[i] : 0.f;
                     // entries of X Y^T above the diagonal may overflow: never read them
@@ -903,10 +895,11 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
                 }
             }
 #pragma unroll
-            for (int q4 = 0; q4 < 2; ++q4)
+            for (int q4 = 0; q4 < 4; ++q4)
                 *reinterpret_cast<float4*>(dpa + dpa_idx(m, s0 + 4 * q4)) =
                     make_float4(g8[4 * q4], g8[4 * q4 + 1], g8[4 * q4 + 2], g8[4 * q4 + 3]);
-            store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + j8, vals);
+            store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + 2 * jh, vals);
+            store_split8(sm + SM_DPHI, sm + SM_DPLO, rho, 4 * hh + 2 * jh + 1, vals + 8);
         }
         if (!kExact && half == 1) atomicAdd(&sh_db[r], red);
     }
