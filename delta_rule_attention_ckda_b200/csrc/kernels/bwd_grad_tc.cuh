@@ -108,10 +108,10 @@ constexpr uint32_t TM_Q1 = 448;         // rows of blocks 2, 3 against block 0 (
 
 }  // namespace cbg
 
-// One out-of-line copy of the 8-value split and store into 16-byte chunk `off` of a hi and a lo
-// tile (shared-memory addresses): called from several phases, it keeps their instruction stream
-// short.
-__device__ __noinline__ void split8_store(uint32_t hi_s, uint32_t lo_s, uint32_t off, float x0, float x1, float x2,
+// The 8-value split and store into 16-byte chunk `off` of a hi and a lo tile (shared-memory
+// addresses). Inlined: as an out-of-line call it saved 2 KB of code but, with every register of
+// the kernel live, its calls cost more than the fetch (the backward 3.7% slower).
+__device__ __forceinline__ void split8_store(uint32_t hi_s, uint32_t lo_s, uint32_t off, float x0, float x1, float x2,
                                           float x3, float x4, float x5, float x6, float x7) {
     uint32_t ph[4], pl[4];
     ctc::split2(x0, x1, ph[0], pl[0]);
@@ -124,9 +124,9 @@ __device__ __noinline__ void split8_store(uint32_t hi_s, uint32_t lo_s, uint32_t
                  "r"(pl[3]) : "memory");
 }
 
-// One out-of-line copy of the 16-value split into packed bf16 hi / lo pairs and their TMEM stores
-// (8 columns each at t_hi and t_lo; every lane of the warp calls it).
-__device__ __noinline__ void split16_tmem(uint32_t t_hi, uint32_t t_lo, float x0, float x1, float x2, float x3,
+// The 16-value split into packed bf16 hi / lo pairs and their TMEM stores (8 columns each at t_hi
+// and t_lo; every lane of the warp calls it). Inlined, as split8_store.
+__device__ __forceinline__ void split16_tmem(uint32_t t_hi, uint32_t t_lo, float x0, float x1, float x2, float x3,
                                           float x4, float x5, float x6, float x7, float x8, float x9, float x10,
                                           float x11, float x12, float x13, float x14, float x15) {
     uint32_t hi[8], lo[8];
@@ -160,12 +160,12 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     using ctc::at_idx;
     using ctc::split2;
     using ctc::split3;
-    // split 16 values into TMEM hi / lo operand columns through the out-of-line copy
+    // split 16 values into TMEM hi / lo operand columns
     auto split_tmem16 = [&](uint32_t t_hi, uint32_t t_lo, const float (&x)[16]) {
         split16_tmem(t_hi, t_lo, x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7], x[8], x[9], x[10], x[11], x[12], x[13],
                      x[14], x[15]);
     };
-    // ctc::store_split8 through the out-of-line copy
+    // ctc::store_split8 on shared-memory addresses
     auto store_split8 = [&](uint8_t* hi, uint8_t* lo, int row, int ch, const float* x) {
         split8_store(tc::smem_u32(hi), tc::smem_u32(lo), ctc::chunk_off(row, ch), x[0], x[1], x[2], x[3], x[4], x[5],
                      x[6], x[7]);
