@@ -489,6 +489,15 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
     }
     // the factored instance leaves a chunk that needs the exact path (flagged above)
     if (sync_or(fail || (!kExact && slow_rt))) goto done;
+    // this thread's column v = m of the entering state, channels 64 hh .. (in L2 since the
+    // kernel's start), in flight during the solve; d_k is 64 or 128, so a half's channels are all
+    // in or all out
+    float s0c[64];
+    {
+        const bool s0ok = 64 * hh < dk && m < dv;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s0c[i] = s0ok ? __ldg(S0 + (size_t)(64 * hh + i) * dv + m) : 0.f;
+    }
 
 
     // solve: X = (I + A)^{-1} (the forward's blocked solve), T = X Diag(b) in three bf16 terms
@@ -603,20 +612,14 @@ grad_chunk(const CUtensorMap& map_k, const CUtensorMap& map_q, const CUtensorMap
         *reinterpret_cast<uint32_t*>(sm + SM_T + 8192 + off1) = m1;
         *reinterpret_cast<uint32_t*>(sm + SM_TL + off1) = l1;
     }
-    // S0 Diag(g) -> TMEM operand [d_v lanes][d_k]: thread (lane v, half hh) takes columns 64 hh ..,
-    // 16 per step from the entering state's column v (in L2 since the kernel's start; d_k is 64 or
-    // 128, so a half's channels are all in or all out)
+    // S0 Diag(g) -> TMEM operand [d_v lanes][d_k]: thread (lane v, half hh) takes columns 64 hh ..
     {
-        const bool s0ok = 64 * hh < dk && m < dv;
-#pragma unroll 1
+#pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             const int c0 = 64 * hh + 16 * cb;
-            const float* p = S0 + (size_t)c0 * dv + m;
             float z[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = s0ok ? __ldg(p + (size_t)i * dv) : 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] *= sh_g[c0 + i];
+            for (int i = 0; i < 16; ++i) z[i] = s0c[16 * cb + i] * sh_g[c0 + i];
             split_tmem16(tl + TM_SA + c0 / 2, tl + TM_SA + 64 + c0 / 2, z);
         }
     }
